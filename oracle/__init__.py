@@ -1,0 +1,105 @@
+"""The oracle: plain, slow, f64 CPU causal attention (forward and backward).
+
+TEST INFRASTRUCTURE. Only tests/, the smoke check in __graft_entry__ and the
+bench's CPU-baseline leg may import this package. The product library neither
+imports it nor links it, and the two share no code.
+
+Parity pins (tests/test_oracle.py): torch SDPA in f64 (causal, band mask, GQA by
+repeat_interleave), torch autograd of SDPA, brute-force softmax Jacobian on tiny
+shapes, central finite differences, and the invariants and closed forms of the
+definition. No function here is left unpinned.
+
+Every function takes and returns numpy float64 arrays in [B, H, T, D] layout.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        i = ctypes.c_int
+        d = ctypes.c_double
+        lib.oracle_attn_fwd.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i, d, i, d]
+        lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, d, i, d]
+        lib.oracle_attn_probs.argtypes = [dp, dp, dp, i, i, i, i, i, d, i, d]
+        lib.oracle_rowdot.argtypes = [dp, dp, dp, ctypes.c_long, i]
+        lib.oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    if hasattr(a, "detach"):  # torch tensor
+        a = a.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _dims(q, k):
+    B, Hq, T, D = q.shape
+    Bk, Hkv, Tk, Dk = k.shape
+    assert (B, T, D) == (Bk, Tk, Dk) and Hq % Hkv == 0
+    return B, Hq, Hkv, T, D
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def attn_fwd(q, k, v, scale: float, window: int = 0, softcap: float = 0.0):
+    """Return (o [B,Hq,T,D], lse [B,Hq,T]) in f64."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Hkv, T, D = _dims(q, k)
+    o = np.empty_like(q)
+    lse = np.empty((B, Hq, T), dtype=np.float64)
+    _load().oracle_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, T, D,
+                            float(scale), int(window), float(softcap))
+    return o, lse
+
+
+def attn_bwd(q, k, v, dO, scale: float, window: int = 0, softcap: float = 0.0):
+    """Return (dq, dk, dv, delta, lse) in f64 for upstream gradient dO."""
+    q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
+    B, Hq, Hkv, T, D = _dims(q, k)
+    dq = np.empty_like(q)
+    dk = np.empty_like(k)
+    dv = np.empty_like(v)
+    delta = np.empty((B, Hq, T), dtype=np.float64)
+    lse = np.empty((B, Hq, T), dtype=np.float64)
+    _load().oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dq), _ptr(dk), _ptr(dv),
+                            _ptr(delta), _ptr(lse), B, Hq, Hkv, T, D, float(scale), int(window),
+                            float(softcap))
+    return dq, dk, dv, delta, lse
+
+
+def attn_probs(q, k, scale: float, window: int = 0, softcap: float = 0.0):
+    """Full probability matrix [B,Hq,T,T] (zero where masked). Small shapes only."""
+    q, k = _f64(q), _f64(k)
+    B, Hq, Hkv, T, D = _dims(q, k)
+    P = np.empty((B, Hq, T, T), dtype=np.float64)
+    _load().oracle_attn_probs(_ptr(q), _ptr(k), _ptr(P), B, Hq, Hkv, T, D, float(scale),
+                              int(window), float(softcap))
+    return P
+
+
+def rowdot(o, dO):
+    """Delta = rowsum(dO * O) over the last axis."""
+    o, dO = _f64(o), _f64(dO)
+    out = np.empty(o.shape[:-1], dtype=np.float64)
+    _load().oracle_rowdot(_ptr(o), _ptr(dO), _ptr(out), int(np.prod(o.shape[:-1])), o.shape[-1])
+    return out

@@ -1,0 +1,235 @@
+/*
+ * oracle/attn_ref.c -- plain f64 CPU causal attention, forward and backward.
+ *
+ * TEST INFRASTRUCTURE ONLY. This file is the oracle the CUDA kernels are checked
+ * against. Only tests/, the smoke check and the bench's CPU-baseline leg may load
+ * it; the product library never links or calls it, and it shares no code, header
+ * or constant with the CUDA path.
+ *
+ * What it computes is the plain definition, row by row, with every score row
+ * materialised in f64: no tiling, no online softmax, no fusion.
+ *
+ * Sources (Forge pages):
+ *  - mask: key k is visible to query q iff  q - W < k <= q  (W = 0: no window).
+ *    Forge ARCHITECTURES.md, "Vague 2" item 8 (sliding_window in the flash kernels
+ *    and the reference); W = 0 is the sliding_window(0) default of the config
+ *    schema (forge-studio RESEARCH.md, section 2).
+ *  - softcap: s -> cap * tanh(s / cap) on the pre-softmax scores, cap = 0 off.
+ *    ARCHITECTURES.md "Vague 2" item 9; src/nn/attention.h commit log, "Wave 2
+ *    (attention kernels)": attn_softcap, exact tanh' chain in all backwards.
+ *  - GQA: n_heads % n_kv_heads == 0 (config schema validation, RESEARCH.md
+ *    section 2). Reading: query head hq uses KV head hq / (Hq / Hkv), i.e. each
+ *    KV head serves a contiguous group of query heads.
+ *  - softmax (max, sum) per row: ARCHITECTURES.md "Vague 2" item 10 and
+ *    "Vague 3" item 12 (the flash kernel keeps the per-row max).
+ *  - Reading: the scale multiplies q.k before the cap: s = cap*tanh(scale*q.k/cap).
+ *  - Reading: LSE is the natural-log log-sum-exp of the (capped) scores of a row.
+ *
+ * Layouts: q, o, dO, dq are [B][Hq][T][D]; k, v, dk, dv are [B][Hkv][T][D];
+ * lse and delta are [B][Hq][T]; all row-major, f64.
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* first key a query row may see */
+static long first_key(long i, long window) {
+    if (window > 0 && i - window + 1 > 0) return i - window + 1;
+    return 0;
+}
+
+static double dot(const double *a, const double *b, int D) {
+    double acc = 0.0;
+#pragma omp simd reduction(+ : acc)
+    for (int d = 0; d < D; d++) acc += a[d] * b[d];
+    return acc;
+}
+
+/* scaled score before the cap (the argument of tanh when a cap is set) */
+static double raw_score(const double *qi, const double *kj, int D, double scale) {
+    return scale * dot(qi, kj, D);
+}
+
+/* the score the softmax sees */
+static double capped(double s, double softcap) {
+    return softcap > 0.0 ? softcap * tanh(s / softcap) : s;
+}
+
+/* derivative of the cap with respect to its argument: 1 - tanh^2(s/cap) */
+static double cap_grad(double s, double softcap) {
+    if (softcap <= 0.0) return 1.0;
+    double t = tanh(s / softcap);
+    return 1.0 - t * t;
+}
+
+/*
+ * Probabilities of one query row: p[j] for j in [lo, i], returns the LSE.
+ * p[j] = exp(s_j - m) / sum_k exp(s_k - m), m = max_k s_k (k allowed).
+ */
+static double row_probs(const double *qi, const double *K, long i, long lo, int D,
+                        double scale, double softcap, double *p) {
+    double m = -INFINITY;
+    for (long j = lo; j <= i; j++) {
+        p[j] = capped(raw_score(qi, K + j * D, D, scale), softcap);
+        if (p[j] > m) m = p[j];
+    }
+    double l = 0.0;
+    for (long j = lo; j <= i; j++) {
+        p[j] = exp(p[j] - m);
+        l += p[j];
+    }
+    for (long j = lo; j <= i; j++) p[j] /= l;
+    return m + log(l);
+}
+
+/* Forward: O_i = sum_j P_ij V_j, LSE_i = log sum_j exp(s_ij). */
+void oracle_attn_fwd(const double *q, const double *k, const double *v, double *o, double *lse,
+                     int B, int Hq, int Hkv, int T, int D, double scale, int window,
+                     double softcap) {
+    const int G = Hq / Hkv;
+#pragma omp parallel
+    {
+        double *p = (double *)malloc(sizeof(double) * (size_t)T);
+#pragma omp for collapse(3) schedule(dynamic, 8)
+        for (int b = 0; b < B; b++)
+            for (int hq = 0; hq < Hq; hq++)
+                for (int i = 0; i < T; i++) {
+                    const int hkv = hq / G;
+                    const size_t qrow = ((size_t)(b * Hq + hq) * T + i);
+                    const double *qi = q + qrow * D;
+                    const double *K = k + (size_t)(b * Hkv + hkv) * T * D;
+                    const double *V = v + (size_t)(b * Hkv + hkv) * T * D;
+                    const long lo = first_key(i, window);
+                    lse[qrow] = row_probs(qi, K, i, lo, D, scale, softcap, p);
+                    double *oi = o + qrow * D;
+                    for (int d = 0; d < D; d++) oi[d] = 0.0;
+                    for (long j = lo; j <= i; j++)
+                        for (int d = 0; d < D; d++) oi[d] += p[j] * V[j * D + d];
+                }
+        free(p);
+    }
+}
+
+/*
+ * Backward of L(O) with upstream gradient dO:
+ *   dP_ij  = dO_i . V_j
+ *   Delta_i = sum_j P_ij dP_ij
+ *   dS_ij  = P_ij (dP_ij - Delta_i) * (1 - tanh^2(S_ij / cap))   [cap factor only if cap > 0]
+ *   dQ_i   = scale * sum_j dS_ij K_j
+ *   dK_j   = scale * sum over the group's query heads and rows i of dS_ij Q_i
+ *   dV_j   =         sum over the group's query heads and rows i of P_ij dO_i
+ * Pass 1 walks query rows (P, Delta, dQ); pass 2 walks key rows (dK, dV), using
+ * P_ij = exp(s_ij - LSE_i), which is the same softmax entry.
+ * delta (may be NULL) receives Delta, lse_out (may be NULL) receives LSE.
+ */
+void oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dO,
+                     double *dq, double *dk, double *dv, double *delta, double *lse_out,
+                     int B, int Hq, int Hkv, int T, int D, double scale, int window,
+                     double softcap) {
+    const int G = Hq / Hkv;
+    const size_t nrows = (size_t)B * Hq * T;
+    double *lse = (double *)malloc(sizeof(double) * nrows);
+    double *dlt = (double *)malloc(sizeof(double) * nrows);
+
+    /* pass 1: query rows */
+#pragma omp parallel
+    {
+        double *p = (double *)malloc(sizeof(double) * (size_t)T);
+        double *dp = (double *)malloc(sizeof(double) * (size_t)T);
+#pragma omp for collapse(3) schedule(dynamic, 8)
+        for (int b = 0; b < B; b++)
+            for (int hq = 0; hq < Hq; hq++)
+                for (int i = 0; i < T; i++) {
+                    const int hkv = hq / G;
+                    const size_t qrow = ((size_t)(b * Hq + hq) * T + i);
+                    const double *qi = q + qrow * D;
+                    const double *doi = dO + qrow * D;
+                    const double *K = k + (size_t)(b * Hkv + hkv) * T * D;
+                    const double *V = v + (size_t)(b * Hkv + hkv) * T * D;
+                    const long lo = first_key(i, window);
+                    lse[qrow] = row_probs(qi, K, i, lo, D, scale, softcap, p);
+                    double dl = 0.0;
+                    for (long j = lo; j <= i; j++) {
+                        dp[j] = dot(doi, V + j * D, D);
+                        dl += p[j] * dp[j];
+                    }
+                    dlt[qrow] = dl;
+                    double *dqi = dq + qrow * D;
+                    for (int d = 0; d < D; d++) dqi[d] = 0.0;
+                    for (long j = lo; j <= i; j++) {
+                        const double s = raw_score(qi, K + j * D, D, scale);
+                        const double ds = p[j] * (dp[j] - dl) * cap_grad(s, softcap);
+                        for (int d = 0; d < D; d++) dqi[d] += scale * ds * K[j * D + d];
+                    }
+                }
+        free(p);
+        free(dp);
+    }
+
+    /* pass 2: key rows, summed over the group's query heads */
+#pragma omp parallel for collapse(3) schedule(dynamic, 8)
+    for (int b = 0; b < B; b++)
+        for (int hkv = 0; hkv < Hkv; hkv++)
+            for (int j = 0; j < T; j++) {
+                const double *K = k + (size_t)(b * Hkv + hkv) * T * D;
+                const double *V = v + (size_t)(b * Hkv + hkv) * T * D;
+                const double *kj = K + (size_t)j * D;
+                const double *vj = V + (size_t)j * D;
+                double *dkj = dk + ((size_t)(b * Hkv + hkv) * T + j) * D;
+                double *dvj = dv + ((size_t)(b * Hkv + hkv) * T + j) * D;
+                for (int d = 0; d < D; d++) dkj[d] = dvj[d] = 0.0;
+                long last = T - 1;
+                if (window > 0 && (long)j + window - 1 < last) last = (long)j + window - 1;
+                for (int g = 0; g < G; g++) {
+                    const int hq = hkv * G + g;
+                    for (long i = j; i <= last; i++) {
+                        const size_t qrow = ((size_t)(b * Hq + hq) * T + i);
+                        const double *qi = q + qrow * D;
+                        const double *doi = dO + qrow * D;
+                        const double s = raw_score(qi, kj, D, scale);
+                        const double pij = exp(capped(s, softcap) - lse[qrow]);
+                        const double dpij = dot(doi, vj, D);
+                        const double ds = pij * (dpij - dlt[qrow]) * cap_grad(s, softcap);
+                        for (int d = 0; d < D; d++) {
+                            dvj[d] += pij * doi[d];
+                            dkj[d] += scale * ds * qi[d];
+                        }
+                    }
+                }
+            }
+
+    if (delta) memcpy(delta, dlt, sizeof(double) * nrows);
+    if (lse_out) memcpy(lse_out, lse, sizeof(double) * nrows);
+    free(lse);
+    free(dlt);
+}
+
+/* Full probability matrix P [B][Hq][T][T] (zeros where masked); small sizes only. */
+void oracle_attn_probs(const double *q, const double *k, double *P, int B, int Hq, int Hkv,
+                       int T, int D, double scale, int window, double softcap) {
+    const int G = Hq / Hkv;
+    for (int b = 0; b < B; b++)
+        for (int hq = 0; hq < Hq; hq++)
+            for (int i = 0; i < T; i++) {
+                const int hkv = hq / G;
+                const size_t qrow = ((size_t)(b * Hq + hq) * T + i);
+                double *pi = P + qrow * T;
+                for (int j = 0; j < T; j++) pi[j] = 0.0;
+                row_probs(q + qrow * D, k + (size_t)(b * Hkv + hkv) * T * D, i,
+                          first_key(i, window), D, scale, softcap, pi);
+            }
+}
+
+/* Delta_i = sum_d dO_id O_id (the identity the backward's first step relies on). */
+void oracle_rowdot(const double *o, const double *dO, double *delta, long rows, int D) {
+    for (long r = 0; r < rows; r++) delta[r] = dot(o + r * D, dO + r * D, D);
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

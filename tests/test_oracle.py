@@ -1,0 +1,346 @@
+"""Pins for the f64 oracle: each test checks it against something other than itself.
+
+- library special cases: torch SDPA (f64, CPU) with is_causal, with an explicit band
+  mask, with GQA by repeat_interleave; torch autograd through SDPA for gradients;
+- brute force on tiny shapes, with the full softmax Jacobian instead of the Delta
+  shortcut;
+- central finite differences of L = sum(O * dO);
+- the page's mask written out (tests/golden/mask_*.txt);
+- invariants and closed forms of the definition.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rnd(shape, seed, sigma=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(*shape, generator=g, dtype=torch.float64) * sigma)
+
+
+def qkv(B, Hq, Hkv, T, D, seed=0, sq=1.0, sk=1.0):
+    q = rnd((B, Hq, T, D), seed, sq)
+    k = rnd((B, Hkv, T, D), seed + 1, sk)
+    v = rnd((B, Hkv, T, D), seed + 2)
+    dO = rnd((B, Hq, T, D), seed + 3)
+    return q, k, v, dO
+
+
+def band_mask(T, W):
+    """Boolean [T, T] mask from torch's triangle routines: keep k <= q, and when
+    W > 0 also k > q - W."""
+    m = torch.ones(T, T, dtype=torch.bool).tril()
+    if W > 0:
+        m = m & torch.ones(T, T, dtype=torch.bool).triu(diagonal=-(W - 1))
+    return m
+
+
+def sdpa_ref(q, k, v, scale, W=0, softcap=0.0):
+    """Attention through torch's own SDPA. Softcap enters as an additive bias
+    (cap*tanh(S/cap) - S) so that SDPA's softmax sees the capped scores."""
+    G = q.shape[1] // k.shape[1]
+    kr = k.repeat_interleave(G, dim=1)
+    vr = v.repeat_interleave(G, dim=1)
+    T = q.shape[2]
+    if softcap == 0.0 and W == 0:
+        return F.scaled_dot_product_attention(q, kr, vr, is_causal=True, scale=scale)
+    mask = band_mask(T, W)
+    if softcap == 0.0:
+        return F.scaled_dot_product_attention(q, kr, vr, attn_mask=mask, scale=scale)
+    S = scale * q @ kr.transpose(-1, -2)
+    bias = softcap * torch.tanh(S / softcap) - S
+    bias = bias.masked_fill(~mask, float("-inf"))
+    return F.scaled_dot_product_attention(q, kr, vr, attn_mask=bias, scale=scale)
+
+
+def sdpa_grads(q, k, v, dO, scale, W=0, softcap=0.0):
+    q = q.clone().requires_grad_(True)
+    k = k.clone().requires_grad_(True)
+    v = v.clone().requires_grad_(True)
+    o = sdpa_ref(q, k, v, scale, W, softcap)
+    o.backward(dO)
+    return o.detach(), q.grad, k.grad, v.grad
+
+
+CASES = [
+    # B, Hq, Hkv, T, D, W, C
+    (1, 1, 1, 1, 4, 0, 0.0),
+    (2, 2, 2, 37, 8, 0, 0.0),
+    (1, 4, 2, 33, 16, 0, 0.0),
+    (1, 6, 2, 40, 8, 7, 0.0),
+    (2, 3, 1, 29, 8, 1, 0.0),
+    (1, 2, 1, 31, 8, 0, 3.0),
+    (1, 4, 4, 45, 8, 9, 2.0),
+    (1, 3, 3, 20, 8, 25, 0.0),  # W > T
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,T,D,W,C", CASES)
+def test_fwd_bwd_match_torch_sdpa_autograd(B, Hq, Hkv, T, D, W, C):
+    q, k, v, dO = qkv(B, Hq, Hkv, T, D, seed=T + D, sq=2.0 if C else 1.0, sk=2.0 if C else 1.0)
+    scale = 1.0 / math.sqrt(D)
+    o_ref, dq_ref, dk_ref, dv_ref = sdpa_grads(q, k, v, dO, scale, W, C)
+    o, lse = oracle.attn_fwd(q, k, v, scale, W, C)
+    np.testing.assert_allclose(o, o_ref.numpy(), rtol=1e-12, atol=1e-12)
+    dq, dk, dv, delta, lse2 = oracle.attn_bwd(q, k, v, dO, scale, W, C)
+    np.testing.assert_allclose(dq, dq_ref.numpy(), rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(dk, dk_ref.numpy(), rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(dv, dv_ref.numpy(), rtol=1e-10, atol=1e-11)
+    np.testing.assert_array_equal(lse, lse2)
+
+
+@pytest.mark.parametrize("W,C", [(0, 0.0), (5, 0.0), (0, 4.0), (6, 3.0)])
+def test_lse_matches_torch_logsumexp(W, C):
+    q, k, _, _ = qkv(1, 2, 1, 23, 8, seed=11, sq=2.0, sk=2.0)
+    scale = 0.3
+    _, lse = oracle.attn_fwd(q, k, k, scale, W, C)
+    S = scale * q @ k.repeat_interleave(2, dim=1).transpose(-1, -2)
+    if C:
+        S = C * torch.tanh(S / C)
+    S = S.masked_fill(~band_mask(23, W), float("-inf"))
+    np.testing.assert_allclose(lse, torch.logsumexp(S, dim=-1).numpy(), rtol=1e-13, atol=1e-13)
+
+
+# ----------------------------------------------------------------- brute force
+
+def brute(q, k, v, dO, scale, W, C):
+    """Tiny shapes only: explicit loops, softmax Jacobian J_ab = P_a (delta_ab - P_b)."""
+    q, k, v, dO = (x.numpy() for x in (q, k, v, dO))
+    B, Hq, T, D = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    o = np.zeros_like(q)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            for i in range(T):
+                keys = [j for j in range(T) if (j <= i and (W == 0 or j > i - W))]
+                raw = {j: scale * sum(q[b, h, i, d] * k[b, g, j, d] for d in range(D)) for j in keys}
+                s = {j: (C * math.tanh(raw[j] / C) if C else raw[j]) for j in keys}
+                z = sum(math.exp(s[j]) for j in keys)
+                P = {j: math.exp(s[j]) / z for j in keys}
+                for j in keys:
+                    o[b, h, i] += P[j] * v[b, g, j]
+                    dv[b, g, j] += P[j] * dO[b, h, i]
+                dP = {j: sum(dO[b, h, i, d] * v[b, g, j, d] for d in range(D)) for j in keys}
+                for a in keys:
+                    dsa = sum(P[a] * ((1.0 if a == c else 0.0) - P[c]) * dP[c] for c in keys)
+                    if C:
+                        dsa *= 1.0 - math.tanh(raw[a] / C) ** 2
+                    dq[b, h, i] += scale * dsa * k[b, g, a]
+                    dk[b, g, a] += scale * dsa * q[b, h, i]
+    return o, dq, dk, dv
+
+
+@pytest.mark.parametrize("T,D,W,C,Hq,Hkv", [(5, 3, 0, 0.0, 2, 1), (6, 2, 2, 0.0, 1, 1),
+                                             (6, 3, 3, 1.5, 4, 2), (4, 1, 1, 0.0, 2, 2),
+                                             (7, 2, 0, 0.7, 3, 1)])
+def test_bruteforce_jacobian(T, D, W, C, Hq, Hkv):
+    q, k, v, dO = qkv(1, Hq, Hkv, T, D, seed=3 * T + D, sq=1.5, sk=1.5)
+    scale = 0.9
+    o_b, dq_b, dk_b, dv_b = brute(q, k, v, dO, scale, W, C)
+    o, _ = oracle.attn_fwd(q, k, v, scale, W, C)
+    dq, dk, dv, _, _ = oracle.attn_bwd(q, k, v, dO, scale, W, C)
+    for a, b in ((o, o_b), (dq, dq_b), (dk, dk_b), (dv, dv_b)):
+        np.testing.assert_allclose(a, b, rtol=1e-11, atol=1e-12)
+
+
+# ----------------------------------------------------- central finite differences
+
+@pytest.mark.parametrize("W,C", [(0, 0.0), (4, 0.0), (0, 2.5), (3, 1.2)])
+def test_central_finite_differences(W, C):
+    B, Hq, Hkv, T, D = 1, 4, 2, 9, 3
+    q, k, v, dO = qkv(B, Hq, Hkv, T, D, seed=40 + W, sq=1.3, sk=1.3)
+    scale = 0.8
+    dq, dk, dv, _, _ = oracle.attn_bwd(q, k, v, dO, scale, W, C)
+    grads = {"q": dq, "k": dk, "v": dv}
+    base = {"q": q.numpy().copy(), "k": k.numpy().copy(), "v": v.numpy().copy()}
+    dOn = dO.numpy()
+    h = 1e-6
+
+    def loss(x):
+        o, _ = oracle.attn_fwd(x["q"], x["k"], x["v"], scale, W, C)
+        return float(np.sum(o * dOn))
+
+    for name in ("q", "k", "v"):
+        arr = base[name]
+        for idx in np.ndindex(arr.shape):
+            xp = {n: a.copy() for n, a in base.items()}
+            xm = {n: a.copy() for n, a in base.items()}
+            xp[name][idx] += h
+            xm[name][idx] -= h
+            fd = (loss(xp) - loss(xm)) / (2 * h)
+            assert abs(fd - grads[name][idx]) <= 1e-7 * (1.0 + abs(fd)), (name, idx, fd, grads[name][idx])
+
+
+# --------------------------------------------------------------- mask (the page)
+
+def read_mask(path):
+    rows = {}
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            q, ks = line.split(":")
+            rows[int(q)] = [int(x) for x in ks.split()]
+    return rows
+
+
+@pytest.mark.parametrize("fname,T,W", [("mask_T6_W3.txt", 6, 3), ("mask_T5_W0.txt", 5, 0)])
+def test_mask_matches_page(fname, T, W):
+    rows = read_mask(os.path.join(GOLDEN, fname))
+    q, k, _, _ = qkv(1, 1, 1, T, 4, seed=5)
+    P = oracle.attn_probs(q, k, 0.5, W, 0.0)[0, 0]
+    for i in range(T):
+        nz = [j for j in range(T) if P[i, j] != 0.0]
+        assert nz == rows[i], (i, nz, rows[i])
+
+
+# --------------------------------------------------------- invariants, closed forms
+
+def test_probability_rows_sum_to_one_and_respect_mask():
+    q, k, _, _ = qkv(2, 4, 2, 30, 8, seed=9, sq=2.0, sk=2.0)
+    for W, C in ((0, 0.0), (6, 0.0), (0, 3.0), (11, 5.0)):
+        P = oracle.attn_probs(q, k, 0.4, W, C)
+        np.testing.assert_allclose(P.sum(-1), 1.0, rtol=0, atol=1e-14)
+        allowed = band_mask(30, W).numpy()
+        assert np.all(P[..., ~allowed] == 0.0)
+        assert np.all(P[..., allowed] > 0.0)
+
+
+def test_ones_value_gives_ones_output():
+    q, k, _, _ = qkv(1, 2, 2, 25, 8, seed=2)
+    v = torch.ones(1, 2, 25, 8, dtype=torch.float64)
+    o, _ = oracle.attn_fwd(q, k, v, 0.35, 4, 2.0)
+    np.testing.assert_allclose(o, 1.0, rtol=0, atol=1e-14)
+
+
+def test_window_at_least_T_is_full_causal_bitwise():
+    q, k, v, dO = qkv(1, 4, 2, 27, 8, seed=4)
+    ref = oracle.attn_fwd(q, k, v, 0.3, 0, 1.5)
+    refb = oracle.attn_bwd(q, k, v, dO, 0.3, 0, 1.5)
+    for W in (27, 28, 1000):
+        o, lse = oracle.attn_fwd(q, k, v, 0.3, W, 1.5)
+        np.testing.assert_array_equal(o, ref[0])
+        np.testing.assert_array_equal(lse, ref[1])
+        for a, b in zip(oracle.attn_bwd(q, k, v, dO, 0.3, W, 1.5), refb):
+            np.testing.assert_array_equal(a, b)
+
+
+def test_huge_softcap_reproduces_no_cap():
+    q, k, v, dO = qkv(1, 2, 1, 21, 8, seed=6)
+    C = 1e8
+    o0, l0 = oracle.attn_fwd(q, k, v, 0.35, 0, 0.0)
+    o1, l1 = oracle.attn_fwd(q, k, v, 0.35, 0, C)
+    smax = float((q.abs().sum(-1).max() * k.abs().sum(-1).max()) * 0.35)
+    bound = 4.0 * (smax ** 3) / (3 * C * C) + 1e-13  # cap*tanh(s/cap) = s - s^3/(3 cap^2) + ...
+    np.testing.assert_allclose(o1, o0, rtol=0, atol=bound)
+    np.testing.assert_allclose(l1, l0, rtol=0, atol=bound)
+    g0 = oracle.attn_bwd(q, k, v, dO, 0.35, 0, 0.0)
+    g1 = oracle.attn_bwd(q, k, v, dO, 0.35, 0, C)
+    for a, b in zip(g0[:3], g1[:3]):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-10)
+
+
+def test_small_softcap_changes_result():
+    """A cap in the tanh regime must move the output (guards a dropped cap term)."""
+    q, k, v, _ = qkv(1, 1, 1, 16, 8, seed=8, sq=3.0, sk=3.0)
+    o0, _ = oracle.attn_fwd(q, k, v, 0.5, 0, 0.0)
+    o1, _ = oracle.attn_fwd(q, k, v, 0.5, 0, 2.0)
+    assert np.max(np.abs(o0 - o1)) > 1e-2
+
+
+def test_gqa_equals_repeated_kv_heads():
+    B, Hq, Hkv, T, D = 2, 6, 2, 19, 8
+    G = Hq // Hkv
+    q, k, v, dO = qkv(B, Hq, Hkv, T, D, seed=12)
+    kr = k.repeat_interleave(G, dim=1)
+    vr = v.repeat_interleave(G, dim=1)
+    for W, C in ((0, 0.0), (5, 2.0)):
+        o, lse = oracle.attn_fwd(q, k, v, 0.4, W, C)
+        o2, lse2 = oracle.attn_fwd(q, kr, vr, 0.4, W, C)
+        np.testing.assert_allclose(o, o2, rtol=0, atol=1e-14)
+        np.testing.assert_allclose(lse, lse2, rtol=0, atol=1e-14)
+        dq, dk, dv, _, _ = oracle.attn_bwd(q, k, v, dO, 0.4, W, C)
+        dq2, dk2, dv2, _, _ = oracle.attn_bwd(q, kr, vr, dO, 0.4, W, C)
+        np.testing.assert_allclose(dq, dq2, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(dk, dk2.reshape(B, Hkv, G, T, D).sum(2), rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dv, dv2.reshape(B, Hkv, G, T, D).sum(2), rtol=0, atol=1e-12)
+
+
+def test_key_shift_invariance():
+    """Adding one vector c to every key adds q.c to a whole score row: P, O and dQ
+    are unchanged (rows of the softmax gradient sum to zero) and LSE moves by
+    scale*q.c. Holds without a cap."""
+    q, k, v, dO = qkv(1, 2, 1, 22, 8, seed=13)
+    c = rnd((8,), 99)
+    k2 = k + c
+    o, lse = oracle.attn_fwd(q, k, v, 0.3, 6, 0.0)
+    o2, lse2 = oracle.attn_fwd(q, k2, v, 0.3, 6, 0.0)
+    np.testing.assert_allclose(o2, o, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse2 - lse, 0.3 * (q @ c).numpy(), rtol=0, atol=1e-12)
+    dq, dk, dv, _, _ = oracle.attn_bwd(q, k, v, dO, 0.3, 6, 0.0)
+    dq2, dk2, dv2, _, _ = oracle.attn_bwd(q, k2, v, dO, 0.3, 6, 0.0)
+    np.testing.assert_allclose(dq2, dq, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dv2, dv, rtol=0, atol=1e-12)
+
+
+def test_delta_identity():
+    q, k, v, dO = qkv(2, 4, 2, 24, 8, seed=14)
+    for W, C in ((0, 0.0), (7, 2.0)):
+        o, _ = oracle.attn_fwd(q, k, v, 0.5, W, C)
+        _, _, _, delta, _ = oracle.attn_bwd(q, k, v, dO, 0.5, W, C)
+        np.testing.assert_allclose(delta, oracle.rowdot(o, dO), rtol=1e-12, atol=1e-13)
+        # and the library form
+        np.testing.assert_allclose(delta, (torch.from_numpy(o) * dO).sum(-1).numpy(),
+                                   rtol=1e-12, atol=1e-13)
+
+
+def test_closed_form_single_token_and_window_one():
+    q, k, v, dO = qkv(1, 4, 2, 1, 8, seed=15)
+    o, lse = oracle.attn_fwd(q, k, v, 0.7, 0, 0.0)
+    np.testing.assert_allclose(o, v.repeat_interleave(2, dim=1).numpy(), rtol=0, atol=1e-15)
+    np.testing.assert_allclose(lse, 0.7 * (q * k.repeat_interleave(2, 1)).sum(-1).numpy(),
+                               rtol=1e-14, atol=1e-14)
+    # W = 1: every query sees only itself
+    q, k, v, dO = qkv(1, 4, 2, 17, 8, seed=16)
+    o, lse = oracle.attn_fwd(q, k, v, 0.7, 1, 2.0)
+    np.testing.assert_allclose(o, v.repeat_interleave(2, dim=1).numpy(), rtol=0, atol=1e-15)
+    s = 0.7 * (q * k.repeat_interleave(2, 1)).sum(-1)
+    np.testing.assert_allclose(lse, (2.0 * torch.tanh(s / 2.0)).numpy(), rtol=1e-13, atol=1e-13)
+    dq, dk, dv, _, _ = oracle.attn_bwd(q, k, v, dO, 0.7, 1, 2.0)
+    assert np.max(np.abs(dq)) < 1e-14 and np.max(np.abs(dk)) < 1e-14
+    np.testing.assert_allclose(dv, dO.reshape(1, 2, 2, 17, 8).sum(2).numpy(), rtol=0, atol=1e-14)
+
+
+def test_closed_form_zero_query_uniform_average():
+    T, D = 26, 8
+    _, k, v, _ = qkv(1, 1, 1, T, D, seed=17)
+    q = torch.zeros(1, 1, T, D, dtype=torch.float64)
+    for W in (0, 5):
+        o, lse = oracle.attn_fwd(q, k, v, 0.6, W, 0.0)
+        for i in range(T):
+            lo = max(0, i - W + 1) if W else 0
+            np.testing.assert_allclose(o[0, 0, i], v[0, 0, lo:i + 1].mean(0).numpy(), rtol=0, atol=1e-14)
+            assert abs(lse[0, 0, i] - math.log(i + 1 - lo)) < 1e-14
+
+
+def test_closed_form_constant_value():
+    q, k, _, dO = qkv(1, 2, 1, 20, 8, seed=18)
+    v = torch.full((1, 1, 20, 8), 0.0, dtype=torch.float64) + torch.arange(8.0, dtype=torch.float64)
+    o, _ = oracle.attn_fwd(q, k, v, 0.5, 0, 3.0)
+    np.testing.assert_allclose(o, np.broadcast_to(np.arange(8.0), o.shape), rtol=0, atol=1e-13)
+    dq, dk, dv, _, _ = oracle.attn_bwd(q, k, v, dO, 0.5, 0, 3.0)
+    assert np.max(np.abs(dq)) < 1e-12 and np.max(np.abs(dk)) < 1e-12
