@@ -1,0 +1,193 @@
+"""B200 (sm_100a) fused causal attention: Python binding of libforge_attn.so.
+
+The functions named ``forge_attn_*`` mirror the C ABI in include/forge_attn.h one
+to one (argument marshalling only: every pointer argument accepts a torch
+tensor or an integer device address). ``attention_fwd`` / ``attention_bwd``
+allocate outputs and workspace with torch and call them.
+
+PyTorch is used for device memory and streams only; all arithmetic runs in the
+library's CUDA kernels. There is no fallback: if the shared library is missing
+or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+__all__ = [
+    "FORGE_OK", "FORGE_ERR_INVALID_ARG", "FORGE_ERR_UNSUPPORTED", "FORGE_ERR_WORKSPACE",
+    "FORGE_ERR_CUDA", "FORGE_ERR_TIMEOUT", "FORGE_DTYPE_F32", "FORGE_DTYPE_BF16", "ForgeError",
+    "library", "library_path", "forge_attn_fwd", "forge_attn_bwd", "forge_attn_bwd_workspace_size",
+    "forge_attn_bwd_preprocess", "forge_attn_bwd_main", "forge_attn_bwd_finalize", "forge_attn_check",
+    "forge_attn_status_string", "forge_attn_selftest_timeout", "forge_attn_version",
+    "attention_fwd", "attention_bwd", "dtype_code",
+]
+
+FORGE_OK = 0
+FORGE_ERR_INVALID_ARG = 1
+FORGE_ERR_UNSUPPORTED = 2
+FORGE_ERR_WORKSPACE = 3
+FORGE_ERR_CUDA = 4
+FORGE_ERR_TIMEOUT = 5
+FORGE_DTYPE_F32 = 0
+FORGE_DTYPE_BF16 = 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libforge_attn.so")
+_lib = None
+
+
+class ForgeError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {forge_attn_status_string(status)}" if what else forge_attn_status_string(status))
+
+
+def library():
+    """Load (once) and return the ctypes handle of libforge_attn.so."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(library_path):
+        raise RuntimeError(f"{library_path} is missing: run `python -m causal_flash_attention_attn_b200.build`")
+    L = ctypes.CDLL(library_path)
+    vp, i, f, st, u = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_uint
+    L.forge_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, f, i, vp]
+    L.forge_attn_fwd.restype = i
+    L.forge_attn_bwd_workspace_size.argtypes = [i, i, i, i, i, i]
+    L.forge_attn_bwd_workspace_size.restype = st
+    L.forge_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, f, i, vp, st, vp]
+    L.forge_attn_bwd.restype = i
+    L.forge_attn_bwd_preprocess.argtypes = [vp, vp, i, i, i, i, i, i, vp, st, vp]
+    L.forge_attn_bwd_preprocess.restype = i
+    L.forge_attn_bwd_main.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, f, i, vp, st, vp]
+    L.forge_attn_bwd_main.restype = i
+    L.forge_attn_bwd_finalize.argtypes = [vp, i, i, i, i, i, i, vp, st, vp]
+    L.forge_attn_bwd_finalize.restype = i
+    L.forge_attn_check.argtypes = [vp]
+    L.forge_attn_check.restype = i
+    L.forge_attn_status_string.argtypes = [i]
+    L.forge_attn_status_string.restype = ctypes.c_char_p
+    L.forge_attn_selftest_timeout.argtypes = [u, vp]
+    L.forge_attn_selftest_timeout.restype = i
+    L.forge_attn_version.argtypes = []
+    L.forge_attn_version.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def dtype_code(dtype) -> int:
+    import torch
+    if dtype == torch.float32:
+        return FORGE_DTYPE_F32
+    if dtype == torch.bfloat16:
+        return FORGE_DTYPE_BF16
+    raise ValueError(f"unsupported dtype {dtype}")
+
+
+# ------------------------------------------------------------------ raw C ABI
+def forge_attn_fwd(q, k, v, o, lse, B, Hq, Hkv, T, D, scale, window, softcap, dtype, stream=None) -> int:
+    return library().forge_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, T, D,
+                                    float(scale), int(window), float(softcap), int(dtype), _stream(stream))
+
+
+def forge_attn_bwd_workspace_size(B, Hq, Hkv, T, D, dtype) -> int:
+    return int(library().forge_attn_bwd_workspace_size(B, Hq, Hkv, T, D, int(dtype)))
+
+
+def forge_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale, window, softcap, dtype,
+                   workspace, workspace_bytes, stream=None) -> int:
+    return library().forge_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
+                                    _ptr(dk), _ptr(dv), B, Hq, Hkv, T, D, float(scale), int(window),
+                                    float(softcap), int(dtype), _ptr(workspace), int(workspace_bytes),
+                                    _stream(stream))
+
+
+def forge_attn_bwd_preprocess(o, dO, B, Hq, Hkv, T, D, dtype, workspace, workspace_bytes, stream=None) -> int:
+    return library().forge_attn_bwd_preprocess(_ptr(o), _ptr(dO), B, Hq, Hkv, T, D, int(dtype),
+                                               _ptr(workspace), int(workspace_bytes), _stream(stream))
+
+
+def forge_attn_bwd_main(q, k, v, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale, window, softcap, dtype,
+                        workspace, workspace_bytes, stream=None) -> int:
+    return library().forge_attn_bwd_main(_ptr(q), _ptr(k), _ptr(v), _ptr(lse), _ptr(dO), _ptr(dq), _ptr(dk),
+                                         _ptr(dv), B, Hq, Hkv, T, D, float(scale), int(window), float(softcap),
+                                         int(dtype), _ptr(workspace), int(workspace_bytes), _stream(stream))
+
+
+def forge_attn_bwd_finalize(dq, B, Hq, Hkv, T, D, dtype, workspace, workspace_bytes, stream=None) -> int:
+    return library().forge_attn_bwd_finalize(_ptr(dq), B, Hq, Hkv, T, D, int(dtype), _ptr(workspace),
+                                             int(workspace_bytes), _stream(stream))
+
+
+def forge_attn_check(stream=None) -> int:
+    return library().forge_attn_check(_stream(stream))
+
+
+def forge_attn_status_string(s: int) -> str:
+    return library().forge_attn_status_string(int(s)).decode()
+
+
+def forge_attn_selftest_timeout(limit_us: int, stream=None) -> int:
+    return library().forge_attn_selftest_timeout(int(limit_us), _stream(stream))
+
+
+def forge_attn_version() -> str:
+    return library().forge_attn_version().decode()
+
+
+# ---------------------------------------------------------- torch conveniences
+def _dims(q, k):
+    B, Hq, T, D = q.shape
+    Hkv = k.shape[1]
+    return B, Hq, Hkv, T, D
+
+
+def attention_fwd(q, k, v, scale=None, window=0, softcap=0.0, stream=None):
+    """Forward on device tensors [B,H,T,D] (bf16 or f32). Returns (o, lse)."""
+    import torch
+    B, Hq, Hkv, T, D = _dims(q, k)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    s = forge_attn_fwd(q, k, v, o, lse, B, Hq, Hkv, T, D, scale, window, softcap, dtype_code(q.dtype), stream)
+    if s != FORGE_OK:
+        raise ForgeError(s, "forge_attn_fwd")
+    return o, lse
+
+
+def attention_bwd(q, k, v, o, lse, dO, scale=None, window=0, softcap=0.0, workspace=None, stream=None):
+    """Backward on device tensors. Returns (dq, dk, dv)."""
+    import torch
+    B, Hq, Hkv, T, D = _dims(q, k)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    dt = dtype_code(q.dtype)
+    nbytes = forge_attn_bwd_workspace_size(B, Hq, Hkv, T, D, dt)
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    s = forge_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale, window, softcap, dt,
+                       workspace, workspace.numel(), stream)
+    if s != FORGE_OK:
+        raise ForgeError(s, "forge_attn_bwd")
+    return dq, dk, dv

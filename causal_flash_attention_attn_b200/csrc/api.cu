@@ -1,0 +1,370 @@
+// api.cu -- the C ABI of libforge_attn.so (declared in include/forge_attn.h):
+// argument validation, TMA tensor maps, workspace layout and kernel dispatch.
+// Single translation unit: every kernel header is included here.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "forge_attn.h"
+
+#include "bwd_aux.cuh"
+#include "bwd_tc.cuh"
+#include "fwd_tc.cuh"
+#include "simt.cuh"
+#include "sm100.cuh"
+
+namespace forge {
+namespace {
+
+// ------------------------------------------------------------------ validation
+bool aligned16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+forge_status check_sizes(int B, int Hq, int Hkv, int T, int D, forge_dtype dtype) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || T < 1 || D < 1) return FORGE_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return FORGE_ERR_INVALID_ARG;  // n_heads % n_kv_heads == 0
+    if (D % 2 != 0) return FORGE_ERR_INVALID_ARG;     // head_dim even
+    if (dtype != FORGE_DTYPE_F32 && dtype != FORGE_DTYPE_BF16) return FORGE_ERR_INVALID_ARG;
+    if (D != 64 && D != 128 && D != 256) return FORGE_ERR_UNSUPPORTED;
+    // index arithmetic limits: grid sizes and per-tensor element counts
+    const long long rows = (long long)B * Hq * T;
+    if ((long long)B * Hq > (1ll << 24) || T > (1 << 30) || rows * D > (1ll << 40)) return FORGE_ERR_INVALID_ARG;
+    const long long ntiles = (long long)((T + 127) / 128) * B * Hq;
+    if (ntiles > 0x7fffffffll) return FORGE_ERR_INVALID_ARG;
+    return FORGE_OK;
+}
+
+forge_status check_scalars(float scale, int window, float softcap) {
+    if (!(scale > 0.0f) || !isfinite(scale)) return FORGE_ERR_INVALID_ARG;
+    if (window < 0) return FORGE_ERR_INVALID_ARG;
+    if (!(softcap >= 0.0f) || !isfinite(softcap)) return FORGE_ERR_INVALID_ARG;
+    return FORGE_OK;
+}
+
+int effective_window(int window, int T) { return (window >= T) ? 0 : window; }
+
+// ------------------------------------------------------------- workspace layout
+// [ delta: B*Hq*T f32, 256-aligned ][ dq accumulator: B*Hq*Tpad*D f32 (bf16 only) ]
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+int tpad_of(int T) { return (T + 127) / 128 * 128; }
+size_t delta_bytes(int B, int Hq, int T) { return round256(sizeof(float) * (size_t)B * Hq * T); }
+size_t acc_bytes(int B, int Hq, int T, int D) { return round256(sizeof(float) * (size_t)B * Hq * tpad_of(T) * D); }
+
+// ----------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (fn == nullptr) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// [BH][T][D] bf16 viewed as a 3D tensor (D innermost); box = 64 columns x rows x 1,
+// 128-byte swizzle (the layout the tcgen05 descriptors describe). Rows past T
+// read as zeros.
+bool make_map(CUtensorMap *map, const void *base, int D, int T, long long BH, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (enc == nullptr) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)D * 2 * (cuuint64_t)T};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+forge_status launch_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? FORGE_OK : FORGE_ERR_CUDA;
+}
+
+template <typename K>
+forge_status set_smem(K kernel, size_t bytes) {
+    if (bytes <= 48 * 1024) return FORGE_OK;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess
+               ? FORGE_OK
+               : FORGE_ERR_CUDA;
+}
+
+// ----------------------------------------------------------------- dispatchers
+template <int D>
+forge_status fwd_tc(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv, int T,
+                    float scale, int window, float softcap, cudaStream_t st) {
+    using C = FwdTc<D>;
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, q, D, T, (long long)B * Hq, 128) || !make_map(&mk, k, D, T, (long long)B * Hkv, 128) ||
+        !make_map(&mv, v, D, T, (long long)B * Hkv, 128))
+        return FORGE_ERR_CUDA;
+    FwdParams p;
+    p.o = static_cast<__nv_bfloat16 *>(o);
+    p.lse = lse;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.T = T; p.window = window;
+    p.num_qt = (T + 127) / 128;
+    p.scale_log2 = scale * kLog2e;
+    p.softcap = softcap;
+    p.cap_in = softcap > 0.0f ? scale / softcap : 0.0f;
+    p.cap_out = softcap * kLog2e;
+    if (set_smem(fwd_tc_kernel<D>, C::SMEM) != FORGE_OK) return FORGE_ERR_CUDA;
+    const unsigned grid = (unsigned)(p.num_qt * B * Hq);
+    fwd_tc_kernel<D><<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, p);
+    return launch_status();
+}
+
+template <typename T_, int D>
+forge_status fwd_simt(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv, int T,
+                      float scale, int window, float softcap, cudaStream_t st) {
+    const size_t sm = simt_fwd_smem<D>();
+    if (set_smem(simt_fwd<T_, D>, sm) != FORGE_OK) return FORGE_ERR_CUDA;
+    dim3 grid((T + kSimtRows - 1) / kSimtRows, B * Hq);
+    simt_fwd<T_, D><<<grid, kSimtThreads, sm, st>>>(static_cast<const T_ *>(q), static_cast<const T_ *>(k),
+                                                     static_cast<const T_ *>(v), static_cast<T_ *>(o), lse, Hq, Hkv,
+                                                     T, scale, window, softcap);
+    return launch_status();
+}
+
+template <typename T_, int D>
+forge_status bwd_simt(const void *q, const void *k, const void *v, const float *lse, const void *dO,
+                      const float *delta, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int T, float scale,
+                      int window, float softcap, cudaStream_t st) {
+    const size_t sm1 = simt_bwd_dq_smem<D>(), sm2 = simt_bwd_dkdv_smem<D>();
+    if (set_smem(simt_bwd_dq<T_, D>, sm1) != FORGE_OK || set_smem(simt_bwd_dkdv<T_, D>, sm2) != FORGE_OK)
+        return FORGE_ERR_CUDA;
+    dim3 g1((T + kSimtRows - 1) / kSimtRows, B * Hq);
+    simt_bwd_dq<T_, D><<<g1, kSimtThreads, sm1, st>>>(
+        static_cast<const T_ *>(q), static_cast<const T_ *>(k), static_cast<const T_ *>(v), lse,
+        static_cast<const T_ *>(dO), delta, static_cast<T_ *>(dq), Hq, Hkv, T, scale, window, softcap);
+    forge_status s = launch_status();
+    if (s != FORGE_OK) return s;
+    dim3 g2((T + kSimtRows - 1) / kSimtRows, B * Hkv);
+    simt_bwd_dkdv<T_, D><<<g2, kSimtThreads, sm2, st>>>(
+        static_cast<const T_ *>(q), static_cast<const T_ *>(k), static_cast<const T_ *>(v), lse,
+        static_cast<const T_ *>(dO), delta, static_cast<T_ *>(dk), static_cast<T_ *>(dv), Hq, Hkv, T, scale, window,
+        softcap);
+    return launch_status();
+}
+
+template <int D>
+forge_status bwd_tc(const void *q, const void *k, const void *v, const float *lse, const void *dO,
+                    const float *delta, float *acc, void *dk, void *dv, int B, int Hq, int Hkv, int T, float scale,
+                    int window, float softcap, cudaStream_t st) {
+    using C = BwdTc<D>;
+    CUtensorMap mq, mk, mv, mdo;
+    if (!make_map(&mq, q, D, T, (long long)B * Hq, C::BM) || !make_map(&mk, k, D, T, (long long)B * Hkv, 128) ||
+        !make_map(&mv, v, D, T, (long long)B * Hkv, 128) || !make_map(&mdo, dO, D, T, (long long)B * Hq, C::BM))
+        return FORGE_ERR_CUDA;
+    BwdParams p;
+    p.lse = lse;
+    p.delta = delta;
+    p.dq_acc = acc;
+    p.dk = static_cast<__nv_bfloat16 *>(dk);
+    p.dv = static_cast<__nv_bfloat16 *>(dv);
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.T = T; p.Tpad = tpad_of(T); p.window = window;
+    p.num_kt = (T + 127) / 128;
+    p.scale = scale;
+    p.scale_log2 = scale * kLog2e;
+    p.softcap = softcap;
+    p.cap_in = softcap > 0.0f ? scale / softcap : 0.0f;
+    p.cap_out = softcap * kLog2e;
+    if (set_smem(bwd_tc_kernel<D>, C::SMEM) != FORGE_OK) return FORGE_ERR_CUDA;
+    const unsigned grid = (unsigned)(p.num_kt * B * Hkv * C::NSPLIT);
+    bwd_tc_kernel<D><<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, mdo, p);
+    return launch_status();
+}
+
+#define FORGE_DISPATCH_D(D, ...)                               \
+    switch (D) {                                               \
+        case 64: { constexpr int kD = 64; __VA_ARGS__ } break;   \
+        case 128: { constexpr int kD = 128; __VA_ARGS__ } break; \
+        case 256: { constexpr int kD = 256; __VA_ARGS__ } break; \
+        default: return FORGE_ERR_UNSUPPORTED;                 \
+    }
+
+}  // namespace
+
+// Timeout self-test: waits on a barrier nothing completes.
+__global__ void selftest_timeout_kernel(unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t barrier;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        mbar_init(smem_u32(&barrier), 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(smem_u32(&barrier), 0, &abort_flag, limit_ns);
+    __syncthreads();
+}
+
+}  // namespace forge
+
+using namespace forge;
+
+extern "C" {
+
+forge_status forge_attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+                            int Hkv, int T, int D, float scale, int window, float softcap, forge_dtype dtype,
+                            void *stream) {
+    forge_status s = check_sizes(B, Hq, Hkv, T, D, dtype);
+    if (s != FORGE_OK) return s;
+    if ((s = check_scalars(scale, window, softcap)) != FORGE_OK) return s;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return FORGE_ERR_INVALID_ARG;
+    window = effective_window(window, T);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dtype == FORGE_DTYPE_BF16) {
+        FORGE_DISPATCH_D(D, return fwd_tc<kD>(q, k, v, o, lse, B, Hq, Hkv, T, scale, window, softcap, st);)
+    } else {
+        FORGE_DISPATCH_D(D, return fwd_simt<float, kD>(q, k, v, o, lse, B, Hq, Hkv, T, scale, window, softcap, st);)
+    }
+    return FORGE_ERR_UNSUPPORTED;
+}
+
+size_t forge_attn_bwd_workspace_size(int B, int Hq, int Hkv, int T, int D, forge_dtype dtype) {
+    if (check_sizes(B, Hq, Hkv, T, D, dtype) != FORGE_OK) return 0;
+    size_t n = delta_bytes(B, Hq, T);
+    if (dtype == FORGE_DTYPE_BF16) n += acc_bytes(B, Hq, T, D);
+    return n;
+}
+
+static forge_status check_workspace(void *ws, size_t bytes, int B, int Hq, int Hkv, int T, int D, forge_dtype dtype) {
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return FORGE_ERR_WORKSPACE;
+    if (bytes < forge_attn_bwd_workspace_size(B, Hq, Hkv, T, D, dtype)) return FORGE_ERR_WORKSPACE;
+    return FORGE_OK;
+}
+
+forge_status forge_attn_bwd_preprocess(const void *o, const void *dO, int B, int Hq, int Hkv, int T, int D,
+                                       forge_dtype dtype, void *workspace, size_t workspace_bytes, void *stream) {
+    forge_status s = check_sizes(B, Hq, Hkv, T, D, dtype);
+    if (s != FORGE_OK) return s;
+    if (!aligned16(o) || !aligned16(dO)) return FORGE_ERR_INVALID_ARG;
+    if ((s = check_workspace(workspace, workspace_bytes, B, Hq, Hkv, T, D, dtype)) != FORGE_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float *delta = static_cast<float *>(workspace);
+    const long rows = (long)B * Hq * T;
+    const unsigned grid = (unsigned)((rows + 7) / 8);
+    if (dtype == FORGE_DTYPE_BF16) {
+        // the dq accumulator receives reductions: zero it in the same pass
+        float *acc = reinterpret_cast<float *>(static_cast<char *>(workspace) + delta_bytes(B, Hq, T));
+        if (D == 256) acc = nullptr;  // head dim 256 writes dq directly
+        FORGE_DISPATCH_D(D, bwd_preprocess<__nv_bfloat16, kD><<<grid, 256, 0, st>>>(
+                                static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dO), delta,
+                                acc, rows, T, tpad_of(T));)
+        return launch_status();
+    }
+    FORGE_DISPATCH_D(D, bwd_preprocess<float, kD><<<grid, 256, 0, st>>>(static_cast<const float *>(o),
+                                                                          static_cast<const float *>(dO), delta,
+                                                                          nullptr, rows, T, tpad_of(T));)
+    return launch_status();
+}
+
+forge_status forge_attn_bwd_main(const void *q, const void *k, const void *v, const float *lse, const void *dO,
+                                 void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int T, int D, float scale,
+                                 int window, float softcap, forge_dtype dtype, void *workspace,
+                                 size_t workspace_bytes, void *stream) {
+    forge_status s = check_sizes(B, Hq, Hkv, T, D, dtype);
+    if (s != FORGE_OK) return s;
+    if ((s = check_scalars(scale, window, softcap)) != FORGE_OK) return s;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(lse) || !aligned16(dO) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv))
+        return FORGE_ERR_INVALID_ARG;
+    if ((s = check_workspace(workspace, workspace_bytes, B, Hq, Hkv, T, D, dtype)) != FORGE_OK) return s;
+    window = effective_window(window, T);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const float *delta = static_cast<const float *>(workspace);
+    if (dtype == FORGE_DTYPE_BF16) {
+        float *acc = reinterpret_cast<float *>(static_cast<char *>(workspace) + delta_bytes(B, Hq, T));
+        if (D == 256) {
+            // head dim 256: CUDA-core backward for dq, dk, dv (f32 arithmetic)
+            return bwd_simt<__nv_bfloat16, 256>(q, k, v, lse, dO, delta, dq, dk, dv, B, Hq, Hkv, T, scale, window,
+                                                softcap, st);
+        }
+        FORGE_DISPATCH_D(D, return bwd_tc<kD>(q, k, v, lse, dO, delta, acc, dk, dv, B, Hq, Hkv, T, scale, window,
+                                              softcap, st);)
+    }
+    FORGE_DISPATCH_D(D, return bwd_simt<float, kD>(q, k, v, lse, dO, delta, dq, dk, dv, B, Hq, Hkv, T, scale, window,
+                                                   softcap, st);)
+    return FORGE_ERR_UNSUPPORTED;
+}
+
+forge_status forge_attn_bwd_finalize(void *dq, int B, int Hq, int Hkv, int T, int D, forge_dtype dtype,
+                                     void *workspace, size_t workspace_bytes, void *stream) {
+    forge_status s = check_sizes(B, Hq, Hkv, T, D, dtype);
+    if (s != FORGE_OK) return s;
+    if (!aligned16(dq)) return FORGE_ERR_INVALID_ARG;
+    if ((s = check_workspace(workspace, workspace_bytes, B, Hq, Hkv, T, D, dtype)) != FORGE_OK) return s;
+    if (dtype != FORGE_DTYPE_BF16 || D == 256) return FORGE_OK;  // dq already written by the main stage
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const float *acc = reinterpret_cast<const float *>(static_cast<char *>(workspace) + delta_bytes(B, Hq, T));
+    const long long total = (long long)B * Hq * T * (D / 8);
+    const unsigned grid = (unsigned)((total + 255) / 256);
+    FORGE_DISPATCH_D(D, bwd_finalize_dq<kD><<<grid, 256, 0, st>>>(acc, static_cast<__nv_bfloat16 *>(dq),
+                                                                  (long)B * Hq, T, tpad_of(T));)
+    return launch_status();
+}
+
+forge_status forge_attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                            const void *dO, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int T, int D,
+                            float scale, int window, float softcap, forge_dtype dtype, void *workspace,
+                            size_t workspace_bytes, void *stream) {
+    forge_status s = check_sizes(B, Hq, Hkv, T, D, dtype);
+    if (s != FORGE_OK) return s;
+    if ((s = check_scalars(scale, window, softcap)) != FORGE_OK) return s;
+    // validate everything before the first launch: on error nothing runs
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dO) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return FORGE_ERR_INVALID_ARG;
+    if ((s = check_workspace(workspace, workspace_bytes, B, Hq, Hkv, T, D, dtype)) != FORGE_OK) return s;
+    s = forge_attn_bwd_preprocess(o, dO, B, Hq, Hkv, T, D, dtype, workspace, workspace_bytes, stream);
+    if (s != FORGE_OK) return s;
+    s = forge_attn_bwd_main(q, k, v, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale, window, softcap, dtype, workspace,
+                            workspace_bytes, stream);
+    if (s != FORGE_OK) return s;
+    return forge_attn_bwd_finalize(dq, B, Hq, Hkv, T, D, dtype, workspace, workspace_bytes, stream);
+}
+
+forge_status forge_attn_check(void *stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return FORGE_ERR_CUDA;
+    int h = 0;
+    if (cudaMemcpyFromSymbol(&h, g_status, sizeof(int)) != cudaSuccess) return FORGE_ERR_CUDA;
+    if (h != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return FORGE_ERR_CUDA;
+        return static_cast<forge_status>(h);
+    }
+    return FORGE_OK;
+}
+
+const char *forge_attn_status_string(forge_status s) {
+    switch (s) {
+        case FORGE_OK: return "FORGE_OK";
+        case FORGE_ERR_INVALID_ARG: return "FORGE_ERR_INVALID_ARG: invalid argument";
+        case FORGE_ERR_UNSUPPORTED: return "FORGE_ERR_UNSUPPORTED: unsupported configuration";
+        case FORGE_ERR_WORKSPACE: return "FORGE_ERR_WORKSPACE: workspace missing, misaligned or too small";
+        case FORGE_ERR_CUDA: return "FORGE_ERR_CUDA: CUDA runtime or launch failure";
+        case FORGE_ERR_TIMEOUT: return "FORGE_ERR_TIMEOUT: a bounded wait inside a kernel ran out";
+    }
+    return "FORGE_ERR_UNKNOWN";
+}
+
+forge_status forge_attn_selftest_timeout(unsigned int limit_us, void *stream) {
+    if (limit_us < 1 || limit_us > 2000000u) return FORGE_ERR_INVALID_ARG;
+    selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(1000ull * limit_us);
+    return launch_status();
+}
+
+const char *forge_attn_version(void) { return "forge_attn 0.1.0 sm_100a"; }
+
+}  // extern "C"

@@ -1,0 +1,441 @@
+// bwd_tc.cuh -- tensor-core backward main kernel (bf16 in, f32 accumulate).
+//
+// One CTA per (KV tile of 128 keys, batch, KV head, head-dim half). The CTA keeps
+// its K and V tiles in shared memory and dK, dV accumulators in tensor memory for
+// the whole run, and walks every (query head of the group, query tile) pair that
+// can see its keys: query tiles from the key tile's diagonal up to the window's
+// reach (or T - 1), so the cost scales with the window. Per step:
+//   S^T  = K Q^T            (tcgen05, 128 x BM, f32 in TMEM)
+//   dP^T = V dO^T           (tcgen05)
+//   P^T  = exp2(s*log2e - LSE*log2e), masked to 0   -> bf16 into TMEM (over S^T)
+//   dS^T = scale * P^T (dP^T - Delta) [* (1 - tanh^2)] -> bf16 into shared memory
+//          (the cap factor is the "exact tanh' chain": src/nn/attention.h
+//           commit log, Wave 2)
+//   dV  += P^T dO           (A from TMEM)
+//   dK  += dS^T Q
+//   dQ   = dS K  (or its transpose K^T dS^T), drained from TMEM by four warps
+//          with f32 reductions into a padded [B*Hq][Tpad][D] workspace.
+// dK and dV sum over the group's query heads inside the CTA, so they need no
+// atomics; dQ rows are shared between key tiles and are reduced in L2.
+//
+// Shapes per head dim (TMEM: S^T BM + dP^T BM + dV DH + dK DH + dQ <= 512 cols):
+//   D = 64 : BM = 128 query rows, dQ = dS K    (M = 128 query rows, N = 64)
+//   D = 128: BM = 64,  dQ^T = K^T dS^T         (M = 128 = D, N = 64 query rows)
+//   D = 256: BM = 64, two CTAs per key tile, each owning half of the head dim
+//            (DH = 128) for dK, dV and dQ; S^T and dP^T use the full head dim.
+//
+// Roles (320 threads): warps 0-3 compute (one thread per key row, TMEM lane),
+// warps 4-7 dQ drain + dK epilogue, warp 8 loads (TMA for tiles, plain loads
+// for LSE and Delta), warp 9 issues MMAs and owns TMEM.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace forge {
+
+template <int D_>
+struct BwdTc {
+    static constexpr int D = D_;
+    static constexpr int BN = 128;                       // keys per CTA
+    static constexpr int BM = D == 64 ? 128 : 64;        // query rows per step
+    static constexpr bool DQT = D != 64;                 // transposed dQ product
+    static constexpr int NSPLIT = D == 256 ? 2 : 1;      // head-dim halves
+    static constexpr int DH = D / NSPLIT;                // output columns per CTA
+    static constexpr int QST = D == 256 ? 1 : 2;         // Q/dO stages
+    static constexpr int NCB = D / 64;
+    static constexpr uint32_t CBK = 128 * 128;           // column block of a 128-row tile
+    static constexpr uint32_t CBQ = BM * 128;            // column block of a BM-row tile
+    static constexpr uint32_t TK = NCB * CBK;            // K (or V) tile bytes
+    static constexpr uint32_t TQ = NCB * CBQ;            // Q (or dO) tile bytes
+    static constexpr uint32_t TS = (BM / 64) * CBK;      // dS^T tile bytes
+    static constexpr uint32_t OFF_K = 0, OFF_V = TK, OFF_Q = 2 * TK;
+    static constexpr uint32_t OFF_DO = OFF_Q + QST * TQ;
+    static constexpr uint32_t OFF_DS = OFF_DO + QST * TQ;
+    static constexpr uint32_t TILES = OFF_DS + TS;
+    static constexpr uint32_t CTRL = 4096;               // barriers, slots, LSE/Delta stages
+    static constexpr uint32_t SMEM = CTRL + TILES + 1024;
+    static constexpr int THREADS = 320;
+    static constexpr uint32_t COL_S = 0, COL_DP = BM, COL_DV = 2 * BM, COL_DK = 2 * BM + DH;
+    static constexpr uint32_t COL_DQ = 2 * BM + 2 * DH;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static_assert(COL_DQ + (DQT ? BM : DH) <= 512, "tensor memory");
+    static_assert(!DQT || DH == 128, "transposed dQ needs M = 128");
+    static_assert(SMEM <= 232448, "shared memory");
+    // barriers
+    static constexpr int B_KV = 0;
+    static constexpr int B_Q_FULL = 1;             // QST
+    static constexpr int B_Q_EMPTY = 1 + QST;      // QST
+    static constexpr int B_S_FULL = 1 + 2 * QST;
+    static constexpr int B_DP_FULL = 2 + 2 * QST;
+    static constexpr int B_PDS_FULL = 3 + 2 * QST;
+    static constexpr int B_DS_EMPTY = 4 + 2 * QST;
+    static constexpr int B_DQ_FULL = 5 + 2 * QST;
+    static constexpr int B_DQ_FREE = 6 + 2 * QST;
+    static constexpr int B_KDONE = 7 + 2 * QST;
+    static constexpr int NBAR = 8 + 2 * QST;
+    static constexpr uint32_t OFF_TMEM_SLOT = 512, OFF_ABORT = 516;
+    static constexpr uint32_t OFF_LSE = 1024;                       // [QST][BM] f32, LSE * log2(e)
+    static constexpr uint32_t OFF_DLT = OFF_LSE + 4 * 2 * 128;      // [QST][BM] f32, Delta
+};
+
+struct BwdParams {
+    const float *lse;      // [B*Hq*T]
+    const float *delta;    // [B*Hq*T]
+    float *dq_acc;         // [B*Hq][Tpad][D]
+    __nv_bfloat16 *dk, *dv;
+    int B, Hq, Hkv, T, Tpad, window, num_kt;
+    float scale;           // softmax scale (folded into dS)
+    float scale_log2;      // scale * log2(e)
+    float softcap;         // 0 = off
+    float cap_in;          // scale / softcap
+    float cap_out;         // softcap * log2(e)
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                  const BwdParams p) {
+    using C = BwdTc<D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t sbase = smem_u32(smem_raw);
+    const uint32_t tiles = (sbase + C::CTRL + 1023u) & ~1023u;
+    const uint32_t sK = tiles + C::OFF_K, sV = tiles + C::OFF_V, sQ0 = tiles + C::OFF_Q;
+    const uint32_t sdO0 = tiles + C::OFF_DO, sdS = tiles + C::OFF_DS;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem_raw + C::OFF_ABORT);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + C::OFF_TMEM_SLOT);
+    float *sLSE = reinterpret_cast<float *>(smem_raw + C::OFF_LSE);
+    float *sDLT = reinterpret_cast<float *>(smem_raw + C::OFF_DLT);
+    auto bar = [&](int i) -> uint32_t { return sbase + 8u * (uint32_t)i; };
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    // work item: key tile n (heaviest = smallest n first), batch b, KV head, half h
+    const int per_n = p.B * p.Hkv * C::NSPLIT;
+    const int n = blockIdx.x / per_n;
+    int rest = blockIdx.x % per_n;
+    const int h = rest % C::NSPLIT;
+    rest /= C::NSPLIT;
+    const int bkv = rest;  // b * Hkv + hkv
+    const int b = bkv / p.Hkv, hkv = bkv % p.Hkv;
+    const int G = p.Hq / p.Hkv;
+    const int k0 = n * C::BN;
+    const int W = p.window;
+    const int m_lo = k0 / C::BM;
+    const int q_last = W > 0 ? min(p.T - 1, k0 + C::BN - 1 + W - 1) : p.T - 1;
+    const int m_hi = q_last / C::BM;
+    const int nm = m_hi - m_lo + 1;
+    const int steps = G * nm;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(C::B_KV), 1);
+        for (int s = 0; s < C::QST; s++) {
+            mbar_init(bar(C::B_Q_FULL + s), 33);
+            mbar_init(bar(C::B_Q_EMPTY + s), 1);
+        }
+        mbar_init(bar(C::B_S_FULL), 1);
+        mbar_init(bar(C::B_DP_FULL), 1);
+        mbar_init(bar(C::B_PDS_FULL), 4);
+        mbar_init(bar(C::B_DS_EMPTY), 1);
+        mbar_init(bar(C::B_DQ_FULL), 1);
+        mbar_init(bar(C::B_DQ_FREE), 4);
+        mbar_init(bar(C::B_KDONE), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 8 && lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        tma_prefetch_desc(&tmdO);
+    }
+    if (warp == 9) {
+        tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 8) {
+        // ------------------------------------------------------------ producer
+        int issued = 0;
+        bool ok = true;
+        if (lane == 0) {
+            mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::TK);
+            for (int c = 0; c < C::NCB; c++) {
+                tma_load_3d(sK + c * C::CBK, &tmK, bar(C::B_KV), c * 64, k0, bkv);
+                tma_load_3d(sV + c * C::CBK, &tmV, bar(C::B_KV), c * 64, k0, bkv);
+            }
+        }
+        for (int i = 0; i < steps; i++) {
+            const int st = i % C::QST;
+            const uint32_t ph = (uint32_t)((i / C::QST) & 1);
+            const int g = i / nm, m = m_lo + i % nm;
+            const int bhq = b * p.Hq + hkv * G + g;
+            if (!mbar_wait_warp(bar(C::B_Q_EMPTY + st), ph ^ 1u, abort_flag)) {
+                ok = false;
+                break;
+            }
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar(C::B_Q_FULL + st), 2 * C::TQ);
+                for (int c = 0; c < C::NCB; c++) {
+                    tma_load_3d(sQ0 + st * C::TQ + c * C::CBQ, &tmQ, bar(C::B_Q_FULL + st), c * 64, m * C::BM, bhq);
+                    tma_load_3d(sdO0 + st * C::TQ + c * C::CBQ, &tmdO, bar(C::B_Q_FULL + st), c * 64, m * C::BM,
+                                bhq);
+                }
+            }
+            issued++;
+            for (int c = lane; c < C::BM; c += 32) {
+                const int q = m * C::BM + c;
+                const size_t idx = (size_t)bhq * p.T + (size_t)min(q, p.T - 1);
+                sLSE[st * C::BM + c] = q < p.T ? p.lse[idx] * kLog2e : INFINITY;
+                sDLT[st * C::BM + c] = q < p.T ? p.delta[idx] : 0.0f;
+            }
+            mbar_arrive(bar(C::B_Q_FULL + st));
+        }
+        if (!ok && lane == 0) {
+            mbar_wait_drain(bar(C::B_KV), 0, 200000000ull);
+            for (int back = 1; back <= min(issued, C::QST); back++) {
+                const int L = issued - back;
+                mbar_wait_drain(bar(C::B_Q_FULL + L % C::QST), (uint32_t)((L / C::QST) & 1), 200000000ull);
+            }
+        }
+    } else if (warp == 9) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t ID_S = idesc_bf16_f32(128, C::BM, false, false);
+            constexpr uint32_t ID_ACC = idesc_bf16_f32(128, C::DH, false, true);
+            constexpr uint32_t ID_DQ =
+                C::DQT ? idesc_bf16_f32(128, C::BM, true, true) : idesc_bf16_f32(128, C::D, true, true);
+            const uint32_t h_q = (uint32_t)h * (C::DH / 64) * C::CBQ;  // column-block offset of half h
+            const uint32_t h_k = (uint32_t)h * (C::DH / 64) * C::CBK;
+            bool ok = mbar_wait(bar(C::B_KV), 0, abort_flag);
+            for (int i = 0; ok && i < steps; i++) {
+                const int st = i % C::QST;
+                const uint32_t ph = (uint32_t)((i / C::QST) & 1);
+                const uint32_t sQ = sQ0 + st * C::TQ, sdO = sdO0 + st * C::TQ;
+                if (!(ok = mbar_wait(bar(C::B_Q_FULL + st), ph, abort_flag))) break;
+                tc_fence_after();
+                // S^T = K Q^T and dP^T = V dO^T over the full head dim
+#pragma unroll
+                for (int kk = 0; kk < D / 16; kk++) {
+                    const uint32_t ok_ = (kk >> 2) * C::CBK + (kk & 3) * 32;
+                    const uint32_t oq = (kk >> 2) * C::CBQ + (kk & 3) * 32;
+                    mma_ss(tmem + C::COL_S, sdesc_sw128(sK + ok_, 16, 1024), sdesc_sw128(sQ + oq, 16, 1024), ID_S,
+                           kk > 0);
+                }
+                tc_commit(bar(C::B_S_FULL));
+#pragma unroll
+                for (int kk = 0; kk < D / 16; kk++) {
+                    const uint32_t ok_ = (kk >> 2) * C::CBK + (kk & 3) * 32;
+                    const uint32_t oq = (kk >> 2) * C::CBQ + (kk & 3) * 32;
+                    mma_ss(tmem + C::COL_DP, sdesc_sw128(sV + ok_, 16, 1024), sdesc_sw128(sdO + oq, 16, 1024), ID_S,
+                           kk > 0);
+                }
+                tc_commit(bar(C::B_DP_FULL));
+                if (!(ok = mbar_wait(bar(C::B_PDS_FULL), (uint32_t)(i & 1), abort_flag))) break;
+                tc_fence_after();
+                // dV += P^T dO (P^T from TMEM), dK += dS^T Q
+#pragma unroll
+                for (int kk = 0; kk < C::BM / 16; kk++)
+                    mma_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8, sdesc_sw128(sdO + h_q + kk * 2048, C::CBQ, 1024),
+                           ID_ACC, (i > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < C::BM / 16; kk++) {
+                    const uint32_t oa = (kk >> 2) * C::CBK + (kk & 3) * 32;
+                    mma_ss(tmem + C::COL_DK, sdesc_sw128(sdS + oa, 16, 1024),
+                           sdesc_sw128(sQ + h_q + kk * 2048, C::CBQ, 1024), ID_ACC, (i > 0 || kk > 0) ? 1u : 0u);
+                }
+                // dQ (the drain warps must have emptied the previous one)
+                if (i > 0) {
+                    if (!(ok = mbar_wait(bar(C::B_DQ_FREE), (uint32_t)((i - 1) & 1), abort_flag))) break;
+                    tc_fence_after();
+                }
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; kk++) {
+                    if constexpr (C::DQT) {
+                        mma_ss(tmem + C::COL_DQ, sdesc_sw128(sK + h_k + kk * 2048, C::CBK, 1024),
+                               sdesc_sw128(sdS + kk * 2048, C::CBK, 1024), ID_DQ, kk > 0);
+                    } else {
+                        mma_ss(tmem + C::COL_DQ, sdesc_sw128(sdS + kk * 2048, C::CBK, 1024),
+                               sdesc_sw128(sK + kk * 2048, C::CBK, 1024), ID_DQ, kk > 0);
+                    }
+                }
+                tc_commit(bar(C::B_DQ_FULL));
+                tc_commit(bar(C::B_Q_EMPTY + st));
+                tc_commit(bar(C::B_DS_EMPTY));
+            }
+            tc_commit(bar(C::B_KDONE));
+            if (!ok) mbar_wait_drain(bar(C::B_KDONE), 0, 200000000ull);
+        }
+    } else if (warp < 4) {
+        // ------------------------------------------- compute (key rows, TMEM lanes)
+        const int kr = threadIdx.x;  // key row within the tile
+        const int kj = k0 + kr;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        bool ok = true;
+        for (int i = 0; i < steps; i++) {
+            const int st = i % C::QST;
+            const uint32_t ph = (uint32_t)((i / C::QST) & 1);
+            const int m = m_lo + i % nm;
+            const int qb = m * C::BM;
+            if (!(ok = mbar_wait_warp(bar(C::B_Q_FULL + st), ph, abort_flag))) break;
+            if (!(ok = mbar_wait_warp(bar(C::B_S_FULL), (uint32_t)(i & 1), abort_flag))) break;
+            if (!(ok = mbar_wait_warp(bar(C::B_DP_FULL), (uint32_t)(i & 1), abort_flag))) break;
+            if (i > 0 && !(ok = mbar_wait_warp(bar(C::B_DS_EMPTY), (uint32_t)((i - 1) & 1), abort_flag))) break;
+            tc_fence_after();
+            const float *lse2 = sLSE + st * C::BM;
+            const float *dlt = sDLT + st * C::BM;
+            const bool need_mask = (k0 + C::BN - 1 > qb) || (W > 0 && k0 <= qb + C::BM - 1 - W);
+#pragma unroll 1
+            for (int c0 = 0; c0 < C::BM; c0 += 32) {
+                uint32_t s[32], dp[32];
+                tmem_ld32(tmem + lane_base + C::COL_S + c0, s);
+                tmem_ld32(tmem + lane_base + C::COL_DP + c0, dp);
+                tmem_ld_wait(s);
+                tmem_ld_wait(dp);
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int c = 0; c < 32; c += 2) {
+                    float pp[2], dd[2];
+#pragma unroll
+                    for (int e = 0; e < 2; e++) {
+                        const int cc = c0 + c + e;
+                        const float x = __uint_as_float(s[c + e]);
+                        float s2, cg = 1.0f;
+                        if (p.softcap > 0.0f) {
+                            const float t = tanh_via_ex2(x * p.cap_in);
+                            s2 = p.cap_out * t;
+                            cg = 1.0f - t * t;
+                        } else {
+                            s2 = x * p.scale_log2;
+                        }
+                        float pr = ex2_approx(s2 - lse2[cc]);
+                        if (need_mask) {
+                            const int qi = qb + cc;
+                            const bool vis = kj <= qi && (W == 0 || kj > qi - W);
+                            pr = vis ? pr : 0.0f;
+                        }
+                        pp[e] = pr;
+                        dd[e] = pr * cg * (__uint_as_float(dp[c + e]) - dlt[cc]) * p.scale;
+                    }
+                    pk[c >> 1] = pack_bf16x2(pp[0], pp[1]);
+                    dk[c >> 1] = pack_bf16x2(dd[0], dd[1]);
+                }
+                // P^T chunk -> TMEM columns [c0/2, c0/2 + 16) of the S^T region
+                // (those S^T columns were already read: c0/2 + 16 <= c0 + 32).
+                tmem_st16(tmem + lane_base + C::COL_S + (uint32_t)(c0 >> 1), pk);
+                // dS^T chunk -> shared memory row kr, columns [c0, c0 + 32): 4 x 16 bytes,
+                // 128-byte swizzle (16-byte chunk index XOR row % 8).
+                const uint32_t blk = sdS + (uint32_t)(c0 >> 6) * C::CBK + (uint32_t)kr * 128u;
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    const uint32_t chunk = (uint32_t)(((c0 & 63) >> 3) + e);
+                    const uint32_t addr = blk + ((chunk ^ (uint32_t)(kr & 7)) << 4);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dk[4 * e]),
+                                 "r"(dk[4 * e + 1]), "r"(dk[4 * e + 2]), "r"(dk[4 * e + 3])
+                                 : "memory");
+                }
+            }
+            tmem_st_wait();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_PDS_FULL));
+        }
+        // epilogue: dV rows
+        if (ok) ok = mbar_wait_warp(bar(C::B_KDONE), 0, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            __nv_bfloat16 *row = p.dv + ((size_t)bkv * p.T + (size_t)min(kj, p.T - 1)) * D + h * C::DH;
+#pragma unroll 1
+            for (int c0 = 0; c0 < C::DH; c0 += 32) {
+                uint32_t o[32];
+                tmem_ld32(tmem + lane_base + C::COL_DV + c0, o);
+                tmem_ld_wait(o);
+                uint32_t w[16];
+#pragma unroll
+                for (int i = 0; i < 16; i++) w[i] = pack_bf16x2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1]));
+                if (kj < p.T) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(row + c0);
+#pragma unroll
+                    for (int i = 0; i < 4; i++) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                }
+            }
+        }
+    } else {
+        // ------------------------------------ dQ drain (warps 4..7), dK epilogue
+        const int t = threadIdx.x - 128;  // TMEM lane of this thread
+        const uint32_t lane_base = (uint32_t)((warp - 4) * 32) << 16;
+        bool ok = true;
+        for (int i = 0; i < steps; i++) {
+            const int g = i / nm, m = m_lo + i % nm;
+            const int bhq = b * p.Hq + hkv * G + g;
+            if (!(ok = mbar_wait_warp(bar(C::B_DQ_FULL), (uint32_t)(i & 1), abort_flag))) break;
+            tc_fence_after();
+            if constexpr (C::DQT) {
+                // lane = head-dim column h*DH + t, columns = BM query rows
+                uint32_t v[C::BM];
+                uint32_t(&v0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
+                uint32_t(&v1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
+                tmem_ld32(tmem + lane_base + C::COL_DQ, v0);
+                tmem_ld32(tmem + lane_base + C::COL_DQ + 32, v1);
+                tmem_ld_wait(v0);
+                tmem_ld_wait(v1);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::B_DQ_FREE));
+                float *base = p.dq_acc + ((size_t)bhq * p.Tpad + (size_t)m * C::BM) * D + h * C::DH + t;
+#pragma unroll 8
+                for (int c = 0; c < C::BM; c++) atomicAdd(base + (size_t)c * D, __uint_as_float(v[c]));
+            } else {
+                // lane = query row t of the tile, columns = D head-dim values
+                uint32_t v[64];
+                uint32_t(&v0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
+                uint32_t(&v1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
+                tmem_ld32(tmem + lane_base + C::COL_DQ, v0);
+                tmem_ld32(tmem + lane_base + C::COL_DQ + 32, v1);
+                tmem_ld_wait(v0);
+                tmem_ld_wait(v1);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::B_DQ_FREE));
+                float4 *base = reinterpret_cast<float4 *>(p.dq_acc + ((size_t)bhq * p.Tpad + (size_t)m * C::BM + t) * D);
+#pragma unroll
+                for (int c = 0; c < 16; c++)
+                    atomicAdd(base + c, make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
+                                                    __uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3])));
+            }
+        }
+        if (ok) ok = mbar_wait_warp(bar(C::B_KDONE), 0, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            const int kj = k0 + t;
+            __nv_bfloat16 *row = p.dk + ((size_t)bkv * p.T + (size_t)min(kj, p.T - 1)) * D + h * C::DH;
+#pragma unroll 1
+            for (int c0 = 0; c0 < C::DH; c0 += 32) {
+                uint32_t o[32];
+                tmem_ld32(tmem + lane_base + C::COL_DK + c0, o);
+                tmem_ld_wait(o);
+                uint32_t w[16];
+#pragma unroll
+                for (int i = 0; i < 16; i++) w[i] = pack_bf16x2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1]));
+                if (kj < p.T) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(row + c0);
+#pragma unroll
+                    for (int i = 0; i < 4; i++) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+}  // namespace forge

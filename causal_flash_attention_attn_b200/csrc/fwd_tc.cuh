@@ -1,0 +1,340 @@
+// fwd_tc.cuh -- tensor-core forward (bf16 in, f32 accumulate) for sm_100a.
+//
+// One CTA per (query tile of 128 rows, batch, query head), heaviest tiles
+// first. Only the KV tiles a tile can see are visited: j from
+// lo = (q0 - W + 1) / 128 (0 without a window) up to the diagonal tile, so the
+// cost scales with the window ("out-of-window KV blocks are skipped, so cost
+// scales with the window": src/nn/attention.h commit log, Wave 2).
+//
+// Roles (192 threads):
+//   warp 4   TMA producer: Q once, then K/V tiles through an NSTAGE ring in the
+//            order the MMA warp consumes them: K0 K1 | V0 K2 | V1 K3 | ...
+//   warp 5   MMA issuer (one thread) and TMEM owner (512 columns):
+//            S_b = Q K_j^T into S buffer b = j % 2 (128 columns each), then
+//            O += P_j V_j with P read from tensor memory (it overwrites S_b).
+//            Two S buffers let QK^T of tile j+1 run while tile j is in softmax.
+//   warps 0-3 softmax + epilogue, one thread per query row (TMEM lane):
+//            s = scale*S (or cap*tanh(scale*S/cap)), masked only on tiles that
+//            straddle the diagonal or the window edge; online softmax in base 2.
+//            The running max is only moved when a row max exceeds it by more
+//            than 8 (a factor 256), so O in TMEM is rescaled rarely; the result
+//            is exact either way because l and O use the same stale max.
+// Online softmax (max, sum) per row: ARCHITECTURES.md "Vague 2" item 10.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace forge {
+
+template <int D>
+struct FwdTc {
+    static constexpr int BM = 128, BN = 128;
+    static constexpr int NCB = D / 64;                 // 64-column (128-byte) blocks
+    static constexpr uint32_t CB = 128 * 128;          // bytes of one column block of a 128-row tile
+    static constexpr uint32_t TILE = NCB * CB;         // one 128 x D bf16 tile
+    static constexpr int NSTAGE = D == 256 ? 2 : (D == 128 ? 4 : 6);
+    static constexpr uint32_t CTRL = 1024;             // barriers, TMEM slot, abort flag
+    static constexpr uint32_t SMEM = CTRL + TILE * (1 + NSTAGE) + 1024;
+    static constexpr int THREADS = 192;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O = 256;
+    // barrier indices
+    static constexpr int B_Q = 0;
+    static constexpr int B_KV_FULL = 1;
+    static constexpr int B_KV_EMPTY = 1 + NSTAGE;
+    static constexpr int B_S_FULL = 1 + 2 * NSTAGE;
+    static constexpr int B_P_FULL = 3 + 2 * NSTAGE;
+    static constexpr int B_O_READY = 5 + 2 * NSTAGE;
+    static constexpr int B_O_FINAL = 6 + 2 * NSTAGE;
+    static constexpr int NBAR = 7 + 2 * NSTAGE;
+    static constexpr uint32_t OFF_TMEM_SLOT = 512;
+    static constexpr uint32_t OFF_ABORT = 516;
+    static_assert(NBAR * 8 <= 512, "control block");
+    static_assert(SMEM <= 232448, "shared memory");
+};
+
+struct FwdParams {
+    __nv_bfloat16 *o;
+    float *lse;
+    int B, Hq, Hkv, T, window, num_qt;
+    float scale_log2;  // scale * log2(e)
+    float softcap;     // 0 = off
+    float cap_in;      // scale / softcap
+    float cap_out;     // softcap * log2(e)
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+    using C = FwdTc<D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t sbase = smem_u32(smem_raw);
+    const uint32_t tiles = (sbase + C::CTRL + 1023u) & ~1023u;
+    const uint32_t sQ = tiles;
+    const uint32_t sKV = tiles + C::TILE;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem_raw + C::OFF_ABORT);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + C::OFF_TMEM_SLOT);
+    auto bar = [&](int i) -> uint32_t { return sbase + 8u * (uint32_t)i; };
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int nbh = p.B * p.Hq;
+    const int qt = p.num_qt - 1 - (int)(blockIdx.x / nbh);
+    const int bh = blockIdx.x % nbh;
+    const int b = bh / p.Hq, hq = bh % p.Hq;
+    const int bkv = b * p.Hkv + hq / (p.Hq / p.Hkv);
+    const int q0 = qt * C::BM;
+    const int lo = p.window > 0 ? max(0, q0 - p.window + 1) / C::BN : 0;
+    const int n = qt - lo + 1;  // KV tiles lo..qt
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(C::B_Q), 1);
+        for (int s = 0; s < C::NSTAGE; s++) {
+            mbar_init(bar(C::B_KV_FULL + s), 1);
+            mbar_init(bar(C::B_KV_EMPTY + s), 1);
+        }
+        for (int s = 0; s < 2; s++) {
+            mbar_init(bar(C::B_S_FULL + s), 1);
+            mbar_init(bar(C::B_P_FULL + s), 4);
+        }
+        mbar_init(bar(C::B_O_READY), 1);
+        mbar_init(bar(C::B_O_FINAL), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 4 && lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+    }
+    if (warp == 5) {
+        tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            const uint64_t keep = policy_evict_last();
+            mbar_arrive_expect_tx(bar(C::B_Q), C::TILE);
+            for (int c = 0; c < C::NCB; c++) tma_load_3d(sQ + c * C::CB, &tmQ, bar(C::B_Q), c * 64, q0, bh);
+            int stage = 0;
+            uint32_t ph = 0;
+            int issued = 0;
+            bool ok = true;
+            auto load = [&](const CUtensorMap *m, int j) -> bool {
+                if (!mbar_wait(bar(C::B_KV_EMPTY + stage), ph ^ 1u, abort_flag)) return false;
+                mbar_arrive_expect_tx(bar(C::B_KV_FULL + stage), C::TILE);
+                for (int c = 0; c < C::NCB; c++)
+                    tma_load_3d_hint(sKV + stage * C::TILE + c * C::CB, m, bar(C::B_KV_FULL + stage), c * 64,
+                                     j * C::BN, bkv, keep);
+                issued++;
+                if (++stage == C::NSTAGE) {
+                    stage = 0;
+                    ph ^= 1u;
+                }
+                return true;
+            };
+            ok = load(&tmK, lo);
+            if (ok && n > 1) ok = load(&tmK, lo + 1);
+            for (int u = 0; ok && u < n; u++) {
+                ok = load(&tmV, lo + u);
+                if (ok && u + 2 < n) ok = load(&tmK, lo + u + 2);
+            }
+            if (!ok) {
+                // Let the copies already issued land before the CTA exits.
+                mbar_wait_drain(bar(C::B_Q), 0, 200000000ull);
+                for (int back = 1; back <= min(issued, C::NSTAGE); back++) {
+                    const int L = issued - back;
+                    mbar_wait_drain(bar(C::B_KV_FULL + L % C::NSTAGE), (uint32_t)((L / C::NSTAGE) & 1),
+                                    200000000ull);
+                }
+            }
+        }
+    } else if (warp == 5) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t ID_QK = idesc_bf16_f32(128, 128, false, false);
+            constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, false, true);
+            int stage = 0;
+            uint32_t ph = 0;
+            auto next = [&]() {
+                if (++stage == C::NSTAGE) {
+                    stage = 0;
+                    ph ^= 1u;
+                }
+            };
+            auto qk = [&](int buf) -> bool {
+                if (!mbar_wait(bar(C::B_KV_FULL + stage), ph, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t sK = sKV + stage * C::TILE;
+                const uint32_t dS = tmem + (buf ? C::COL_S1 : C::COL_S0);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; kk++) {
+                    const uint32_t off = (kk >> 2) * C::CB + (kk & 3) * 32;
+                    mma_ss(dS, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), ID_QK, kk > 0);
+                }
+                tc_commit(bar(C::B_S_FULL + buf));
+                tc_commit(bar(C::B_KV_EMPTY + stage));
+                next();
+                return true;
+            };
+            auto pv = [&](int buf, bool acc) -> bool {
+                if (!mbar_wait(bar(C::B_KV_FULL + stage), ph, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t sV = sKV + stage * C::TILE;
+                const uint32_t aP = tmem + (buf ? C::COL_S1 : C::COL_S0);
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; kk++)
+                    mma_ts(tmem + C::COL_O, aP + kk * 8, sdesc_sw128(sV + kk * 2048, C::CB, 1024), ID_PV,
+                           (acc || kk > 0) ? 1u : 0u);
+                tc_commit(bar(C::B_O_READY));
+                tc_commit(bar(C::B_KV_EMPTY + stage));
+                next();
+                return true;
+            };
+            bool ok = mbar_wait(bar(C::B_Q), 0, abort_flag);
+            if (ok) ok = qk(0);
+            if (ok && n > 1) ok = qk(1);
+            for (int u = 0; ok && u < n; u++) {
+                const int buf = u & 1;
+                ok = mbar_wait(bar(C::B_P_FULL + buf), (uint32_t)((u >> 1) & 1), abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                ok = pv(buf, u > 0);
+                if (ok && u + 2 < n) ok = qk(buf);
+            }
+            // Whether or not the loop finished, O_FINAL fires once every MMA
+            // issued so far has completed (the softmax warps or the abort path
+            // wait on it before tensor memory is released).
+            tc_commit(bar(C::B_O_FINAL));
+            if (!ok) mbar_wait_drain(bar(C::B_O_FINAL), 0, 200000000ull);
+        }
+    } else {
+        // ---------------------------------------------- softmax (warps 0..3)
+        const int row = threadIdx.x;
+        const int qi = q0 + row;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const int W = p.window;
+        float m = -INFINITY, l = 0.0f;
+        bool ok = true;
+        for (int u = 0; u < n; u++) {
+            const int buf = u & 1;
+            const int k0 = (lo + u) * C::BN;
+            if (!mbar_wait_warp(bar(C::B_S_FULL + buf), (uint32_t)((u >> 1) & 1), abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tS = tmem + lane_base + (buf ? C::COL_S1 : C::COL_S0);
+            uint32_t s[4][32];
+            tmem_ld32(tS + 0, s[0]);
+            tmem_ld32(tS + 32, s[1]);
+            tmem_ld32(tS + 64, s[2]);
+            tmem_ld32(tS + 96, s[3]);
+            tmem_ld_wait(s[0]);
+            tmem_ld_wait(s[1]);
+            tmem_ld_wait(s[2]);
+            tmem_ld_wait(s[3]);
+            // scores in log2 units
+            if (p.softcap > 0.0f) {
+#pragma unroll
+                for (int c = 0; c < 128; c++) {
+                    const float x = __uint_as_float(s[c >> 5][c & 31]);
+                    s[c >> 5][c & 31] = __float_as_uint(p.cap_out * tanh_via_ex2(x * p.cap_in));
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 128; c++)
+                    s[c >> 5][c & 31] = __float_as_uint(__uint_as_float(s[c >> 5][c & 31]) * p.scale_log2);
+            }
+            const bool need_mask = (k0 + C::BN - 1 > q0) || (W > 0 && k0 <= q0 + C::BM - 1 - W);
+            if (need_mask) {
+#pragma unroll
+                for (int c = 0; c < 128; c++) {
+                    const int kj = k0 + c;
+                    const bool vis = kj <= qi && (W == 0 || kj > qi - W);
+                    if (!vis) s[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+                }
+            }
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 128; c++) mx = fmaxf(mx, __uint_as_float(s[c >> 5][c & 31]));
+            const float m_new = (mx > m + 8.0f) ? mx : m;
+            const bool moved = (m_new != m);
+            const float factor = moved ? ex2_approx(m - m_new) : 1.0f;
+            if (__any_sync(0xffffffffu, moved && u > 0)) {
+                // rescale O (row-wise) once PV of the previous tile has landed
+                if (!mbar_wait_warp(bar(C::B_O_READY), (uint32_t)((u - 1) & 1), abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const float f = (moved && u > 0) ? factor : 1.0f;
+#pragma unroll 1
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(tmem + lane_base + C::COL_O + c0, o);
+                    tmem_ld_wait(o);
+#pragma unroll
+                    for (int i = 0; i < 32; i++) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+                    tmem_st32(tmem + lane_base + C::COL_O + c0, o);
+                }
+                tmem_st_wait();
+            }
+            m = m_new;
+            const float msub = (m == -INFINITY) ? 0.0f : m;
+            float rs = 0.0f;
+            uint32_t pk[2][32];
+#pragma unroll
+            for (int c = 0; c < 64; c++) {
+                const float p0 = ex2_approx(__uint_as_float(s[(2 * c) >> 5][(2 * c) & 31]) - msub);
+                const float p1 = ex2_approx(__uint_as_float(s[(2 * c + 1) >> 5][(2 * c + 1) & 31]) - msub);
+                rs += p0 + p1;
+                pk[c >> 5][c & 31] = pack_bf16x2(p0, p1);
+            }
+            tmem_st32(tS + 0, pk[0]);
+            tmem_st32(tS + 32, pk[1]);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_P_FULL + buf));
+            l = l * factor + rs;
+        }
+        if (ok) ok = mbar_wait_warp(bar(C::B_O_FINAL), 0, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            const float inv_l = 1.0f / l;
+            __nv_bfloat16 *orow = p.o + ((size_t)bh * p.T + (size_t)min(qi, p.T - 1)) * D;
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t o[32];
+                tmem_ld32(tmem + lane_base + C::COL_O + c0, o);
+                tmem_ld_wait(o);
+                uint32_t w[16];
+#pragma unroll
+                for (int i = 0; i < 16; i++)
+                    w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+                if (qi < p.T) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
+#pragma unroll
+                    for (int i = 0; i < 4; i++) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                }
+            }
+            if (qi < p.T) p.lse[(size_t)bh * p.T + qi] = (m + __log2f(l)) * kLn2;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+}  // namespace forge

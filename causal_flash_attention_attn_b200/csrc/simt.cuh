@@ -1,0 +1,311 @@
+// simt.cuh -- CUDA-core attention kernels (f32 arithmetic throughout).
+//
+// This is the f32 path of the library (FORGE_DTYPE_F32): exact f32 FMAs, no
+// tensor cores, so the result stays within the 1e-4 parity bar the Forge pages
+// set for their CPU-vs-GPU checks (README "85 parity checks, <=1e-4"). The
+// same templates instantiated for bf16 storage serve the bf16 backward at head
+// dim 256 until the tensor-core backward covers it.
+//
+// Structure: a block owns 16 rows (4 warps x 4 rows); keys (or queries) stream
+// through shared memory 32 at a time; lane j of a warp scores element j of the
+// tile, and lane d owns output columns d, d+32, ...
+//  - simt_fwd:   rows = queries; online softmax over key tiles -> o, lse.
+//  - simt_bwd_dq: rows = queries; P = exp(s - lse), dS = P (dP - Delta) [* cap'],
+//                 dq = scale * sum dS k.
+//  - simt_bwd_dkdv: rows = keys; loops over the group's query heads and the
+//                 queries that see the key; dv = sum P dO, dk = scale * sum dS q.
+// No atomics: every output element has one writer, so results are deterministic.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+namespace forge {
+
+constexpr int kSimtRows = 16;  // rows per block
+constexpr int kSimtTile = 32;  // streamed rows per tile
+constexpr int kSimtThreads = 128;
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ void from_f32(float *p, float x) { *p = x; }
+__device__ __forceinline__ void from_f32(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    return x;
+}
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// Visible iff kj <= qi and (window == 0 or kj > qi - window).
+__device__ __forceinline__ bool visible(int qi, int kj, int window) {
+    return kj <= qi && (window == 0 || kj > qi - window);
+}
+
+// Capped score from the scaled dot product (natural units).
+__device__ __forceinline__ float simt_capped(float s, float softcap) {
+    return softcap > 0.0f ? softcap * tanhf(s / softcap) : s;
+}
+
+template <typename T, int D>
+__device__ __forceinline__ void load_rows(float *dst, int ld, const T *src, int row0, int nrows,
+                                          int T_) {
+    for (int idx = threadIdx.x; idx < nrows * D; idx += blockDim.x) {
+        const int r = idx / D, d = idx % D;
+        dst[r * ld + d] = (row0 + r < T_ && row0 + r >= 0) ? to_f32(src[(size_t)(row0 + r) * D + d]) : 0.0f;
+    }
+}
+
+template <int D>
+constexpr size_t simt_fwd_smem() {
+    return sizeof(float) * (size_t)(kSimtRows * D + 2 * kSimtTile * (D + 1));
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kSimtThreads) simt_fwd(const T *__restrict__ q, const T *__restrict__ k,
+                                                         const T *__restrict__ v, T *__restrict__ o,
+                                                         float *__restrict__ lse, int Hq, int Hkv, int T_,
+                                                         float scale, int window, float softcap) {
+    extern __shared__ float sm[];
+    float *sQ = sm;
+    float *sK = sQ + kSimtRows * D;
+    float *sV = sK + kSimtTile * (D + 1);
+    constexpr int NT = D / 32;
+    const int bh = blockIdx.y, b = bh / Hq, hq = bh % Hq, hkv = hq / (Hq / Hkv);
+    const int r0 = blockIdx.x * kSimtRows;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const T *Qb = q + (size_t)bh * T_ * D;
+    const T *Kb = k + (size_t)(b * Hkv + hkv) * T_ * D;
+    const T *Vb = v + (size_t)(b * Hkv + hkv) * T_ * D;
+    load_rows<T, D>(sQ, D, Qb, r0, kSimtRows, T_);
+
+    float m[4], l[4], acc[4][NT];
+#pragma unroll
+    for (int rr = 0; rr < 4; rr++) {
+        m[rr] = -INFINITY;
+        l[rr] = 0.0f;
+#pragma unroll
+        for (int t = 0; t < NT; t++) acc[rr][t] = 0.0f;
+    }
+    const int last = min(r0 + kSimtRows - 1, T_ - 1);
+    int first = (window > 0) ? max(0, r0 - window + 1) : 0;
+    first = (first / kSimtTile) * kSimtTile;
+    for (int k0 = first; k0 <= last; k0 += kSimtTile) {
+        __syncthreads();
+        load_rows<T, D>(sK, D + 1, Kb, k0, kSimtTile, T_);
+        load_rows<T, D>(sV, D + 1, Vb, k0, kSimtTile, T_);
+        __syncthreads();
+#pragma unroll
+        for (int rr = 0; rr < 4; rr++) {
+            const int r = warp * 4 + rr, qi = r0 + r;
+            if (qi >= T_) continue;
+            const int kj = k0 + lane;
+            float s = 0.0f;
+#pragma unroll 8
+            for (int d = 0; d < D; d++) s = fmaf(sQ[r * D + d], sK[lane * (D + 1) + d], s);
+            s = simt_capped(s * scale, softcap);
+            const bool ok = visible(qi, kj, window) && kj < T_;
+            s = ok ? s : -INFINITY;
+            const float mnew = fmaxf(m[rr], warp_max(s));
+            if (mnew == -INFINITY) continue;
+            const float corr = expf(m[rr] - mnew);
+            const float p = ok ? expf(s - mnew) : 0.0f;
+            l[rr] = l[rr] * corr + warp_sum(p);
+#pragma unroll
+            for (int t = 0; t < NT; t++) acc[rr][t] *= corr;
+            for (int j = 0; j < kSimtTile; j++) {
+                const float pj = __shfl_sync(0xffffffffu, p, j);
+#pragma unroll
+                for (int t = 0; t < NT; t++) acc[rr][t] = fmaf(pj, sV[j * (D + 1) + lane + 32 * t], acc[rr][t]);
+            }
+            m[rr] = mnew;
+        }
+    }
+#pragma unroll
+    for (int rr = 0; rr < 4; rr++) {
+        const int qi = r0 + warp * 4 + rr;
+        if (qi >= T_) continue;
+        const float inv = 1.0f / l[rr];
+        T *orow = o + ((size_t)bh * T_ + qi) * D;
+#pragma unroll
+        for (int t = 0; t < NT; t++) from_f32(orow + lane + 32 * t, acc[rr][t] * inv);
+        if (lane == 0) lse[(size_t)bh * T_ + qi] = m[rr] + logf(l[rr]);
+    }
+}
+
+template <int D>
+constexpr size_t simt_bwd_dq_smem() {
+    return sizeof(float) * (size_t)(2 * kSimtRows * D + 2 * kSimtTile * (D + 1));
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kSimtThreads) simt_bwd_dq(const T *__restrict__ q, const T *__restrict__ k,
+                                                            const T *__restrict__ v, const float *__restrict__ lse,
+                                                            const T *__restrict__ dO, const float *__restrict__ delta,
+                                                            T *__restrict__ dq, int Hq, int Hkv, int T_, float scale,
+                                                            int window, float softcap) {
+    extern __shared__ float sm[];
+    float *sQ = sm;
+    float *sdO = sQ + kSimtRows * D;
+    float *sK = sdO + kSimtRows * D;
+    float *sV = sK + kSimtTile * (D + 1);
+    constexpr int NT = D / 32;
+    const int bh = blockIdx.y, b = bh / Hq, hq = bh % Hq, hkv = hq / (Hq / Hkv);
+    const int r0 = blockIdx.x * kSimtRows;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const T *Kb = k + (size_t)(b * Hkv + hkv) * T_ * D;
+    const T *Vb = v + (size_t)(b * Hkv + hkv) * T_ * D;
+    load_rows<T, D>(sQ, D, q + (size_t)bh * T_ * D, r0, kSimtRows, T_);
+    load_rows<T, D>(sdO, D, dO + (size_t)bh * T_ * D, r0, kSimtRows, T_);
+    float acc[4][NT], L[4], Dl[4];
+#pragma unroll
+    for (int rr = 0; rr < 4; rr++) {
+        const int qi = min(r0 + warp * 4 + rr, T_ - 1);
+        L[rr] = lse[(size_t)bh * T_ + qi];
+        Dl[rr] = delta[(size_t)bh * T_ + qi];
+#pragma unroll
+        for (int t = 0; t < NT; t++) acc[rr][t] = 0.0f;
+    }
+    const int last = min(r0 + kSimtRows - 1, T_ - 1);
+    int first = (window > 0) ? max(0, r0 - window + 1) : 0;
+    first = (first / kSimtTile) * kSimtTile;
+    for (int k0 = first; k0 <= last; k0 += kSimtTile) {
+        __syncthreads();
+        load_rows<T, D>(sK, D + 1, Kb, k0, kSimtTile, T_);
+        load_rows<T, D>(sV, D + 1, Vb, k0, kSimtTile, T_);
+        __syncthreads();
+#pragma unroll
+        for (int rr = 0; rr < 4; rr++) {
+            const int r = warp * 4 + rr, qi = r0 + r;
+            if (qi >= T_) continue;
+            const int kj = k0 + lane;
+            float s = 0.0f, dp = 0.0f;
+#pragma unroll 8
+            for (int d = 0; d < D; d++) {
+                s = fmaf(sQ[r * D + d], sK[lane * (D + 1) + d], s);
+                dp = fmaf(sdO[r * D + d], sV[lane * (D + 1) + d], dp);
+            }
+            const float sc = simt_capped(s * scale, softcap);
+            const bool ok = visible(qi, kj, window) && kj < T_;
+            const float p = ok ? expf(sc - L[rr]) : 0.0f;
+            float ds = p * (dp - Dl[rr]);
+            if (softcap > 0.0f) {
+                const float t = sc / softcap;
+                ds *= 1.0f - t * t;
+            }
+            for (int j = 0; j < kSimtTile; j++) {
+                const float dsj = __shfl_sync(0xffffffffu, ds, j);
+#pragma unroll
+                for (int t = 0; t < NT; t++) acc[rr][t] = fmaf(dsj, sK[j * (D + 1) + lane + 32 * t], acc[rr][t]);
+            }
+        }
+    }
+#pragma unroll
+    for (int rr = 0; rr < 4; rr++) {
+        const int qi = r0 + warp * 4 + rr;
+        if (qi >= T_) continue;
+        T *row = dq + ((size_t)bh * T_ + qi) * D;
+#pragma unroll
+        for (int t = 0; t < NT; t++) from_f32(row + lane + 32 * t, acc[rr][t] * scale);
+    }
+}
+
+template <int D>
+constexpr size_t simt_bwd_dkdv_smem() {
+    return sizeof(float) * (size_t)(2 * kSimtRows * D + 2 * kSimtTile * (D + 1) + 2 * kSimtTile);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kSimtThreads) simt_bwd_dkdv(const T *__restrict__ q, const T *__restrict__ k,
+                                                              const T *__restrict__ v, const float *__restrict__ lse,
+                                                              const T *__restrict__ dO,
+                                                              const float *__restrict__ delta, T *__restrict__ dk,
+                                                              T *__restrict__ dv, int Hq, int Hkv, int T_,
+                                                              float scale, int window, float softcap) {
+    extern __shared__ float sm[];
+    float *sK = sm;                        // [16][D] key rows of this block
+    float *sV = sK + kSimtRows * D;        // [16][D]
+    float *sQ = sV + kSimtRows * D;        // [32][D+1] query tile
+    float *sdO = sQ + kSimtTile * (D + 1); // [32][D+1]
+    float *sL = sdO + kSimtTile * (D + 1); // [32]
+    float *sD = sL + kSimtTile;            // [32]
+    constexpr int NT = D / 32;
+    const int bkv = blockIdx.y, b = bkv / Hkv, hkv = bkv % Hkv;
+    const int G = Hq / Hkv;
+    const int r0 = blockIdx.x * kSimtRows;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    load_rows<T, D>(sK, D, k + (size_t)bkv * T_ * D, r0, kSimtRows, T_);
+    load_rows<T, D>(sV, D, v + (size_t)bkv * T_ * D, r0, kSimtRows, T_);
+    float adk[4][NT], adv[4][NT];
+#pragma unroll
+    for (int rr = 0; rr < 4; rr++)
+#pragma unroll
+        for (int t = 0; t < NT; t++) adk[rr][t] = adv[rr][t] = 0.0f;
+    const int qfirst = (r0 / kSimtTile) * kSimtTile;
+    int qlast = T_ - 1;
+    if (window > 0) qlast = min(qlast, r0 + kSimtRows - 1 + window - 1);
+    for (int g = 0; g < G; g++) {
+        const int bh = b * Hq + hkv * G + g;
+        for (int q0 = qfirst; q0 <= qlast; q0 += kSimtTile) {
+            __syncthreads();
+            load_rows<T, D>(sQ, D + 1, q + (size_t)bh * T_ * D, q0, kSimtTile, T_);
+            load_rows<T, D>(sdO, D + 1, dO + (size_t)bh * T_ * D, q0, kSimtTile, T_);
+            if (threadIdx.x < kSimtTile) {
+                const int qi = q0 + threadIdx.x;
+                sL[threadIdx.x] = qi < T_ ? lse[(size_t)bh * T_ + qi] : 0.0f;
+                sD[threadIdx.x] = qi < T_ ? delta[(size_t)bh * T_ + qi] : 0.0f;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int rr = 0; rr < 4; rr++) {
+                const int r = warp * 4 + rr, kj = r0 + r;
+                if (kj >= T_) continue;
+                const int qi = q0 + lane;
+                float s = 0.0f, dp = 0.0f;
+#pragma unroll 8
+                for (int d = 0; d < D; d++) {
+                    s = fmaf(sK[r * D + d], sQ[lane * (D + 1) + d], s);
+                    dp = fmaf(sV[r * D + d], sdO[lane * (D + 1) + d], dp);
+                }
+                const float sc = simt_capped(s * scale, softcap);
+                const bool ok = qi < T_ && visible(qi, kj, window);
+                const float p = ok ? expf(sc - sL[lane]) : 0.0f;
+                float ds = p * (dp - sD[lane]);
+                if (softcap > 0.0f) {
+                    const float t = sc / softcap;
+                    ds *= 1.0f - t * t;
+                }
+                for (int j = 0; j < kSimtTile; j++) {
+                    const float pj = __shfl_sync(0xffffffffu, p, j);
+                    const float dsj = __shfl_sync(0xffffffffu, ds, j);
+#pragma unroll
+                    for (int t = 0; t < NT; t++) {
+                        adv[rr][t] = fmaf(pj, sdO[j * (D + 1) + lane + 32 * t], adv[rr][t]);
+                        adk[rr][t] = fmaf(dsj, sQ[j * (D + 1) + lane + 32 * t], adk[rr][t]);
+                    }
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int rr = 0; rr < 4; rr++) {
+        const int kj = r0 + warp * 4 + rr;
+        if (kj >= T_) continue;
+        T *krow = dk + ((size_t)bkv * T_ + kj) * D;
+        T *vrow = dv + ((size_t)bkv * T_ + kj) * D;
+#pragma unroll
+        for (int t = 0; t < NT; t++) {
+            from_f32(krow + lane + 32 * t, adk[rr][t] * scale);
+            from_f32(vrow + lane + 32 * t, adv[rr][t]);
+        }
+    }
+}
+
+}  // namespace forge

@@ -1,0 +1,141 @@
+/*
+ * forge_attn.h -- C ABI of the B200 (sm_100a) fused causal attention library
+ * (libforge_attn.so): forward and backward of causal multi-head attention with
+ * GQA head mapping, an optional sliding window and an optional attention-logit
+ * softcap.
+ *
+ * What the operation is (Forge pages):
+ *   S_ij  = scale * (q_i . k_j)
+ *   s_ij  = softcap * tanh(S_ij / softcap)      if softcap > 0, else S_ij
+ *           ("cap*tanh on scores pre-softmax": src/nn/attention.h commit log,
+ *            Wave 2 (attention kernels); ARCHITECTURES.md "Vague 2" item 9)
+ *   key j is visible to query i iff  i - window < j <= i   (window = 0: j <= i)
+ *           (ARCHITECTURES.md "Vague 2" item 8; sliding_window(0) default,
+ *            forge-studio RESEARCH.md section 2)
+ *   P_i   = softmax over the visible j of s_ij,   o_i = sum_j P_ij v_j,
+ *   lse_i = log sum_j exp(s_ij)  (natural log)
+ *   Query head hq reads KV head hq / (Hq / Hkv) (GQA; Hq % Hkv == 0 is the
+ *   config rule n_heads % n_kv_heads == 0, RESEARCH.md section 2).
+ *   The backward is the exact gradient of o with respect to q, k, v, including
+ *   the tanh' factor of the cap ("exact tanh' chain in all backwards").
+ *   A per-layer pattern (sliding_global_every) is chosen by the caller: a global
+ *   layer passes window = 0.
+ *
+ * Layouts (all row-major, contiguous, device memory, 16-byte aligned):
+ *   q, o, dO, dq : [B][Hq][T][D]      k, v, dk, dv : [B][Hkv][T][D]
+ *   lse          : [B][Hq][T] float32
+ *   `dtype` gives the element type of q, k, v, o, dO, dq, dk, dv.
+ *   FORGE_DTYPE_BF16 runs the tensor-core kernels (bf16 operands, f32
+ *   accumulation, P and dS rounded to bf16 before their products);
+ *   FORGE_DTYPE_F32 runs f32 CUDA-core kernels (f32 arithmetic throughout).
+ *   Supported head dims: 64, 128, 256.
+ *
+ * Ownership and behaviour:
+ *   The caller allocates and frees every buffer, including the backward
+ *   workspace. The library never allocates, frees or synchronises (except
+ *   forge_attn_check, which synchronises the stream it is given), and launches
+ *   only on `stream` (a cudaStream_t; NULL is the legacy default stream).
+ *   Calls are asynchronous; outputs are fully overwritten (dq, dk, dv are not
+ *   accumulated into). Errors are returned, never thrown or aborted.
+ *   Every wait inside a kernel is bounded; a wait that runs out records
+ *   FORGE_ERR_TIMEOUT in a device status word that forge_attn_check reports.
+ */
+#ifndef FORGE_ATTN_H
+#define FORGE_ATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FORGE_OK = 0,
+    FORGE_ERR_INVALID_ARG = 1, /* null or misaligned pointer, bad size, bad scalar */
+    FORGE_ERR_UNSUPPORTED = 2, /* valid but not built: head dim not in {64,128,256} */
+    FORGE_ERR_WORKSPACE = 3,   /* backward workspace missing, misaligned or too small */
+    FORGE_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+    FORGE_ERR_TIMEOUT = 5      /* a bounded wait inside a kernel ran out */
+} forge_status;
+
+typedef enum { FORGE_DTYPE_F32 = 0, FORGE_DTYPE_BF16 = 1 } forge_dtype;
+
+/*
+ * Forward. Writes o and lse (lse is kept for the backward).
+ * scale: finite, > 0 (usually 1/sqrt(D)); window: >= 0, 0 = off, >= T acts as
+ * off; softcap: finite, >= 0, 0 = off.
+ * Returns FORGE_OK or an error; on error nothing is launched.
+ */
+forge_status forge_attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                            int B, int Hq, int Hkv, int T, int D, float scale, int window,
+                            float softcap, forge_dtype dtype, void *stream);
+
+/*
+ * Bytes of device workspace forge_attn_bwd needs for these sizes (0 on invalid
+ * sizes). Holds rowsum(dO * o) as f32 and, for bf16, an f32 dq accumulator.
+ */
+size_t forge_attn_bwd_workspace_size(int B, int Hq, int Hkv, int T, int D, forge_dtype dtype);
+
+/*
+ * Backward. Given q, k, v, the o and lse of the matching forward call and the
+ * upstream gradient dO, writes dq, dk, dv. `workspace` is caller-owned device
+ * memory of at least forge_attn_bwd_workspace_size(...) bytes, 256-byte
+ * aligned; its contents on entry do not matter and are overwritten.
+ * Launches three kernels in order: forge_attn_bwd_preprocess,
+ * forge_attn_bwd_main, forge_attn_bwd_finalize (below), on `stream`.
+ */
+forge_status forge_attn_bwd(const void *q, const void *k, const void *v, const void *o,
+                            const float *lse, const void *dO, void *dq, void *dk, void *dv,
+                            int B, int Hq, int Hkv, int T, int D, float scale, int window,
+                            float softcap, forge_dtype dtype, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/*
+ * The three stages of forge_attn_bwd, callable one by one on the same stream
+ * with the same arguments and workspace (used to time the stages separately).
+ *  preprocess: Delta_i = sum_d dO_id o_id into the workspace (f32) and, for
+ *              bf16, zeroes the dq accumulator;
+ *  main:       recomputes P from q, k and lse, and produces dk, dv (written
+ *              out) and dq (accumulated in the workspace for bf16; written
+ *              out for f32);
+ *  finalize:   bf16 only, converts the dq accumulator to dq (no-op for f32).
+ */
+forge_status forge_attn_bwd_preprocess(const void *o, const void *dO, int B, int Hq, int Hkv,
+                                       int T, int D, forge_dtype dtype, void *workspace,
+                                       size_t workspace_bytes, void *stream);
+forge_status forge_attn_bwd_main(const void *q, const void *k, const void *v, const float *lse,
+                                 const void *dO, void *dq, void *dk, void *dv, int B, int Hq,
+                                 int Hkv, int T, int D, float scale, int window, float softcap,
+                                 forge_dtype dtype, void *workspace, size_t workspace_bytes,
+                                 void *stream);
+forge_status forge_attn_bwd_finalize(void *dq, int B, int Hq, int Hkv, int T, int D,
+                                     forge_dtype dtype, void *workspace, size_t workspace_bytes,
+                                     void *stream);
+
+/*
+ * Synchronises `stream`, then reports (and clears) any error a kernel of this
+ * library recorded on the current device since the last check: FORGE_OK,
+ * FORGE_ERR_TIMEOUT, or FORGE_ERR_CUDA for an asynchronous CUDA error.
+ */
+forge_status forge_attn_check(void *stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *forge_attn_status_string(forge_status s);
+
+/*
+ * Self-test of the bounded-wait machinery: launches one tiny kernel that waits
+ * on a barrier nothing will ever complete, with a wait limit of `limit_us`
+ * microseconds (1..2000000). The wait runs out, the kernel records
+ * FORGE_ERR_TIMEOUT and returns normally, leaving the context usable; the next
+ * forge_attn_check reports it. Used by the tests of failure detection.
+ */
+forge_status forge_attn_selftest_timeout(unsigned int limit_us, void *stream);
+
+/* Library version, e.g. "forge_attn 0.1.0 sm_100a". */
+const char *forge_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FORGE_ATTN_H */

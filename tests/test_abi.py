@@ -1,0 +1,111 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/forge_attn.h declares, and rejects bad arguments with the
+documented status codes before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import causal_flash_attention_attn_b200 as fa
+from causal_flash_attention_attn_b200 import build as fa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "forge_attn.h")
+
+A = 0x10000  # a 16-byte (and 256-byte) aligned fake device address: never dereferenced
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    fa_build.build()
+    yield
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"\b(forge_attn_\w+)\s*\(", text)))
+
+
+def test_header_functions_are_exported():
+    names = declared_functions()
+    assert len(names) >= 10
+    lib = ctypes.CDLL(fa.library_path)
+    for n in names:
+        assert hasattr(lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", fa.library_path], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (forge_attn_\w+)", out))
+    assert set(names) <= exported, set(names) - exported
+
+
+def test_status_strings_and_version():
+    for code in range(6):
+        s = fa.forge_attn_status_string(code)
+        assert s.startswith("FORGE_")
+    assert fa.forge_attn_status_string(99) == "FORGE_ERR_UNKNOWN"
+    assert "sm_100a" in fa.forge_attn_version()
+
+
+def fwd(**kw):
+    a = dict(q=A, k=A, v=A, o=A, lse=A, B=1, Hq=4, Hkv=2, T=128, D=128, scale=0.1, window=0, softcap=0.0,
+             dtype=fa.FORGE_DTYPE_BF16, stream=0)
+    a.update(kw)
+    return fa.forge_attn_fwd(**a)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hkv=3), fa.FORGE_ERR_INVALID_ARG),           # Hq % Hkv != 0
+    (dict(D=63), fa.FORGE_ERR_INVALID_ARG),            # odd head dim
+    (dict(D=96), fa.FORGE_ERR_UNSUPPORTED),            # even but not built
+    (dict(D=512), fa.FORGE_ERR_UNSUPPORTED),
+    (dict(B=0), fa.FORGE_ERR_INVALID_ARG),
+    (dict(T=0), fa.FORGE_ERR_INVALID_ARG),
+    (dict(Hq=0), fa.FORGE_ERR_INVALID_ARG),
+    (dict(window=-1), fa.FORGE_ERR_INVALID_ARG),
+    (dict(softcap=-1.0), fa.FORGE_ERR_INVALID_ARG),
+    (dict(softcap=float("inf")), fa.FORGE_ERR_INVALID_ARG),
+    (dict(scale=0.0), fa.FORGE_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), fa.FORGE_ERR_INVALID_ARG),
+    (dict(q=0), fa.FORGE_ERR_INVALID_ARG),             # null
+    (dict(o=A + 8), fa.FORGE_ERR_INVALID_ARG),         # misaligned
+    (dict(dtype=7), fa.FORGE_ERR_INVALID_ARG),
+])
+def test_fwd_rejects(kw, code):
+    assert fwd(**kw) == code
+
+
+def test_workspace_size_and_rejection():
+    bf, f32 = fa.FORGE_DTYPE_BF16, fa.FORGE_DTYPE_F32
+    n = fa.forge_attn_bwd_workspace_size(2, 28, 4, 4096, 128, bf)
+    delta = 2 * 28 * 4096 * 4
+    acc = 2 * 28 * 4096 * 128 * 4
+    assert n >= delta + acc and n <= delta + acc + 512
+    assert fa.forge_attn_bwd_workspace_size(2, 28, 4, 4096, 128, f32) >= delta
+    assert fa.forge_attn_bwd_workspace_size(2, 28, 3, 4096, 128, bf) == 0
+    # ragged T pads the accumulator to a multiple of 128 rows
+    assert fa.forge_attn_bwd_workspace_size(1, 1, 1, 129, 64, bf) >= 256 * 64 * 4
+    args = dict(q=A, k=A, v=A, o=A, lse=A, dO=A, dq=A, dk=A, dv=A, B=1, Hq=2, Hkv=1, T=100, D=64, scale=0.1,
+                window=0, softcap=0.0, dtype=bf, stream=0)
+    need = fa.forge_attn_bwd_workspace_size(1, 2, 1, 100, 64, bf)
+    assert fa.forge_attn_bwd(workspace=A, workspace_bytes=need - 1, **args) == fa.FORGE_ERR_WORKSPACE
+    assert fa.forge_attn_bwd(workspace=0, workspace_bytes=need, **args) == fa.FORGE_ERR_WORKSPACE
+    assert fa.forge_attn_bwd(workspace=A + 16, workspace_bytes=need, **args) == fa.FORGE_ERR_WORKSPACE
+    bad = dict(args, Hkv=3)
+    assert fa.forge_attn_bwd(workspace=A, workspace_bytes=need, **bad) == fa.FORGE_ERR_INVALID_ARG
+    bad = dict(args, dk=A + 4)
+    assert fa.forge_attn_bwd(workspace=A, workspace_bytes=need, **bad) == fa.FORGE_ERR_INVALID_ARG
+
+
+def test_selftest_rejects_bad_limit():
+    assert fa.forge_attn_selftest_timeout(0, 0) == fa.FORGE_ERR_INVALID_ARG
+    assert fa.forge_attn_selftest_timeout(3000000, 0) == fa.FORGE_ERR_INVALID_ARG
+
+
+def test_layer_window_pattern():
+    from causal_flash_attention_attn_b200.inputs import layer_window
+    # Gemma 3-like 5 local : 1 global
+    assert [layer_window(l, 1024, 6) for l in range(12)] == [1024] * 5 + [0] + [1024] * 5 + [0]
+    # alternating
+    assert [layer_window(l, 4096, 2) for l in range(4)] == [4096, 0, 4096, 0]
+    assert [layer_window(l, 4096, 0) for l in range(3)] == [4096] * 3
