@@ -1,0 +1,443 @@
+"""Throughput of causal attention forward + backward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+One step = forward + backward (forge_attn_fwd, then forge_attn_bwd's three
+stages) over one batch of the workload, inputs resident in HBM. The metric is
+TFLOPS counting only causal / in-window score pairs: forward 4*D*pairs, backward
+10*D*pairs (five D-deep products per pair, the recompute of S included).
+
+N > 1 (torchrun, one process per GPU): every rank runs its own copy of the
+workload (independent batches, no collective on the data path: weak scaling);
+time is the max over ranks of the device-timed region.
+
+--impl reference times the f64 CPU oracle on the host cores on a bounded sample
+of the same workload (rank 0 only), in the same unit.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "causal attention fwd+bwd TFLOPS on 1 B200 and % of dense BF16 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def flops_of(w):
+    from causal_flash_attention_attn_b200.inputs import allowed_pairs
+    pairs = allowed_pairs(w.T, w.window) * w.B * w.Hq
+    return 4.0 * w.D * pairs, 10.0 * w.D * pairs
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "causal_flash_attention_attn_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel, workload):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None
+    when the summary is missing or was taken on different kernel sources."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    e = d.get(f"{kernel}@{workload}")
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ distributed
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity when world == 1)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world == 1:
+        return
+    import torch.distributed as dist
+    if device is not None and device.type == "cuda":
+        dist.barrier(device_ids=[device.index])
+    else:
+        dist.barrier()
+
+
+# ------------------------------------------------------------ CPU baseline
+def cpu_oracle_sample(w, budget_s=12.0, max_groups=None):
+    """Time the f64 oracle (fwd + bwd) on whole KV groups of the workload, adding
+    groups until ~budget_s of CPU work. Returns (tflops, seconds, description, cores)."""
+    import oracle
+    from causal_flash_attention_attn_b200 import inputs
+    from causal_flash_attention_attn_b200.inputs import allowed_pairs
+    q, k, v, dO = inputs.make_inputs(w)
+    G = w.G
+    groups = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+    if max_groups:
+        groups = groups[:max_groups]
+    done, secs, flops = 0, 0.0, 0.0
+    for b, h in groups:
+        hs = slice(h * G, (h + 1) * G)
+        ks, vs = k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1]
+        qs, ds = q[b:b + 1, hs], dO[b:b + 1, hs]
+        t0 = time.perf_counter()
+        oracle.attn_fwd(qs, ks, vs, w.sm_scale, w.window, w.softcap)
+        oracle.attn_bwd(qs, ks, vs, ds, w.sm_scale, w.window, w.softcap)
+        secs += time.perf_counter() - t0
+        flops += 14.0 * w.D * allowed_pairs(w.T, w.window) * G
+        done += 1
+        if secs >= budget_s:
+            break
+    desc = (f"f64 oracle fwd+bwd on {done} of {w.B * w.Hkv} KV groups (b, kv-head) of {w.name}, "
+            f"each {G} query heads x T={w.T}")
+    return flops / secs / 1e12, secs, desc, oracle.num_threads()
+
+
+# -------------------------------------------------------------------- ours
+def run_ours(args, w):
+    import torch
+    import causal_flash_attention_attn_b200 as fa
+    from causal_flash_attention_attn_b200 import inputs
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    fa.library()
+    stream = torch.cuda.Stream(device=dev)
+
+    # inputs: each rank its own batch of the workload (seed offset by rank)
+    wr = w.with_(seed=w.seed + 1000 * rank) if rank else w
+    q, k, v, dO = inputs.make_inputs(wr)
+    B, Hq, Hkv, T, D = w.B, w.Hq, w.Hkv, w.T, w.D
+    dt = fa.dtype_code(inputs.torch_dtype(w.dtype))
+    qd, kd, vd, dOd = (x.to(dev) for x in (q, k, v, dO))
+    o = torch.empty_like(qd)
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    nws = fa.forge_attn_bwd_workspace_size(B, Hq, Hkv, T, D, dt)
+    ws = torch.empty(nws, dtype=torch.uint8, device=dev)
+    sc, W, C = w.sm_scale, w.window, w.softcap
+    sh = stream.cuda_stream
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        s = fa.forge_attn_fwd(qd, kd, vd, o, lse, B, Hq, Hkv, T, D, sc, W, C, dt, sh)
+        if ev:
+            ev[1].record(stream)
+        s |= fa.forge_attn_bwd_preprocess(o, dOd, B, Hq, Hkv, T, D, dt, ws, nws, sh)
+        if ev:
+            ev[2].record(stream)
+        s |= fa.forge_attn_bwd_main(qd, kd, vd, lse, dOd, dq, dk, dv, B, Hq, Hkv, T, D, sc, W, C, dt, ws, nws, sh)
+        if ev:
+            ev[3].record(stream)
+        s |= fa.forge_attn_bwd_finalize(dq, B, Hq, Hkv, T, D, dt, ws, nws, sh)
+        if ev:
+            ev[4].record(stream)
+        if s != fa.FORGE_OK:
+            raise fa.ForgeError(s, "step")
+
+    launches_per_step = 4
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize(dev)
+    st = fa.forge_attn_check(sh)
+    if st != fa.FORGE_OK:
+        raise fa.ForgeError(st, "warmup")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    clk = ClockSampler(dev.index)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    clk.start()
+    time.sleep(0.3)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = clk.stop()
+    barrier(world, dev)
+    st = fa.forge_attn_check(sh)
+    if st != fa.FORGE_OK:
+        raise fa.ForgeError(st, "timed run")
+    ms_local = start.elapsed_time(end)
+    ms = max_over_ranks(ms_local, world, dev)
+    per = {"fwd": [], "bwd_preprocess": [], "bwd_main": [], "bwd_finalize": []}
+    for e in evs:
+        per["fwd"].append(e[0].elapsed_time(e[1]))
+        per["bwd_preprocess"].append(e[1].elapsed_time(e[2]))
+        per["bwd_main"].append(e[2].elapsed_time(e[3]))
+        per["bwd_finalize"].append(e[3].elapsed_time(e[4]))
+    avg = {kname: sum(v) / len(v) for kname, v in per.items()}
+
+    # end to end through the same C ABI from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        hq_, hk_, hv_, hdo = (x.pin_memory() for x in (q, k, v, dO))
+        hdq, hdk, hdv = (torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in (qd, kd, vd))
+        h2d = sum(x.numel() * x.element_size() for x in (hq_, hk_, hv_, hdo))
+        d2h = sum(x.numel() * x.element_size() for x in (hdq, hdk, hdv))
+
+        def e2e_step():
+            for dst, src in ((qd, hq_), (kd, hk_), (vd, hv_), (dOd, hdo)):
+                dst.copy_(src, non_blocking=True)
+            step()
+            for dst, src in ((hdq, dq), (hdk, dk), (hdv, dv)):
+                dst.copy_(src, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier(world, dev)
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            s0.record(stream)
+            for _ in range(args.steps):
+                e2e_step()
+            s1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(s0.elapsed_time(s1), world, dev) / args.steps
+        fl_f, fl_b = flops_of(w)
+        e2e = {"value": round(world * (fl_f + fl_b) / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOPS",
+               "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    fl_f, fl_b = flops_of(w)
+    ms_step = ms / args.steps
+    tflops = world * (fl_f + fl_b) / (ms_step * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    timed_s = ms * 1e-3
+    peak_key = "bf16_tflops_sustained" if timed_s > 2.0 else "bf16_tflops"
+    peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
+    # dominant kernel: the larger of forward and backward-main by time
+    dom = "bwd_main" if avg["bwd_main"] >= avg["fwd"] else "fwd"
+    dom_flops = fl_b if dom == "bwd_main" else fl_f
+    achieved = dom_flops / (avg[dom] * 1e-3) / 1e12
+    kname = {"fwd": "fwd_tc_kernel", "bwd_main": "bwd_tc_kernel"}[dom]
+    traffic = ncu_traffic(kname, w.name)
+    line = {
+        "metric": METRIC,
+        "value": round(tflops, 3),
+        "unit": "TFLOPS",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded N(0, sigma^2) Q, K, V, dO)",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "T": w.T, "D": w.D,
+                   "window": w.window, "softcap": w.softcap, "scale": w.sm_scale,
+                   "parallelism": f"replicas x{world} (independent batches, no collective)",
+                   "flops_per_step_per_gpu": fl_f + fl_b,
+                   "flop_count": "only causal/in-window pairs; fwd 4*D*pairs, bwd 10*D*pairs",
+                   "l2": "not flushed: per-step working set (q,k,v,o,dO,dq,dk,dv,lse + f32 dq accumulator) "
+                         "exceeds the 126 MB L2"},
+        "pct_of_bf16_peak": round(100.0 * tflops / world / peak, 2),
+        "kernels_ms": {k_: round(v_, 4) for k_, v_ in avg.items()},
+        "roofline": {"kernel": kname, "bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "peak_source": f"{peak_src} {peak_key}",
+                     "achieved_def": f"{'10' if dom == 'bwd_main' else '4'}*D*pairs per launch / "
+                                     "CUDA-event launch time"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if world == 1 and not args.no_cpu:
+        v_, secs, desc, cores = cpu_oracle_sample(w, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(v_, 6), "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                                "sample": desc, "seconds": round(secs, 2)}
+    return line
+
+
+def run_reference(args, w):
+    """The oracle as it stands, on the host cores: W untimed then K timed steps,
+    each step one bounded sample (one whole KV group of the workload, cycling
+    through the groups)."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    import oracle
+    from causal_flash_attention_attn_b200 import inputs
+    from causal_flash_attention_attn_b200.inputs import allowed_pairs
+    q, k, v, dO = inputs.make_inputs(w)
+    G = w.G
+    groups = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+
+    def sample(i):
+        b, h = groups[i % len(groups)]
+        hs = slice(h * G, (h + 1) * G)
+        qs, ds = q[b:b + 1, hs], dO[b:b + 1, hs]
+        ks, vs = k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1]
+        t0 = time.perf_counter()
+        oracle.attn_fwd(qs, ks, vs, w.sm_scale, w.window, w.softcap)
+        oracle.attn_bwd(qs, ks, vs, ds, w.sm_scale, w.window, w.softcap)
+        return time.perf_counter() - t0
+
+    for i in range(args.warmup):
+        sample(i)
+    secs = sum(sample(i) for i in range(args.steps))
+    flops = 14.0 * w.D * allowed_pairs(w.T, w.window) * G * args.steps
+    value = flops / secs / 1e12
+    fl_f, fl_b = flops_of(w)
+    desc = (f"f64 oracle fwd+bwd, one KV group (b, kv-head: {G} query heads x T={w.T}) of {w.name} per step")
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 6),
+        "unit": "TFLOPS",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(1e3 * secs / args.steps, 2),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded N(0, sigma^2) Q, K, V, dO)",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "T": w.T, "D": w.D,
+                   "window": w.window, "softcap": w.softcap, "flops_per_step_full": fl_f + fl_b},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=None)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args(argv)
+    from causal_flash_attention_attn_b200 import inputs
+    w = inputs.WORKLOADS[args.workload or inputs.HEADLINE]
+    if args.warmup < 3:
+        args.warmup = 3
+    line = run_reference(args, w) if args.impl == "reference" else run_ours(args, w)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()
