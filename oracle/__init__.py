@@ -32,7 +32,8 @@ def _load():
         i = ctypes.c_int
         d = ctypes.c_double
         lib.oracle_attn_fwd.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i, d, i, d]
-        lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, d, i, d]
+        lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, d, i, d, i]
+        lib.oracle_round.argtypes = [dp, dp, ctypes.c_long, i]
         lib.oracle_attn_probs.argtypes = [dp, dp, dp, i, i, i, i, i, d, i, d]
         lib.oracle_rowdot.argtypes = [dp, dp, dp, ctypes.c_long, i]
         lib.oracle_num_threads.restype = ctypes.c_int
@@ -72,8 +73,23 @@ def attn_fwd(q, k, v, scale: float, window: int = 0, softcap: float = 0.0):
     return o, lse
 
 
-def attn_bwd(q, k, v, dO, scale: float, window: int = 0, softcap: float = 0.0):
-    """Return (dq, dk, dv, delta, lse) in f64 for upstream gradient dO."""
+_ROUND = {None: 0, "f64": 0, "f32": 1, "bf16": 2}
+
+
+def round_to(x, dtype: str):
+    """Round f64 values to a storage type ("f32" or "bf16", nearest even) and back."""
+    x = _f64(x)
+    y = np.empty_like(x)
+    _load().oracle_round(_ptr(x), _ptr(y), x.size, _ROUND[dtype])
+    return y
+
+
+def attn_bwd(q, k, v, dO, scale: float, window: int = 0, softcap: float = 0.0, o_round=None):
+    """Return (dq, dk, dv, delta, lse) in f64 for upstream gradient dO.
+
+    o_round=None uses Delta_i = sum_j P_ij dP_ij. o_round="f32"/"bf16" uses
+    Delta_i = rowsum(dO * o) with the oracle's own o rounded to that storage type,
+    i.e. the O a forward call of that dtype returns to the backward."""
     q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
     B, Hq, Hkv, T, D = _dims(q, k)
     dq = np.empty_like(q)
@@ -83,7 +99,7 @@ def attn_bwd(q, k, v, dO, scale: float, window: int = 0, softcap: float = 0.0):
     lse = np.empty((B, Hq, T), dtype=np.float64)
     _load().oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dq), _ptr(dk), _ptr(dv),
                             _ptr(delta), _ptr(lse), B, Hq, Hkv, T, D, float(scale), int(window),
-                            float(softcap))
+                            float(softcap), _ROUND[o_round])
     return dq, dk, dv, delta, lse
 
 

@@ -29,6 +29,7 @@
  * lse and delta are [B][Hq][T]; all row-major, f64.
  */
 #include <math.h>
+#include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -60,6 +61,29 @@ static double cap_grad(double s, double softcap) {
     if (softcap <= 0.0) return 1.0;
     double t = tanh(s / softcap);
     return 1.0 - t * t;
+}
+
+/*
+ * Rounding of an output value to the storage type of the call: 1 = f32
+ * (round to nearest even), 2 = bf16 (to f32, then to the 8 significant bits of
+ * bf16, round to nearest even on the f32 bit pattern), 0 = none.
+ */
+static double round_to(double x, int mode) {
+    if (mode == 0) return x;
+    float f = (float)x;
+    if (mode == 1) return (double)f;
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7f800000u) != 0x7f800000u) {
+        u += 0x7fffu + ((u >> 16) & 1u);
+        u &= 0xffff0000u;
+    }
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+void oracle_round(const double *x, double *y, long n, int mode) {
+    for (long i = 0; i < n; i++) y[i] = round_to(x[i], mode);
 }
 
 /*
@@ -121,11 +145,17 @@ void oracle_attn_fwd(const double *q, const double *k, const double *v, double *
  * Pass 1 walks query rows (P, Delta, dQ); pass 2 walks key rows (dK, dV), using
  * P_ij = exp(s_ij - LSE_i), which is the same softmax entry.
  * delta (may be NULL) receives Delta, lse_out (may be NULL) receives LSE.
+ *
+ * o_round selects how Delta is formed. 0: Delta_i = sum_j P_ij dP_ij (the
+ * definition). 1 or 2: Delta_i = sum_d dO_id * o_id with o_i = sum_j P_ij V_j
+ * rounded to the storage type of the call (1 = f32, 2 = bf16): the backward's
+ * first step takes rowsum(dO * O) of the O the forward returned, and in a bf16
+ * call that O is bf16. With exact O both forms are equal (sum_j P_ij = 1).
  */
 void oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dO,
                      double *dq, double *dk, double *dv, double *delta, double *lse_out,
                      int B, int Hq, int Hkv, int T, int D, double scale, int window,
-                     double softcap) {
+                     double softcap, int o_round) {
     const int G = Hq / Hkv;
     const size_t nrows = (size_t)B * Hq * T;
     double *lse = (double *)malloc(sizeof(double) * nrows);
@@ -136,6 +166,7 @@ void oracle_attn_bwd(const double *q, const double *k, const double *v, const do
     {
         double *p = (double *)malloc(sizeof(double) * (size_t)T);
         double *dp = (double *)malloc(sizeof(double) * (size_t)T);
+        double *oi = (double *)malloc(sizeof(double) * (size_t)D);
 #pragma omp for collapse(3) schedule(dynamic, 8)
         for (int b = 0; b < B; b++)
             for (int hq = 0; hq < Hq; hq++)
@@ -153,6 +184,13 @@ void oracle_attn_bwd(const double *q, const double *k, const double *v, const do
                         dp[j] = dot(doi, V + j * D, D);
                         dl += p[j] * dp[j];
                     }
+                    if (o_round != 0) {
+                        for (int d = 0; d < D; d++) oi[d] = 0.0;
+                        for (long j = lo; j <= i; j++)
+                            for (int d = 0; d < D; d++) oi[d] += p[j] * V[j * D + d];
+                        dl = 0.0;
+                        for (int d = 0; d < D; d++) dl += doi[d] * round_to(oi[d], o_round);
+                    }
                     dlt[qrow] = dl;
                     double *dqi = dq + qrow * D;
                     for (int d = 0; d < D; d++) dqi[d] = 0.0;
@@ -164,6 +202,7 @@ void oracle_attn_bwd(const double *q, const double *k, const double *v, const do
                 }
         free(p);
         free(dp);
+        free(oi);
     }
 
     /* pass 2: key rows, summed over the group's query heads */

@@ -65,7 +65,7 @@ def compare_all(q, k, v, dO, scale, window, softcap, dtype, gpu=None, subset=Fal
     pairs = groups_to_check(B, Hkv) if subset else [(b, h) for b in range(B) for h in range(Hkv)]
     if not subset:
         ro, rl = oracle.attn_fwd(q, k, v, scale, window, softcap)
-        rdq, rdk, rdv, _, _ = oracle.attn_bwd(q, k, v, dO, scale, window, softcap)
+        rdq, rdk, rdv, _, _ = oracle.attn_bwd(q, k, v, dO, scale, window, softcap, o_round=dtype)
         check_close("o", o, ro, dtype)
         check_close("lse", lse, rl, dtype)
         check_close("dq", dq, rdq, dtype)
@@ -76,7 +76,7 @@ def compare_all(q, k, v, dO, scale, window, softcap, dtype, gpu=None, subset=Fal
         hs = slice(h * G, (h + 1) * G)
         qs, ks, vs, ds = q[b:b + 1, hs], k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1], dO[b:b + 1, hs]
         ro, rl = oracle.attn_fwd(qs, ks, vs, scale, window, softcap)
-        rdq, rdk, rdv, _, _ = oracle.attn_bwd(qs, ks, vs, ds, scale, window, softcap)
+        rdq, rdk, rdv, _, _ = oracle.attn_bwd(qs, ks, vs, ds, scale, window, softcap, o_round=dtype)
         tag = f"[b={b},kv={h}]"
         check_close("o" + tag, o[b:b + 1, hs], ro, dtype)
         check_close("lse" + tag, lse[b:b + 1, hs], rl, dtype)

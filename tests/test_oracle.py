@@ -344,3 +344,39 @@ def test_closed_form_constant_value():
     np.testing.assert_allclose(o, np.broadcast_to(np.arange(8.0), o.shape), rtol=0, atol=1e-13)
     dq, dk, dv, _, _ = oracle.attn_bwd(q, k, v, dO, 0.5, 0, 3.0)
     assert np.max(np.abs(dq)) < 1e-12 and np.max(np.abs(dk)) < 1e-12
+
+
+# ------------------------------------------- Delta from the stored (rounded) O
+
+def test_rounding_matches_torch_conversions():
+    g = torch.Generator().manual_seed(21)
+    x = torch.cat([torch.randn(20000, generator=g, dtype=torch.float64) * 10 ** torch.randint(-6, 6, (20000,),
+                                                                                                 generator=g),
+                   torch.tensor([0.0, -0.0, 1.0, 1.00390625, 1.01171875, 1.0078125, 65504.0, 3.3e38, -2.5e-40,
+                                 1e-45, float("inf"), -float("inf")], dtype=torch.float64)])
+    np.testing.assert_array_equal(oracle.round_to(x, "f32"), x.to(torch.float32).double().numpy())
+    np.testing.assert_array_equal(oracle.round_to(x, "bf16"),
+                                  x.to(torch.float32).to(torch.bfloat16).double().numpy())
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_delta_from_rounded_output(dtype):
+    q, k, v, dO = qkv(1, 4, 2, 30, 8, seed=22)
+    for W, C in ((0, 0.0), (7, 2.0)):
+        o, _ = oracle.attn_fwd(q, k, v, 0.5, W, C)
+        tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+        o_stored = torch.from_numpy(o).to(torch.float32).to(tdt).double()
+        want = (o_stored * dO).sum(-1).numpy()
+        _, _, _, delta, _ = oracle.attn_bwd(q, k, v, dO, 0.5, W, C, o_round=dtype)
+        np.testing.assert_allclose(delta, want, rtol=1e-12, atol=1e-12)
+        # the gradient moves only through Delta: dV is unchanged, and dQ moves by
+        # -scale * dDelta_i * sum_j P_ij cap'_ij K_j
+        ex = oracle.attn_bwd(q, k, v, dO, 0.5, W, C)
+        rd = oracle.attn_bwd(q, k, v, dO, 0.5, W, C, o_round=dtype)
+        np.testing.assert_array_equal(rd[2], ex[2])
+        P = oracle.attn_probs(q, k, 0.5, W, C)
+        kr = k.repeat_interleave(2, dim=1).numpy()
+        S = 0.5 * np.einsum("bhid,bhjd->bhij", q.numpy(), kr)
+        cg = (1 - np.tanh(S / C) ** 2) if C else 1.0
+        U = np.einsum("bhij,bhjd->bhid", P * cg, kr)
+        np.testing.assert_allclose(rd[0] - ex[0], -0.5 * (rd[3] - ex[3])[..., None] * U, rtol=1e-9, atol=1e-13)
