@@ -85,6 +85,21 @@ bool make_map(CUtensorMap *map, const void *base, int D, int T, long long BH, in
     return r == CUDA_SUCCESS;
 }
 
+// [BH][Tpad][D] f32 accumulator as a 3D tensor; box = 32 columns (128 bytes) x
+// rows x 1 with the 128-byte swizzle, the layout of the dQ staging tiles.
+bool make_map_acc(CUtensorMap *map, const float *base, int D, int Tpad, long long BH, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (enc == nullptr) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Tpad, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)D * 4 * (cuuint64_t)Tpad};
+    cuuint32_t box[3] = {32, (cuuint32_t)box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 forge_status launch_status() {
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? FORGE_OK : FORGE_ERR_CUDA;
@@ -160,9 +175,10 @@ forge_status bwd_tc(const void *q, const void *k, const void *v, const float *ls
                     const float *delta, float *acc, void *dk, void *dv, int B, int Hq, int Hkv, int T, float scale,
                     int window, float softcap, cudaStream_t st) {
     using C = BwdTc<D>;
-    CUtensorMap mq, mk, mv, mdo;
+    CUtensorMap mq, mk, mv, mdo, macc;
     if (!make_map(&mq, q, D, T, (long long)B * Hq, C::BM) || !make_map(&mk, k, D, T, (long long)B * Hkv, 128) ||
-        !make_map(&mv, v, D, T, (long long)B * Hkv, 128) || !make_map(&mdo, dO, D, T, (long long)B * Hq, C::BM))
+        !make_map(&mv, v, D, T, (long long)B * Hkv, 128) || !make_map(&mdo, dO, D, T, (long long)B * Hq, C::BM) ||
+        !make_map_acc(&macc, acc, D, tpad_of(T), (long long)B * Hq, C::BM))
         return FORGE_ERR_CUDA;
     BwdParams p;
     p.lse = lse;
@@ -179,7 +195,7 @@ forge_status bwd_tc(const void *q, const void *k, const void *v, const float *ls
     p.cap_out = softcap * kLog2e;
     if (set_smem(bwd_tc_kernel<D>, C::SMEM) != FORGE_OK) return FORGE_ERR_CUDA;
     const unsigned grid = (unsigned)(p.num_kt * B * Hkv * C::NSPLIT);
-    bwd_tc_kernel<D><<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, mdo, p);
+    bwd_tc_kernel<D><<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, mdo, macc, p);
     return launch_status();
 }
 
@@ -257,7 +273,6 @@ forge_status forge_attn_bwd_preprocess(const void *o, const void *dO, int B, int
     if (dtype == FORGE_DTYPE_BF16) {
         // the dq accumulator receives reductions: zero it in the same pass
         float *acc = reinterpret_cast<float *>(static_cast<char *>(workspace) + delta_bytes(B, Hq, T));
-        if (D == 256) acc = nullptr;  // head dim 256 writes dq directly
         FORGE_DISPATCH_D(D, bwd_preprocess<__nv_bfloat16, kD><<<grid, 256, 0, st>>>(
                                 static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dO), delta,
                                 acc, rows, T, tpad_of(T));)
@@ -285,11 +300,6 @@ forge_status forge_attn_bwd_main(const void *q, const void *k, const void *v, co
     const float *delta = static_cast<const float *>(workspace);
     if (dtype == FORGE_DTYPE_BF16) {
         float *acc = reinterpret_cast<float *>(static_cast<char *>(workspace) + delta_bytes(B, Hq, T));
-        if (D == 256) {
-            // head dim 256: CUDA-core backward for dq, dk, dv (f32 arithmetic)
-            return bwd_simt<__nv_bfloat16, 256>(q, k, v, lse, dO, delta, dq, dk, dv, B, Hq, Hkv, T, scale, window,
-                                                softcap, st);
-        }
         FORGE_DISPATCH_D(D, return bwd_tc<kD>(q, k, v, lse, dO, delta, acc, dk, dv, B, Hq, Hkv, T, scale, window,
                                               softcap, st);)
     }
@@ -304,7 +314,7 @@ forge_status forge_attn_bwd_finalize(void *dq, int B, int Hq, int Hkv, int T, in
     if (s != FORGE_OK) return s;
     if (!aligned16(dq)) return FORGE_ERR_INVALID_ARG;
     if ((s = check_workspace(workspace, workspace_bytes, B, Hq, Hkv, T, D, dtype)) != FORGE_OK) return s;
-    if (dtype != FORGE_DTYPE_BF16 || D == 256) return FORGE_OK;  // dq already written by the main stage
+    if (dtype != FORGE_DTYPE_BF16) return FORGE_OK;  // f32: dq already written by the main stage
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const float *acc = reinterpret_cast<const float *>(static_cast<char *>(workspace) + delta_bytes(B, Hq, T));
     const long long total = (long long)B * Hq * T * (D / 8);

@@ -14,7 +14,10 @@
 //   dV  += P^T dO           (A from TMEM)
 //   dK  += dS^T Q
 //   dQ   = dS K  (or its transpose K^T dS^T), drained from TMEM by four warps
-//          with f32 reductions into a padded [B*Hq][Tpad][D] workspace.
+//          into a swizzled f32 staging tile in shared memory and added into a
+//          padded [B*Hq][Tpad][D] f32 workspace with TMA bulk reduce-add (head
+//          dim 256, which has no shared memory left for staging, adds with
+//          per-element f32 reductions instead).
 // dK and dV sum over the group's query heads inside the CTA, so they need no
 // atomics; dQ rows are shared between key tiles and are reduced in L2.
 //
@@ -51,7 +54,10 @@ struct BwdTc {
     static constexpr uint32_t OFF_K = 0, OFF_V = TK, OFF_Q = 2 * TK;
     static constexpr uint32_t OFF_DO = OFF_Q + QST * TQ;
     static constexpr uint32_t OFF_DS = OFF_DO + QST * TQ;
-    static constexpr uint32_t TILES = OFF_DS + TS;
+    static constexpr bool BULK_DQ = D != 256;            // staged TMA reduce-add of dQ
+    static constexpr uint32_t STG = BM * DH * 4;         // one f32 dQ staging tile
+    static constexpr uint32_t OFF_STG = OFF_DS + TS;     // two staging tiles (double buffer)
+    static constexpr uint32_t TILES = OFF_STG + (BULK_DQ ? 2 * STG : 0);
     static constexpr uint32_t CTRL = 4096;               // barriers, slots, LSE/Delta stages
     static constexpr uint32_t SMEM = CTRL + TILES + 1024;
     static constexpr int THREADS = 320;
@@ -95,13 +101,13 @@ template <int D>
 __global__ void __launch_bounds__(320, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tmAcc, const BwdParams p) {
     using C = BwdTc<D>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = smem_u32(smem_raw);
     const uint32_t tiles = (sbase + C::CTRL + 1023u) & ~1023u;
     const uint32_t sK = tiles + C::OFF_K, sV = tiles + C::OFF_V, sQ0 = tiles + C::OFF_Q;
-    const uint32_t sdO0 = tiles + C::OFF_DO, sdS = tiles + C::OFF_DS;
+    const uint32_t sdO0 = tiles + C::OFF_DO, sdS = tiles + C::OFF_DS, sStg = tiles + C::OFF_STG;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem_raw + C::OFF_ABORT);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + C::OFF_TMEM_SLOT);
     float *sLSE = reinterpret_cast<float *>(smem_raw + C::OFF_LSE);
@@ -374,39 +380,69 @@ __global__ void __launch_bounds__(320, 1)
             const int bhq = b * p.Hq + hkv * G + g;
             if (!(ok = mbar_wait_warp(bar(C::B_DQ_FULL), (uint32_t)(i & 1), abort_flag))) break;
             tc_fence_after();
-            if constexpr (C::DQT) {
-                // lane = head-dim column h*DH + t, columns = BM query rows
-                uint32_t v[C::BM];
-                uint32_t(&v0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
-                uint32_t(&v1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
-                tmem_ld32(tmem + lane_base + C::COL_DQ, v0);
-                tmem_ld32(tmem + lane_base + C::COL_DQ + 32, v1);
-                tmem_ld_wait(v0);
-                tmem_ld_wait(v1);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(C::B_DQ_FREE));
-                float *base = p.dq_acc + ((size_t)bhq * p.Tpad + (size_t)m * C::BM) * D + h * C::DH + t;
-#pragma unroll 8
-                for (int c = 0; c < C::BM; c++) atomicAdd(base + (size_t)c * D, __uint_as_float(v[c]));
-            } else {
-                // lane = query row t of the tile, columns = D head-dim values
-                uint32_t v[64];
-                uint32_t(&v0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
-                uint32_t(&v1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
-                tmem_ld32(tmem + lane_base + C::COL_DQ, v0);
-                tmem_ld32(tmem + lane_base + C::COL_DQ + 32, v1);
-                tmem_ld_wait(v0);
-                tmem_ld_wait(v1);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(C::B_DQ_FREE));
-                float4 *base = reinterpret_cast<float4 *>(p.dq_acc + ((size_t)bhq * p.Tpad + (size_t)m * C::BM + t) * D);
+            // two 32-column TMEM loads: this thread's 64 dQ values
+            uint32_t v0[32], v1[32];
+            tmem_ld32(tmem + lane_base + C::COL_DQ, v0);
+            tmem_ld32(tmem + lane_base + C::COL_DQ + 32, v1);
+            tmem_ld_wait(v0);
+            tmem_ld_wait(v1);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_DQ_FREE));
+            if constexpr (C::BULK_DQ) {
+                // Staging tile [BM rows][DH cols] f32, stored as DH/32 column blocks of
+                // [BM][32] with the 128-byte swizzle (16-byte chunk ^ row % 8), the
+                // layout of a TMA box {32, BM, 1}. Buffer i % 2 was last read by the
+                // reduce issued two steps ago.
+                const uint32_t stg = sStg + (uint32_t)(i & 1) * C::STG;
+                if (t == 0) bulk_wait_read<1>();
+                named_barrier_sync(1, 128);
+                if constexpr (C::DQT) {
+                    // thread t = head-dim column t of this half; v = 64 query rows
+                    const uint32_t cb = (uint32_t)t >> 5, ch = ((uint32_t)t & 31u) >> 2, w4 = ((uint32_t)t & 3u) << 2;
+                    const uint32_t base = stg + cb * (uint32_t)(C::BM * 128) + w4;
 #pragma unroll
-                for (int c = 0; c < 16; c++)
-                    atomicAdd(base + c, make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
-                                                    __uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3])));
+                    for (int c = 0; c < 32; c++) {
+                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(base + (uint32_t)c * 128u + ((ch ^ ((uint32_t)c & 7u)) << 4)),
+                                     "r"(v0[c]) : "memory");
+                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(base + (uint32_t)(c + 32) * 128u +
+                                                                     ((ch ^ ((uint32_t)(c + 32) & 7u)) << 4)),
+                                     "r"(v1[c]) : "memory");
+                    }
+                } else {
+                    // thread t = query row t; v = the 64 head-dim values of that row
+                    const uint32_t row = stg + (uint32_t)t * 128u;
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; c4++) {
+                        const uint32_t sw = (((uint32_t)c4 ^ ((uint32_t)t & 7u)) << 4);
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + sw), "r"(v0[4 * c4]),
+                                     "r"(v0[4 * c4 + 1]), "r"(v0[4 * c4 + 2]), "r"(v0[4 * c4 + 3]) : "memory");
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + (uint32_t)(C::BM * 128) + sw),
+                                     "r"(v1[4 * c4]), "r"(v1[4 * c4 + 1]), "r"(v1[4 * c4 + 2]), "r"(v1[4 * c4 + 3])
+                                     : "memory");
+                    }
+                }
+                fence_proxy_async_smem();
+                named_barrier_sync(1, 128);
+                if (t == 0) {
+#pragma unroll
+                    for (int cb = 0; cb < C::DH / 32; cb++)
+                        tma_reduce_add_3d(&tmAcc, stg + (uint32_t)cb * (uint32_t)(C::BM * 128), h * C::DH + 32 * cb,
+                                          m * C::BM, bhq);
+                    bulk_commit();
+                }
+            } else {
+                // head dim 256: lane = head-dim column h*DH + t, 64 query rows
+                float *base = p.dq_acc + ((size_t)bhq * p.Tpad + (size_t)m * C::BM) * D + h * C::DH + t;
+#pragma unroll
+                for (int c = 0; c < 32; c++) {
+                    atomicAdd(base + (size_t)c * D, __uint_as_float(v0[c]));
+                    atomicAdd(base + (size_t)(c + 32) * D, __uint_as_float(v1[c]));
+                }
             }
+        }
+        if constexpr (C::BULK_DQ) {
+            if (t == 0) bulk_wait<0>();  // reductions complete before the CTA retires
         }
         if (ok) ok = mbar_wait_warp(bar(C::B_KDONE), 0, abort_flag);
         if (ok) {

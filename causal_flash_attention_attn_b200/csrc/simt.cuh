@@ -2,9 +2,7 @@
 //
 // This is the f32 path of the library (FORGE_DTYPE_F32): exact f32 FMAs, no
 // tensor cores, so the result stays within the 1e-4 parity bar the Forge pages
-// set for their CPU-vs-GPU checks (README "85 parity checks, <=1e-4"). The
-// same templates instantiated for bf16 storage serve the bf16 backward at head
-// dim 256 until the tensor-core backward covers it.
+// set for their CPU-vs-GPU checks (README "85 parity checks, <=1e-4").
 //
 // Structure: a block owns 16 rows (4 warps x 4 rows); keys (or queries) stream
 // through shared memory 32 at a time; lane j of a warp scores element j of the
