@@ -29,6 +29,12 @@ namespace forge {
 template <int D>
 struct FwdTc {
     static constexpr int BM = 128, BN = 128;
+    // O += P V with P split into two bf16 terms, P = hi + lo (hi = bf16(P),
+    // lo = bf16(P - hi)): O is then accurate to f32 before its final rounding
+    // instead of carrying the 2^-9 relative error of a single bf16 P. The
+    // backward's Delta = rowsum(dO * O) inherits that accuracy; at head dim 256 a
+    // single-term P moves Delta by up to ~0.2 on logits in the tanh regime.
+    static constexpr bool PSPLIT = (D == 256);
     static constexpr int NCB = D / 64;                 // 64-column (128-byte) blocks
     static constexpr uint32_t CB = 128 * 128;          // bytes of one column block of a 128-row tile
     static constexpr uint32_t TILE = NCB * CB;         // one 128 x D bf16 tile
@@ -192,6 +198,12 @@ __global__ void __launch_bounds__(192, 1)
                 for (int kk = 0; kk < C::BN / 16; kk++)
                     mma_ts(tmem + C::COL_O, aP + kk * 8, sdesc_sw128(sV + kk * 2048, C::CB, 1024), ID_PV,
                            (acc || kk > 0) ? 1u : 0u);
+                if constexpr (C::PSPLIT) {
+                    // low parts of P live in columns [64, 128) of the same S buffer
+#pragma unroll
+                    for (int kk = 0; kk < C::BN / 16; kk++)
+                        mma_ts(tmem + C::COL_O, aP + 64 + kk * 8, sdesc_sw128(sV + kk * 2048, C::CB, 1024), ID_PV, 1u);
+                }
                 tc_commit(bar(C::B_O_READY));
                 tc_commit(bar(C::B_KV_EMPTY + stage));
                 next();
@@ -296,9 +308,24 @@ __global__ void __launch_bounds__(192, 1)
                 const float p1 = ex2_approx(__uint_as_float(s[(2 * c + 1) >> 5][(2 * c + 1) & 31]) - msub);
                 rs += p0 + p1;
                 pk[c >> 5][c & 31] = pack_bf16x2(p0, p1);
+                if constexpr (C::PSPLIT) {
+                    // keep the residuals where the scores were (columns no longer needed)
+                    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(&pk[c >> 5][c & 31]);
+                    const float2 hf = __bfloat1622float2(hi);
+                    s[(2 * c) >> 5][(2 * c) & 31] = __float_as_uint(p0 - hf.x);
+                    s[(2 * c + 1) >> 5][(2 * c + 1) & 31] = __float_as_uint(p1 - hf.y);
+                }
             }
             tmem_st32(tS + 0, pk[0]);
             tmem_st32(tS + 32, pk[1]);
+            if constexpr (C::PSPLIT) {
+#pragma unroll
+                for (int c = 0; c < 64; c++)
+                    pk[c >> 5][c & 31] = pack_bf16x2(__uint_as_float(s[(2 * c) >> 5][(2 * c) & 31]),
+                                                     __uint_as_float(s[(2 * c + 1) >> 5][(2 * c + 1) & 31]));
+                tmem_st32(tS + 64, pk[0]);
+                tmem_st32(tS + 96, pk[1]);
+            }
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
