@@ -223,6 +223,15 @@ __global__ void selftest_timeout_kernel(unsigned long long limit_ns) {
     __syncthreads();
 }
 
+// exp2 self-test: the kernels' FMA-pipe exp2 next to CUDA's exp2f.
+__global__ void selftest_exp2_kernel(const float *x, float *y, float *y_ref, int n) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) {
+        y[i] = exp2_poly(x[i]);
+        y_ref[i] = exp2f(x[i]);
+    }
+}
+
 }  // namespace forge
 
 using namespace forge;
@@ -372,6 +381,13 @@ const char *forge_attn_status_string(forge_status s) {
 forge_status forge_attn_selftest_timeout(unsigned int limit_us, void *stream) {
     if (limit_us < 1 || limit_us > 2000000u) return FORGE_ERR_INVALID_ARG;
     selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(1000ull * limit_us);
+    return launch_status();
+}
+
+forge_status forge_attn_selftest_exp2(const float *x, float *y, float *y_ref, int n, void *stream) {
+    if (n < 0 || (n > 0 && (x == nullptr || y == nullptr || y_ref == nullptr))) return FORGE_ERR_INVALID_ARG;
+    if (n == 0) return FORGE_OK;
+    selftest_exp2_kernel<<<(n + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, y_ref, n);
     return launch_status();
 }
 

@@ -59,6 +59,51 @@ struct FwdTc {
     static_assert(SMEM <= 232448, "shared memory");
 };
 
+// Row max of a 128-column tile held as 4 x 32 registers (8 independent chains).
+__device__ __forceinline__ float fwd_row_max(const uint32_t (&s)[4][32]) {
+    float mx[8];
+#pragma unroll
+    for (int j = 0; j < 8; j++) mx[j] = __uint_as_float(s[0][j]);
+#pragma unroll
+    for (int c = 8; c < 128; c++) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(s[c >> 5][c & 31]));
+    return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+}
+
+// Exponentials, row sum and bf16 packing of one tile row.
+//   CAP:    s holds scores in log2 units; otherwise raw products, y = s*sl2 - m.
+//   EMU:    every fourth column pair goes through the FMA-pipe exp2 (only for
+//           tiles without masked scores), the rest through MUFU ex2.
+//   PSPLIT: also leaves the residuals p - bf16(p) in s for a second PV term.
+// Returns the row sum of p (f32, 4 chains).
+template <bool CAP, bool EMU, bool PSPLIT>
+__device__ __forceinline__ float fwd_exp_tile(uint32_t (&s)[4][32], uint32_t (&pk)[2][32], float sl2, float msub) {
+    float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int c = 0; c < 64; c++) {
+        const float x0 = __uint_as_float(s[(2 * c) >> 5][(2 * c) & 31]);
+        const float x1 = __uint_as_float(s[(2 * c + 1) >> 5][(2 * c + 1) & 31]);
+        const float y0 = CAP ? x0 - msub : fmaf(x0, sl2, -msub);
+        const float y1 = CAP ? x1 - msub : fmaf(x1, sl2, -msub);
+        float p0, p1;
+        if (EMU && (c & 3) == 3) {
+            p0 = exp2_poly(y0);
+            p1 = exp2_poly(y1);
+        } else {
+            p0 = ex2_approx(y0);
+            p1 = ex2_approx(y1);
+        }
+        rs[c & 3] += p0 + p1;
+        pk[c >> 5][c & 31] = pack_bf16x2(p0, p1);
+        if constexpr (PSPLIT) {
+            const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(&pk[c >> 5][c & 31]);
+            const float2 hf = __bfloat1622float2(hi);
+            s[(2 * c) >> 5][(2 * c) & 31] = __float_as_uint(p0 - hf.x);
+            s[(2 * c + 1) >> 5][(2 * c + 1) & 31] = __float_as_uint(p1 - hf.y);
+        }
+    }
+    return (rs[0] + rs[1]) + (rs[2] + rs[3]);
+}
+
 struct FwdParams {
     __nv_bfloat16 *o;
     float *lse;
@@ -252,17 +297,16 @@ __global__ void __launch_bounds__(192, 1)
             tmem_ld_wait(s[1]);
             tmem_ld_wait(s[2]);
             tmem_ld_wait(s[3]);
-            // scores in log2 units
-            if (p.softcap > 0.0f) {
+            // capped scores are turned into log2 units here; plain ones stay raw
+            // (the scale is folded into the exponent's FMA, and max commutes
+            // with a positive scale)
+            const bool cap = p.softcap > 0.0f;
+            if (cap) {
 #pragma unroll
                 for (int c = 0; c < 128; c++) {
                     const float x = __uint_as_float(s[c >> 5][c & 31]);
                     s[c >> 5][c & 31] = __float_as_uint(p.cap_out * tanh_via_ex2(x * p.cap_in));
                 }
-            } else {
-#pragma unroll
-                for (int c = 0; c < 128; c++)
-                    s[c >> 5][c & 31] = __float_as_uint(__uint_as_float(s[c >> 5][c & 31]) * p.scale_log2);
             }
             const bool need_mask = (k0 + C::BN - 1 > q0) || (W > 0 && k0 <= q0 + C::BM - 1 - W);
             if (need_mask) {
@@ -273,9 +317,8 @@ __global__ void __launch_bounds__(192, 1)
                     if (!vis) s[c >> 5][c & 31] = __float_as_uint(-INFINITY);
                 }
             }
-            float mx = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 128; c++) mx = fmaxf(mx, __uint_as_float(s[c >> 5][c & 31]));
+            float mx = fwd_row_max(s);
+            if (!cap) mx *= p.scale_log2;
             const float m_new = (mx > m + 8.0f) ? mx : m;
             const bool moved = (m_new != m);
             const float factor = moved ? ex2_approx(m - m_new) : 1.0f;
@@ -300,21 +343,14 @@ __global__ void __launch_bounds__(192, 1)
             }
             m = m_new;
             const float msub = (m == -INFINITY) ? 0.0f : m;
-            float rs = 0.0f;
             uint32_t pk[2][32];
-#pragma unroll
-            for (int c = 0; c < 64; c++) {
-                const float p0 = ex2_approx(__uint_as_float(s[(2 * c) >> 5][(2 * c) & 31]) - msub);
-                const float p1 = ex2_approx(__uint_as_float(s[(2 * c + 1) >> 5][(2 * c + 1) & 31]) - msub);
-                rs += p0 + p1;
-                pk[c >> 5][c & 31] = pack_bf16x2(p0, p1);
-                if constexpr (C::PSPLIT) {
-                    // keep the residuals where the scores were (columns no longer needed)
-                    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(&pk[c >> 5][c & 31]);
-                    const float2 hf = __bfloat1622float2(hi);
-                    s[(2 * c) >> 5][(2 * c) & 31] = __float_as_uint(p0 - hf.x);
-                    s[(2 * c + 1) >> 5][(2 * c + 1) & 31] = __float_as_uint(p1 - hf.y);
-                }
+            float rs;
+            if (cap) {
+                rs = need_mask ? fwd_exp_tile<true, false, C::PSPLIT>(s, pk, p.scale_log2, msub)
+                               : fwd_exp_tile<true, true, C::PSPLIT>(s, pk, p.scale_log2, msub);
+            } else {
+                rs = need_mask ? fwd_exp_tile<false, false, C::PSPLIT>(s, pk, p.scale_log2, msub)
+                               : fwd_exp_tile<false, true, C::PSPLIT>(s, pk, p.scale_log2, msub);
             }
             tmem_st32(tS + 0, pk[0]);
             tmem_st32(tS + 32, pk[1]);

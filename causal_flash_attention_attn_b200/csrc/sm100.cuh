@@ -295,6 +295,25 @@ __device__ __forceinline__ float tanh_via_ex2(float y) {
     const float e = ex2_approx(y * 2.8853900817779268f);  // 2 * log2(e)
     return 1.0f - 2.0f * rcp_approx(1.0f + e);
 }
+// 2^y on the FMA pipe, to share the exponential work with the MUFU unit.
+// Cody-Waite argument reduction: y = n + f with n = round(y) (the 1.5*2^23
+// rounding constant), f in [-1/2, 1/2]; 2^f from a degree-4 polynomial that is
+// minimax in relative error on [-1/2, 1/2] (Remez exchange; coefficients and
+// their f32 error bound, 2.7e-6, from csrc/gen_exp2_poly.py); 2^n applied by
+// adding n to the exponent field. Valid for -125 <= y < 2^22; smaller y
+// returns ~2^-125 (not 0), so callers use it only where no score is masked.
+__device__ __forceinline__ float exp2_poly(float y) {
+    y = fmaxf(y, -125.0f);
+    const float t = y + 12582912.0f;
+    const float n = t - 12582912.0f;
+    const float f = y - n;
+    float p = fmaf(f, 9.570102207e-03f, 5.591785908e-02f);
+    p = fmaf(p, f, 2.402474433e-01f);
+    p = fmaf(p, f, 6.931217909e-01f);
+    p = fmaf(p, f, 9.999992847e-01f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);

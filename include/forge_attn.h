@@ -131,6 +131,14 @@ const char *forge_attn_status_string(forge_status s);
  */
 forge_status forge_attn_selftest_timeout(unsigned int limit_us, void *stream);
 
+/*
+ * Self-test of the FMA-pipe exponential the kernels use for part of their
+ * exp2 work (Cody-Waite reduction + degree-4 minimax polynomial): for each of
+ * the n device floats x[i], writes that exp2 to y[i] and CUDA's exp2f(x[i]) to
+ * y_ref[i]. Device pointers, asynchronous on `stream`. Used by the tests.
+ */
+forge_status forge_attn_selftest_exp2(const float *x, float *y, float *y_ref, int n, void *stream);
+
 /* Library version, e.g. "forge_attn 0.1.0 sm_100a". */
 const char *forge_attn_version(void);
 
