@@ -12,6 +12,7 @@
 
 #include "bwd_aux.cuh"
 #include "bwd_tc.cuh"
+#include "fwd2_tc.cuh"
 #include "fwd_tc.cuh"
 #include "simt.cuh"
 #include "sm100.cuh"
@@ -131,9 +132,18 @@ forge_status fwd_tc(const void *q, const void *k, const void *v, void *o, float 
     p.softcap = softcap;
     p.cap_in = softcap > 0.0f ? scale / softcap : 0.0f;
     p.cap_out = softcap * kLog2e;
-    if (set_smem(fwd_tc_kernel<D>, C::SMEM) != FORGE_OK) return FORGE_ERR_CUDA;
-    const unsigned grid = (unsigned)(p.num_qt * B * Hq);
-    fwd_tc_kernel<D><<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, p);
+    if constexpr (D == 256) {
+        // one query tile per CTA: S0, S1 and the 256-column O fill TMEM
+        if (set_smem(fwd_tc_kernel<D>, C::SMEM) != FORGE_OK) return FORGE_ERR_CUDA;
+        const unsigned grid = (unsigned)(p.num_qt * B * Hq);
+        fwd_tc_kernel<D><<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, p);
+    } else {
+        // two query tiles per CTA
+        using C2 = Fwd2Tc<D>;
+        if (set_smem(fwd2_tc_kernel<D>, C2::SMEM) != FORGE_OK) return FORGE_ERR_CUDA;
+        const unsigned grid = (unsigned)(((p.num_qt + 1) / 2) * B * Hq);
+        fwd2_tc_kernel<D><<<grid, C2::THREADS, C2::SMEM, st>>>(mq, mk, mv, p);
+    }
     return launch_status();
 }
 

@@ -1,0 +1,387 @@
+// fwd2_tc.cuh -- tensor-core forward with two query tiles per CTA (head dims 64
+// and 128; head dim 256 uses fwd_tc.cuh, whose single tile fills TMEM).
+//
+// One CTA per (pair of consecutive 128-row query tiles A, B of one head), so the
+// CTA streams each K/V tile once for 256 query rows and runs two softmax streams
+// side by side (8 softmax warps, two per SM sub-partition): while one tile's
+// scores are in softmax, the tensor cores work on the other tile. Tile A sees
+// KV tiles [loA, tA], tile B [loB, tB] (tB = tA + 1); both ranges are the
+// causal/window ranges of their rows, so out-of-window KV tiles are never loaded
+// ("out-of-window KV blocks are skipped, so cost scales with the window":
+// src/nn/attention.h commit log, Wave 2).
+//
+// Roles (320 threads): warps 0-3 softmax of tile A, warps 4-7 softmax of tile
+// B (one thread per query row / TMEM lane), warp 8 TMA producer, warp 9 MMA
+// issuer and TMEM owner. TMEM: S_A, S_B (128 columns each; P overwrites its S
+// as bf16), O_A, O_B (D columns each).
+// MMA order per KV tile j: PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1). Because
+// QK_x(j+1) is committed after PV_x(j), a softmax warp that sees S_x(j+1) also
+// knows O_x holds every PV up to j, so it may rescale O_x without a wait.
+// Online softmax (max, sum) per row: ARCHITECTURES.md "Vague 2" item 10.
+#pragma once
+
+#include "fwd_tc.cuh"
+#include "sm100.cuh"
+
+namespace forge {
+
+template <int D>
+struct Fwd2Tc {
+    static constexpr int BM = 128, BN = 128;
+    static constexpr int NCB = D / 64;
+    static constexpr uint32_t CB = 128 * 128;          // column block of a 128-row tile
+    static constexpr uint32_t TILE = NCB * CB;         // one 128 x D bf16 tile
+    static constexpr int NSTAGE = D == 128 ? 4 : 8;
+    static constexpr uint32_t CTRL = 1024;
+    static constexpr uint32_t SMEM = CTRL + TILE * (2 + NSTAGE) + 1024;
+    static constexpr int THREADS = 320;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t col_s(int x) { return (uint32_t)(x * 128); }
+    static constexpr uint32_t col_o(int x) { return (uint32_t)(256 + x * D); }
+    static constexpr int B_Q = 0;
+    static constexpr int B_KV_FULL = 1;
+    static constexpr int B_KV_EMPTY = 1 + NSTAGE;
+    static constexpr int B_S_FULL = 1 + 2 * NSTAGE;   // [2]
+    static constexpr int B_P_FULL = 3 + 2 * NSTAGE;   // [2]
+    static constexpr int B_O_FINAL = 5 + 2 * NSTAGE;  // [2]
+    static constexpr int NBAR = 7 + 2 * NSTAGE;
+    static constexpr uint32_t OFF_TMEM_SLOT = 512, OFF_ABORT = 516;
+    static constexpr int EMU_MASK = 7;                 // pairs with (c & 7) == 7 use the FMA-pipe exp2
+    static_assert(NBAR * 8 <= 512, "control block");
+    static_assert(SMEM <= 232448, "shared memory");
+    static_assert(256 + 2 * D <= 512, "tensor memory");
+};
+
+// Row max over 128 scores with three-input maxima (4 chains).
+__device__ __forceinline__ float row_max128(const uint32_t (&s)[4][32]) {
+    float mx[4];
+#pragma unroll
+    for (int j = 0; j < 4; j++) mx[j] = fmaxf(__uint_as_float(s[0][2 * j]), __uint_as_float(s[0][2 * j + 1]));
+#pragma unroll
+    for (int c = 8; c < 128; c += 8) {
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const int a = c + 2 * j;
+            mx[j] = fmax3(mx[j], __uint_as_float(s[a >> 5][a & 31]), __uint_as_float(s[(a + 1) >> 5][(a + 1) & 31]));
+        }
+    }
+    return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+}
+
+// Exponentials of 64 scores (columns [64*half, 64*half + 64)), their sum (added
+// to rs) and bf16 packing into pk (column pairs, low half = even column).
+//   CAP: s holds log2-unit scores (y = s - m); else raw products (y = s*sl2 - m).
+//   EMU: pairs with (c & EMU_MASK) == EMU_MASK use the FMA-pipe exp2.
+template <bool CAP, bool EMU, int EMU_MASK>
+__device__ __forceinline__ void exp_half64(const uint32_t (&s)[4][32], int half, uint64_t sl2x2, uint64_t negm2,
+                                           uint64_t (&rs)[2], uint32_t (&pk)[32]) {
+#pragma unroll
+    for (int c = 0; c < 32; c++) {
+        const int e = 64 * half + 2 * c;
+        const uint64_t x2 = f2_make(__uint_as_float(s[e >> 5][e & 31]), __uint_as_float(s[(e + 1) >> 5][(e + 1) & 31]));
+        const uint64_t y2 = CAP ? f2_add(x2, negm2) : f2_fma(x2, sl2x2, negm2);
+        float y0, y1;
+        f2_split(y2, y0, y1);
+        float p0, p1;
+        if (EMU && (c & EMU_MASK) == EMU_MASK) {
+            p0 = exp2_poly(y0);
+            p1 = exp2_poly(y1);
+        } else {
+            p0 = ex2_approx(y0);
+            p1 = ex2_approx(y1);
+        }
+        rs[c & 1] = f2_add(rs[c & 1], f2_make(p0, p1));
+        pk[c] = pack_bf16x2(p0, p1);
+    }
+}
+
+template <int D>
+__global__ void __maxnreg__(200)
+    fwd2_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+    using C = Fwd2Tc<D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t sbase = smem_u32(smem_raw);
+    const uint32_t tiles = (sbase + C::CTRL + 1023u) & ~1023u;
+    const uint32_t sQ = tiles;                  // Q_A then Q_B
+    const uint32_t sKV = tiles + 2 * C::TILE;   // NSTAGE K/V tiles
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem_raw + C::OFF_ABORT);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + C::OFF_TMEM_SLOT);
+    auto bar = [&](int i) -> uint32_t { return sbase + 8u * (uint32_t)i; };
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int nbh = p.B * p.Hq;
+    const int npairs = (p.num_qt + 1) / 2;
+    const int pr = npairs - 1 - (int)(blockIdx.x / nbh);
+    const int bh = blockIdx.x % nbh;
+    const int b = bh / p.Hq, hq = bh % p.Hq;
+    const int bkv = b * p.Hkv + hq / (p.Hq / p.Hkv);
+    const int W = p.window;
+    const int tA = 2 * pr, tB = 2 * pr + 1;
+    const bool hasB = tB < p.num_qt;
+    const int qA0 = tA * C::BM, qB0 = tB * C::BM;
+    const int loA = W > 0 ? max(0, qA0 - W + 1) / C::BN : 0;
+    const int loB = W > 0 ? max(0, qB0 - W + 1) / C::BN : 0;
+    const int lo = loA, hi = hasB ? tB : tA;
+    auto active = [&](int x, int j) -> bool { return x == 0 ? (j >= loA && j <= tA) : (hasB && j >= loB && j <= tB); };
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(C::B_Q), 1);
+        for (int s = 0; s < C::NSTAGE; s++) {
+            mbar_init(bar(C::B_KV_FULL + s), 1);
+            mbar_init(bar(C::B_KV_EMPTY + s), 1);
+        }
+        for (int x = 0; x < 2; x++) {
+            mbar_init(bar(C::B_S_FULL + x), 1);
+            mbar_init(bar(C::B_P_FULL + x), 4);
+            mbar_init(bar(C::B_O_FINAL + x), 1);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 8 && lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+    }
+    if (warp == 9) {
+        tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 8) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            const uint64_t keep = policy_evict_last();
+            mbar_arrive_expect_tx(bar(C::B_Q), hasB ? 2 * C::TILE : C::TILE);
+            for (int c = 0; c < C::NCB; c++) {
+                tma_load_3d(sQ + c * C::CB, &tmQ, bar(C::B_Q), c * 64, qA0, bh);
+                if (hasB) tma_load_3d(sQ + C::TILE + c * C::CB, &tmQ, bar(C::B_Q), c * 64, qB0, bh);
+            }
+            // ring slots in order K(lo), V(lo), K(lo+1), V(lo+1), ...
+            int issued = 0;
+            bool ok = true;
+            for (int j = lo; ok && j <= hi; j++) {
+                for (int kv = 0; kv < 2 && ok; kv++) {
+                    const int st = issued % C::NSTAGE;
+                    const uint32_t ph = (uint32_t)((issued / C::NSTAGE) & 1);
+                    if (!mbar_wait(bar(C::B_KV_EMPTY + st), ph ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(bar(C::B_KV_FULL + st), C::TILE);
+                    for (int c = 0; c < C::NCB; c++)
+                        tma_load_3d_hint(sKV + st * C::TILE + c * C::CB, kv ? &tmV : &tmK, bar(C::B_KV_FULL + st),
+                                         c * 64, j * C::BN, bkv, keep);
+                    issued++;
+                }
+            }
+            if (!ok) {
+                mbar_wait_drain(bar(C::B_Q), 0, 200000000ull);
+                for (int back = 1; back <= min(issued, C::NSTAGE); back++) {
+                    const int L = issued - back;
+                    mbar_wait_drain(bar(C::B_KV_FULL + L % C::NSTAGE), (uint32_t)((L / C::NSTAGE) & 1), 200000000ull);
+                }
+            }
+        }
+    } else if (warp == 9) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t ID_QK = idesc_bf16_f32(128, 128, false, false);
+            constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, false, true);
+            auto wait_full = [&](int slot) -> bool {
+                return mbar_wait(bar(C::B_KV_FULL + slot % C::NSTAGE), (uint32_t)((slot / C::NSTAGE) & 1), abort_flag);
+            };
+            auto release = [&](int slot) { tc_commit(bar(C::B_KV_EMPTY + slot % C::NSTAGE)); };
+            auto issue_qk = [&](int x, int slot) {
+                const uint32_t sK = sKV + (slot % C::NSTAGE) * C::TILE;
+                const uint32_t sQx = sQ + (uint32_t)x * C::TILE;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; kk++) {
+                    const uint32_t off = (kk >> 2) * C::CB + (kk & 3) * 32;
+                    mma_ss(tmem + C::col_s(x), sdesc_sw128(sQx + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), ID_QK,
+                           kk > 0);
+                }
+                tc_commit(bar(C::B_S_FULL + x));
+            };
+            auto issue_pv = [&](int x, int slot, bool acc) {
+                const uint32_t sV = sKV + (slot % C::NSTAGE) * C::TILE;
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; kk++)
+                    mma_ts(tmem + C::col_o(x), tmem + C::col_s(x) + kk * 8, sdesc_sw128(sV + kk * 2048, C::CB, 1024),
+                           ID_PV, (acc || kk > 0) ? 1u : 0u);
+            };
+            bool ok = mbar_wait(bar(C::B_Q), 0, abort_flag);
+            if (ok) ok = wait_full(0);
+            if (ok) {
+                tc_fence_after();
+                if (active(0, lo)) issue_qk(0, 0);
+                if (active(1, lo)) issue_qk(1, 0);
+                release(0);
+            }
+            int cnt[2] = {0, 0};
+            for (int j = lo; ok && j <= hi; j++) {
+                const int slotV = 2 * (j - lo) + 1, slotK = slotV + 1;
+                if (!(ok = wait_full(slotV))) break;
+                bool k_ready = false;
+                for (int x = 0; x < 2 && ok; x++) {
+                    if (active(x, j)) {
+                        if (!(ok = mbar_wait(bar(C::B_P_FULL + x), (uint32_t)(cnt[x] & 1), abort_flag))) break;
+                        tc_fence_after();
+                        issue_pv(x, slotV, cnt[x] > 0);
+                        cnt[x]++;
+                    }
+                    if (j < hi && active(x, j + 1)) {
+                        if (!k_ready) {
+                            if (!(ok = wait_full(slotK))) break;
+                            tc_fence_after();
+                            k_ready = true;
+                        }
+                        issue_qk(x, slotK);
+                    }
+                }
+                if (!ok) break;
+                release(slotV);
+                if (j < hi) release(slotK);
+            }
+            // O_FINAL fires once every MMA issued so far has completed
+            tc_commit(bar(C::B_O_FINAL + 0));
+            tc_commit(bar(C::B_O_FINAL + 1));
+            if (!ok) mbar_wait_drain(bar(C::B_O_FINAL + 0), 0, 200000000ull);
+        }
+    } else {
+        // ---------------------------------------- softmax: warps 0-3 tile A, 4-7 tile B
+        const int x = warp / 4;
+        const int row = threadIdx.x % 128;
+        const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
+        const uint32_t tS = tmem + lane_base + C::col_s(x);
+        const uint32_t tO = tmem + lane_base + C::col_o(x);
+        const int q0 = x ? qB0 : qA0;
+        const int lox = x ? loB : loA, hix = x ? tB : tA;
+        const int qi = q0 + row;
+        const bool cap = p.softcap > 0.0f;
+        const uint64_t sl2x2 = f2_make(p.scale_log2, p.scale_log2);
+        float m = -INFINITY, l = 0.0f;
+        bool ok = (x == 0) || hasB;
+        if (ok) {
+            int cnt = 0;
+            for (int j = lox; j <= hix; j++, cnt++) {
+                const int k0 = j * C::BN;
+                if (!(ok = mbar_wait_warp(bar(C::B_S_FULL + x), (uint32_t)(cnt & 1), abort_flag))) break;
+                tc_fence_after();
+                uint32_t s[4][32];
+                tmem_ld32(tS + 0, s[0]);
+                tmem_ld32(tS + 32, s[1]);
+                tmem_ld32(tS + 64, s[2]);
+                tmem_ld32(tS + 96, s[3]);
+                tmem_ld_wait(s[0]);
+                tmem_ld_wait(s[1]);
+                tmem_ld_wait(s[2]);
+                tmem_ld_wait(s[3]);
+                if (cap) {
+#pragma unroll
+                    for (int c = 0; c < 128; c++) {
+                        const float v = __uint_as_float(s[c >> 5][c & 31]);
+                        s[c >> 5][c & 31] = __float_as_uint(p.cap_out * tanh_via_ex2(v * p.cap_in));
+                    }
+                }
+                const bool need_mask = (k0 + C::BN - 1 > q0) || (W > 0 && k0 <= q0 + C::BM - 1 - W);
+                if (need_mask) {
+#pragma unroll
+                    for (int c = 0; c < 128; c++) {
+                        const int kj = k0 + c;
+                        const bool vis = kj <= qi && (W == 0 || kj > qi - W);
+                        if (!vis) s[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+                    }
+                }
+                float mx = row_max128(s);
+                if (!cap) mx *= p.scale_log2;
+                const float m_new = (mx > m + 8.0f) ? mx : m;
+                const bool moved = (m_new != m);
+                const float factor = moved ? ex2_approx(m - m_new) : 1.0f;
+                if (__any_sync(0xffffffffu, moved && cnt > 0)) {
+                    // O_x already holds every PV of this tile's earlier KV tiles
+                    const float f = (moved && cnt > 0) ? factor : 1.0f;
+                    const uint64_t f2 = f2_make(f, f);
+#pragma unroll 1
+                    for (int c0 = 0; c0 < D; c0 += 32) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + c0, o);
+                        tmem_ld_wait(o);
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2) {
+                            float a, bb;
+                            f2_split(f2_mul(f2_make(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), f2), a, bb);
+                            o[i] = __float_as_uint(a);
+                            o[i + 1] = __float_as_uint(bb);
+                        }
+                        tmem_st32(tO + c0, o);
+                    }
+                }
+                m = m_new;
+                const float msub = (m == -INFINITY) ? 0.0f : m;
+                const uint64_t negm2 = f2_make(-msub, -msub);
+                uint64_t rs[2] = {f2_make(0.0f, 0.0f), f2_make(0.0f, 0.0f)};
+#pragma unroll
+                for (int half = 0; half < 2; half++) {
+                    uint32_t pk[32];
+                    if (cap) {
+                        if (need_mask) exp_half64<true, false, C::EMU_MASK>(s, half, sl2x2, negm2, rs, pk);
+                        else exp_half64<true, true, C::EMU_MASK>(s, half, sl2x2, negm2, rs, pk);
+                    } else {
+                        if (need_mask) exp_half64<false, false, C::EMU_MASK>(s, half, sl2x2, negm2, rs, pk);
+                        else exp_half64<false, true, C::EMU_MASK>(s, half, sl2x2, negm2, rs, pk);
+                    }
+                    tmem_st32(tS + 32 * half, pk);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::B_P_FULL + x));
+                float r0, r1, r2, r3;
+                f2_split(rs[0], r0, r1);
+                f2_split(rs[1], r2, r3);
+                l = l * factor + ((r0 + r1) + (r2 + r3));
+            }
+        }
+        if (ok) ok = mbar_wait_warp(bar(C::B_O_FINAL + x), 0, abort_flag);
+        if (ok && ((x == 0) || hasB)) {
+            tc_fence_after();
+            const float inv_l = 1.0f / l;
+            const uint64_t inv2 = f2_make(inv_l, inv_l);
+            __nv_bfloat16 *orow = p.o + ((size_t)bh * p.T + (size_t)min(qi, p.T - 1)) * D;
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t o[32];
+                tmem_ld32(tO + c0, o);
+                tmem_ld_wait(o);
+                uint32_t w[16];
+#pragma unroll
+                for (int i = 0; i < 16; i++) {
+                    float a, bb;
+                    f2_split(f2_mul(f2_make(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), inv2), a, bb);
+                    w[i] = pack_bf16x2(a, bb);
+                }
+                if (qi < p.T) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
+#pragma unroll
+                    for (int i = 0; i < 4; i++) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                }
+            }
+            if (qi < p.T) p.lse[(size_t)bh * p.T + qi] = (m + __log2f(l)) * kLn2;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+}  // namespace forge

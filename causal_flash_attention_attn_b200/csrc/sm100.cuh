@@ -295,6 +295,37 @@ __device__ __forceinline__ float tanh_via_ex2(float y) {
     const float e = ex2_approx(y * 2.8853900817779268f);  // 2 * log2(e)
     return 1.0f - 2.0f * rcp_approx(1.0f + e);
 }
+// ------------------------------------------------ packed f32x2 (sm_100) helpers
+__device__ __forceinline__ uint64_t f2_make(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float &a, float &b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// three-input maximum
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // 2^y on the FMA pipe, to share the exponential work with the MUFU unit.
 // Cody-Waite argument reduction: y = n + f with n = round(y) (the 1.5*2^23
 // rounding constant), f in [-1/2, 1/2]; 2^f from a degree-4 polynomial that is
