@@ -20,7 +20,7 @@ __all__ = [
     "FORGE_ERR_CUDA", "FORGE_ERR_TIMEOUT", "FORGE_DTYPE_F32", "FORGE_DTYPE_BF16", "ForgeError",
     "library", "library_path", "forge_attn_fwd", "forge_attn_bwd", "forge_attn_bwd_workspace_size",
     "forge_attn_bwd_preprocess", "forge_attn_bwd_main", "forge_attn_bwd_finalize", "forge_attn_check",
-    "forge_attn_status_string", "forge_attn_selftest_timeout", "forge_attn_selftest_exp2", "forge_attn_version",
+    "forge_attn_status_string", "forge_attn_selftest_timeout", "forge_attn_selftest_exp2", "forge_attn_last_cuda_error", "forge_attn_version",
     "attention_fwd", "attention_bwd", "dtype_code",
 ]
 
@@ -41,7 +41,10 @@ _lib = None
 class ForgeError(RuntimeError):
     def __init__(self, status: int, what: str = ""):
         self.status = status
-        super().__init__(f"{what}: {forge_attn_status_string(status)}" if what else forge_attn_status_string(status))
+        msg = forge_attn_status_string(status)
+        if status == FORGE_ERR_CUDA:
+            msg += f" ({forge_attn_last_cuda_error()})"
+        super().__init__(f"{what}: {msg}" if what else msg)
 
 
 def library():
@@ -73,6 +76,8 @@ def library():
     L.forge_attn_selftest_timeout.restype = i
     L.forge_attn_selftest_exp2.argtypes = [vp, vp, vp, i, vp]
     L.forge_attn_selftest_exp2.restype = i
+    L.forge_attn_last_cuda_error.argtypes = []
+    L.forge_attn_last_cuda_error.restype = ctypes.c_char_p
     L.forge_attn_version.argtypes = []
     L.forge_attn_version.restype = ctypes.c_char_p
     _lib = L
@@ -154,6 +159,10 @@ def forge_attn_selftest_timeout(limit_us: int, stream=None) -> int:
 
 def forge_attn_selftest_exp2(x, y, y_ref, n, stream=None) -> int:
     return library().forge_attn_selftest_exp2(_ptr(x), _ptr(y), _ptr(y_ref), int(n), _stream(stream))
+
+
+def forge_attn_last_cuda_error() -> str:
+    return library().forge_attn_last_cuda_error().decode()
 
 
 def forge_attn_version() -> str:

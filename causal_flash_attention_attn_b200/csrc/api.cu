@@ -101,17 +101,21 @@ bool make_map_acc(CUtensorMap *map, const float *base, int D, int Tpad, long lon
     return r == CUDA_SUCCESS;
 }
 
-forge_status launch_status() {
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? FORGE_OK : FORGE_ERR_CUDA;
+// Text of the last CUDA error a call of this thread ran into (for diagnostics).
+thread_local const char *t_last_cuda_error = "no error";
+
+forge_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return FORGE_OK;
+    t_last_cuda_error = cudaGetErrorString(e);
+    return FORGE_ERR_CUDA;
 }
+
+forge_status launch_status() { return cuda_status(cudaGetLastError()); }
 
 template <typename K>
 forge_status set_smem(K kernel, size_t bytes) {
     if (bytes <= 48 * 1024) return FORGE_OK;
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess
-               ? FORGE_OK
-               : FORGE_ERR_CUDA;
+    return cuda_status(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes));
 }
 
 // ----------------------------------------------------------------- dispatchers
@@ -122,7 +126,10 @@ forge_status fwd_tc(const void *q, const void *k, const void *v, void *o, float 
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, q, D, T, (long long)B * Hq, 128) || !make_map(&mk, k, D, T, (long long)B * Hkv, 128) ||
         !make_map(&mv, v, D, T, (long long)B * Hkv, 128))
+    {
+        t_last_cuda_error = "cuTensorMapEncodeTiled failed";
         return FORGE_ERR_CUDA;
+    }
     FwdParams p;
     p.o = static_cast<__nv_bfloat16 *>(o);
     p.lse = lse;
@@ -188,8 +195,10 @@ forge_status bwd_tc(const void *q, const void *k, const void *v, const float *ls
     CUtensorMap mq, mk, mv, mdo, macc;
     if (!make_map(&mq, q, D, T, (long long)B * Hq, C::BM) || !make_map(&mk, k, D, T, (long long)B * Hkv, 128) ||
         !make_map(&mv, v, D, T, (long long)B * Hkv, 128) || !make_map(&mdo, dO, D, T, (long long)B * Hq, C::BM) ||
-        !make_map_acc(&macc, acc, D, tpad_of(T), (long long)B * Hq, C::BM))
+        !make_map_acc(&macc, acc, D, tpad_of(T), (long long)B * Hq, C::BM)) {
+        t_last_cuda_error = "cuTensorMapEncodeTiled failed";
         return FORGE_ERR_CUDA;
+    }
     BwdParams p;
     p.lse = lse;
     p.delta = delta;
@@ -365,12 +374,13 @@ forge_status forge_attn_bwd(const void *q, const void *k, const void *v, const v
 
 forge_status forge_attn_check(void *stream) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (cudaStreamSynchronize(st) != cudaSuccess) return FORGE_ERR_CUDA;
+    forge_status s = cuda_status(cudaStreamSynchronize(st));
+    if (s != FORGE_OK) return s;
     int h = 0;
-    if (cudaMemcpyFromSymbol(&h, g_status, sizeof(int)) != cudaSuccess) return FORGE_ERR_CUDA;
+    if ((s = cuda_status(cudaMemcpyFromSymbol(&h, g_status, sizeof(int)))) != FORGE_OK) return s;
     if (h != 0) {
         const int zero = 0;
-        if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return FORGE_ERR_CUDA;
+        if ((s = cuda_status(cudaMemcpyToSymbol(g_status, &zero, sizeof(int)))) != FORGE_OK) return s;
         return static_cast<forge_status>(h);
     }
     return FORGE_OK;
@@ -400,6 +410,8 @@ forge_status forge_attn_selftest_exp2(const float *x, float *y, float *y_ref, in
     selftest_exp2_kernel<<<(n + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, y_ref, n);
     return launch_status();
 }
+
+const char *forge_attn_last_cuda_error(void) { return t_last_cuda_error; }
 
 const char *forge_attn_version(void) { return "forge_attn 0.1.0 sm_100a"; }
 

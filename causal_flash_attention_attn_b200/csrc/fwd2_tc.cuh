@@ -96,7 +96,7 @@ __device__ __forceinline__ void exp_half64(const uint32_t (&s)[4][32], int half,
 }
 
 template <int D>
-__global__ void __maxnreg__(200)
+__global__ void __maxnreg__(192)
     fwd2_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
     using C = Fwd2Tc<D>;

@@ -119,6 +119,13 @@ forge_status forge_attn_bwd_finalize(void *dq, int B, int Hq, int Hkv, int T, in
  */
 forge_status forge_attn_check(void *stream);
 
+/*
+ * Text of the last CUDA runtime error that a call made on this host thread ran
+ * into (the detail behind a FORGE_ERR_CUDA return); "no error" if none.
+ * Static storage, never NULL.
+ */
+const char *forge_attn_last_cuda_error(void);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *forge_attn_status_string(forge_status s);
 
