@@ -68,17 +68,16 @@ __device__ __forceinline__ float row_max128(const uint32_t (&s)[4][32]) {
     return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
 }
 
-// Exponentials of 64 scores (columns [64*half, 64*half + 64)), their sum (added
-// to rs) and bf16 packing into pk (column pairs, low half = even column).
+// Exponentials of 32 scores (columns [32*q, 32*q + 32)), their sum (added to rs)
+// and bf16 packing into pk (column pairs, low half = even column).
 //   CAP: s holds log2-unit scores (y = s - m); else raw products (y = s*sl2 - m).
 //   EMU: pairs with (c & EMU_MASK) == EMU_MASK use the FMA-pipe exp2.
 template <bool CAP, bool EMU, int EMU_MASK>
-__device__ __forceinline__ void exp_half64(const uint32_t (&s)[4][32], int half, uint64_t sl2x2, uint64_t negm2,
-                                           uint64_t (&rs)[2], uint32_t (&pk)[32]) {
+__device__ __forceinline__ void exp_chunk32(const uint32_t (&s)[32], uint64_t sl2x2, uint64_t negm2, uint64_t (&rs)[2],
+                                            uint32_t (&pk)[16]) {
 #pragma unroll
-    for (int c = 0; c < 32; c++) {
-        const int e = 64 * half + 2 * c;
-        const uint64_t x2 = f2_make(__uint_as_float(s[e >> 5][e & 31]), __uint_as_float(s[(e + 1) >> 5][(e + 1) & 31]));
+    for (int c = 0; c < 16; c++) {
+        const uint64_t x2 = f2_make(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1]));
         const uint64_t y2 = CAP ? f2_add(x2, negm2) : f2_fma(x2, sl2x2, negm2);
         float y0, y1;
         f2_split(y2, y0, y1);
@@ -96,7 +95,7 @@ __device__ __forceinline__ void exp_half64(const uint32_t (&s)[4][32], int half,
 }
 
 template <int D>
-__global__ void __maxnreg__(192)
+__global__ void __launch_bounds__(320, 1)
     fwd2_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
     using C = Fwd2Tc<D>;
@@ -327,16 +326,17 @@ __global__ void __maxnreg__(192)
                 const uint64_t negm2 = f2_make(-msub, -msub);
                 uint64_t rs[2] = {f2_make(0.0f, 0.0f), f2_make(0.0f, 0.0f)};
 #pragma unroll
-                for (int half = 0; half < 2; half++) {
-                    uint32_t pk[32];
+                for (int q4 = 0; q4 < 4; q4++) {
+                    // 32 scores -> 16 packed P columns; P column c holds scores 2c, 2c+1
+                    uint32_t pk[16];
                     if (cap) {
-                        if (need_mask) exp_half64<true, false, C::EMU_MASK>(s, half, sl2x2, negm2, rs, pk);
-                        else exp_half64<true, true, C::EMU_MASK>(s, half, sl2x2, negm2, rs, pk);
+                        if (need_mask) exp_chunk32<true, false, C::EMU_MASK>(s[q4], sl2x2, negm2, rs, pk);
+                        else exp_chunk32<true, true, C::EMU_MASK>(s[q4], sl2x2, negm2, rs, pk);
                     } else {
-                        if (need_mask) exp_half64<false, false, C::EMU_MASK>(s, half, sl2x2, negm2, rs, pk);
-                        else exp_half64<false, true, C::EMU_MASK>(s, half, sl2x2, negm2, rs, pk);
+                        if (need_mask) exp_chunk32<false, false, C::EMU_MASK>(s[q4], sl2x2, negm2, rs, pk);
+                        else exp_chunk32<false, true, C::EMU_MASK>(s[q4], sl2x2, negm2, rs, pk);
                     }
-                    tmem_st32(tS + 32 * half, pk);
+                    tmem_st16(tS + 16 * q4, pk);
                 }
                 tmem_st_wait();
                 tc_fence_before();
