@@ -20,7 +20,7 @@ __all__ = [
     "FORGE_ERR_CUDA", "FORGE_ERR_TIMEOUT", "FORGE_DTYPE_F32", "FORGE_DTYPE_BF16", "ForgeError",
     "library", "library_path", "forge_attn_fwd", "forge_attn_bwd", "forge_attn_bwd_workspace_size",
     "forge_attn_bwd_preprocess", "forge_attn_bwd_main", "forge_attn_bwd_finalize", "forge_attn_check",
-    "forge_attn_status_string", "forge_attn_selftest_timeout", "forge_attn_selftest_exp2", "forge_attn_last_cuda_error", "forge_attn_version",
+    "forge_attn_status_string", "forge_attn_selftest_timeout", "forge_attn_selftest_exp2", "forge_attn_last_cuda_error", "forge_attn_timeout_info", "forge_attn_version",
     "attention_fwd", "attention_bwd", "dtype_code",
 ]
 
@@ -44,6 +44,11 @@ class ForgeError(RuntimeError):
         msg = forge_attn_status_string(status)
         if status == FORGE_ERR_CUDA:
             msg += f" ({forge_attn_last_cuda_error()})"
+        if status == FORGE_ERR_TIMEOUT:
+            try:
+                msg += f" (wait info {forge_attn_timeout_info()[1]})"
+            except Exception:
+                pass
         super().__init__(f"{what}: {msg}" if what else msg)
 
 
@@ -76,6 +81,8 @@ def library():
     L.forge_attn_selftest_timeout.restype = i
     L.forge_attn_selftest_exp2.argtypes = [vp, vp, vp, i, vp]
     L.forge_attn_selftest_exp2.restype = i
+    L.forge_attn_timeout_info.argtypes = [vp]
+    L.forge_attn_timeout_info.restype = i
     L.forge_attn_last_cuda_error.argtypes = []
     L.forge_attn_last_cuda_error.restype = ctypes.c_char_p
     L.forge_attn_version.argtypes = []
@@ -159,6 +166,13 @@ def forge_attn_selftest_timeout(limit_us: int, stream=None) -> int:
 
 def forge_attn_selftest_exp2(x, y, y_ref, n, stream=None) -> int:
     return library().forge_attn_selftest_exp2(_ptr(x), _ptr(y), _ptr(y_ref), int(n), _stream(stream))
+
+
+def forge_attn_timeout_info():
+    """(status, [barrier+1, block, thread, (threads << 20) | blocks]) of the first wait that ran out."""
+    arr = (ctypes.c_uint * 4)()
+    s = library().forge_attn_timeout_info(arr)
+    return s, list(arr)
 
 
 def forge_attn_last_cuda_error() -> str:

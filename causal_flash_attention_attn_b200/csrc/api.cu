@@ -413,6 +413,14 @@ forge_status forge_attn_selftest_exp2(const float *x, float *y, float *y_ref, in
 
 const char *forge_attn_last_cuda_error(void) { return t_last_cuda_error; }
 
+forge_status forge_attn_timeout_info(unsigned int *info4) {
+    if (info4 == nullptr) return FORGE_ERR_INVALID_ARG;
+    forge_status s = cuda_status(cudaMemcpyFromSymbol(info4, g_timeout_info, 4 * sizeof(unsigned)));
+    if (s != FORGE_OK) return s;
+    const unsigned zero[4] = {0, 0, 0, 0};
+    return cuda_status(cudaMemcpyToSymbol(g_timeout_info, zero, sizeof(zero)));
+}
+
 const char *forge_attn_version(void) { return "forge_attn 0.1.0 sm_100a"; }
 
 }  // extern "C"

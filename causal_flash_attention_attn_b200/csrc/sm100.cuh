@@ -18,6 +18,11 @@ __device__ int g_status;
 
 enum : int { kStatusTimeout = 5 };
 
+// Where the first timed-out wait happened: [0] = 1 + barrier shared-memory
+// address, [1] = block index, [2] = thread index, [3] = (block size << 20) |
+// grid size, which tells the kernels apart. All zero if no wait ran out.
+__device__ unsigned g_timeout_info[4];
+
 // Wait limit for every barrier wait: 2 s of %globaltimer. No correct wait in
 // these kernels comes within orders of magnitude of it.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
@@ -73,6 +78,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
         if (*abort_flag) return false;
         if (globaltimer_ns() - t0 > limit_ns) {
             record_status(kStatusTimeout);
+            if (atomicCAS(&g_timeout_info[0], 0u, 1u + (bar & 0xFFFFFu)) == 0u) {
+                g_timeout_info[1] = blockIdx.x;
+                g_timeout_info[2] = threadIdx.x;
+                g_timeout_info[3] = (blockDim.x << 20) | (gridDim.x & 0xFFFFFu);
+            }
             *abort_flag = 1;
             return false;
         }

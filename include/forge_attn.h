@@ -126,6 +126,14 @@ forge_status forge_attn_check(void *stream);
  */
 const char *forge_attn_last_cuda_error(void);
 
+/*
+ * Where the first bounded wait that ran out (FORGE_ERR_TIMEOUT) gave up, for
+ * diagnosis, then cleared: info4[0] = 1 + the barrier's shared-memory address
+ * (0 if no wait ran out), [1] = block index, [2] = thread index, [3] = (threads
+ * per block << 20) | blocks in the grid. Host array of 4; synchronous.
+ */
+forge_status forge_attn_timeout_info(unsigned int *info4);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *forge_attn_status_string(forge_status s);
 
