@@ -196,27 +196,23 @@ __global__ void __launch_bounds__(320, 1)
                 return mbar_wait(bar(C::B_KV_FULL + slot % C::NSTAGE), (uint32_t)((slot / C::NSTAGE) & 1), abort_flag);
             };
             auto release = [&](int slot) { tc_commit(bar(C::B_KV_EMPTY + slot % C::NSTAGE)); };
-            // descriptor words: K-major operands use LBO 16 / SBO 1024, the MN-major
-            // V uses LBO = one column block; walking K only adds to the low word
-            const uint32_t hi = sdesc_hi(1024);
-            const uint32_t lbo16 = sdesc_lbo_bits(16), lbo_cb = sdesc_lbo_bits(C::CB);
             auto issue_qk = [&](int x, int slot) {
-                const uint32_t qlo = sdesc_lo(sQ + (uint32_t)x * C::TILE) | lbo16;
-                const uint32_t klo = sdesc_lo(sKV + (slot % C::NSTAGE) * C::TILE) | lbo16;
-                const uint32_t d = tmem + C::col_s(x);
+                const uint32_t sK = sKV + (slot % C::NSTAGE) * C::TILE;
+                const uint32_t sQx = sQ + (uint32_t)x * C::TILE;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; kk++) {
-                    const uint32_t o = ((kk >> 2) * C::CB + (kk & 3) * 32) >> 4;
-                    mma_ss_lh(d, qlo + o, hi, klo + o, hi, ID_QK, kk > 0);
+                    const uint32_t off = (kk >> 2) * C::CB + (kk & 3) * 32;
+                    mma_ss(tmem + C::col_s(x), sdesc_sw128(sQx + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), ID_QK,
+                           kk > 0);
                 }
                 tc_commit(bar(C::B_S_FULL + x));
             };
             auto issue_pv = [&](int x, int slot, bool acc) {
-                const uint32_t vlo = sdesc_lo(sKV + (slot % C::NSTAGE) * C::TILE) | lbo_cb;
-                const uint32_t d = tmem + C::col_o(x), a = tmem + C::col_s(x);
+                const uint32_t sV = sKV + (slot % C::NSTAGE) * C::TILE;
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; kk++)
-                    mma_ts_lh(d, a + kk * 8, vlo + (uint32_t)kk * 128u, hi, ID_PV, (acc || kk > 0) ? 1u : 0u);
+                    mma_ts(tmem + C::col_o(x), tmem + C::col_s(x) + kk * 8, sdesc_sw128(sV + kk * 2048, C::CB, 1024),
+                           ID_PV, (acc || kk > 0) ? 1u : 0u);
             };
             bool ok = mbar_wait(bar(C::B_Q), 0, abort_flag);
             if (ok) ok = wait_full(0);
