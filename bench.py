@@ -325,7 +325,7 @@ def run_ours(args, w):
     dom = "bwd_main" if avg["bwd_main"] >= avg["fwd"] else "fwd"
     dom_flops = fl_b if dom == "bwd_main" else fl_f
     achieved = dom_flops / (avg[dom] * 1e-3) / 1e12
-    kname = {"fwd": "fwd_tc_kernel", "bwd_main": "bwd_tc_kernel"}[dom]
+    kname = {"fwd": "fwd_tc_kernel" if w.D == 256 else "fwd2_tc_kernel", "bwd_main": "bwd_tc_kernel"}[dom]
     traffic = ncu_traffic(kname, w.name)
     line = {
         "metric": METRIC,
