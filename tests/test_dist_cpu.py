@@ -1,0 +1,61 @@
+"""The N > 1 host path of bench.py on CPU: two gloo ranks, the max-over-ranks timing
+reduction, the barrier, the rank environment and the weak-scaling aggregate."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    from datetime import timedelta
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    import bench
+    w, r, l = bench.dist_env()
+    t = bench.max_over_ranks(10.0 + 5.0 * rank, w)
+    bench.barrier(w)
+    out.put((r, w, l, t))
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_reduce_max_and_agree():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [x[0] for x in res] == [0, 1]
+    assert all(x[1] == 2 for x in res)
+    assert [x[2] for x in res] == [0, 1]
+    assert all(x[3] == 15.0 for x in res)  # every rank sees the slowest rank's time
+
+
+def test_single_process_paths_and_aggregate():
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(3.5, 1) == 3.5
+    bench.barrier(1)
+    # N ranks, each its own batch: N x the work over the slowest rank's time
+    one = bench.aggregate_tflops(1, 8.42e11, 1.4)
+    assert abs(bench.aggregate_tflops(4, 8.42e11, 1.4) - 4 * one) < 1e-9
+    assert abs(one - 8.42e11 / 1.4e-3 / 1e12) < 1e-9
