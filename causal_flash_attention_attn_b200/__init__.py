@@ -19,6 +19,7 @@ __all__ = [
     "FORGE_OK", "FORGE_ERR_INVALID_ARG", "FORGE_ERR_UNSUPPORTED", "FORGE_ERR_WORKSPACE",
     "FORGE_ERR_CUDA", "FORGE_ERR_TIMEOUT", "FORGE_DTYPE_F32", "FORGE_DTYPE_BF16", "ForgeError",
     "library", "library_path", "forge_attn_fwd", "forge_attn_bwd", "forge_attn_bwd_workspace_size",
+    "forge_attn_bwd_noalloc",
     "forge_attn_bwd_preprocess", "forge_attn_bwd_main", "forge_attn_bwd_finalize", "forge_attn_check",
     "forge_attn_status_string", "forge_attn_selftest_timeout", "forge_attn_selftest_exp2", "forge_attn_last_cuda_error", "forge_attn_timeout_info", "forge_attn_version",
     "attention_fwd", "attention_bwd", "dtype_code",
@@ -67,6 +68,8 @@ def library():
     L.forge_attn_bwd_workspace_size.restype = st
     L.forge_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, f, i, vp, st, vp]
     L.forge_attn_bwd.restype = i
+    L.forge_attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, f, i, vp]
+    L.forge_attn_bwd_noalloc.restype = i
     L.forge_attn_bwd_preprocess.argtypes = [vp, vp, i, i, i, i, i, i, vp, st, vp]
     L.forge_attn_bwd_preprocess.restype = i
     L.forge_attn_bwd_main.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, f, i, vp, st, vp]
@@ -133,6 +136,14 @@ def forge_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale, win
                                     _ptr(dk), _ptr(dv), B, Hq, Hkv, T, D, float(scale), int(window),
                                     float(softcap), int(dtype), _ptr(workspace), int(workspace_bytes),
                                     _stream(stream))
+
+
+def forge_attn_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale, window, softcap, dtype,
+                           stream=None) -> int:
+    """forge_attn_bwd with the library's fixed 32 MiB internal scratch instead of a workspace."""
+    return library().forge_attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
+                                            _ptr(dk), _ptr(dv), B, Hq, Hkv, T, D, float(scale), int(window),
+                                            float(softcap), int(dtype), _stream(stream))
 
 
 def forge_attn_bwd_preprocess(o, dO, B, Hq, Hkv, T, D, dtype, workspace, workspace_bytes, stream=None) -> int:

@@ -8,6 +8,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "forge_attn.h"
 
 #include "bwd_aux.cuh"
@@ -253,6 +255,41 @@ __global__ void selftest_exp2_kernel(const float *x, float *y, float *y_ref, int
 
 }  // namespace forge
 
+// ---------------------------------------------------------------------------
+// Backward without caller-provided workspace.
+//
+// Some callers cannot allocate device memory at all: a host program that only
+// receives device buffers from another runtime and has no allocator of its own
+// (plain C or a foreign-language binding), or a process whose memory pool owns
+// the whole device and forbids allocations outside it. forge_attn_bwd_noalloc
+// serves them with scratch that lives in this fixed-size device array instead
+// of a caller workspace. Every GPU that loads the library holds the array until
+// the process exits. Its device address is looked up once per device (on the
+// first call made with that device current) and cached.
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+forge_status noalloc_scratch_for_current_device(void **out) {
+    int dev = -1;
+    forge_status s = forge::cuda_status(cudaGetDevice(&dev));
+    if (s != FORGE_OK) return s;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return FORGE_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        s = forge::cuda_status(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+        if (s != FORGE_OK) return s;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return FORGE_OK;
+}
+}  // namespace
+
 using namespace forge;
 
 extern "C" {
@@ -370,6 +407,23 @@ forge_status forge_attn_bwd(const void *q, const void *k, const void *v, const v
                             workspace_bytes, stream);
     if (s != FORGE_OK) return s;
     return forge_attn_bwd_finalize(dq, B, Hq, Hkv, T, D, dtype, workspace, workspace_bytes, stream);
+}
+
+forge_status forge_attn_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                                    const void *dO, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int T, int D,
+                                    float scale, int window, float softcap, forge_dtype dtype, void *stream) {
+    forge_status s = check_sizes(B, Hq, Hkv, T, D, dtype);
+    if (s != FORGE_OK) return s;
+    if (forge_attn_bwd_workspace_size(B, Hq, Hkv, T, D, dtype) > kNoAllocScratchBytes) {
+        t_last_cuda_error = "problem too large for forge_attn_bwd_noalloc's 32 MiB scratch";
+        return FORGE_ERR_WORKSPACE;
+    }
+    void *scratch = nullptr;
+    if ((s = noalloc_scratch_for_current_device(&scratch)) != FORGE_OK) return s;
+    // the preprocess stage zeroes the dq accumulator rows and overwrites Delta,
+    // so whatever the previous call left in the array does not matter
+    return forge_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale, window, softcap, dtype, scratch,
+                          kNoAllocScratchBytes, stream);
 }
 
 forge_status forge_attn_check(void *stream) {

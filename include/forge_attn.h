@@ -91,6 +91,32 @@ forge_status forge_attn_bwd(const void *q, const void *k, const void *v, const v
                             size_t workspace_bytes, void *stream);
 
 /*
+ * Backward for callers that cannot allocate device memory (no counterpart on
+ * the Forge pages: it exists for callers, not for the method). Some hosts only
+ * receive device buffers from another runtime and have no device allocator of
+ * their own, or run in a process whose memory pool owns the whole device; they
+ * cannot provide the workspace forge_attn_bwd needs. This entry point takes the
+ * same arguments as forge_attn_bwd minus the workspace and uses scratch that
+ * lives in a fixed 32 MiB device array inside the library instead (held by
+ * every GPU that loads the library until the process exits). It allocates and
+ * frees nothing.
+ *  - Limit: forge_attn_bwd_workspace_size(B, Hq, Hkv, T, D, dtype) must be at
+ *    most 32 MiB (33554432 bytes); larger problems return FORGE_ERR_WORKSPACE
+ *    (forge_attn_last_cuda_error says why) and launch nothing.
+ *  - The array's device address is looked up the first time the entry point is
+ *    called with a given device current; make that first call on each device
+ *    before any stream capture.
+ *  - All calls share the one array per device. It keeps the previous call's
+ *    contents; the call clears what must start at zero itself. Calls whose work
+ *    overlaps on the GPU (other streams, other host threads) race on the array:
+ *    serialise them.
+ */
+forge_status forge_attn_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
+                                    const float *lse, const void *dO, void *dq, void *dk, void *dv,
+                                    int B, int Hq, int Hkv, int T, int D, float scale, int window,
+                                    float softcap, forge_dtype dtype, void *stream);
+
+/*
  * The three stages of forge_attn_bwd, callable one by one on the same stream
  * with the same arguments and workspace (used to time the stages separately).
  *  preprocess: Delta_i = sum_d dO_id o_id into the workspace (f32) and, for
