@@ -149,9 +149,14 @@ forge_status fwd_tc(const void *q, const void *k, const void *v, void *o, float 
     } else {
         // two query tiles per CTA
         using C2 = Fwd2Tc<D>;
+        CUtensorMap mo;
+        if (!make_map(&mo, o, D, T, (long long)B * Hq, 128)) {
+            t_last_cuda_error = "cuTensorMapEncodeTiled failed";
+            return FORGE_ERR_CUDA;
+        }
         if (set_smem(fwd2_tc_kernel<D>, C2::SMEM) != FORGE_OK) return FORGE_ERR_CUDA;
         const unsigned grid = (unsigned)(((p.num_qt + 1) / 2) * B * Hq);
-        fwd2_tc_kernel<D><<<grid, C2::THREADS, C2::SMEM, st>>>(mq, mk, mv, p);
+        fwd2_tc_kernel<D><<<grid, C2::THREADS, C2::SMEM, st>>>(mq, mk, mv, mo, p);
     }
     return launch_status();
 }

@@ -10,9 +10,10 @@
 // ("out-of-window KV blocks are skipped, so cost scales with the window":
 // src/nn/attention.h commit log, Wave 2).
 //
-// Roles (320 threads): warps 0-3 softmax of tile A, warps 4-7 softmax of tile
+// Roles (384 threads): warps 0-3 softmax of tile A, warps 4-7 softmax of tile
 // B (one thread per query row / TMEM lane), warp 8 TMA producer, warp 9 MMA
-// issuer and TMEM owner. TMEM: S_A, S_B (128 columns each; P overwrites its S
+// issuer and TMEM owner, warps 10-11 idle (they complete the third warpgroup,
+// whose registers the softmax warpgroups take over). TMEM: S_A, S_B (128 columns each; P overwrites its S
 // as bf16), O_A, O_B (D columns each).
 // MMA order per KV tile j: PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1). Because
 // QK_x(j+1) is committed after PV_x(j), a softmax warp that sees S_x(j+1) also
@@ -34,7 +35,15 @@ struct Fwd2Tc {
     static constexpr int NSTAGE = D == 128 ? 4 : 8;
     static constexpr uint32_t CTRL = 1024;
     static constexpr uint32_t SMEM = CTRL + TILE * (2 + NSTAGE) + 1024;
-    static constexpr int THREADS = 320;
+    // warpgroups 0, 1: softmax of tiles A, B; warpgroup 2: producer (warp 8),
+    // MMA issuer (warp 9), two idle warps. Launched at 168 registers a thread
+    // (three warps per SM sub-partition); warpgroup 2 gives back down to
+    // REG_CTRL so the softmax warpgroups can grow to REG_SOFTMAX:
+    // 4 * (168 - REG_CTRL) = 8 * (REG_SOFTMAX - 168).
+    static constexpr int THREADS = 384;
+    static constexpr int REG_LAUNCH = 168, REG_CTRL = 56, REG_SOFTMAX = 224;
+    static_assert(4 * (REG_LAUNCH - REG_CTRL) >= 8 * (REG_SOFTMAX - REG_LAUNCH), "register split");
+    static_assert((2 * REG_SOFTMAX + REG_CTRL) * 32 <= 16384, "registers of one SM sub-partition");
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t col_s(int x) { return (uint32_t)(x * 128); }
     static constexpr uint32_t col_o(int x) { return (uint32_t)(256 + x * D); }
@@ -95,9 +104,10 @@ __device__ __forceinline__ void exp_chunk32(const uint32_t (&s)[32], uint64_t sl
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     fwd2_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   const FwdParams p) {
     using C = Fwd2Tc<D>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = smem_u32(smem_raw);
@@ -142,6 +152,7 @@ __global__ void __launch_bounds__(320, 1)
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
+        tma_prefetch_desc(&tmO);
     }
     if (warp == 9) {
         tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -152,107 +163,111 @@ __global__ void __launch_bounds__(320, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 8) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            const uint64_t keep = policy_evict_last();
-            mbar_arrive_expect_tx(bar(C::B_Q), hasB ? 2 * C::TILE : C::TILE);
-            for (int c = 0; c < C::NCB; c++) {
-                tma_load_3d(sQ + c * C::CB, &tmQ, bar(C::B_Q), c * 64, qA0, bh);
-                if (hasB) tma_load_3d(sQ + C::TILE + c * C::CB, &tmQ, bar(C::B_Q), c * 64, qB0, bh);
-            }
-            // ring slots in order K(lo), V(lo), K(lo+1), V(lo+1), ...
-            int issued = 0;
-            bool ok = true;
-            for (int j = lo; ok && j <= hi; j++) {
-                for (int kv = 0; kv < 2 && ok; kv++) {
-                    const int st = issued % C::NSTAGE;
-                    const uint32_t ph = (uint32_t)((issued / C::NSTAGE) & 1);
-                    if (!mbar_wait(bar(C::B_KV_EMPTY + st), ph ^ 1u, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(bar(C::B_KV_FULL + st), C::TILE);
-                    for (int c = 0; c < C::NCB; c++)
-                        tma_load_3d_hint(sKV + st * C::TILE + c * C::CB, kv ? &tmV : &tmK, bar(C::B_KV_FULL + st),
-                                         c * 64, j * C::BN, bkv, keep);
-                    issued++;
+    if (warp >= 8) {
+        setmaxnreg_dec<C::REG_CTRL>();
+        if (warp == 8) {
+            // ------------------------------------------------------------ producer
+            if (lane == 0) {
+                const uint64_t keep = policy_evict_last();
+                mbar_arrive_expect_tx(bar(C::B_Q), hasB ? 2 * C::TILE : C::TILE);
+                for (int c = 0; c < C::NCB; c++) {
+                    tma_load_3d(sQ + c * C::CB, &tmQ, bar(C::B_Q), c * 64, qA0, bh);
+                    if (hasB) tma_load_3d(sQ + C::TILE + c * C::CB, &tmQ, bar(C::B_Q), c * 64, qB0, bh);
                 }
-            }
-            if (!ok) {
-                mbar_wait_drain(bar(C::B_Q), 0, 200000000ull);
-                for (int back = 1; back <= min(issued, C::NSTAGE); back++) {
-                    const int L = issued - back;
-                    mbar_wait_drain(bar(C::B_KV_FULL + L % C::NSTAGE), (uint32_t)((L / C::NSTAGE) & 1), 200000000ull);
-                }
-            }
-        }
-    } else if (warp == 9) {
-        // ---------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t ID_QK = idesc_bf16_f32(128, 128, false, false);
-            constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, false, true);
-            auto wait_full = [&](int slot) -> bool {
-                return mbar_wait(bar(C::B_KV_FULL + slot % C::NSTAGE), (uint32_t)((slot / C::NSTAGE) & 1), abort_flag);
-            };
-            auto release = [&](int slot) { tc_commit(bar(C::B_KV_EMPTY + slot % C::NSTAGE)); };
-            auto issue_qk = [&](int x, int slot) {
-                const uint32_t sK = sKV + (slot % C::NSTAGE) * C::TILE;
-                const uint32_t sQx = sQ + (uint32_t)x * C::TILE;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; kk++) {
-                    const uint32_t off = (kk >> 2) * C::CB + (kk & 3) * 32;
-                    mma_ss(tmem + C::col_s(x), sdesc_sw128(sQx + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), ID_QK,
-                           kk > 0);
-                }
-                tc_commit(bar(C::B_S_FULL + x));
-            };
-            auto issue_pv = [&](int x, int slot, bool acc) {
-                const uint32_t sV = sKV + (slot % C::NSTAGE) * C::TILE;
-#pragma unroll
-                for (int kk = 0; kk < C::BN / 16; kk++)
-                    mma_ts(tmem + C::col_o(x), tmem + C::col_s(x) + kk * 8, sdesc_sw128(sV + kk * 2048, C::CB, 1024),
-                           ID_PV, (acc || kk > 0) ? 1u : 0u);
-            };
-            bool ok = mbar_wait(bar(C::B_Q), 0, abort_flag);
-            if (ok) ok = wait_full(0);
-            if (ok) {
-                tc_fence_after();
-                if (active(0, lo)) issue_qk(0, 0);
-                if (active(1, lo)) issue_qk(1, 0);
-                release(0);
-            }
-            int cnt[2] = {0, 0};
-            for (int j = lo; ok && j <= hi; j++) {
-                const int slotV = 2 * (j - lo) + 1, slotK = slotV + 1;
-                if (!(ok = wait_full(slotV))) break;
-                bool k_ready = false;
-                for (int x = 0; x < 2 && ok; x++) {
-                    if (active(x, j)) {
-                        if (!(ok = mbar_wait(bar(C::B_P_FULL + x), (uint32_t)(cnt[x] & 1), abort_flag))) break;
-                        tc_fence_after();
-                        issue_pv(x, slotV, cnt[x] > 0);
-                        cnt[x]++;
-                    }
-                    if (j < hi && active(x, j + 1)) {
-                        if (!k_ready) {
-                            if (!(ok = wait_full(slotK))) break;
-                            tc_fence_after();
-                            k_ready = true;
+                // ring slots in order K(lo), V(lo), K(lo+1), V(lo+1), ...
+                int issued = 0;
+                bool ok = true;
+                for (int j = lo; ok && j <= hi; j++) {
+                    for (int kv = 0; kv < 2 && ok; kv++) {
+                        const int st = issued % C::NSTAGE;
+                        const uint32_t ph = (uint32_t)((issued / C::NSTAGE) & 1);
+                        if (!mbar_wait(bar(C::B_KV_EMPTY + st), ph ^ 1u, abort_flag)) {
+                            ok = false;
+                            break;
                         }
-                        issue_qk(x, slotK);
+                        mbar_arrive_expect_tx(bar(C::B_KV_FULL + st), C::TILE);
+                        for (int c = 0; c < C::NCB; c++)
+                            tma_load_3d_hint(sKV + st * C::TILE + c * C::CB, kv ? &tmV : &tmK, bar(C::B_KV_FULL + st),
+                                             c * 64, j * C::BN, bkv, keep);
+                        issued++;
                     }
                 }
-                if (!ok) break;
-                release(slotV);
-                if (j < hi) release(slotK);
+                if (!ok) {
+                    mbar_wait_drain(bar(C::B_Q), 0, 200000000ull);
+                    for (int back = 1; back <= min(issued, C::NSTAGE); back++) {
+                        const int L = issued - back;
+                        mbar_wait_drain(bar(C::B_KV_FULL + L % C::NSTAGE), (uint32_t)((L / C::NSTAGE) & 1), 200000000ull);
+                    }
+                }
             }
-            // O_FINAL fires once every MMA issued so far has completed
-            tc_commit(bar(C::B_O_FINAL + 0));
-            tc_commit(bar(C::B_O_FINAL + 1));
-            if (!ok) mbar_wait_drain(bar(C::B_O_FINAL + 0), 0, 200000000ull);
+        } else if (warp == 9) {
+            // ---------------------------------------------------------- MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t ID_QK = idesc_bf16_f32(128, 128, false, false);
+                constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, false, true);
+                auto wait_full = [&](int slot) -> bool {
+                    return mbar_wait(bar(C::B_KV_FULL + slot % C::NSTAGE), (uint32_t)((slot / C::NSTAGE) & 1), abort_flag);
+                };
+                auto release = [&](int slot) { tc_commit(bar(C::B_KV_EMPTY + slot % C::NSTAGE)); };
+                auto issue_qk = [&](int x, int slot) {
+                    const uint32_t sK = sKV + (slot % C::NSTAGE) * C::TILE;
+                    const uint32_t sQx = sQ + (uint32_t)x * C::TILE;
+    #pragma unroll
+                    for (int kk = 0; kk < D / 16; kk++) {
+                        const uint32_t off = (kk >> 2) * C::CB + (kk & 3) * 32;
+                        mma_ss(tmem + C::col_s(x), sdesc_sw128(sQx + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), ID_QK,
+                               kk > 0);
+                    }
+                    tc_commit(bar(C::B_S_FULL + x));
+                };
+                auto issue_pv = [&](int x, int slot, bool acc) {
+                    const uint32_t sV = sKV + (slot % C::NSTAGE) * C::TILE;
+    #pragma unroll
+                    for (int kk = 0; kk < C::BN / 16; kk++)
+                        mma_ts(tmem + C::col_o(x), tmem + C::col_s(x) + kk * 8, sdesc_sw128(sV + kk * 2048, C::CB, 1024),
+                               ID_PV, (acc || kk > 0) ? 1u : 0u);
+                };
+                bool ok = mbar_wait(bar(C::B_Q), 0, abort_flag);
+                if (ok) ok = wait_full(0);
+                if (ok) {
+                    tc_fence_after();
+                    if (active(0, lo)) issue_qk(0, 0);
+                    if (active(1, lo)) issue_qk(1, 0);
+                    release(0);
+                }
+                int cnt[2] = {0, 0};
+                for (int j = lo; ok && j <= hi; j++) {
+                    const int slotV = 2 * (j - lo) + 1, slotK = slotV + 1;
+                    if (!(ok = wait_full(slotV))) break;
+                    bool k_ready = false;
+                    for (int x = 0; x < 2 && ok; x++) {
+                        if (active(x, j)) {
+                            if (!(ok = mbar_wait(bar(C::B_P_FULL + x), (uint32_t)(cnt[x] & 1), abort_flag))) break;
+                            tc_fence_after();
+                            issue_pv(x, slotV, cnt[x] > 0);
+                            cnt[x]++;
+                        }
+                        if (j < hi && active(x, j + 1)) {
+                            if (!k_ready) {
+                                if (!(ok = wait_full(slotK))) break;
+                                tc_fence_after();
+                                k_ready = true;
+                            }
+                            issue_qk(x, slotK);
+                        }
+                    }
+                    if (!ok) break;
+                    release(slotV);
+                    if (j < hi) release(slotK);
+                }
+                // O_FINAL fires once every MMA issued so far has completed
+                tc_commit(bar(C::B_O_FINAL + 0));
+                tc_commit(bar(C::B_O_FINAL + 1));
+                if (!ok) mbar_wait_drain(bar(C::B_O_FINAL + 0), 0, 200000000ull);
+            }
         }
     } else {
+        setmaxnreg_inc<C::REG_SOFTMAX>();
         // ---------------------------------------- softmax: warps 0-3 tile A, 4-7 tile B
         const int x = warp / 4;
         const int row = threadIdx.x % 128;
@@ -262,6 +277,7 @@ __global__ void __launch_bounds__(320, 1)
         const int q0 = x ? qB0 : qA0;
         const int lox = x ? loB : loA, hix = x ? tB : tA;
         const int qi = q0 + row;
+        const int r0 = q0 + 32 * (warp % 4);
         const bool cap = p.softcap > 0.0f;
         const uint64_t sl2x2 = f2_make(p.scale_log2, p.scale_log2);
         float m = -INFINITY, l = 0.0f;
@@ -282,13 +298,32 @@ __global__ void __launch_bounds__(320, 1)
                         s[c >> 5][c & 31] = __float_as_uint(p.cap_out * tanh_via_ex2(v * p.cap_in));
                     }
                 }
-                const bool need_mask = (k0 + C::BN - 1 > q0) || (W > 0 && k0 <= q0 + C::BM - 1 - W);
-                if (need_mask) {
+                // Classes of the four 32-key chunks for this warp's 32 rows
+                // [r0, r0 + 31] (warp-uniform): bit q of `dead` = no key of chunk q
+                // is visible to any of the rows, bit q of `part` = some are.
+                unsigned dead = 0, part = 0;
 #pragma unroll
-                    for (int c = 0; c < 128; c++) {
-                        const int kj = k0 + c;
-                        const bool vis = kj <= qi && (W == 0 || kj > qi - W);
-                        if (!vis) s[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+                for (int q4 = 0; q4 < 4; q4++) {
+                    const int c0 = k0 + 32 * q4;
+                    const bool all_vis = (c0 + 31 <= r0) && (W == 0 || c0 > r0 + 31 - W);
+                    const bool none = (c0 > r0 + 31) || (W > 0 && c0 + 31 <= r0 - W);
+                    dead |= (unsigned)none << q4;
+                    part |= (unsigned)(!all_vis && !none) << q4;
+                }
+                if (dead | part) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; q4++) {
+                        // bit c of vm: key k0 + 32 q4 + c is visible to row qi,
+                        // i.e. lo_c < c <= hi_c
+                        const int hi_c = qi - (k0 + 32 * q4);
+                        uint32_t vm = hi_c < 0 ? 0u : (hi_c >= 31 ? ~0u : (~0u >> (31 - hi_c)));
+                        if (W > 0) {
+                            const int lo_c = hi_c - W;
+                            vm &= lo_c < 0 ? ~0u : (lo_c >= 31 ? 0u : (~0u << (lo_c + 1)));
+                        }
+#pragma unroll
+                        for (int c = 0; c < 32; c++)
+                            if (!((vm >> c) & 1u)) s[q4][c] = __float_as_uint(-INFINITY);
                     }
                 }
                 float mx = row_max128(s);
@@ -319,18 +354,37 @@ __global__ void __launch_bounds__(320, 1)
                 const float msub = (m == -INFINITY) ? 0.0f : m;
                 const uint64_t negm2 = f2_make(-msub, -msub);
                 uint64_t rs[2] = {f2_make(0.0f, 0.0f), f2_make(0.0f, 0.0f)};
+                // 32 scores -> 16 packed P columns; P column c holds scores 2c, 2c+1.
+                // Masked scores are -inf and need the MUFU exp2 (the FMA-pipe one
+                // is only valid for finite arguments); chunks no row sees are 0.
+                if (dead | part) {
 #pragma unroll
-                for (int q4 = 0; q4 < 4; q4++) {
-                    // 32 scores -> 16 packed P columns; P column c holds scores 2c, 2c+1
-                    uint32_t pk[16];
-                    if (cap) {
-                        if (need_mask) exp_chunk32<true, false, C::EMU_MASK>(s[q4], sl2x2, negm2, rs, pk);
-                        else exp_chunk32<true, true, C::EMU_MASK>(s[q4], sl2x2, negm2, rs, pk);
-                    } else {
-                        if (need_mask) exp_chunk32<false, false, C::EMU_MASK>(s[q4], sl2x2, negm2, rs, pk);
-                        else exp_chunk32<false, true, C::EMU_MASK>(s[q4], sl2x2, negm2, rs, pk);
+                    for (int q4 = 0; q4 < 4; q4++) {
+                        uint32_t pk[16];
+                        if ((dead >> q4) & 1u) {
+#pragma unroll
+                            for (int c = 0; c < 16; c++) pk[c] = 0u;
+                        } else if (cap) {
+                            exp_chunk32<true, false, C::EMU_MASK>(s[q4], sl2x2, negm2, rs, pk);
+                        } else {
+                            exp_chunk32<false, false, C::EMU_MASK>(s[q4], sl2x2, negm2, rs, pk);
+                        }
+                        tmem_st16(tS + 16 * q4, pk);
                     }
-                    tmem_st16(tS + 16 * q4, pk);
+                } else if (cap) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; q4++) {
+                        uint32_t pk[16];
+                        exp_chunk32<true, true, C::EMU_MASK>(s[q4], sl2x2, negm2, rs, pk);
+                        tmem_st16(tS + 16 * q4, pk);
+                    }
+                } else {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; q4++) {
+                        uint32_t pk[16];
+                        exp_chunk32<false, true, C::EMU_MASK>(s[q4], sl2x2, negm2, rs, pk);
+                        tmem_st16(tS + 16 * q4, pk);
+                    }
                 }
                 tmem_st_wait();
                 tc_fence_before();
@@ -347,7 +401,11 @@ __global__ void __launch_bounds__(320, 1)
             tc_fence_after();
             const float inv_l = 1.0f / l;
             const uint64_t inv2 = f2_make(inv_l, inv_l);
-            __nv_bfloat16 *orow = p.o + ((size_t)bh * p.T + (size_t)min(qi, p.T - 1)) * D;
+            // Stage this tile's O (bf16) in its Q buffer, which every MMA has
+            // finished reading once O_FINAL fired, in the 128-byte-swizzled
+            // layout of the O tensor map, then store it with TMA (rows >= T
+            // are clipped by the map).
+            const uint32_t sO = sQ + (uint32_t)x * C::TILE;
 #pragma unroll 1
             for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t o[32];
@@ -360,11 +418,19 @@ __global__ void __launch_bounds__(320, 1)
                     f2_split(f2_mul(f2_make(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), inv2), a, bb);
                     w[i] = pack_bf16x2(a, bb);
                 }
-                if (qi < p.T) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
+                const uint32_t rowaddr = sO + (uint32_t)(c0 / 64) * C::CB + (uint32_t)row * 128u;
+                const uint32_t ch0 = (uint32_t)((c0 % 64) / 8);
 #pragma unroll
-                    for (int i = 0; i < 4; i++) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-                }
+                for (int i = 0; i < 4; i++)
+                    st_shared_v4(rowaddr + ((((ch0 + i) ^ (uint32_t)(row & 7))) << 4), w[4 * i], w[4 * i + 1],
+                                 w[4 * i + 2], w[4 * i + 3]);
+            }
+            fence_proxy_async_smem();
+            named_barrier_sync(1 + x, 128);
+            if (row == 0) {
+                for (int cb = 0; cb < C::NCB; cb++) tma_store_3d(&tmO, sO + cb * C::CB, cb * 64, q0, bh);
+                bulk_commit();
+                bulk_wait_read<0>();
             }
             if (qi < p.T) p.lse[(size_t)bh * p.T + qi] = (m + __log2f(l)) * kLn2;
         }

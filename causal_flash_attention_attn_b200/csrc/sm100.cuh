@@ -138,6 +138,15 @@ __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap *map, uint32
         "r"(src), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
+// 3D tiled store from this CTA's shared memory (bulk group; pair with bulk_commit
+// and bulk_wait_read before the source is reused or the CTA exits).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t src, int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(src), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until at most N bulk groups of this thread still have to READ their source.
 template <int N>
@@ -164,8 +173,23 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
 }
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (tensor core operand reads).
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Warpgroup-wide register re-allocation (every warp of the warpgroup executes it).
+// The block's launch allocation is the pool: the decreases must free at least
+// what the increases take.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ---------------------------------------------------------------------- tcgen05
