@@ -14,24 +14,25 @@
 //   dV  += P^T dO           (A from TMEM)
 //   dK  += dS^T Q
 //   dQ   = dS K  (or its transpose K^T dS^T), drained from TMEM by four warps
-//          into a swizzled f32 staging tile in shared memory and added into a
-//          padded [B*Hq][Tpad][D] f32 workspace with TMA bulk reduce-add (head
-//          dim 256, which has no shared memory left for staging, adds with
-//          per-element f32 reductions instead).
+//          and added into a padded [B*Hq][Tpad][D] f32 workspace: head dim 64
+//          through a swizzled f32 staging tile in shared memory and TMA bulk
+//          reduce-add; head dims 128 and 256, which have no shared memory left
+//          for staging, with warp-coalesced f32 reductions from registers.
 // dK and dV sum over the group's query heads inside the CTA, so they need no
 // atomics; dQ rows are shared between key tiles and are reduced in L2.
 //
-// Overlap (head dim 128): S^T and dS^T are double-buffered and the compute warps
-// copy dP^T into registers as soon as it lands, so the MMA warp issues
-// S^T(i+1) and dP^T(i+1) while step i's P and dS are being formed, and step
-// i+1's P/dS math runs while dV, dK, dQ of step i are on the tensor cores.
+// Steps of 128 query rows keep every product at N = 128 (or M = N = 128 for
+// dQ^T): a tcgen05.mma with both operands in shared memory reads A and B
+// (4 KB + N/32 KB per K = 16 slice) at the shared-memory port's rate, so
+// narrower products are bound by that port rather than by the tensor cores.
 //
-// Shapes per head dim (TMEM columns: NSB x S^T + dP^T + dV + dK + dQ <= 512):
-//   D = 64 : BM = 128 query rows, one S buffer, dQ = dS K (M = 128 rows, N = 64)
-//   D = 128: BM = 64, two S buffers, dQ^T = K^T dS^T (M = 128 = D, N = 64 rows)
-//   D = 256: BM = 64, one S buffer, two CTAs per key tile, each owning half of
-//            the head dim (DH = 128) for dK, dV and dQ; S^T and dP^T use the
-//            full head dim.
+// Shapes per head dim (TMEM columns: S^T + dP^T + dV + dK (+ dQ) <= 512):
+//   D = 64 : BM = 128 query rows, dQ = dS K (M = 128 rows, N = 64)
+//   D = 128: BM = 128, dQ^T = K^T dS^T (M = 128 = D, N = 128 rows) in the
+//            columns of dP^T (already copied to registers when dQ^T is issued;
+//            dP^T of the next step waits until the drain warps copied dQ^T)
+//   D = 256: BM = 64, two CTAs per key tile, each owning half of the head dim
+//            (DH = 128) for dK, dV and dQ; S^T and dP^T use the full head dim.
 //
 // Roles (320 threads): warps 0-3 compute (one thread per key row, TMEM lane),
 // warps 4-7 dQ drain + dK epilogue, warp 8 loads (TMA for tiles, plain loads
@@ -46,13 +47,15 @@ template <int D_>
 struct BwdTc {
     static constexpr int D = D_;
     static constexpr int BN = 128;                       // keys per CTA
-    static constexpr int BM = D == 64 ? 128 : 64;        // query rows per step
+    static constexpr int BM = D == 256 ? 64 : 128;       // query rows per step
     static constexpr bool DQT = D != 64;                 // transposed dQ product
     static constexpr int NSPLIT = D == 256 ? 2 : 1;      // head-dim halves
     static constexpr int DH = D / NSPLIT;                // output columns per CTA
-    static constexpr int QST = D == 256 ? 1 : (D == 128 ? 3 : 2);  // Q/dO stages
-    static constexpr int NSB = D == 128 ? 2 : 1;         // S^T / dS^T buffers
-    static constexpr bool PRELOAD = (BM == 64);          // whole S^T/dP^T rows in registers
+    static constexpr int QST = D == 256 ? 1 : 2;         // Q/dO stages
+    // head dim 128: dQ^T takes the TMEM columns of dP^T, which the compute warps
+    // have copied out by the time dQ^T is issued (dP^T of the next step then
+    // waits for the drain warps to copy dQ^T out)
+    static constexpr bool DQ_ALIAS = D == 128;
     static constexpr int NCB = D / 64;
     static constexpr uint32_t CBK = 128 * 128;           // column block of a 128-row tile
     static constexpr uint32_t CBQ = BM * 128;            // column block of a BM-row tile
@@ -62,35 +65,57 @@ struct BwdTc {
     static constexpr uint32_t OFF_K = 0, OFF_V = TK, OFF_Q = 2 * TK;
     static constexpr uint32_t OFF_DO = OFF_Q + QST * TQ;
     static constexpr uint32_t OFF_DS = OFF_DO + QST * TQ;
-    static constexpr bool BULK_DQ = D != 256;            // staged TMA reduce-add of dQ
+    static constexpr bool BULK_DQ = D == 64;             // staged TMA reduce-add of dQ
     static constexpr int NSTG = D == 64 ? 2 : 1;         // dQ staging tiles
     static constexpr uint32_t STG = BM * DH * 4;         // one f32 dQ staging tile
-    static constexpr uint32_t OFF_STG = OFF_DS + NSB * TS;
+    static constexpr uint32_t OFF_STG = OFF_DS + TS;
     static constexpr uint32_t TILES = OFF_STG + (BULK_DQ ? NSTG * STG : 0);
-    // control block: barriers, TMEM slot, abort flag, per-stage LSE/Delta rows
+    // control block after the tiles: barriers, TMEM slot, abort flag, per-stage
+    // LSE/Delta rows. The tiles need 1024-byte alignment (128-byte swizzle); the
+    // dynamic shared memory base is 1024-aligned in practice, and SLACK covers
+    // a base that is not wherever the budget leaves room (the kernel checks).
     static constexpr uint32_t OFF_TMEM_SLOT = 240, OFF_ABORT = 244;
-    static constexpr uint32_t OFF_LSE = 256;                        // [QST][BM] f32, LSE * log2(e)
-    static constexpr uint32_t OFF_DLT = OFF_LSE + QST * BM * 4;     // [QST][BM] f32, scale * Delta
-    static constexpr uint32_t CTRL = (OFF_DLT + QST * BM * 4 + 1023) / 1024 * 1024;
-    static constexpr uint32_t SMEM = CTRL + TILES + 1024;
-    static constexpr int THREADS = 320;
-    static constexpr uint32_t COL_DP = NSB * BM, COL_DV = COL_DP + BM, COL_DK = COL_DV + DH;
-    static constexpr uint32_t COL_DQ = COL_DK + DH;
+    static constexpr uint32_t OFF_LSE = 256;                        // [QST][BM] f32, -LSE * log2(e)
+    static constexpr uint32_t OFF_DLT = OFF_LSE + QST * BM * 4;     // [QST][BM] f32, -scale * Delta
+    static constexpr uint32_t CTRL = OFF_DLT + QST * BM * 4;
+    static constexpr uint32_t SLACK = (TILES + CTRL + 1024 <= 232448) ? 1024 : 0;
+    static constexpr uint32_t SMEM = SLACK + TILES + CTRL;
+    // Roles: warps 0-7 compute (warp w: TMEM lanes 32 (w % 4).., query-row half
+    // w / 4 of the step), 8-11 dQ drain and dK epilogue, 12 loads, 13 MMA issue
+    // and TMEM owner, 14-15 idle (they complete the fourth warpgroup). Launched
+    // at 128 registers a thread; the fourth warpgroup gives back down to
+    // REG_CTRL, the compute warpgroups grow to REG_COMPUTE, the drain
+    // warpgroup to REG_DRAIN.
+    static constexpr int THREADS = 512;
+    static constexpr int W_DRAIN = 8, W_LOAD = 12, W_MMA = 13;
+    static constexpr int REG_LAUNCH = 128, REG_CTRL = 80, REG_COMPUTE = 144, REG_DRAIN = 144;
+    static_assert(4 * (REG_LAUNCH - REG_CTRL) >= 8 * (REG_COMPUTE - REG_LAUNCH) + 4 * (REG_DRAIN - REG_LAUNCH),
+                  "register split");
+    static_assert((2 * REG_COMPUTE + REG_DRAIN + REG_CTRL) * 32 <= 16384, "registers of one SM sub-partition");
+    static constexpr int HALF = BM / 2;                  // query rows of one compute warp
+    static constexpr uint32_t COL_S = 0;
+    static constexpr uint32_t COL_DP = BM, COL_DV = COL_DP + BM, COL_DK = COL_DV + DH;
+    static constexpr uint32_t COL_DQ = DQ_ALIAS ? COL_DP : COL_DK + DH;
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t col_s(int b) { return (uint32_t)(b * BM); }
-    static_assert(COL_DQ + (DQT ? BM : DH) <= 512, "tensor memory");
+    // P^T (bf16 pairs) of query rows [16 kk, 16 kk + 16): each compute warp
+    // writes its half's P^T into the first columns of its own half of S^T
+    static constexpr uint32_t col_p(int kk) {
+        return COL_S + (uint32_t)((16 * kk / HALF) * HALF + 8 * (kk % (HALF / 16)));
+    }
+    static_assert(COL_DK + DH <= 512 && COL_DQ + (DQT ? BM : DH) <= 512, "tensor memory");
+    static_assert(!DQ_ALIAS || (DQT ? BM : DH) <= BM, "dQ fits in the dP^T columns");
     static_assert(!DQT || DH == 128, "transposed dQ needs M = 128");
     static_assert(SMEM <= 232448, "shared memory");
     // barriers
     static constexpr int B_KV = 0;
     static constexpr int B_Q_FULL = 1;                   // [QST]
     static constexpr int B_Q_EMPTY = B_Q_FULL + QST;     // [QST]
-    static constexpr int B_S_FULL = B_Q_EMPTY + QST;     // [NSB]
-    static constexpr int B_DS_EMPTY = B_S_FULL + NSB;    // [NSB]
-    static constexpr int B_PDS_FULL = B_DS_EMPTY + NSB;  // [NSB] P^T and dS^T of a buffer ready
-    static constexpr int B_DP_FULL = B_PDS_FULL + NSB;
-    static constexpr int B_DP_FREE = B_DP_FULL + 1;
-    static constexpr int B_DQ_FULL = B_DP_FREE + 1;
+    static constexpr int B_S_FULL = B_Q_EMPTY + QST;
+    static constexpr int B_DS_EMPTY = B_S_FULL + 1;
+    static constexpr int B_P_FULL = B_DS_EMPTY + 1;       // P^T in TMEM (8 compute warps)
+    static constexpr int B_DS_FULL = B_P_FULL + 1;        // dS^T in shared memory (8 compute warps)
+    static constexpr int B_DP_FULL = B_DS_FULL + 1;
+    static constexpr int B_DQ_FULL = B_DP_FULL + 1;
     static constexpr int B_DQ_FREE = B_DQ_FULL + 1;
     static constexpr int B_KDONE = B_DQ_FREE + 1;
     static constexpr int NBAR = B_KDONE + 1;
@@ -110,100 +135,120 @@ struct BwdParams {
     float cap_out;         // softcap * log2(e)
 };
 
-// P and dS for 32 query columns of one key row (this thread's TMEM lane).
-//   s, dp : raw S^T and dP^T accumulators of the 32 columns
-//   l2, dl: LSE*log2(e) and scale*Delta of the 32 columns
-//   pk, dk: bf16x2-packed P^T and dS^T (column pairs, low half = even column)
-// CAP and MASK are compile-time so the unrolled loop is one basic block.
+// The two phases of one key row's P / dS work (this thread's TMEM lane), 32
+// query columns at a time:
+//   phase A (needs S^T): P = exp2(s * scale * log2(e) - LSE * log2(e)), masked
+//            to 0, as bf16 pairs pk (P^T for dV += P^T dO), and the factor g of
+//            dS = g * (dP - Delta): g = P, or P (1 - tanh^2) under the cap
+//            (the "exact tanh' chain": src/nn/attention.h commit log, Wave 2);
+//   phase B (needs dP^T): dS = g * (dP * scale - Delta * scale) as bf16 pairs.
+//   nl, nd: -LSE*log2(e) and -scale*Delta of the 32 columns (shared memory).
+// CAP and MASK are compile-time so each unrolled loop is one basic block; the
+// common case (neither) runs on packed f32x2 arithmetic.
 template <bool CAP, bool MASK>
-__device__ __forceinline__ void bwd_math32(const uint32_t (&s)[32], const uint32_t (&dp)[32], const float *l2s,
-                                           const float *dls, const BwdParams &p, int kj, int q0, int W,
-                                           uint32_t (&pk)[16], uint32_t (&dk)[16]) {
-    float l2[4], dl[4];
+__device__ __forceinline__ void bwd_p32(const uint32_t (&s)[32], const float *nl, const BwdParams &p, int kj, int q0,
+                                        int W, uint32_t (&pk)[16], float (&g)[32]) {
+    if constexpr (!CAP && !MASK) {
+        const uint64_t sl2 = f2_make(p.scale_log2, p.scale_log2);
 #pragma unroll
-    for (int c = 0; c < 32; c += 2) {
-        if ((c & 3) == 0) {
-            const float4 a = *reinterpret_cast<const float4 *>(l2s + c);
-            const float4 d4 = *reinterpret_cast<const float4 *>(dls + c);
-            l2[0] = a.x; l2[1] = a.y; l2[2] = a.z; l2[3] = a.w;
-            dl[0] = d4.x; dl[1] = d4.y; dl[2] = d4.z; dl[3] = d4.w;
+        for (int c = 0; c < 32; c += 4) {
+            const float4 a = *reinterpret_cast<const float4 *>(nl + c);
+#pragma unroll
+            for (int e = 0; e < 4; e += 2) {
+                const uint64_t y2 = f2_fma(f2_make(__uint_as_float(s[c + e]), __uint_as_float(s[c + e + 1])), sl2,
+                                           e ? f2_make(a.z, a.w) : f2_make(a.x, a.y));
+                float y0, y1;
+                f2_split(y2, y0, y1);
+                // a quarter of the exponentials on the FMA pipe
+                const bool emu = ((c + e) & 6) == 6;
+                g[c + e] = emu ? exp2_poly(y0) : ex2_approx(y0);
+                g[c + e + 1] = emu ? exp2_poly(y1) : ex2_approx(y1);
+                pk[(c + e) >> 1] = pack_bf16x2(g[c + e], g[c + e + 1]);
+            }
         }
-        float pp[2], dd[2];
+    } else {
 #pragma unroll
-        for (int e = 0; e < 2; e++) {
-            const float x = __uint_as_float(s[c + e]);
-            float pr, g;
-            // a quarter of the exponentials on the FMA pipe when nothing is masked
+        for (int c = 0; c < 32; c++) {
+            const float x = __uint_as_float(s[c]);
+            float pr, gg;
             const bool emu = !MASK && (c & 6) == 6;
             if constexpr (CAP) {
                 const float t = tanh_via_ex2(x * p.cap_in);
-                const float y = fmaf(p.cap_out, t, -l2[(c & 3) + e]);
+                const float y = fmaf(p.cap_out, t, nl[c]);
                 pr = emu ? exp2_poly(y) : ex2_approx(y);
-                g = pr * (1.0f - t * t);
+                gg = pr * (1.0f - t * t);
             } else {
-                const float y = fmaf(x, p.scale_log2, -l2[(c & 3) + e]);
+                const float y = fmaf(x, p.scale_log2, nl[c]);
                 pr = emu ? exp2_poly(y) : ex2_approx(y);
-                g = pr;
+                gg = pr;
             }
             if constexpr (MASK) {
-                const int qi = q0 + c + e;
+                const int qi = q0 + c;
                 const bool vis = kj <= qi && (W == 0 || kj > qi - W);
                 pr = vis ? pr : 0.0f;
-                g = vis ? g : 0.0f;
+                gg = vis ? gg : 0.0f;
             }
-            pp[e] = pr;
-            dd[e] = g * fmaf(__uint_as_float(dp[c + e]), p.scale, -dl[(c & 3) + e]);
+            g[c] = gg;
+            if (c & 1) pk[c >> 1] = pack_bf16x2(__uint_as_float(pk[c >> 1]), pr);
+            else pk[c >> 1] = __float_as_uint(pr);
         }
-        pk[c >> 1] = pack_bf16x2(pp[0], pp[1]);
-        dk[c >> 1] = pack_bf16x2(dd[0], dd[1]);
     }
 }
 
-// One 32-column chunk: LSE/Delta terms from shared memory, P/dS math, P^T into
-// TMEM (columns [c0/2, c0/2 + 16) of the S buffer, already read), dS^T into the
-// swizzled shared-memory tile (row kr, 16-byte chunk index XOR row % 8).
-template <int D>
-__device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], const float *l2s,
-                                          const float *dls, const BwdParams &p, bool cap, bool mask, int kj, int q0,
-                                          int W, int c0, int kr, uint32_t tS, uint32_t sdS) {
-    using C = BwdTc<D>;
-    const float *l2 = l2s + c0, *dl = dls + c0;
-    uint32_t pk[16], dk[16];
-    if (cap) {
-        if (mask) bwd_math32<true, true>(s, dp, l2, dl, p, kj, q0, W, pk, dk);
-        else bwd_math32<true, false>(s, dp, l2, dl, p, kj, q0, W, pk, dk);
-    } else {
-        if (mask) bwd_math32<false, true>(s, dp, l2, dl, p, kj, q0, W, pk, dk);
-        else bwd_math32<false, false>(s, dp, l2, dl, p, kj, q0, W, pk, dk);
+__device__ __forceinline__ void bwd_ds32(const uint32_t (&dp)[32], const float (&g)[32], const float *nd,
+                                         const BwdParams &p, uint32_t (&dk)[16]) {
+    const uint64_t sc2 = f2_make(p.scale, p.scale);
+#pragma unroll
+    for (int c = 0; c < 32; c += 4) {
+        const float4 d4 = *reinterpret_cast<const float4 *>(nd + c);
+#pragma unroll
+        for (int e = 0; e < 4; e += 2) {
+            const uint64_t t2 = f2_fma(f2_make(__uint_as_float(dp[c + e]), __uint_as_float(dp[c + e + 1])), sc2,
+                                       e ? f2_make(d4.z, d4.w) : f2_make(d4.x, d4.y));
+            float d0, d1;
+            f2_split(f2_mul(f2_make(g[c + e], g[c + e + 1]), t2), d0, d1);
+            dk[(c + e) >> 1] = pack_bf16x2(d0, d1);
+        }
     }
-    tmem_st16(tS + (uint32_t)(c0 >> 1), pk);
+}
+
+// dS^T pairs of 32 query columns (starting at column c0 of the step) into the
+// swizzled shared-memory tile: row kr, 16-byte chunk index XOR row % 8.
+template <int D>
+__device__ __forceinline__ void bwd_store_ds(const uint32_t (&dk)[16], int c0, int kr, uint32_t sdS) {
+    using C = BwdTc<D>;
     const uint32_t blk = sdS + (uint32_t)(c0 >> 6) * C::CBK + (uint32_t)kr * 128u;
 #pragma unroll
     for (int e = 0; e < 4; e++) {
         const uint32_t chunk = (uint32_t)(((c0 & 63) >> 3) + e);
-        const uint32_t addr = blk + ((chunk ^ (uint32_t)(kr & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dk[4 * e]), "r"(dk[4 * e + 1]),
-                     "r"(dk[4 * e + 2]), "r"(dk[4 * e + 3])
-                     : "memory");
+        st_shared_v4(blk + ((chunk ^ (uint32_t)(kr & 7)) << 4), dk[4 * e], dk[4 * e + 1], dk[4 * e + 2],
+                     dk[4 * e + 3]);
     }
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(512, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                   const __grid_constant__ CUtensorMap tmAcc, const BwdParams p) {
     using C = BwdTc<D>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = smem_u32(smem_raw);
-    const uint32_t tiles = (sbase + C::CTRL + 1023u) & ~1023u;
+    const uint32_t tiles = (sbase + 1023u) & ~1023u;
+    const uint32_t ctrl = tiles + C::TILES;
+    uint8_t *const ctrl_p = smem_raw + (ctrl - sbase);
     const uint32_t sK = tiles + C::OFF_K, sV = tiles + C::OFF_V, sQ0 = tiles + C::OFF_Q;
-    const uint32_t sdO0 = tiles + C::OFF_DO, sdS0 = tiles + C::OFF_DS, sStg = tiles + C::OFF_STG;
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem_raw + C::OFF_ABORT);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + C::OFF_TMEM_SLOT);
-    float *sLSE = reinterpret_cast<float *>(smem_raw + C::OFF_LSE);
-    float *sDLT = reinterpret_cast<float *>(smem_raw + C::OFF_DLT);
-    auto bar = [&](int i) -> uint32_t { return sbase + 8u * (uint32_t)i; };
+    const uint32_t sdO0 = tiles + C::OFF_DO, sdS = tiles + C::OFF_DS, sStg = tiles + C::OFF_STG;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl_p + C::OFF_ABORT);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ctrl_p + C::OFF_TMEM_SLOT);
+    float *sLSE = reinterpret_cast<float *>(ctrl_p + C::OFF_LSE);
+    float *sDLT = reinterpret_cast<float *>(ctrl_p + C::OFF_DLT);
+    auto bar = [&](int i) -> uint32_t { return ctrl + 8u * (uint32_t)i; };
+    if (tiles - sbase > C::SLACK) {
+        // the layout does not fit this shared-memory base: nothing is touched
+        if (threadIdx.x == 0) record_status(kStatusUnsupported);
+        return;
+    }
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     // work item: key tile n (heaviest = smallest n first), batch b, KV head, half h
@@ -229,27 +274,25 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(bar(C::B_Q_FULL + s), 33);
             mbar_init(bar(C::B_Q_EMPTY + s), 1);
         }
-        for (int s = 0; s < C::NSB; s++) {
-            mbar_init(bar(C::B_S_FULL + s), 1);
-            mbar_init(bar(C::B_DS_EMPTY + s), 1);
-            mbar_init(bar(C::B_PDS_FULL + s), 4);
-        }
+        mbar_init(bar(C::B_S_FULL), 1);
+        mbar_init(bar(C::B_DS_EMPTY), 1);
+        mbar_init(bar(C::B_P_FULL), 8);
+        mbar_init(bar(C::B_DS_FULL), 8);
         mbar_init(bar(C::B_DP_FULL), 1);
-        mbar_init(bar(C::B_DP_FREE), 4);
         mbar_init(bar(C::B_DQ_FULL), 1);
         mbar_init(bar(C::B_DQ_FREE), 4);
         mbar_init(bar(C::B_KDONE), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 8 && lane == 0) {
+    if (warp == C::W_LOAD && lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
         tma_prefetch_desc(&tmdO);
         tma_prefetch_desc(&tmAcc);
     }
-    if (warp == 9) {
+    if (warp == C::W_MMA) {
         tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -258,82 +301,84 @@ __global__ void __launch_bounds__(320, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 8) {
-        // ------------------------------------------------------------ producer
-        int issued = 0;
-        bool ok = true;
-        if (lane == 0) {
-            mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::TK);
-            for (int c = 0; c < C::NCB; c++) {
-                tma_load_3d(sK + c * C::CBK, &tmK, bar(C::B_KV), c * 64, k0, bkv);
-                tma_load_3d(sV + c * C::CBK, &tmV, bar(C::B_KV), c * 64, k0, bkv);
-            }
-        }
-        for (int i = 0; i < steps; i++) {
-            const int st = i % C::QST;
-            const uint32_t ph = (uint32_t)((i / C::QST) & 1);
-            const int g = i / nm, m = m_lo + i % nm;
-            const int bhq = b * p.Hq + hkv * G + g;
-            // this step's LSE and Delta into registers first: their global-load
-            // latency overlaps the wait for a free stage
-            float lv[C::BM / 32], dv[C::BM / 32];
-#pragma unroll
-            for (int r = 0; r < C::BM / 32; r++) {
-                const int q = m * C::BM + lane + 32 * r;
-                const size_t idx = (size_t)bhq * p.T + (size_t)min(q, p.T - 1);
-                lv[r] = q < p.T ? p.lse[idx] * kLog2e : INFINITY;
-                dv[r] = q < p.T ? p.delta[idx] * p.scale : 0.0f;
-            }
-            if (!mbar_wait_warp(bar(C::B_Q_EMPTY + st), ph ^ 1u, abort_flag)) {
-                ok = false;
-                break;
-            }
+    if (warp >= C::W_LOAD) {
+        setmaxnreg_dec<C::REG_CTRL>();
+        if (warp == C::W_LOAD) {
+            // -------------------------------------------------------- producer
+            int issued = 0;
+            bool ok = true;
             if (lane == 0) {
-                mbar_arrive_expect_tx(bar(C::B_Q_FULL + st), 2 * C::TQ);
+                mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::TK);
                 for (int c = 0; c < C::NCB; c++) {
-                    tma_load_3d(sQ0 + st * C::TQ + c * C::CBQ, &tmQ, bar(C::B_Q_FULL + st), c * 64, m * C::BM, bhq);
-                    tma_load_3d(sdO0 + st * C::TQ + c * C::CBQ, &tmdO, bar(C::B_Q_FULL + st), c * 64, m * C::BM,
-                                bhq);
+                    tma_load_3d(sK + c * C::CBK, &tmK, bar(C::B_KV), c * 64, k0, bkv);
+                    tma_load_3d(sV + c * C::CBK, &tmV, bar(C::B_KV), c * 64, k0, bkv);
                 }
             }
-            issued++;
+            for (int i = 0; i < steps; i++) {
+                const int st = i % C::QST;
+                const uint32_t ph = (uint32_t)((i / C::QST) & 1);
+                const int g = i / nm, m = m_lo + i % nm;
+                const int bhq = b * p.Hq + hkv * G + g;
+                // this step's LSE and Delta into registers first: their global-load
+                // latency overlaps the wait for a free stage
+                float lv[C::BM / 32], dv[C::BM / 32];
 #pragma unroll
-            for (int r = 0; r < C::BM / 32; r++) {
-                sLSE[st * C::BM + lane + 32 * r] = lv[r];
-                sDLT[st * C::BM + lane + 32 * r] = dv[r];
+                for (int r = 0; r < C::BM / 32; r++) {
+                    const int q = m * C::BM + lane + 32 * r;
+                    const size_t idx = (size_t)bhq * p.T + (size_t)min(q, p.T - 1);
+                    lv[r] = q < p.T ? p.lse[idx] * kLog2e : INFINITY;
+                    dv[r] = q < p.T ? p.delta[idx] * p.scale : 0.0f;
+                }
+                if (!mbar_wait_warp(bar(C::B_Q_EMPTY + st), ph ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar(C::B_Q_FULL + st), 2 * C::TQ);
+                    for (int c = 0; c < C::NCB; c++) {
+                        tma_load_3d(sQ0 + st * C::TQ + c * C::CBQ, &tmQ, bar(C::B_Q_FULL + st), c * 64, m * C::BM,
+                                    bhq);
+                        tma_load_3d(sdO0 + st * C::TQ + c * C::CBQ, &tmdO, bar(C::B_Q_FULL + st), c * 64,
+                                    m * C::BM, bhq);
+                    }
+                }
+                issued++;
+#pragma unroll
+                for (int r = 0; r < C::BM / 32; r++) {
+                    sLSE[st * C::BM + lane + 32 * r] = -lv[r];
+                    sDLT[st * C::BM + lane + 32 * r] = -dv[r];
+                }
+                mbar_arrive(bar(C::B_Q_FULL + st));
             }
-            mbar_arrive(bar(C::B_Q_FULL + st));
-        }
-        if (!ok && lane == 0) {
-            mbar_wait_drain(bar(C::B_KV), 0, 200000000ull);
-            for (int back = 1; back <= min(issued, C::QST); back++) {
-                const int L = issued - back;
-                mbar_wait_drain(bar(C::B_Q_FULL + L % C::QST), (uint32_t)((L / C::QST) & 1), 200000000ull);
+            if (!ok && lane == 0) {
+                mbar_wait_drain(bar(C::B_KV), 0, 200000000ull);
+                for (int back = 1; back <= min(issued, C::QST); back++) {
+                    const int L = issued - back;
+                    mbar_wait_drain(bar(C::B_Q_FULL + L % C::QST), (uint32_t)((L / C::QST) & 1), 200000000ull);
+                }
             }
-        }
-    } else if (warp == 9) {
-        // ---------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        } else if (warp == C::W_MMA && lane == 0) {
+            // ------------------------------------------------------ MMA issuer
             constexpr uint32_t ID_S = idesc_bf16_f32(128, C::BM, false, false);
             constexpr uint32_t ID_ACC = idesc_bf16_f32(128, C::DH, false, true);
             constexpr uint32_t ID_DQ =
                 C::DQT ? idesc_bf16_f32(128, C::BM, true, true) : idesc_bf16_f32(128, C::D, true, true);
             const uint32_t h_q = (uint32_t)h * (C::DH / 64) * C::CBQ;  // column-block offset of half h
             const uint32_t h_k = (uint32_t)h * (C::DH / 64) * C::CBK;
-            // S^T(j) = K Q(j)^T into S buffer j % NSB, over the full head dim
+            // S^T(j) = K Q(j)^T, over the full head dim
             auto issue_s = [&](int j) -> bool {
                 const int st = j % C::QST;
                 if (!mbar_wait(bar(C::B_Q_FULL + st), (uint32_t)((j / C::QST) & 1), abort_flag)) return false;
                 tc_fence_after();
                 const uint32_t sQ = sQ0 + st * C::TQ;
-                const uint32_t dS = tmem + C::col_s(j % C::NSB);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; kk++) {
                     const uint32_t ok_ = (kk >> 2) * C::CBK + (kk & 3) * 32;
                     const uint32_t oq = (kk >> 2) * C::CBQ + (kk & 3) * 32;
-                    mma_ss(dS, sdesc_sw128(sK + ok_, 16, 1024), sdesc_sw128(sQ + oq, 16, 1024), ID_S, kk > 0);
+                    mma_ss(tmem + C::COL_S, sdesc_sw128(sK + ok_, 16, 1024), sdesc_sw128(sQ + oq, 16, 1024), ID_S,
+                           kk > 0);
                 }
-                tc_commit(bar(C::B_S_FULL + j % C::NSB));
+                tc_commit(bar(C::B_S_FULL));
                 return true;
             };
             // dP^T(j) = V dO(j)^T (the stage of j is already known to be full)
@@ -343,38 +388,43 @@ __global__ void __launch_bounds__(320, 1)
                 for (int kk = 0; kk < D / 16; kk++) {
                     const uint32_t ok_ = (kk >> 2) * C::CBK + (kk & 3) * 32;
                     const uint32_t oq = (kk >> 2) * C::CBQ + (kk & 3) * 32;
-                    mma_ss(tmem + C::COL_DP, sdesc_sw128(sV + ok_, 16, 1024), sdesc_sw128(sdO + oq, 16, 1024), ID_S,
-                           kk > 0);
+                    mma_ss(tmem + C::COL_DP, sdesc_sw128(sV + ok_, 16, 1024), sdesc_sw128(sdO + oq, 16, 1024),
+                           ID_S, kk > 0);
                 }
                 tc_commit(bar(C::B_DP_FULL));
             };
             bool ok = mbar_wait(bar(C::B_KV), 0, abort_flag);
             if (ok && (ok = issue_s(0))) issue_dp(0);
             for (int i = 0; ok && i < steps; i++) {
-                const int st = i % C::QST, sb = i % C::NSB;
-                const uint32_t sQ = sQ0 + st * C::TQ, sdO = sdO0 + st * C::TQ, sdS = sdS0 + sb * C::TS;
+                const int st = i % C::QST;
+                const uint32_t sQ = sQ0 + st * C::TQ, sdO = sdO0 + st * C::TQ;
                 const bool more = i + 1 < steps;
-                if (C::NSB == 2 && more) {
-                    // next step's products while this step's P and dS are formed
-                    if (!(ok = issue_s(i + 1))) break;
-                    if (!(ok = mbar_wait(bar(C::B_DP_FREE), (uint32_t)(i & 1), abort_flag))) break;
-                    issue_dp(i + 1);
-                }
-                if (!(ok = mbar_wait(bar(C::B_PDS_FULL + sb), (uint32_t)((i / C::NSB) & 1), abort_flag))) break;
+                // dV += P^T dO, P^T from TMEM (phase A of step i)
+                if (!(ok = mbar_wait(bar(C::B_P_FULL), (uint32_t)(i & 1), abort_flag))) break;
                 tc_fence_after();
-                // dV += P^T dO (P^T from TMEM), dK += dS^T Q
 #pragma unroll
                 for (int kk = 0; kk < C::BM / 16; kk++)
-                    mma_ts(tmem + C::COL_DV, tmem + C::col_s(sb) + kk * 8,
-                           sdesc_sw128(sdO + h_q + kk * 2048, C::CBQ, 1024), ID_ACC, (i > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts(tmem + C::COL_DV, tmem + C::col_p(kk), sdesc_sw128(sdO + h_q + kk * 2048, C::CBQ, 1024),
+                           ID_ACC, (i > 0 || kk > 0) ? 1u : 0u);
+                // S^T(i + 1) over S^T(i) / P^T(i): phase A has read S^T(i), and dV(i)
+                // is ahead of it on the tensor cores. It runs while the compute warps
+                // form dS of step i. With a single Q/dO stage Q(i + 1) can only be
+                // loaded once dK(i) has read Q(i), so S^T(i + 1) then comes after dQ(i).
+                constexpr bool EARLY_S = C::QST > 1;
+                if (EARLY_S && more && !(ok = issue_s(i + 1))) break;
+                // dK += dS^T Q, dQ (phase B of step i)
+                if (!(ok = mbar_wait(bar(C::B_DS_FULL), (uint32_t)(i & 1), abort_flag))) break;
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < C::BM / 16; kk++) {
                     const uint32_t oa = (kk >> 2) * C::CBK + (kk & 3) * 32;
                     mma_ss(tmem + C::COL_DK, sdesc_sw128(sdS + oa, 16, 1024),
                            sdesc_sw128(sQ + h_q + kk * 2048, C::CBQ, 1024), ID_ACC, (i > 0 || kk > 0) ? 1u : 0u);
                 }
-                // dQ (the drain warps must have emptied the previous one)
-                if (i > 0) {
+                tc_commit(bar(C::B_Q_EMPTY + st));  // Q(i), dO(i) read by every product issued so far
+                // dQ (the drain warps must have emptied the previous one; in the
+                // aliased layout they did so before dP^T(i) was issued)
+                if (!C::DQ_ALIAS && i > 0) {
                     if (!(ok = mbar_wait(bar(C::B_DQ_FREE), (uint32_t)((i - 1) & 1), abort_flag))) break;
                     tc_fence_after();
                 }
@@ -389,94 +439,87 @@ __global__ void __launch_bounds__(320, 1)
                     }
                 }
                 tc_commit(bar(C::B_DQ_FULL));
-                tc_commit(bar(C::B_Q_EMPTY + st));
-                tc_commit(bar(C::B_DS_EMPTY + sb));
-                if (C::NSB == 1 && more) {
-                    if (!(ok = issue_s(i + 1))) break;
+                tc_commit(bar(C::B_DS_EMPTY));
+                if (!EARLY_S && more && !(ok = issue_s(i + 1))) break;
+                if (more) {
+                    // dP^T(i + 1): phase B has read dP^T(i); in the aliased layout it
+                    // also overwrites dQ^T(i), so wait for the drain warps
+                    if (C::DQ_ALIAS) {
+                        if (!(ok = mbar_wait(bar(C::B_DQ_FREE), (uint32_t)(i & 1), abort_flag))) break;
+                        tc_fence_after();
+                    }
                     issue_dp(i + 1);
                 }
             }
             tc_commit(bar(C::B_KDONE));
             if (!ok) mbar_wait_drain(bar(C::B_KDONE), 0, 200000000ull);
         }
-    } else if (warp < 4) {
-        // ------------------------------------------- compute (key rows, TMEM lanes)
-        const int kr = threadIdx.x;  // key row within the tile
+    } else if (warp < C::W_DRAIN) {
+        setmaxnreg_inc<C::REG_COMPUTE>();
+        // ------------------------------- compute (key rows = TMEM lanes, row halves)
+        const int hc = warp / 4;             // query-row half of the step
+        const int kr = (warp % 4) * 32 + lane;  // key row within the tile
         const int kj = k0 + kr;
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
         const bool cap = p.softcap > 0.0f;
         bool ok = true;
         for (int i = 0; i < steps; i++) {
-            const int st = i % C::QST, sb = i % C::NSB;
+            const int st = i % C::QST;
             const int m = m_lo + i % nm;
             const int qb = m * C::BM;
+            // phase A: S^T -> P^T (TMEM) and the dS factors g (registers)
             if (!(ok = mbar_wait_warp(bar(C::B_Q_FULL + st), (uint32_t)((i / C::QST) & 1), abort_flag))) break;
-            if (!(ok = mbar_wait_warp(bar(C::B_S_FULL + sb), (uint32_t)((i / C::NSB) & 1), abort_flag))) break;
-            if (!(ok = mbar_wait_warp(bar(C::B_DP_FULL), (uint32_t)(i & 1), abort_flag))) break;
+            if (!(ok = mbar_wait_warp(bar(C::B_S_FULL), (uint32_t)(i & 1), abort_flag))) break;
             tc_fence_after();
-            const uint32_t tS = tmem + lane_base + C::col_s(sb);
-            const uint32_t tP = tmem + lane_base + C::COL_DP;
-            const float *l2s = sLSE + st * C::BM;
-            const float *dls = sDLT + st * C::BM;
-            const uint32_t sdS = sdS0 + sb * C::TS;
+            const float *nls = sLSE + st * C::BM;
+            const float *nds = sDLT + st * C::BM;
             const bool mask = (k0 + C::BN - 1 > qb) || (W > 0 && k0 <= qb + C::BM - 1 - W);
-            if constexpr (C::PRELOAD) {
-                // the whole dP^T row (64 columns) into registers: dP^T is then free
-                // for the next step's product; S^T is read chunk by chunk
-                uint32_t d0[32], d1[32];
-                tmem_ld32(tP, d0);
-                tmem_ld32(tP + 32, d1);
-                tmem_ld_wait(d0);
-                tmem_ld_wait(d1);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(C::B_DP_FREE));
-                // dS^T buffer sb was last read by the dK/dQ products of step i - NSB
-                if (i >= C::NSB &&
-                    !(ok = mbar_wait_warp(bar(C::B_DS_EMPTY + sb), (uint32_t)(((i / C::NSB) - 1) & 1), abort_flag)))
-                    break;
-                {
-                    uint32_t sc[32];
-                    tmem_ld32(tS, sc);
-                    tmem_ld_wait(sc);
-                    bwd_chunk<D>(sc, d0, l2s, dls, p, cap, mask, kj, qb, W, 0, kr, tS, sdS);
+            float g[C::HALF / 32][32];
+#pragma unroll
+            for (int c = 0; c < C::HALF / 32; c++) {
+                const int c0 = hc * C::HALF + 32 * c;
+                uint32_t sc[32], pk[16];
+                tmem_ld32(tmem + lane_base + C::COL_S + c0, sc);
+                tmem_ld_wait(sc);
+                if (cap) {
+                    if (mask) bwd_p32<true, true>(sc, nls + c0, p, kj, qb + c0, W, pk, g[c]);
+                    else bwd_p32<true, false>(sc, nls + c0, p, kj, qb + c0, W, pk, g[c]);
+                } else {
+                    if (mask) bwd_p32<false, true>(sc, nls + c0, p, kj, qb + c0, W, pk, g[c]);
+                    else bwd_p32<false, false>(sc, nls + c0, p, kj, qb + c0, W, pk, g[c]);
                 }
-                {
-                    uint32_t sc[32];
-                    tmem_ld32(tS + 32, sc);
-                    tmem_ld_wait(sc);
-                    bwd_chunk<D>(sc, d1, l2s, dls, p, cap, mask, kj, qb + 32, W, 32, kr, tS, sdS);
-                }
-            } else {
-                if (i >= C::NSB &&
-                    !(ok = mbar_wait_warp(bar(C::B_DS_EMPTY + sb), (uint32_t)(((i / C::NSB) - 1) & 1), abort_flag)))
-                    break;
-#pragma unroll 1
-                for (int c0 = 0; c0 < C::BM; c0 += 32) {
-                    uint32_t sc[32], dc[32];
-                    tmem_ld32(tS + c0, sc);
-                    tmem_ld32(tP + c0, dc);
-                    tmem_ld_wait(sc);
-                    tmem_ld_wait(dc);
-                    bwd_chunk<D>(sc, dc, l2s, dls, p, cap, mask, kj, qb + c0, W, c0, kr, tS, sdS);
-                }
+                tmem_st16(tmem + lane_base + C::COL_S + hc * C::HALF + 16 * c, pk);
             }
             tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_P_FULL));
+            // phase B: dP^T -> dS^T (shared memory); the dS^T tile was last read
+            // by the dK/dQ products of step i - 1
+            if (!(ok = mbar_wait_warp(bar(C::B_DP_FULL), (uint32_t)(i & 1), abort_flag))) break;
+            if (i > 0 && !(ok = mbar_wait_warp(bar(C::B_DS_EMPTY), (uint32_t)((i - 1) & 1), abort_flag))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < C::HALF / 32; c++) {
+                const int c0 = hc * C::HALF + 32 * c;
+                uint32_t dc[32], dk[16];
+                tmem_ld32(tmem + lane_base + C::COL_DP + c0, dc);
+                tmem_ld_wait(dc);
+                bwd_ds32(dc, g[c], nds + c0, p, dk);
+                bwd_store_ds<D>(dk, c0, kr, sdS);
+            }
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                if constexpr (!C::PRELOAD) mbar_arrive(bar(C::B_DP_FREE));
-                mbar_arrive(bar(C::B_PDS_FULL + sb));
-            }
+            if (lane == 0) mbar_arrive(bar(C::B_DS_FULL));
         }
-        // epilogue: dV rows
+        // epilogue: dV rows, this warp's half of the columns
         if (ok) ok = mbar_wait_warp(bar(C::B_KDONE), 0, abort_flag);
         if (ok) {
             tc_fence_after();
             __nv_bfloat16 *row = p.dv + ((size_t)bkv * p.T + (size_t)min(kj, p.T - 1)) * D + h * C::DH;
 #pragma unroll 1
-            for (int c0 = 0; c0 < C::DH; c0 += 32) {
+            for (int c0 = hc * (C::DH / 2); c0 < (hc + 1) * (C::DH / 2); c0 += 32) {
                 uint32_t o[32];
                 tmem_ld32(tmem + lane_base + C::COL_DV + c0, o);
                 tmem_ld_wait(o);
@@ -491,25 +534,31 @@ __global__ void __launch_bounds__(320, 1)
             }
         }
     } else {
-        // ------------------------------------ dQ drain (warps 4..7), dK epilogue
-        const int t = threadIdx.x - 128;  // TMEM lane of this thread
-        const uint32_t lane_base = (uint32_t)((warp - 4) * 32) << 16;
+        setmaxnreg_inc<C::REG_DRAIN>();
+        // -------------------------------- dQ drain (warps 8..11), dK epilogue
+        const int t = threadIdx.x - 32 * C::W_DRAIN;  // TMEM lane of this thread
+        const uint32_t lane_base = (uint32_t)((warp - C::W_DRAIN) * 32) << 16;
         bool ok = true;
         for (int i = 0; i < steps; i++) {
             const int g = i / nm, m = m_lo + i % nm;
             const int bhq = b * p.Hq + hkv * G + g;
             if (!(ok = mbar_wait_warp(bar(C::B_DQ_FULL), (uint32_t)(i & 1), abort_flag))) break;
             tc_fence_after();
-            // two 32-column TMEM loads: this thread's 64 dQ values
-            uint32_t v0[32], v1[32];
-            tmem_ld32(tmem + lane_base + C::COL_DQ, v0);
-            tmem_ld32(tmem + lane_base + C::COL_DQ + 32, v1);
-            tmem_ld_wait(v0);
-            tmem_ld_wait(v1);
+            // this thread's dQ values: a query row's DH columns, or (transposed)
+            // a head-dim column's BM rows, in 32-column TMEM loads
+            constexpr int NQC = (C::DQT ? C::BM : C::DH) / 32;
+            uint32_t v[NQC][32];
+#pragma unroll
+            for (int j = 0; j < NQC; j++) tmem_ld32(tmem + lane_base + C::COL_DQ + 32 * j, v[j]);
+#pragma unroll
+            for (int j = 0; j < NQC; j++) tmem_ld_wait(v[j]);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(C::B_DQ_FREE));
             if constexpr (C::BULK_DQ) {
+                static_assert(!C::BULK_DQ || NQC == 2, "staging covers 64 dQ values a thread");
+                const uint32_t(&v0)[32] = v[0];
+                const uint32_t(&v1)[32] = v[1 % NQC];
                 // Staging tile [BM rows][DH cols] f32, stored as DH/32 column blocks of
                 // [BM][32] with the 128-byte swizzle (16-byte chunk ^ row % 8), the
                 // layout of a TMA box {32, BM, 1}. The tile is reused once the reduce
@@ -517,30 +566,14 @@ __global__ void __launch_bounds__(320, 1)
                 const uint32_t stg = sStg + (uint32_t)(i % C::NSTG) * C::STG;
                 if (t == 0) bulk_wait_read<C::NSTG - 1>();
                 named_barrier_sync(1, 128);
-                if constexpr (C::DQT) {
-                    // thread t = head-dim column t of this half; v = 64 query rows
-                    const uint32_t cb = (uint32_t)t >> 5, ch = ((uint32_t)t & 31u) >> 2, w4 = ((uint32_t)t & 3u) << 2;
-                    const uint32_t base = stg + cb * (uint32_t)(C::BM * 128) + w4;
+                // thread t = query row t; v = the 64 head-dim values of that row
+                const uint32_t row = stg + (uint32_t)t * 128u;
 #pragma unroll
-                    for (int c = 0; c < 32; c++) {
-                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(base + (uint32_t)c * 128u + ((ch ^ ((uint32_t)c & 7u)) << 4)),
-                                     "r"(v0[c]) : "memory");
-                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(base + (uint32_t)(c + 32) * 128u +
-                                                                     ((ch ^ ((uint32_t)(c + 32) & 7u)) << 4)),
-                                     "r"(v1[c]) : "memory");
-                    }
-                } else {
-                    // thread t = query row t; v = the 64 head-dim values of that row
-                    const uint32_t row = stg + (uint32_t)t * 128u;
-#pragma unroll
-                    for (int c4 = 0; c4 < 8; c4++) {
-                        const uint32_t sw = (((uint32_t)c4 ^ ((uint32_t)t & 7u)) << 4);
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + sw), "r"(v0[4 * c4]),
-                                     "r"(v0[4 * c4 + 1]), "r"(v0[4 * c4 + 2]), "r"(v0[4 * c4 + 3]) : "memory");
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + (uint32_t)(C::BM * 128) + sw),
-                                     "r"(v1[4 * c4]), "r"(v1[4 * c4 + 1]), "r"(v1[4 * c4 + 2]), "r"(v1[4 * c4 + 3])
-                                     : "memory");
-                    }
+                for (int c4 = 0; c4 < 8; c4++) {
+                    const uint32_t sw = (((uint32_t)c4 ^ ((uint32_t)t & 7u)) << 4);
+                    st_shared_v4(row + sw, v0[4 * c4], v0[4 * c4 + 1], v0[4 * c4 + 2], v0[4 * c4 + 3]);
+                    st_shared_v4(row + (uint32_t)(C::BM * 128) + sw, v1[4 * c4], v1[4 * c4 + 1], v1[4 * c4 + 2],
+                                 v1[4 * c4 + 3]);
                 }
                 fence_proxy_async_smem();
                 named_barrier_sync(1, 128);
@@ -552,12 +585,15 @@ __global__ void __launch_bounds__(320, 1)
                     bulk_commit();
                 }
             } else {
-                // head dim 256: lane = head-dim column h*DH + t, 64 query rows
+                // lane = head-dim column h*DH + t, BM query rows: each warp-wide
+                // reduction covers 32 consecutive floats of one dQ row
+                static_assert(C::BULK_DQ || C::DQT, "per-element reduction expects the transposed dQ");
+
                 float *base = p.dq_acc + ((size_t)bhq * p.Tpad + (size_t)m * C::BM) * D + h * C::DH + t;
 #pragma unroll
-                for (int c = 0; c < 32; c++) {
-                    atomicAdd(base + (size_t)c * D, __uint_as_float(v0[c]));
-                    atomicAdd(base + (size_t)(c + 32) * D, __uint_as_float(v1[c]));
+                for (int j = 0; j < NQC; j++) {
+#pragma unroll
+                    for (int c = 0; c < 32; c++) atomicAdd(base + (size_t)(32 * j + c) * D, __uint_as_float(v[j][c]));
                 }
             }
         }
@@ -588,7 +624,7 @@ __global__ void __launch_bounds__(320, 1)
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == C::W_MMA) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
