@@ -31,6 +31,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+L2_BYTES = 126 * 1000 * 1000
 METRIC = "causal attention fwd+bwd TFLOPS on 1 B200 and % of dense BF16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -225,8 +226,17 @@ def run_ours(args, w):
     ws = torch.empty(nws, dtype=torch.uint8, device=dev)
     sc, W, C = w.sm_scale, w.window, w.softcap
     sh = stream.cuda_stream
+    # Timing hygiene: when the per-step working set is not well above the L2
+    # size, every step first overwrites a 256 MB scratch buffer (outside the
+    # timed kernels) so that no step starts with the previous one's data in L2.
+    working_set = sum(x.numel() * x.element_size() for x in (qd, kd, vd, o, lse, dOd, dq, dk, dv, ws))
+    flush = working_set < 2 * L2_BYTES
+    scratch = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush else None
 
     def step(ev=None):
+        if flush:
+            with torch.cuda.stream(stream):
+                scratch.fill_(1)
         if ev:
             ev[0].record(stream)
         s = fa.forge_attn_fwd(qd, kd, vd, o, lse, B, Hq, Hkv, T, D, sc, W, C, dt, sh)
@@ -272,6 +282,9 @@ def run_ours(args, w):
     if st != fa.FORGE_OK:
         raise fa.ForgeError(st, "timed run")
     ms_local = start.elapsed_time(end)
+    if flush:
+        # the flushes sit between the timed kernels: time the kernels only
+        ms_local = sum(e[0].elapsed_time(e[4]) for e in evs)
     ms = max_over_ranks(ms_local, world, dev)
     per = {"fwd": [], "bwd_preprocess": [], "bwd_main": [], "bwd_finalize": []}
     for e in evs:
@@ -351,8 +364,10 @@ def run_ours(args, w):
                    "parallelism": f"replicas x{world} (independent batches, no collective)",
                    "flops_per_step_per_gpu": fl_f + fl_b,
                    "flop_count": "only causal/in-window pairs; fwd 4*D*pairs, bwd 10*D*pairs",
-                   "l2": "not flushed: per-step working set (q,k,v,o,dO,dq,dk,dv,lse + f32 dq accumulator) "
-                         "exceeds the 126 MB L2"},
+                   "l2": ("flushed: a 256 MB buffer is written before each step (working set "
+                          f"{working_set / 1e6:.0f} MB); step time = sum of the kernels' CUDA-event times") if flush
+                         else (f"not flushed: per-step working set (q,k,v,o,dO,dq,dk,dv,lse + workspace) "
+                               f"{working_set / 1e6:.0f} MB exceeds twice the 126 MB L2")},
         "pct_of_bf16_peak": round(100.0 * tflops / world / peak, 2),
         "kernels_ms": {k_: round(v_, 4) for k_, v_ in avg.items()},
         "roofline": {"kernel": kname, "bound": "tensor", "achieved": round(achieved, 2), "peak": peak,

@@ -159,8 +159,8 @@ __device__ __forceinline__ void bwd_p32(const uint32_t (&s)[32], const float *nl
                                            e ? f2_make(a.z, a.w) : f2_make(a.x, a.y));
                 float y0, y1;
                 f2_split(y2, y0, y1);
-                // a quarter of the exponentials on the FMA pipe
-                const bool emu = ((c + e) & 6) == 6;
+                // one pair in eight of the exponentials on the FMA pipe
+                const bool emu = ((c + e) & 14) == 14;
                 g[c + e] = emu ? exp2_poly(y0) : ex2_approx(y0);
                 g[c + e + 1] = emu ? exp2_poly(y1) : ex2_approx(y1);
                 pk[(c + e) >> 1] = pack_bf16x2(g[c + e], g[c + e + 1]);
