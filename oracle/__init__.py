@@ -7,7 +7,11 @@ imports it nor links it, and the two share no code.
 Parity pins (tests/test_oracle.py): torch SDPA in f64 (causal, band mask, GQA by
 repeat_interleave), torch autograd of SDPA, brute-force softmax Jacobian on tiny
 shapes, central finite differences, and the invariants and closed forms of the
-definition. No function here is left unpinned.
+definition. The sink and max-logit extensions are pinned by: sink = -inf being the
+plain softmax bit for bit; a sink being an extra zero-value key at position 0
+(checked through the pinned plain oracle, forward, dq/dk/dv and dsink); a one-key
+closed form; central differences of dsink; a hand-worked max-logit example. No
+function here is left unpinned.
 
 Every function takes and returns numpy float64 arrays in [B, H, T, D] layout.
 """
@@ -32,6 +36,8 @@ def _load():
         i = ctypes.c_int
         d = ctypes.c_double
         lib.oracle_attn_fwd.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i, d, i, d]
+        lib.oracle_attn_fwd_ext.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, d, i, d]
+        lib.oracle_attn_bwd_ext.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, d, i, d, i]
         lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, d, i, d, i]
         lib.oracle_round.argtypes = [dp, dp, ctypes.c_long, i]
         lib.oracle_attn_probs.argtypes = [dp, dp, dp, i, i, i, i, i, d, i, d]
@@ -101,6 +107,43 @@ def attn_bwd(q, k, v, dO, scale: float, window: int = 0, softcap: float = 0.0, o
                             _ptr(delta), _ptr(lse), B, Hq, Hkv, T, D, float(scale), int(window),
                             float(softcap), _ROUND[o_round])
     return dq, dk, dv, delta, lse
+
+
+def _ptr_or_null(a):
+    return None if a is None else _ptr(a)
+
+
+def attn_fwd_ext(q, k, v, scale: float, window: int = 0, softcap: float = 0.0, sink=None):
+    """Forward with an optional per-head sink logit sink [Hq]. Returns (o, lse,
+    max_logit [B, Hq]); max_logit is the per-(b, hq) maximum of the scores the
+    softmax sees over the allowed pairs (the sink not included)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Hkv, T, D = _dims(q, k)
+    sk = None if sink is None else _f64(sink).reshape(Hq)
+    o = np.empty_like(q)
+    lse = np.empty((B, Hq, T), dtype=np.float64)
+    ml = np.empty((B, Hq), dtype=np.float64)
+    _load().oracle_attn_fwd_ext(_ptr(q), _ptr(k), _ptr(v), _ptr_or_null(sk), _ptr(o), _ptr(lse), _ptr(ml),
+                                B, Hq, Hkv, T, D, float(scale), int(window), float(softcap))
+    return o, lse, ml
+
+
+def attn_bwd_ext(q, k, v, dO, scale: float, window: int = 0, softcap: float = 0.0, sink=None, o_round=None):
+    """Backward with an optional per-head sink logit sink [Hq]. Returns (dq, dk,
+    dv, dsink [Hq] (zeros without a sink), delta, lse)."""
+    q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
+    B, Hq, Hkv, T, D = _dims(q, k)
+    sk = None if sink is None else _f64(sink).reshape(Hq)
+    dq = np.empty_like(q)
+    dk = np.empty_like(k)
+    dv = np.empty_like(v)
+    dsink = np.empty((Hq,), dtype=np.float64)
+    delta = np.empty((B, Hq, T), dtype=np.float64)
+    lse = np.empty((B, Hq, T), dtype=np.float64)
+    _load().oracle_attn_bwd_ext(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr_or_null(sk), _ptr(dq), _ptr(dk),
+                                _ptr(dv), _ptr(dsink), _ptr(delta), _ptr(lse), B, Hq, Hkv, T, D, float(scale),
+                                int(window), float(softcap), _ROUND[o_round])
+    return dq, dk, dv, dsink, delta, lse
 
 
 def attn_probs(q, k, scale: float, window: int = 0, softcap: float = 0.0):

@@ -24,6 +24,17 @@
  *    "Vague 3" item 12 (the flash kernel keeps the per-row max).
  *  - Reading: the scale multiplies q.k before the cap: s = cap*tanh(scale*q.k/cap).
  *  - Reading: LSE is the natural-log log-sum-exp of the (capped) scores of a row.
+ *  - attention sinks: a learned logit per head that joins the softmax
+ *    denominator and has no value vector ("biais par tête dans le dénominateur
+ *    softmax": ARCHITECTURES.md family table, GPT-OSS row; "Vague 2" item 10,
+ *    which seeds the online softmax's (max, sum) with it; SMALL_MODELS_RESEARCH.md
+ *    section 2.4). Readings: one logit sigma_h per query head, shared by every
+ *    batch entry and row, in the units of the scores the softmax sees (it is
+ *    not capped); LSE includes it; its gradient is -sum_i P_i,sink Delta_i.
+ *  - max logit: the per-head maximum attention logit that QK-Clip monitors
+ *    (ARCHITECTURES.md "Vague 3" item 12; family table, Kimi K2 row). Reading:
+ *    per (batch, query head), the maximum over the allowed (i, j) of the score
+ *    the softmax sees (after scale and cap), the sink not included.
  *
  * Layouts: q, o, dO, dq are [B][Hq][T][D]; k, v, dk, dv are [B][Hkv][T][D];
  * lse and delta are [B][Hq][T]; all row-major, f64.
@@ -88,16 +99,21 @@ void oracle_round(const double *x, double *y, long n, int mode) {
 
 /*
  * Probabilities of one query row: p[j] for j in [lo, i], returns the LSE.
- * p[j] = exp(s_j - m) / sum_k exp(s_k - m), m = max_k s_k (k allowed).
+ * p[j] = exp(s_j - m) / (exp(sink - m) + sum_k exp(s_k - m)), m = the max of the
+ * allowed s_k and the sink (sink = -inf: no sink; then exp(sink - m) = 0 and the
+ * arithmetic is that of the plain softmax). *smax (may be NULL) receives the
+ * max of the s_k alone.
  */
 static double row_probs(const double *qi, const double *K, long i, long lo, int D,
-                        double scale, double softcap, double *p) {
+                        double scale, double softcap, double sink, double *p, double *smax) {
     double m = -INFINITY;
     for (long j = lo; j <= i; j++) {
         p[j] = capped(raw_score(qi, K + j * D, D, scale), softcap);
         if (p[j] > m) m = p[j];
     }
-    double l = 0.0;
+    if (smax) *smax = m;
+    if (sink > m) m = sink;
+    double l = exp(sink - m);
     for (long j = lo; j <= i; j++) {
         p[j] = exp(p[j] - m);
         l += p[j];
@@ -106,11 +122,17 @@ static double row_probs(const double *qi, const double *K, long i, long lo, int 
     return m + log(l);
 }
 
-/* Forward: O_i = sum_j P_ij V_j, LSE_i = log sum_j exp(s_ij). */
-void oracle_attn_fwd(const double *q, const double *k, const double *v, double *o, double *lse,
-                     int B, int Hq, int Hkv, int T, int D, double scale, int window,
-                     double softcap) {
+static double sink_of(const double *sink, int hq) { return sink ? sink[hq] : -INFINITY; }
+
+/*
+ * Forward: O_i = sum_j P_ij V_j, LSE_i = log (exp(sigma) + sum_j exp(s_ij)).
+ * sink [Hq] may be NULL (no sink); max_logit [B][Hq] may be NULL.
+ */
+void oracle_attn_fwd_ext(const double *q, const double *k, const double *v, const double *sink,
+                         double *o, double *lse, double *max_logit, int B, int Hq, int Hkv, int T,
+                         int D, double scale, int window, double softcap) {
     const int G = Hq / Hkv;
+    double *rowmax = (double *)malloc(sizeof(double) * (size_t)B * Hq * T);
 #pragma omp parallel
     {
         double *p = (double *)malloc(sizeof(double) * (size_t)T);
@@ -124,7 +146,8 @@ void oracle_attn_fwd(const double *q, const double *k, const double *v, double *
                     const double *K = k + (size_t)(b * Hkv + hkv) * T * D;
                     const double *V = v + (size_t)(b * Hkv + hkv) * T * D;
                     const long lo = first_key(i, window);
-                    lse[qrow] = row_probs(qi, K, i, lo, D, scale, softcap, p);
+                    lse[qrow] = row_probs(qi, K, i, lo, D, scale, softcap, sink_of(sink, hq), p,
+                                          rowmax + qrow);
                     double *oi = o + qrow * D;
                     for (int d = 0; d < D; d++) oi[d] = 0.0;
                     for (long j = lo; j <= i; j++)
@@ -132,6 +155,21 @@ void oracle_attn_fwd(const double *q, const double *k, const double *v, double *
                 }
         free(p);
     }
+    if (max_logit)
+        for (long bh = 0; bh < (long)B * Hq; bh++) {
+            double m = -INFINITY;
+            for (long i = 0; i < T; i++)
+                if (rowmax[bh * T + i] > m) m = rowmax[bh * T + i];
+            max_logit[bh] = m;
+        }
+    free(rowmax);
+}
+
+/* Forward without sink or max logit. */
+void oracle_attn_fwd(const double *q, const double *k, const double *v, double *o, double *lse,
+                     int B, int Hq, int Hkv, int T, int D, double scale, int window,
+                     double softcap) {
+    oracle_attn_fwd_ext(q, k, v, NULL, o, lse, NULL, B, Hq, Hkv, T, D, scale, window, softcap);
 }
 
 /*
@@ -146,16 +184,21 @@ void oracle_attn_fwd(const double *q, const double *k, const double *v, double *
  * P_ij = exp(s_ij - LSE_i), which is the same softmax entry.
  * delta (may be NULL) receives Delta, lse_out (may be NULL) receives LSE.
  *
+ * With a sink (sink [Hq] non-NULL) P and LSE include it, and dsink [Hq] (may be
+ * NULL) receives d/d sigma_h = -sum over batches and rows of P_i,sink Delta_i,
+ * P_i,sink = exp(sigma_h - LSE_i): the sink's column of the softmax Jacobian,
+ * whose upstream dP is 0 (it has no value vector).
+ *
  * o_round selects how Delta is formed. 0: Delta_i = sum_j P_ij dP_ij (the
  * definition). 1 or 2: Delta_i = sum_d dO_id * o_id with o_i = sum_j P_ij V_j
  * rounded to the storage type of the call (1 = f32, 2 = bf16): the backward's
  * first step takes rowsum(dO * O) of the O the forward returned, and in a bf16
  * call that O is bf16. With exact O both forms are equal (sum_j P_ij = 1).
  */
-void oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dO,
-                     double *dq, double *dk, double *dv, double *delta, double *lse_out,
-                     int B, int Hq, int Hkv, int T, int D, double scale, int window,
-                     double softcap, int o_round) {
+void oracle_attn_bwd_ext(const double *q, const double *k, const double *v, const double *dO,
+                         const double *sink, double *dq, double *dk, double *dv, double *dsink,
+                         double *delta, double *lse_out, int B, int Hq, int Hkv, int T, int D,
+                         double scale, int window, double softcap, int o_round) {
     const int G = Hq / Hkv;
     const size_t nrows = (size_t)B * Hq * T;
     double *lse = (double *)malloc(sizeof(double) * nrows);
@@ -178,7 +221,7 @@ void oracle_attn_bwd(const double *q, const double *k, const double *v, const do
                     const double *K = k + (size_t)(b * Hkv + hkv) * T * D;
                     const double *V = v + (size_t)(b * Hkv + hkv) * T * D;
                     const long lo = first_key(i, window);
-                    lse[qrow] = row_probs(qi, K, i, lo, D, scale, softcap, p);
+                    lse[qrow] = row_probs(qi, K, i, lo, D, scale, softcap, sink_of(sink, hq), p, NULL);
                     double dl = 0.0;
                     for (long j = lo; j <= i; j++) {
                         dp[j] = dot(doi, V + j * D, D);
@@ -237,10 +280,31 @@ void oracle_attn_bwd(const double *q, const double *k, const double *v, const do
                 }
             }
 
+    if (dsink) {
+        for (int hq = 0; hq < Hq; hq++) {
+            double acc = 0.0;
+            if (sink)
+                for (int b = 0; b < B; b++)
+                    for (int i = 0; i < T; i++) {
+                        const size_t qrow = ((size_t)(b * Hq + hq) * T + i);
+                        acc -= exp(sink[hq] - lse[qrow]) * dlt[qrow];
+                    }
+            dsink[hq] = acc;
+        }
+    }
     if (delta) memcpy(delta, dlt, sizeof(double) * nrows);
     if (lse_out) memcpy(lse_out, lse, sizeof(double) * nrows);
     free(lse);
     free(dlt);
+}
+
+/* Backward without sink. */
+void oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dO,
+                     double *dq, double *dk, double *dv, double *delta, double *lse_out,
+                     int B, int Hq, int Hkv, int T, int D, double scale, int window,
+                     double softcap, int o_round) {
+    oracle_attn_bwd_ext(q, k, v, dO, NULL, dq, dk, dv, NULL, delta, lse_out, B, Hq, Hkv, T, D,
+                        scale, window, softcap, o_round);
 }
 
 /* Full probability matrix P [B][Hq][T][T] (zeros where masked); small sizes only. */
@@ -255,7 +319,7 @@ void oracle_attn_probs(const double *q, const double *k, double *P, int B, int H
                 double *pi = P + qrow * T;
                 for (int j = 0; j < T; j++) pi[j] = 0.0;
                 row_probs(q + qrow * D, k + (size_t)(b * Hkv + hkv) * T * D, i,
-                          first_key(i, window), D, scale, softcap, pi);
+                          first_key(i, window), D, scale, softcap, -INFINITY, pi, NULL);
             }
 }
 

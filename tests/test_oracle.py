@@ -380,3 +380,128 @@ def test_delta_from_rounded_output(dtype):
         cg = (1 - np.tanh(S / C) ** 2) if C else 1.0
         U = np.einsum("bhij,bhjd->bhid", P * cg, kr)
         np.testing.assert_allclose(rd[0] - ex[0], -0.5 * (rd[3] - ex[3])[..., None] * U, rtol=1e-9, atol=1e-13)
+
+
+# ---------------------------------------------------------------- attention sinks
+# A sink is a learned logit per query head in the softmax denominator with no
+# value vector (ARCHITECTURES.md family table, GPT-OSS row; "Vague 2" item 10;
+# SMALL_MODELS_RESEARCH.md section 2.4).
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def test_sink_minus_infinity_is_plain_softmax_bitwise():
+    q, k, v, dO = _rand((2, 4, 9, 8), 1), _rand((2, 2, 9, 8), 2), _rand((2, 2, 9, 8), 3), _rand((2, 4, 9, 8), 4)
+    sink = np.full(4, -np.inf)
+    o, lse = oracle.attn_fwd(q, k, v, 0.3, 4, 2.0)
+    o2, lse2, _ = oracle.attn_fwd_ext(q, k, v, 0.3, 4, 2.0, sink=sink)
+    assert np.array_equal(o, o2) and np.array_equal(lse, lse2)
+    g = oracle.attn_bwd(q, k, v, dO, 0.3, 4, 2.0)
+    g2 = oracle.attn_bwd_ext(q, k, v, dO, 0.3, 4, 2.0, sink=sink)
+    for a, b in zip(g[:3] + g[3:], g2[:3] + g2[4:]):
+        assert np.array_equal(a, b)
+    assert np.all(g2[3] == 0.0)
+
+
+def _augment_with_sink_key(q, k, v, dO, sink, scale, c=0.75):
+    """The sink as a real key: one extra feature (query h: sink_h / (scale * c),
+    keys: c for a new key at position 0, 0 elsewhere) and a zero value vector, so
+    every query's score with the new key is sink_h and it adds nothing to O."""
+    B, Hq, T, D = q.shape
+    Hkv = k.shape[1]
+    qa = np.zeros((B, Hq, T + 1, D + 1)); ka = np.zeros((B, Hkv, T + 1, D + 1))
+    va = np.zeros((B, Hkv, T + 1, D + 1)); doa = np.zeros((B, Hq, T + 1, D + 1))
+    qa[:, :, 1:, :D] = q
+    qa[:, :, :, D] = (sink / (scale * c))[None, :, None]
+    ka[:, :, 1:, :D] = k
+    ka[:, :, 0, D] = c
+    va[:, :, 1:, :D] = v   # the new key's value and every value's extra feature are 0
+    doa[:, :, 1:, :D] = dO  # the new position 0 is not a real query: no upstream gradient
+    return qa, ka, va, doa
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(2, 2), (4, 2)])
+def test_sink_equals_an_extra_zero_value_key(Hq, Hkv):
+    B, T, D, scale = 2, 11, 6, 0.4
+    q, k, v, dO = _rand((B, Hq, T, D), 5), _rand((B, Hkv, T, D), 6), _rand((B, Hkv, T, D), 7), _rand((B, Hq, T, D), 8)
+    sink = np.linspace(-1.0, 1.5, Hq)
+    o, lse, _ = oracle.attn_fwd_ext(q, k, v, scale, 0, 0.0, sink=sink)
+    qa, ka, va, doa = _augment_with_sink_key(q, k, v, dO, sink, scale)
+    oa, lsea = oracle.attn_fwd(qa, ka, va, scale)
+    np.testing.assert_allclose(o, oa[:, :, 1:, :D], rtol=0, atol=1e-12)
+    assert np.all(oa[:, :, 1:, D] == 0.0)
+    np.testing.assert_allclose(lse, lsea[:, :, 1:], rtol=0, atol=1e-12)
+    dq, dk, dv, dsink, _, _ = oracle.attn_bwd_ext(q, k, v, dO, scale, 0, 0.0, sink=sink)
+    dqa, dka, dva, _, _ = oracle.attn_bwd(qa, ka, va, doa, scale)
+    np.testing.assert_allclose(dq, dqa[:, :, 1:, :D], rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dk, dka[:, :, 1:, :D], rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dv, dva[:, :, 1:, :D], rtol=0, atol=1e-11)
+    # d/d sink_h: through the extra query feature, d s_sink / d qa_extra = scale * c
+    np.testing.assert_allclose(dsink, dqa[:, :, 1:, D].sum(axis=(0, 2)) / (scale * 0.75), rtol=0, atol=1e-11)
+
+
+def test_sink_closed_form_single_key():
+    # T = 1: s = scale * q.k = 0.5 * 2 = 1; P(key) = e / (e + e^sigma), sigma = ln 3
+    q = np.array([1.0, 0.0]).reshape(1, 1, 1, 2)
+    k = np.array([2.0, 0.0]).reshape(1, 1, 1, 2)
+    v = np.array([4.0, -2.0]).reshape(1, 1, 1, 2)
+    o, lse, ml = oracle.attn_fwd_ext(q, k, v, 0.5, sink=np.array([math.log(3.0)]))
+    p = math.e / (math.e + 3.0)
+    np.testing.assert_allclose(o.ravel(), [4.0 * p, -2.0 * p], rtol=1e-15)
+    np.testing.assert_allclose(lse.ravel(), [math.log(math.e + 3.0)], rtol=1e-15)
+    assert ml.ravel()[0] == 1.0
+    # dO = (1, 0): loss = O_0 = 4 p(sigma); d/dsigma = -4 p (1 - p)
+    dO = np.array([1.0, 0.0]).reshape(1, 1, 1, 2)
+    _, _, _, dsink, _, _ = oracle.attn_bwd_ext(q, k, v, dO, 0.5, sink=np.array([math.log(3.0)]))
+    np.testing.assert_allclose(dsink, [-4.0 * p * (1.0 - p)], rtol=1e-13)
+
+
+@pytest.mark.parametrize("W,C", [(0, 0.0), (3, 0.0), (0, 1.5), (4, 2.0)])
+def test_dsink_central_finite_differences(W, C):
+    B, Hq, Hkv, T, D, scale = 2, 4, 2, 10, 5, 0.6
+    q, k, v, dO = _rand((B, Hq, T, D), 9), _rand((B, Hkv, T, D), 10), _rand((B, Hkv, T, D), 11), _rand((B, Hq, T, D), 12)
+    sink = np.array([0.2, -0.7, 1.1, 0.0])
+    _, _, _, dsink, _, _ = oracle.attn_bwd_ext(q, k, v, dO, scale, W, C, sink=sink)
+    h = 1e-6
+    for i in range(Hq):
+        sp, sm = sink.copy(), sink.copy()
+        sp[i] += h
+        sm[i] -= h
+        lp = np.sum(oracle.attn_fwd_ext(q, k, v, scale, W, C, sink=sp)[0] * dO)
+        lm = np.sum(oracle.attn_fwd_ext(q, k, v, scale, W, C, sink=sm)[0] * dO)
+        np.testing.assert_allclose(dsink[i], (lp - lm) / (2 * h), rtol=1e-6, atol=1e-9)
+
+
+# ---------------------------------------------------------------- max logit
+# The per-head maximum attention logit that QK-Clip monitors (ARCHITECTURES.md
+# "Vague 3" item 12; family table, Kimi K2 row).
+
+def test_max_logit_hand_example():
+    # D = 1, scale 1: q = (1, 2, -1), k = (3, -1, 0.5). Allowed scores (i, j):
+    # causal (0,0)=3 (1,0)=6 (1,1)=-2 (2,0)=-3 (2,1)=1 (2,2)=-0.5 -> max 6;
+    # window 1 keeps the diagonal 3, -2, -0.5 -> max 3; a cap of 2 maps them to
+    # 2 tanh(6/2) and 2 tanh(3/2).
+    q = np.array([1.0, 2.0, -1.0]).reshape(1, 1, 3, 1)
+    k = np.array([3.0, -1.0, 0.5]).reshape(1, 1, 3, 1)
+    v = np.ones((1, 1, 3, 1))
+    assert oracle.attn_fwd_ext(q, k, v, 1.0)[2].ravel()[0] == 6.0
+    assert oracle.attn_fwd_ext(q, k, v, 1.0, 1)[2].ravel()[0] == 3.0
+    np.testing.assert_allclose(oracle.attn_fwd_ext(q, k, v, 1.0, 0, 2.0)[2].ravel()[0], 2 * math.tanh(3.0), rtol=1e-15)
+    np.testing.assert_allclose(oracle.attn_fwd_ext(q, k, v, 1.0, 1, 2.0)[2].ravel()[0], 2 * math.tanh(1.5), rtol=1e-15)
+    # the sink is not a logit of the max
+    assert oracle.attn_fwd_ext(q, k, v, 1.0, sink=np.array([50.0]))[2].ravel()[0] == 6.0
+
+
+def test_max_logit_is_attained_by_an_allowed_pair_and_bounds_the_rest():
+    B, Hq, Hkv, T, D, scale, W = 2, 4, 2, 13, 6, 0.5, 5
+    q, k, v = _rand((B, Hq, T, D), 13), _rand((B, Hkv, T, D), 14), _rand((B, Hkv, T, D), 15)
+    ml = oracle.attn_fwd_ext(q, k, v, scale, W)[2]
+    kk = np.repeat(k, Hq // Hkv, axis=1)
+    s = scale * np.einsum("bhid,bhjd->bhij", q, kk)
+    i, j = np.arange(T)[:, None], np.arange(T)[None, :]
+    allowed = (j <= i) & (j > i - W)
+    s_allowed = np.where(allowed, s, -np.inf)
+    assert np.all(s_allowed <= ml[:, :, None, None] + 0.0)
+    hits = np.isclose(s_allowed, ml[:, :, None, None], rtol=0, atol=1e-12) & allowed
+    assert np.all(hits.any(axis=(2, 3)))
