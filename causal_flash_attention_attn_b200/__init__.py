@@ -19,7 +19,7 @@ __all__ = [
     "FORGE_OK", "FORGE_ERR_INVALID_ARG", "FORGE_ERR_UNSUPPORTED", "FORGE_ERR_WORKSPACE",
     "FORGE_ERR_CUDA", "FORGE_ERR_TIMEOUT", "FORGE_DTYPE_F32", "FORGE_DTYPE_BF16", "ForgeError",
     "library", "library_path", "forge_attn_fwd", "forge_attn_bwd", "forge_attn_bwd_workspace_size",
-    "forge_attn_bwd_noalloc",
+    "forge_attn_bwd_noalloc", "forge_attn_fwd_ext", "forge_attn_bwd_ext",
     "forge_attn_bwd_preprocess", "forge_attn_bwd_main", "forge_attn_bwd_finalize", "forge_attn_check",
     "forge_attn_status_string", "forge_attn_selftest_timeout", "forge_attn_selftest_exp2", "forge_attn_last_cuda_error", "forge_attn_timeout_info", "forge_attn_version",
     "attention_fwd", "attention_bwd", "dtype_code",
@@ -68,6 +68,10 @@ def library():
     L.forge_attn_bwd_workspace_size.restype = st
     L.forge_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, f, i, vp, st, vp]
     L.forge_attn_bwd.restype = i
+    L.forge_attn_fwd_ext.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, f, vp, vp, i, vp]
+    L.forge_attn_fwd_ext.restype = i
+    L.forge_attn_bwd_ext.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, f, vp, vp, i, vp, st, vp]
+    L.forge_attn_bwd_ext.restype = i
     L.forge_attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, f, i, vp]
     L.forge_attn_bwd_noalloc.restype = i
     L.forge_attn_bwd_preprocess.argtypes = [vp, vp, i, i, i, i, i, i, vp, st, vp]
@@ -136,6 +140,21 @@ def forge_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale, win
                                     _ptr(dk), _ptr(dv), B, Hq, Hkv, T, D, float(scale), int(window),
                                     float(softcap), int(dtype), _ptr(workspace), int(workspace_bytes),
                                     _stream(stream))
+
+
+def forge_attn_fwd_ext(q, k, v, o, lse, B, Hq, Hkv, T, D, scale, window, softcap, sink, max_logit, dtype,
+                       stream=None) -> int:
+    return library().forge_attn_fwd_ext(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, T, D,
+                                        float(scale), int(window), float(softcap), _ptr(sink), _ptr(max_logit),
+                                        int(dtype), _stream(stream))
+
+
+def forge_attn_bwd_ext(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale, window, softcap, sink, dsink,
+                       dtype, workspace, workspace_bytes, stream=None) -> int:
+    return library().forge_attn_bwd_ext(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
+                                        _ptr(dk), _ptr(dv), B, Hq, Hkv, T, D, float(scale), int(window),
+                                        float(softcap), _ptr(sink), _ptr(dsink), int(dtype), _ptr(workspace),
+                                        int(workspace_bytes), _stream(stream))
 
 
 def forge_attn_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale, window, softcap, dtype,

@@ -24,6 +24,7 @@ namespace {
 
 // ------------------------------------------------------------------ validation
 bool aligned16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 forge_status check_sizes(int B, int Hq, int Hkv, int T, int D, forge_dtype dtype) {
     if (B < 1 || Hq < 1 || Hkv < 1 || T < 1 || D < 1) return FORGE_ERR_INVALID_ARG;
@@ -123,7 +124,7 @@ forge_status set_smem(K kernel, size_t bytes) {
 // ----------------------------------------------------------------- dispatchers
 template <int D>
 forge_status fwd_tc(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv, int T,
-                    float scale, int window, float softcap, cudaStream_t st) {
+                    float scale, int window, float softcap, const float *sink, float *max_logit, cudaStream_t st) {
     using C = FwdTc<D>;
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, q, D, T, (long long)B * Hq, 128) || !make_map(&mk, k, D, T, (long long)B * Hkv, 128) ||
@@ -141,6 +142,8 @@ forge_status fwd_tc(const void *q, const void *k, const void *v, void *o, float 
     p.softcap = softcap;
     p.cap_in = softcap > 0.0f ? scale / softcap : 0.0f;
     p.cap_out = softcap * kLog2e;
+    p.sink = sink;
+    p.max_logit = max_logit;
     if constexpr (D == 256) {
         // one query tile per CTA: S0, S1 and the 256-column O fill TMEM
         if (set_smem(fwd_tc_kernel<D>, C::SMEM) != FORGE_OK) return FORGE_ERR_CUDA;
@@ -163,13 +166,13 @@ forge_status fwd_tc(const void *q, const void *k, const void *v, void *o, float 
 
 template <typename T_, int D>
 forge_status fwd_simt(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv, int T,
-                      float scale, int window, float softcap, cudaStream_t st) {
+                      float scale, int window, float softcap, const float *sink, float *max_logit, cudaStream_t st) {
     const size_t sm = simt_fwd_smem<D>();
     if (set_smem(simt_fwd<T_, D>, sm) != FORGE_OK) return FORGE_ERR_CUDA;
     dim3 grid((T + kSimtRows - 1) / kSimtRows, B * Hq);
     simt_fwd<T_, D><<<grid, kSimtThreads, sm, st>>>(static_cast<const T_ *>(q), static_cast<const T_ *>(k),
                                                      static_cast<const T_ *>(v), static_cast<T_ *>(o), lse, Hq, Hkv,
-                                                     T, scale, window, softcap);
+                                                     T, scale, window, softcap, sink, max_logit);
     return launch_status();
 }
 
@@ -223,6 +226,37 @@ forge_status bwd_tc(const void *q, const void *k, const void *v, const float *ls
     const unsigned grid = (unsigned)(p.num_kt * B * Hkv * C::NSPLIT);
     bwd_tc_kernel<D><<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, mdo, macc, p);
     return launch_status();
+}
+
+// out[i] = value for i < n
+__global__ void fill_f32_kernel(float *out, long n, float value) {
+    const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) out[i] = value;
+}
+
+// dsink[hq] = -sum over b, t of exp(sink[hq] - lse[b][hq][t]) * delta[b][hq][t]:
+// the gradient of a per-head sink logit (its softmax column times (0 - Delta),
+// the sink having no value vector). One block per query head, deterministic.
+__global__ void __launch_bounds__(256) sink_grad_kernel(const float *lse, const float *delta, const float *sink,
+                                                        float *dsink, int B, int Hq, int T) {
+    __shared__ float part[8];
+    const int hq = blockIdx.x;
+    const float sg = sink[hq];
+    float acc = 0.0f;
+    for (long idx = threadIdx.x; idx < (long)B * T; idx += blockDim.x) {
+        const long b = idx / T, t = idx % T;
+        const size_t row = ((size_t)b * Hq + hq) * T + t;
+        acc -= expf(sg - lse[row]) * delta[row];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float sum = 0.0f;
+        for (int w = 0; w < 8; w++) sum += part[w];
+        dsink[hq] = sum;
+    }
 }
 
 #define FORGE_DISPATCH_D(D, ...)                               \
@@ -299,22 +333,38 @@ using namespace forge;
 
 extern "C" {
 
-forge_status forge_attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
-                            int Hkv, int T, int D, float scale, int window, float softcap, forge_dtype dtype,
-                            void *stream) {
+forge_status forge_attn_fwd_ext(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+                                int Hkv, int T, int D, float scale, int window, float softcap, const float *sink,
+                                float *max_logit, forge_dtype dtype, void *stream) {
     forge_status s = check_sizes(B, Hq, Hkv, T, D, dtype);
     if (s != FORGE_OK) return s;
     if ((s = check_scalars(scale, window, softcap)) != FORGE_OK) return s;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return FORGE_ERR_INVALID_ARG;
+    if ((sink != nullptr && !aligned4(sink)) || (max_logit != nullptr && !aligned4(max_logit)))
+        return FORGE_ERR_INVALID_ARG;
     window = effective_window(window, T);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (max_logit != nullptr) {
+        const long n = (long)B * Hq;
+        fill_f32_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(max_logit, n, -INFINITY);
+        if ((s = launch_status()) != FORGE_OK) return s;
+    }
     if (dtype == FORGE_DTYPE_BF16) {
-        FORGE_DISPATCH_D(D, return fwd_tc<kD>(q, k, v, o, lse, B, Hq, Hkv, T, scale, window, softcap, st);)
+        FORGE_DISPATCH_D(D, return fwd_tc<kD>(q, k, v, o, lse, B, Hq, Hkv, T, scale, window, softcap, sink,
+                                               max_logit, st);)
     } else {
-        FORGE_DISPATCH_D(D, return fwd_simt<float, kD>(q, k, v, o, lse, B, Hq, Hkv, T, scale, window, softcap, st);)
+        FORGE_DISPATCH_D(D, return fwd_simt<float, kD>(q, k, v, o, lse, B, Hq, Hkv, T, scale, window, softcap, sink,
+                                                        max_logit, st);)
     }
     return FORGE_ERR_UNSUPPORTED;
+}
+
+forge_status forge_attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+                            int Hkv, int T, int D, float scale, int window, float softcap, forge_dtype dtype,
+                            void *stream) {
+    return forge_attn_fwd_ext(q, k, v, o, lse, B, Hq, Hkv, T, D, scale, window, softcap, nullptr, nullptr, dtype,
+                              stream);
 }
 
 size_t forge_attn_bwd_workspace_size(int B, int Hq, int Hkv, int T, int D, forge_dtype dtype) {
@@ -394,10 +444,10 @@ forge_status forge_attn_bwd_finalize(void *dq, int B, int Hq, int Hkv, int T, in
     return launch_status();
 }
 
-forge_status forge_attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
-                            const void *dO, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int T, int D,
-                            float scale, int window, float softcap, forge_dtype dtype, void *workspace,
-                            size_t workspace_bytes, void *stream) {
+forge_status forge_attn_bwd_ext(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                                const void *dO, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int T, int D,
+                                float scale, int window, float softcap, const float *sink, float *dsink,
+                                forge_dtype dtype, void *workspace, size_t workspace_bytes, void *stream) {
     forge_status s = check_sizes(B, Hq, Hkv, T, D, dtype);
     if (s != FORGE_OK) return s;
     if ((s = check_scalars(scale, window, softcap)) != FORGE_OK) return s;
@@ -405,13 +455,29 @@ forge_status forge_attn_bwd(const void *q, const void *k, const void *v, const v
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dO) ||
         !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
         return FORGE_ERR_INVALID_ARG;
+    if (dsink != nullptr && (!aligned4(dsink) || !aligned4(sink))) return FORGE_ERR_INVALID_ARG;
+    if (sink != nullptr && !aligned4(sink)) return FORGE_ERR_INVALID_ARG;
     if ((s = check_workspace(workspace, workspace_bytes, B, Hq, Hkv, T, D, dtype)) != FORGE_OK) return s;
     s = forge_attn_bwd_preprocess(o, dO, B, Hq, Hkv, T, D, dtype, workspace, workspace_bytes, stream);
     if (s != FORGE_OK) return s;
+    if (dsink != nullptr) {
+        // the sink enters dq, dk, dv only through lse; its own gradient needs Delta
+        sink_grad_kernel<<<(unsigned)Hq, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+            lse, static_cast<const float *>(workspace), sink, dsink, B, Hq, T);
+        if ((s = launch_status()) != FORGE_OK) return s;
+    }
     s = forge_attn_bwd_main(q, k, v, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale, window, softcap, dtype, workspace,
                             workspace_bytes, stream);
     if (s != FORGE_OK) return s;
     return forge_attn_bwd_finalize(dq, B, Hq, Hkv, T, D, dtype, workspace, workspace_bytes, stream);
+}
+
+forge_status forge_attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                            const void *dO, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int T, int D,
+                            float scale, int window, float softcap, forge_dtype dtype, void *workspace,
+                            size_t workspace_bytes, void *stream) {
+    return forge_attn_bwd_ext(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale, window, softcap, nullptr,
+                              nullptr, dtype, workspace, workspace_bytes, stream);
 }
 
 forge_status forge_attn_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, const float *lse,

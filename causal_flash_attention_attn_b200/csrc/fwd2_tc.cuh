@@ -280,7 +280,8 @@ __global__ void __launch_bounds__(384, 1)
         const int r0 = q0 + 32 * (warp % 4);
         const bool cap = p.softcap > 0.0f;
         const uint64_t sl2x2 = f2_make(p.scale_log2, p.scale_log2);
-        float m = -INFINITY, l = 0.0f;
+        float m = p.sink ? p.sink[hq] * kLog2e : -INFINITY, l = p.sink ? 1.0f : 0.0f;
+        float mraw = -INFINITY;  // row max of the (log2-unit) scores, the sink excluded
         bool ok = (x == 0) || hasB;
         if (ok) {
             int cnt = 0;
@@ -328,6 +329,7 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 float mx = row_max128(s);
                 if (!cap) mx *= p.scale_log2;
+                mraw = fmaxf(mraw, mx);
                 const float m_new = (mx > m + 8.0f) ? mx : m;
                 const bool moved = (m_new != m);
                 const float factor = moved ? ex2_approx(m - m_new) : 1.0f;
@@ -433,6 +435,10 @@ __global__ void __launch_bounds__(384, 1)
                 bulk_wait_read<0>();
             }
             if (qi < p.T) p.lse[(size_t)bh * p.T + qi] = (m + __log2f(l)) * kLn2;
+            if (p.max_logit) {
+                const float r = warp_max_f32(qi < p.T ? mraw * kLn2 : -INFINITY);
+                if (lane == 0) atomic_max_f32(p.max_logit + bh, r);
+            }
         }
     }
 

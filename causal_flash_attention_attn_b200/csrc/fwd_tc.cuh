@@ -112,6 +112,14 @@ struct FwdParams {
     float softcap;     // 0 = off
     float cap_in;      // scale / softcap
     float cap_out;     // softcap * log2(e)
+    // attention sinks: per query head logit in the softmax denominator (natural
+    // units; nullptr = none). ARCHITECTURES.md family table, GPT-OSS row; "Vague
+    // 2" item 10: the online softmax starts from (max, sum) = (sink, 1).
+    const float *sink;
+    // per (batch, query head) maximum of the scores the softmax sees, the sink
+    // not included (QK-Clip's monitor, "Vague 3" item 12); nullptr = not wanted.
+    // Must hold -inf (or a lower bound) before the launch: kernels atomic-max it.
+    float *max_logit;
 };
 
 template <int D>
@@ -277,7 +285,8 @@ __global__ void __launch_bounds__(192, 1)
         const int qi = q0 + row;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         const int W = p.window;
-        float m = -INFINITY, l = 0.0f;
+        float m = p.sink ? p.sink[hq] * kLog2e : -INFINITY, l = p.sink ? 1.0f : 0.0f;
+        float mraw = -INFINITY;  // row max of the (log2-unit) scores, the sink excluded
         bool ok = true;
         for (int u = 0; u < n; u++) {
             const int buf = u & 1;
@@ -319,6 +328,7 @@ __global__ void __launch_bounds__(192, 1)
             }
             float mx = fwd_row_max(s);
             if (!cap) mx *= p.scale_log2;
+            mraw = fmaxf(mraw, mx);
             const float m_new = (mx > m + 8.0f) ? mx : m;
             const bool moved = (m_new != m);
             const float factor = moved ? ex2_approx(m - m_new) : 1.0f;
@@ -389,6 +399,10 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
             if (qi < p.T) p.lse[(size_t)bh * p.T + qi] = (m + __log2f(l)) * kLn2;
+            if (p.max_logit) {
+                const float r = warp_max_f32(qi < p.T ? mraw * kLn2 : -INFINITY);
+                if ((threadIdx.x & 31) == 0) atomic_max_f32(p.max_logit + bh, r);
+            }
         }
     }
 

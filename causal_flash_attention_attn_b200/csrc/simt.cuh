@@ -70,7 +70,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kSimtThreads) simt_fwd(const T *__restrict__ q, const T *__restrict__ k,
                                                          const T *__restrict__ v, T *__restrict__ o,
                                                          float *__restrict__ lse, int Hq, int Hkv, int T_,
-                                                         float scale, int window, float softcap) {
+                                                         float scale, int window, float softcap,
+                                                         const float *__restrict__ sink, float *__restrict__ max_logit) {
     extern __shared__ float sm[];
     float *sQ = sm;
     float *sK = sQ + kSimtRows * D;
@@ -84,11 +85,13 @@ __global__ void __launch_bounds__(kSimtThreads) simt_fwd(const T *__restrict__ q
     const T *Vb = v + (size_t)(b * Hkv + hkv) * T_ * D;
     load_rows<T, D>(sQ, D, Qb, r0, kSimtRows, T_);
 
-    float m[4], l[4], acc[4][NT];
+    // a sink (natural units) starts each row's (max, sum) at (sink, 1)
+    float m[4], l[4], acc[4][NT], mraw[4];
 #pragma unroll
     for (int rr = 0; rr < 4; rr++) {
-        m[rr] = -INFINITY;
-        l[rr] = 0.0f;
+        m[rr] = sink ? sink[hq] : -INFINITY;
+        l[rr] = sink ? 1.0f : 0.0f;
+        mraw[rr] = -INFINITY;
 #pragma unroll
         for (int t = 0; t < NT; t++) acc[rr][t] = 0.0f;
     }
@@ -111,7 +114,9 @@ __global__ void __launch_bounds__(kSimtThreads) simt_fwd(const T *__restrict__ q
             s = simt_capped(s * scale, softcap);
             const bool ok = visible(qi, kj, window) && kj < T_;
             s = ok ? s : -INFINITY;
-            const float mnew = fmaxf(m[rr], warp_max(s));
+            const float smax = warp_max(s);
+            mraw[rr] = fmaxf(mraw[rr], smax);
+            const float mnew = fmaxf(m[rr], smax);
             if (mnew == -INFINITY) continue;
             const float corr = expf(m[rr] - mnew);
             const float p = ok ? expf(s - mnew) : 0.0f;
@@ -135,6 +140,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_fwd(const T *__restrict__ q
 #pragma unroll
         for (int t = 0; t < NT; t++) from_f32(orow + lane + 32 * t, acc[rr][t] * inv);
         if (lane == 0) lse[(size_t)bh * T_ + qi] = m[rr] + logf(l[rr]);
+        if (max_logit != nullptr && lane == 0) atomic_max_f32(max_logit + bh, mraw[rr]);
     }
 }
 

@@ -173,6 +173,18 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
 }
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (tensor core operand reads).
+// atomic max of a float (the location must hold a float, initially -inf or any
+// value): non-negative values order like their int bit patterns, negative ones
+// inversely like their unsigned bit patterns.
+__device__ __forceinline__ void atomic_max_f32(float *addr, float v) {
+    if (v >= 0.0f) atomicMax(reinterpret_cast<int *>(addr), __float_as_int(v));
+    else atomicMin(reinterpret_cast<unsigned int *>(addr), __float_as_uint(v));
+}
+__device__ __forceinline__ float warp_max_f32(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }

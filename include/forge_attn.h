@@ -71,6 +71,28 @@ forge_status forge_attn_fwd(const void *q, const void *k, const void *v, void *o
                             float softcap, forge_dtype dtype, void *stream);
 
 /*
+ * Forward with two optional extras (either pointer may be NULL; with both NULL
+ * this is forge_attn_fwd):
+ *  - sink [Hq] f32 (device): a learned logit per query head that joins every
+ *    row's softmax denominator and has no value vector (attention sinks:
+ *    ARCHITECTURES.md family table, GPT-OSS row, "biais par tête dans le
+ *    dénominateur softmax"; "Vague 2" item 10, which starts the online softmax's
+ *    (max, sum) from it). In the units of the scores the softmax sees (after
+ *    scale and cap; the sink itself is not capped). P_ij = exp(s_ij) /
+ *    (exp(sink[hq]) + sum_j exp(s_ij)); lse includes it.
+ *  - max_logit [B][Hq] f32 (device, written): per (batch, query head) the
+ *    maximum over the allowed (i, j) of the score the softmax sees, the sink not
+ *    included: the per-head maximum attention logit that QK-Clip monitors
+ *    ("Vague 3" item 12; family table, Kimi K2 row). The call first sets it to
+ *    -inf, then the kernels raise it with atomic maxima.
+ * Both 4-byte aligned. Same errors as forge_attn_fwd.
+ */
+forge_status forge_attn_fwd_ext(const void *q, const void *k, const void *v, void *o, float *lse,
+                                int B, int Hq, int Hkv, int T, int D, float scale, int window,
+                                float softcap, const float *sink, float *max_logit, forge_dtype dtype,
+                                void *stream);
+
+/*
  * Bytes of device workspace forge_attn_bwd needs for these sizes (0 on invalid
  * sizes). Holds rowsum(dO * o) as f32 and, for bf16, an f32 dq accumulator.
  */
@@ -89,6 +111,21 @@ forge_status forge_attn_bwd(const void *q, const void *k, const void *v, const v
                             int B, int Hq, int Hkv, int T, int D, float scale, int window,
                             float softcap, forge_dtype dtype, void *workspace,
                             size_t workspace_bytes, void *stream);
+
+/*
+ * Backward of forge_attn_fwd_ext. `lse` (from that forward) already includes the
+ * sink, which is all dq, dk and dv need of it. dsink [Hq] f32 (device, written;
+ * NULL = not wanted; then sink may be NULL too) receives the gradient of the
+ * loss with respect to sink[hq]: -sum over b and rows t of
+ * exp(sink[hq] - lse[b][hq][t]) * Delta[b][hq][t], Delta = rowsum(dO * o) (the
+ * sink's softmax column times (0 - Delta), the sink having no value vector).
+ * With dsink non-NULL, sink must be non-NULL. Otherwise as forge_attn_bwd.
+ */
+forge_status forge_attn_bwd_ext(const void *q, const void *k, const void *v, const void *o,
+                                const float *lse, const void *dO, void *dq, void *dk, void *dv,
+                                int B, int Hq, int Hkv, int T, int D, float scale, int window,
+                                float softcap, const float *sink, float *dsink, forge_dtype dtype,
+                                void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Backward for callers that cannot allocate device memory (no counterpart on

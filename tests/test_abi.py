@@ -109,3 +109,19 @@ def test_layer_window_pattern():
     # alternating
     assert [layer_window(l, 4096, 2) for l in range(4)] == [4096, 0, 4096, 0]
     assert [layer_window(l, 4096, 0) for l in range(3)] == [4096] * 3
+
+
+def test_dsink_without_sink_is_rejected_before_any_launch():
+    # validation fails before any device access, so fake device addresses are safe
+    A = 0x10000
+    s = fa.forge_attn_bwd_ext(A, A, A, A, A, A, A, A, A, 1, 2, 2, 128, 64, 0.125, 0, 0.0, None, A,
+                              fa.FORGE_DTYPE_BF16, A, 1 << 20, 0)
+    assert s == fa.FORGE_ERR_INVALID_ARG
+
+
+def test_ext_entry_points_reject_misaligned_extras():
+    A = 0x10000
+    s = fa.forge_attn_fwd_ext(A, A, A, A, A, 1, 2, 2, 128, 64, 0.125, 0, 0.0, A + 2, None, fa.FORGE_DTYPE_BF16, 0)
+    assert s == fa.FORGE_ERR_INVALID_ARG
+    s = fa.forge_attn_fwd_ext(A, A, A, A, A, 1, 2, 2, 128, 64, 0.125, 0, 0.0, None, A + 1, fa.FORGE_DTYPE_BF16, 0)
+    assert s == fa.FORGE_ERR_INVALID_ARG
