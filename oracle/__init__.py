@@ -10,8 +10,10 @@ shapes, central finite differences, and the invariants and closed forms of the
 definition. The sink and max-logit extensions are pinned by: sink = -inf being the
 plain softmax bit for bit; a sink being an extra zero-value key at position 0
 (checked through the pinned plain oracle, forward, dq/dk/dv and dsink); a one-key
-closed form; central differences of dsink; a hand-worked max-logit example. No
-function here is left unpinned.
+closed form; central differences of dsink; a hand-worked max-logit example. The
+decode function is pinned to the last row of the pinned forward (bit for bit, with
+window, cap and sink), to per-entry lengths with the cache tail poisoned, and to the
+length-1 closed form. No function here is left unpinned.
 
 Every function takes and returns numpy float64 arrays in [B, H, T, D] layout.
 """
@@ -39,6 +41,8 @@ def _load():
         lib.oracle_attn_fwd_ext.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, d, i, d]
         lib.oracle_attn_bwd_ext.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, d, i, d, i]
         lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, d, i, d, i]
+        lib.oracle_attn_decode.argtypes = [dp, dp, dp, dp, ctypes.POINTER(ctypes.c_int), dp, dp, i, i, i, i, i, i, d,
+                                           i, d]
         lib.oracle_round.argtypes = [dp, dp, ctypes.c_long, i]
         lib.oracle_attn_probs.argtypes = [dp, dp, dp, i, i, i, i, i, d, i, d]
         lib.oracle_rowdot.argtypes = [dp, dp, dp, ctypes.c_long, i]
@@ -144,6 +148,31 @@ def attn_bwd_ext(q, k, v, dO, scale: float, window: int = 0, softcap: float = 0.
                                 _ptr(dv), _ptr(dsink), _ptr(delta), _ptr(lse), B, Hq, Hkv, T, D, float(scale),
                                 int(window), float(softcap), _ROUND[o_round])
     return dq, dk, dv, dsink, delta, lse
+
+
+def attn_decode(q, k_cache, v_cache, scale: float, T: int, window: int = 0, softcap: float = 0.0, sink=None,
+                seq_lens=None):
+    """Decode: q [B, Hq, D] (the new token's queries), caches [B, Hkv, Tmax, D]; entry
+    b's query sits at position len_b - 1 with len_b = seq_lens[b] (or T). Returns
+    (o [B, Hq, D], lse [B, Hq])."""
+    q, kc, vc = _f64(q), _f64(k_cache), _f64(v_cache)
+    B, Hq, D = q.shape
+    Bk, Hkv, Tmax, Dk = kc.shape
+    assert (B, D) == (Bk, Dk) and Hq % Hkv == 0 and vc.shape == kc.shape
+    sk = None if sink is None else _f64(sink).reshape(Hq)
+    sl = None
+    if seq_lens is not None:
+        sl = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32).reshape(B))
+        assert np.all((sl >= 1) & (sl <= Tmax))
+    else:
+        assert 1 <= T <= Tmax
+    o = np.empty((B, Hq, D), dtype=np.float64)
+    lse = np.empty((B, Hq), dtype=np.float64)
+    _load().oracle_attn_decode(_ptr(q), _ptr(kc), _ptr(vc), _ptr_or_null(sk),
+                               None if sl is None else sl.ctypes.data_as(ctypes.POINTER(ctypes.c_int)),
+                               _ptr(o), _ptr(lse), B, Hq, Hkv, int(T), Tmax, D, float(scale), int(window),
+                               float(softcap))
+    return o, lse
 
 
 def attn_probs(q, k, scale: float, window: int = 0, softcap: float = 0.0):

@@ -307,6 +307,38 @@ void oracle_attn_bwd(const double *q, const double *k, const double *v, const do
                         scale, window, softcap, o_round);
 }
 
+/*
+ * Decode: one new query per (b, hq) at position len_b - 1 attends the keys of a
+ * KV cache (INFERENCE_RESEARCH.md section 2: cache pre-allocated to the maximum
+ * length, [layer][head][seq][d] per layer, a dedicated one-query kernel).
+ * q, o [B][Hq][D]; k, v [B][Hkv][Tmax][D]; lse [B][Hq]; seq_lens [B] (NULL: every
+ * entry has T valid positions). Keys visible: [len - W, len - 1] clipped at 0
+ * (W = 0: all len), the same mask as row len - 1 of the forward. sink as in the
+ * forward (may be NULL).
+ */
+void oracle_attn_decode(const double *q, const double *k, const double *v, const double *sink,
+                        const int *seq_lens, double *o, double *lse, int B, int Hq, int Hkv, int T,
+                        int Tmax, int D, double scale, int window, double softcap) {
+    const int G = Hq / Hkv;
+    double *p = (double *)malloc(sizeof(double) * (size_t)Tmax);
+    for (int b = 0; b < B; b++)
+        for (int hq = 0; hq < Hq; hq++) {
+            const int hkv = hq / G;
+            const long len = seq_lens ? seq_lens[b] : T;
+            const long i = len - 1;
+            const size_t qrow = (size_t)(b * Hq + hq);
+            const double *K = k + (size_t)(b * Hkv + hkv) * Tmax * D;
+            const double *V = v + (size_t)(b * Hkv + hkv) * Tmax * D;
+            const long lo = first_key(i, window);
+            lse[qrow] = row_probs(q + qrow * D, K, i, lo, D, scale, softcap, sink_of(sink, hq), p, NULL);
+            double *oi = o + qrow * D;
+            for (int d = 0; d < D; d++) oi[d] = 0.0;
+            for (long j = lo; j <= i; j++)
+                for (int d = 0; d < D; d++) oi[d] += p[j] * V[j * D + d];
+        }
+    free(p);
+}
+
 /* Full probability matrix P [B][Hq][T][T] (zeros where masked); small sizes only. */
 void oracle_attn_probs(const double *q, const double *k, double *P, int B, int Hq, int Hkv,
                        int T, int D, double scale, int window, double softcap) {

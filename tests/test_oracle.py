@@ -505,3 +505,36 @@ def test_max_logit_is_attained_by_an_allowed_pair_and_bounds_the_rest():
     assert np.all(s_allowed <= ml[:, :, None, None] + 0.0)
     hits = np.isclose(s_allowed, ml[:, :, None, None], rtol=0, atol=1e-12) & allowed
     assert np.all(hits.any(axis=(2, 3)))
+
+
+# ---------------------------------------------------------------- decode
+# One new query per (b, hq) against a KV cache (INFERENCE_RESEARCH.md section 2).
+
+@pytest.mark.parametrize("W,C,use_sink", [(0, 0.0, False), (5, 0.0, False), (0, 2.0, True), (4, 1.5, True)])
+def test_decode_equals_last_row_of_the_forward(W, C, use_sink):
+    B, Hq, Hkv, T, Tmax, D, scale = 2, 4, 2, 13, 16, 6, 0.45
+    qf, kc, vc = _rand((B, Hq, T, D), 21), _rand((B, Hkv, Tmax, D), 22), _rand((B, Hkv, Tmax, D), 23)
+    sink = np.array([0.5, -0.3, 1.2, 0.1]) if use_sink else None
+    o, lse = oracle.attn_decode(qf[:, :, T - 1], kc, vc, scale, T, W, C, sink=sink)
+    ro, rl, _ = oracle.attn_fwd_ext(qf, kc[:, :, :T], vc[:, :, :T], scale, W, C, sink=sink)
+    np.testing.assert_array_equal(o, ro[:, :, T - 1])
+    np.testing.assert_array_equal(lse, rl[:, :, T - 1])
+
+
+def test_decode_per_entry_lengths_and_cache_tail_ignored():
+    B, Hq, Hkv, Tmax, D, scale = 3, 2, 1, 12, 5, 0.5
+    q, kc, vc = _rand((B, Hq, D), 24), _rand((B, Hkv, Tmax, D), 25), _rand((B, Hkv, Tmax, D), 26)
+    lens = [12, 1, 7]
+    o, lse = oracle.attn_decode(q, kc, vc, scale, Tmax, seq_lens=lens)
+    kc2, vc2 = kc.copy(), vc.copy()
+    for b, n in enumerate(lens):
+        kc2[b, :, n:] = 1e6   # positions past the entry's length are never read
+        vc2[b, :, n:] = np.nan
+        ob, lb = oracle.attn_decode(q[b:b + 1], kc[b:b + 1], vc[b:b + 1], scale, n)
+        np.testing.assert_array_equal(o[b:b + 1], ob)
+        np.testing.assert_array_equal(lse[b:b + 1], lb)
+    o2, lse2 = oracle.attn_decode(q, kc2, vc2, scale, Tmax, seq_lens=lens)
+    np.testing.assert_array_equal(o, o2)
+    # length 1 sees only position 0: o = v[0], lse = the one score
+    np.testing.assert_allclose(o[1], np.repeat(vc[1, :, 0], Hq // Hkv, axis=0), rtol=1e-15)
+    np.testing.assert_allclose(lse[1], scale * (q[1] @ kc[1, 0, 0]), rtol=1e-14)
