@@ -440,6 +440,73 @@ def run_reference(args, w):
     }
 
 
+# KV-cache decode workload: a long-context batch, one new token per entry
+DECODE = {"workload": "decode_b16_h32_kv8_t16k_d128", "B": 16, "Hq": 32, "Hkv": 8, "T": 16384, "Tmax": 16384,
+          "D": 128, "dtype": "bf16", "window": 0, "softcap": 0.0}
+
+
+def run_decode(args):
+    """--decode: the KV-cache decode kernels (split + combine) on one GPU, HBM-bound:
+    achieved = bytes of the K and V cache (plus q and o) per call / CUDA-event time."""
+    import torch
+    import causal_flash_attention_attn_b200 as fa
+
+    c = DECODE
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    fa.library()
+    stream = torch.cuda.Stream(device=dev)
+    g = torch.Generator(device="cpu").manual_seed(5)
+    B, Hq, Hkv, T, Tmax, D = c["B"], c["Hq"], c["Hkv"], c["T"], c["Tmax"], c["D"]
+    q = torch.randn(B, Hq, D, generator=g).to(torch.bfloat16).to(dev)
+    kc = torch.randn(B, Hkv, Tmax, D, generator=g).to(torch.bfloat16).to(dev)
+    vc = torch.randn(B, Hkv, Tmax, D, generator=g).to(torch.bfloat16).to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    nws = fa.forge_attn_decode_workspace_size(B, Hq, Hkv, T, D)
+    ws = torch.empty(nws, dtype=torch.uint8, device=dev)
+    sc = 1.0 / math.sqrt(D)
+
+    def call():
+        s = fa.forge_attn_decode(q, kc, vc, o, lse, None, B, Hq, Hkv, T, Tmax, D, sc, c["window"], c["softcap"],
+                                 None, fa.FORGE_DTYPE_BF16, ws, nws, stream.cuda_stream)
+        if s != fa.FORGE_OK:
+            raise fa.ForgeError(s, "decode")
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    clk = ClockSampler(dev.index)
+    clk.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = clk.stop()
+    st = fa.forge_attn_check(stream.cuda_stream)
+    if st != fa.FORGE_OK:
+        raise fa.ForgeError(st, "decode timed run")
+    ms = e0.elapsed_time(e1) / args.steps
+    cache_bytes = 2 * B * Hkv * T * D * 2
+    io_bytes = 2 * B * Hq * D * 2 + B * Hq * 4
+    gbs = (cache_bytes + io_bytes) / (ms * 1e-3) / 1e9
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    return {"metric": "KV-cache decode bandwidth (one query per entry and head, K and V read once)",
+            "value": round(gbs, 1), "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded N(0,1) q and caches)",
+            "config": dict(c, l2="not flushed: the 1.07 GB cache exceeds the 126 MB L2"),
+            "roofline": {"kernel": "decode_split", "bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(gbs / peak, 4), "traffic": None,
+                         "peak_source": f"{peak_src} hbm_gbs",
+                         "achieved_def": "K+V cache bytes + q, o, lse bytes per call / CUDA-event time of both kernels"},
+            "gpu_launches": 2 * args.steps, "clocks": clocks}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -450,11 +517,15 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--decode", action="store_true", help="time the KV-cache decode kernels instead")
     args = ap.parse_args(argv)
     from causal_flash_attention_attn_b200 import inputs
     w = inputs.WORKLOADS[args.workload or inputs.HEADLINE]
     if args.warmup < 3:
         args.warmup = 3
+    if args.decode:
+        print(json.dumps(run_decode(args)), flush=True)
+        return
     line = run_reference(args, w) if args.impl == "reference" else run_ours(args, w)
     if line is not None:
         print(json.dumps(line), flush=True)

@@ -19,7 +19,8 @@ __all__ = [
     "FORGE_OK", "FORGE_ERR_INVALID_ARG", "FORGE_ERR_UNSUPPORTED", "FORGE_ERR_WORKSPACE",
     "FORGE_ERR_CUDA", "FORGE_ERR_TIMEOUT", "FORGE_DTYPE_F32", "FORGE_DTYPE_BF16", "ForgeError",
     "library", "library_path", "forge_attn_fwd", "forge_attn_bwd", "forge_attn_bwd_workspace_size",
-    "forge_attn_bwd_noalloc", "forge_attn_fwd_ext", "forge_attn_bwd_ext",
+    "forge_attn_bwd_noalloc", "forge_attn_fwd_ext", "forge_attn_bwd_ext", "forge_attn_decode",
+    "forge_attn_decode_workspace_size", "attention_decode",
     "forge_attn_bwd_preprocess", "forge_attn_bwd_main", "forge_attn_bwd_finalize", "forge_attn_check",
     "forge_attn_status_string", "forge_attn_selftest_timeout", "forge_attn_selftest_exp2", "forge_attn_last_cuda_error", "forge_attn_timeout_info", "forge_attn_version",
     "attention_fwd", "attention_bwd", "dtype_code",
@@ -72,6 +73,10 @@ def library():
     L.forge_attn_fwd_ext.restype = i
     L.forge_attn_bwd_ext.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, f, vp, vp, i, vp, st, vp]
     L.forge_attn_bwd_ext.restype = i
+    L.forge_attn_decode_workspace_size.argtypes = [i, i, i, i, i]
+    L.forge_attn_decode_workspace_size.restype = st
+    L.forge_attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, f, vp, i, vp, st, vp]
+    L.forge_attn_decode.restype = i
     L.forge_attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, f, i, vp]
     L.forge_attn_bwd_noalloc.restype = i
     L.forge_attn_bwd_preprocess.argtypes = [vp, vp, i, i, i, i, i, i, vp, st, vp]
@@ -157,6 +162,18 @@ def forge_attn_bwd_ext(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale,
                                         int(workspace_bytes), _stream(stream))
 
 
+def forge_attn_decode_workspace_size(B, Hq, Hkv, T, D) -> int:
+    return int(library().forge_attn_decode_workspace_size(B, Hq, Hkv, T, D))
+
+
+def forge_attn_decode(q, k_cache, v_cache, o, lse, seq_lens, B, Hq, Hkv, T, Tmax, D, scale, window, softcap, sink,
+                      dtype, workspace, workspace_bytes, stream=None) -> int:
+    return library().forge_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse), _ptr(seq_lens),
+                                       B, Hq, Hkv, T, Tmax, D, float(scale), int(window), float(softcap),
+                                       _ptr(sink), int(dtype), _ptr(workspace), int(workspace_bytes),
+                                       _stream(stream))
+
+
 def forge_attn_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale, window, softcap, dtype,
                            stream=None) -> int:
     """forge_attn_bwd with the library's fixed 32 MiB internal scratch instead of a workspace."""
@@ -230,6 +247,26 @@ def attention_fwd(q, k, v, scale=None, window=0, softcap=0.0, stream=None):
     s = forge_attn_fwd(q, k, v, o, lse, B, Hq, Hkv, T, D, scale, window, softcap, dtype_code(q.dtype), stream)
     if s != FORGE_OK:
         raise ForgeError(s, "forge_attn_fwd")
+    return o, lse
+
+
+def attention_decode(q, k_cache, v_cache, T=None, scale=None, window=0, softcap=0.0, seq_lens=None, sink=None,
+                     stream=None):
+    """Decode on device tensors: q [B,Hq,D], caches [B,Hkv,Tmax,D]; T defaults to
+    Tmax (or the largest of seq_lens, an int32 device tensor [B]). Returns (o, lse)."""
+    import torch
+    B, Hq, D = q.shape
+    Hkv, Tmax = k_cache.shape[1], k_cache.shape[2]
+    if T is None:
+        T = int(seq_lens.max().item()) if seq_lens is not None else Tmax
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    ws = torch.empty(forge_attn_decode_workspace_size(B, Hq, Hkv, T, D), dtype=torch.uint8, device=q.device)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    s = forge_attn_decode(q, k_cache, v_cache, o, lse, seq_lens, B, Hq, Hkv, T, Tmax, D, scale, window, softcap, sink,
+                          dtype_code(q.dtype), ws, ws.numel(), stream)
+    if s != FORGE_OK:
+        raise ForgeError(s, "forge_attn_decode")
     return o, lse
 
 

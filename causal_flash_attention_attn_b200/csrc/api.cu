@@ -14,6 +14,7 @@
 
 #include "bwd_aux.cuh"
 #include "bwd_tc.cuh"
+#include "decode.cuh"
 #include "fwd2_tc.cuh"
 #include "fwd_tc.cuh"
 #include "simt.cuh"
@@ -259,6 +260,36 @@ __global__ void __launch_bounds__(256) sink_grad_kernel(const float *lse, const 
     }
 }
 
+// Keys per decode chunk: enough chunks for about eight CTAs per SM (short tail
+// wave), multiples of 64.
+int decode_chunk(int B, int Hkv, int T) {
+    const long per = (long)B * Hkv;
+    const long splits = (8L * 148 + per - 1) / per;
+    long chunk = ((T + splits - 1) / splits + 63) / 64 * 64;
+    return (int)(chunk < 64 ? 64 : chunk);
+}
+
+template <typename T_, int D, int MG>
+forge_status decode_split_launch(const void *q, const void *kc, const void *vc, const DecParams &p, cudaStream_t st) {
+    using C = DecCfg<T_, D>;
+    if (set_smem(decode_split<T_, D, MG>, C::smem(MG)) != FORGE_OK) return FORGE_ERR_CUDA;
+    decode_split<T_, D, MG><<<dim3((unsigned)p.nsplit, (unsigned)(p.B * p.Hkv)), kDecThreads,
+                              C::smem(p.Hq / p.Hkv), st>>>(static_cast<const T_ *>(q), static_cast<const T_ *>(kc),
+                                                           static_cast<const T_ *>(vc), p);
+    return launch_status();
+}
+
+template <typename T_, int D>
+forge_status decode_run(const void *q, const void *kc, const void *vc, void *o, DecParams p, cudaStream_t st) {
+    const int G = p.Hq / p.Hkv;
+    forge_status s = G <= 4   ? decode_split_launch<T_, D, 4>(q, kc, vc, p, st)
+                     : G <= 8 ? decode_split_launch<T_, D, 8>(q, kc, vc, p, st)
+                              : decode_split_launch<T_, D, 16>(q, kc, vc, p, st);
+    if (s != FORGE_OK) return s;
+    decode_combine<T_, D><<<(unsigned)(p.B * p.Hq), D, 0, st>>>(static_cast<T_ *>(o), p);
+    return launch_status();
+}
+
 #define FORGE_DISPATCH_D(D, ...)                               \
     switch (D) {                                               \
         case 64: { constexpr int kD = 64; __VA_ARGS__ } break;   \
@@ -495,6 +526,47 @@ forge_status forge_attn_bwd_noalloc(const void *q, const void *k, const void *v,
     // so whatever the previous call left in the array does not matter
     return forge_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale, window, softcap, dtype, scratch,
                           kNoAllocScratchBytes, stream);
+}
+
+size_t forge_attn_decode_workspace_size(int B, int Hq, int Hkv, int T, int D) {
+    if (check_sizes(B, Hq, Hkv, T, D, FORGE_DTYPE_BF16) != FORGE_OK) return 0;
+    const int chunk = decode_chunk(B, Hkv, T);
+    const long nsplit = (T + chunk - 1) / chunk;
+    return ((size_t)B * Hq * nsplit * (size_t)(D + 2) * sizeof(float) + 255) / 256 * 256;
+}
+
+forge_status forge_attn_decode(const void *q, const void *k_cache, const void *v_cache, void *o, float *lse,
+                               const int *seq_lens, int B, int Hq, int Hkv, int T, int Tmax, int D, float scale,
+                               int window, float softcap, const float *sink, forge_dtype dtype, void *workspace,
+                               size_t workspace_bytes, void *stream) {
+    forge_status s = check_sizes(B, Hq, Hkv, T, D, dtype);
+    if (s != FORGE_OK) return s;
+    if ((s = check_scalars(scale, window, softcap)) != FORGE_OK) return s;
+    if (Tmax < T || (long)Tmax * D * B * Hkv > (1L << 40)) return FORGE_ERR_INVALID_ARG;
+    if (Hq / Hkv > kDecMaxG) return FORGE_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return FORGE_ERR_INVALID_ARG;
+    if ((lse && !aligned4(lse)) || (seq_lens && !aligned4(seq_lens)) || (sink && !aligned4(sink)))
+        return FORGE_ERR_INVALID_ARG;
+    const size_t need = forge_attn_decode_workspace_size(B, Hq, Hkv, T, D);
+    if (!aligned16(workspace) || workspace_bytes < need) return FORGE_ERR_WORKSPACE;
+    DecParams p;
+    p.seq_lens = seq_lens;
+    p.sink = sink;
+    p.part = static_cast<float *>(workspace);
+    p.lse = lse;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.T = T; p.Tmax = Tmax;
+    p.window = effective_window(window, T);
+    p.chunk = decode_chunk(B, Hkv, T);
+    p.nsplit = (T + p.chunk - 1) / p.chunk;
+    p.qscale = softcap > 0.0f ? scale / softcap : scale * kLog2e;
+    p.cap_out = softcap > 0.0f ? softcap * kLog2e : 0.0f;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dtype == FORGE_DTYPE_BF16) {
+        FORGE_DISPATCH_D(D, return decode_run<__nv_bfloat16, kD>(q, k_cache, v_cache, o, p, st);)
+    } else {
+        FORGE_DISPATCH_D(D, return decode_run<float, kD>(q, k_cache, v_cache, o, p, st);)
+    }
+    return FORGE_ERR_UNSUPPORTED;
 }
 
 forge_status forge_attn_check(void *stream) {

@@ -20,6 +20,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include "sm100.cuh"
+
 namespace forge {
 
 constexpr int kSimtRows = 16;  // rows per block

@@ -16,7 +16,7 @@ namespace forge {
 // wins); forge_attn_check reads and clears it.
 __device__ int g_status;
 
-enum : int { kStatusUnsupported = 2, kStatusTimeout = 5 };
+enum : int { kStatusInvalidArg = 1, kStatusUnsupported = 2, kStatusTimeout = 5 };
 
 // Where the first timed-out wait happened: [0] = 1 + barrier shared-memory
 // address, [1] = block index, [2] = thread index, [3] = (block size << 20) |

@@ -176,6 +176,35 @@ forge_status forge_attn_bwd_finalize(void *dq, int B, int Hq, int Hkv, int T, in
                                      void *stream);
 
 /*
+ * Decode: one new query per (batch entry, query head) against a KV cache
+ * (INFERENCE_RESEARCH.md section 2: the cache is pre-allocated to the maximum
+ * length, laid out [layer][head][seq][d], and decoding gets a dedicated kernel
+ * with one query, split along the cache for long contexts).
+ *   q, o               : [B][Hq][D] (dtype), the new token's queries / outputs
+ *   k_cache, v_cache   : [B][Hkv][Tmax][D] (dtype), one layer's cache
+ *   lse                : [B][Hq] f32 (may be NULL)
+ *   seq_lens           : [B] int32 (device, may be NULL): entry b holds
+ *                        seq_lens[b] valid positions, 1 <= seq_lens[b] <= T; NULL
+ *                        means every entry holds T. Entry b's query sits at
+ *                        position len - 1 and sees keys [len - window, len - 1]
+ *                        clipped at 0 (window 0: all len), capped and scaled as in
+ *                        the forward; sink (may be NULL) as in forge_attn_fwd_ext.
+ *                        A length outside [1, T] is reported as
+ *                        FORGE_ERR_INVALID_ARG by the next forge_attn_check.
+ *   T <= Tmax; Hq / Hkv <= 16; D in {64, 128, 256}; dtype bf16 or f32.
+ * workspace: device memory of at least forge_attn_decode_workspace_size(B, Hq,
+ * Hkv, T, D) bytes, 16-byte aligned (per-chunk partial results), overwritten.
+ * Two kernels on `stream`: the split pass (one CTA per key chunk, batch entry and
+ * KV head, all of the group's query heads at once) and the combine pass.
+ */
+size_t forge_attn_decode_workspace_size(int B, int Hq, int Hkv, int T, int D);
+forge_status forge_attn_decode(const void *q, const void *k_cache, const void *v_cache, void *o,
+                               float *lse, const int *seq_lens, int B, int Hq, int Hkv, int T,
+                               int Tmax, int D, float scale, int window, float softcap,
+                               const float *sink, forge_dtype dtype, void *workspace,
+                               size_t workspace_bytes, void *stream);
+
+/*
  * Synchronises `stream`, then reports (and clears) any error a kernel of this
  * library recorded on the current device since the last check: FORGE_OK,
  * FORGE_ERR_TIMEOUT, or FORGE_ERR_CUDA for an asynchronous CUDA error.
