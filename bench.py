@@ -501,7 +501,8 @@ def run_decode(args):
             "dtype": "bf16", "data": "synthetic (seeded N(0,1) q and caches)",
             "config": dict(c, l2="not flushed: the 1.07 GB cache exceeds the 126 MB L2"),
             "roofline": {"kernel": "decode_split", "bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
-                         "unit": "GB/s", "frac": round(gbs / peak, 4), "traffic": None,
+                         "unit": "GB/s", "frac": round(gbs / peak, 4),
+                         "traffic": ncu_traffic("decode_split", c["workload"]),
                          "peak_source": f"{peak_src} hbm_gbs",
                          "achieved_def": "K+V cache bytes + q, o, lse bytes per call / CUDA-event time of both kernels"},
             "gpu_launches": 2 * args.steps, "clocks": clocks}
