@@ -52,13 +52,39 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def _strip_comments(text):
+    """C/C++ source without // and /* */ comments (string literals kept), so that
+    the hash below changes with the code and not with its comments."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"':
+            j = i + 1
+            while j < n and text[j] != '"':
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return "".join(out)
+
+
 def kernel_source_hash():
+    """sha256 prefix of causal_flash_attention_attn_b200/csrc/* without comments,
+    whitespace runs collapsed (layout and comment edits leave it unchanged)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "causal_flash_attention_attn_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
+        with open(os.path.join(csrc, name), "r", encoding="utf-8") as f:
             h.update(name.encode())
-            h.update(f.read())
+            h.update(" ".join(_strip_comments(f.read()).split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -34,9 +34,17 @@
 //   D = 256: BM = 64, two CTAs per key tile, each owning half of the head dim
 //            (DH = 128) for dK, dV and dQ; S^T and dP^T use the full head dim.
 //
-// Roles (320 threads): warps 0-3 compute (one thread per key row, TMEM lane),
-// warps 4-7 dQ drain + dK epilogue, warp 8 loads (TMA for tiles, plain loads
-// for LSE and Delta), warp 9 issues MMAs and owns TMEM.
+// Each step runs in two phases on the compute warps: phase A (needs S^T) forms
+// P^T into TMEM and keeps the factors of dS in registers; phase B (needs dP^T)
+// forms dS^T into shared memory. The MMA warp issues dV(i) as soon as phase A
+// of step i ends and S^T(i + 1) right after it, so S^T(i + 1) and dV(i) run
+// during phase B, and dP^T(i + 1) during phase A of step i + 1.
+//
+// Roles (512 threads): warps 0-7 compute (warp w: key rows = TMEM lanes
+// 32 (w % 4).., query-row half w / 4 of the step), warps 8-11 dQ drain + dK
+// epilogue, warp 12 loads (TMA for tiles, plain loads for LSE and Delta), warp
+// 13 issues MMAs and owns TMEM, warps 14-15 idle (see BwdTc for the register
+// split).
 #pragma once
 
 #include "sm100.cuh"
