@@ -13,7 +13,9 @@ plain softmax bit for bit; a sink being an extra zero-value key at position 0
 closed form; central differences of dsink; a hand-worked max-logit example. The
 decode function is pinned to the last row of the pinned forward (bit for bit, with
 window, cap and sink), to per-entry lengths with the cache tail poisoned, and to the
-length-1 closed form. No function here is left unpinned.
+length-1 closed form. The d_k != d_v form of attn_fwd_ext / attn_bwd_ext is pinned to
+torch SDPA autograd in f64 (SDPA takes a value head dim of its own) and to the
+independence of the value columns. No function here is left unpinned.
 
 Every function takes and returns numpy float64 arrays in [B, H, T, D] layout.
 """
@@ -38,8 +40,8 @@ def _load():
         i = ctypes.c_int
         d = ctypes.c_double
         lib.oracle_attn_fwd.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i, d, i, d]
-        lib.oracle_attn_fwd_ext.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, d, i, d]
-        lib.oracle_attn_bwd_ext.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, d, i, d, i]
+        lib.oracle_attn_fwd_ext.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, d, i, d]
+        lib.oracle_attn_bwd_ext.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, d, i, d, i]
         lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, d, i, d, i]
         lib.oracle_attn_decode.argtypes = [dp, dp, dp, dp, ctypes.POINTER(ctypes.c_int), dp, dp, i, i, i, i, i, i, d,
                                            i, d]
@@ -66,6 +68,13 @@ def _dims(q, k):
     Bk, Hkv, Tk, Dk = k.shape
     assert (B, T, D) == (Bk, Tk, Dk) and Hq % Hkv == 0
     return B, Hq, Hkv, T, D
+
+
+def _dims_kv(q, k, v):
+    """(B, Hq, Hkv, T, Dk, Dv): the key head dim of q and k, the value head dim of v."""
+    B, Hq, Hkv, T, Dk = _dims(q, k)
+    assert v.shape[:3] == (B, Hkv, T)
+    return B, Hq, Hkv, T, Dk, v.shape[3]
 
 
 def num_threads() -> int:
@@ -118,17 +127,18 @@ def _ptr_or_null(a):
 
 
 def attn_fwd_ext(q, k, v, scale: float, window: int = 0, softcap: float = 0.0, sink=None):
-    """Forward with an optional per-head sink logit sink [Hq]. Returns (o, lse,
+    """Forward with an optional per-head sink logit sink [Hq]; v (and o) may have a
+    head dim other than q and k (d_k != d_v). Returns (o, lse,
     max_logit [B, Hq]); max_logit is the per-(b, hq) maximum of the scores the
     softmax sees over the allowed pairs (the sink not included)."""
     q, k, v = _f64(q), _f64(k), _f64(v)
-    B, Hq, Hkv, T, D = _dims(q, k)
+    B, Hq, Hkv, T, Dk, Dv = _dims_kv(q, k, v)
     sk = None if sink is None else _f64(sink).reshape(Hq)
-    o = np.empty_like(q)
+    o = np.empty((B, Hq, T, Dv), dtype=np.float64)
     lse = np.empty((B, Hq, T), dtype=np.float64)
     ml = np.empty((B, Hq), dtype=np.float64)
     _load().oracle_attn_fwd_ext(_ptr(q), _ptr(k), _ptr(v), _ptr_or_null(sk), _ptr(o), _ptr(lse), _ptr(ml),
-                                B, Hq, Hkv, T, D, float(scale), int(window), float(softcap))
+                                B, Hq, Hkv, T, Dk, Dv, float(scale), int(window), float(softcap))
     return o, lse, ml
 
 
@@ -136,7 +146,8 @@ def attn_bwd_ext(q, k, v, dO, scale: float, window: int = 0, softcap: float = 0.
     """Backward with an optional per-head sink logit sink [Hq]. Returns (dq, dk,
     dv, dsink [Hq] (zeros without a sink), delta, lse)."""
     q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
-    B, Hq, Hkv, T, D = _dims(q, k)
+    B, Hq, Hkv, T, Dk, Dv = _dims_kv(q, k, v)
+    assert dO.shape == (B, Hq, T, Dv)
     sk = None if sink is None else _f64(sink).reshape(Hq)
     dq = np.empty_like(q)
     dk = np.empty_like(k)
@@ -145,7 +156,7 @@ def attn_bwd_ext(q, k, v, dO, scale: float, window: int = 0, softcap: float = 0.
     delta = np.empty((B, Hq, T), dtype=np.float64)
     lse = np.empty((B, Hq, T), dtype=np.float64)
     _load().oracle_attn_bwd_ext(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr_or_null(sk), _ptr(dq), _ptr(dk),
-                                _ptr(dv), _ptr(dsink), _ptr(delta), _ptr(lse), B, Hq, Hkv, T, D, float(scale),
+                                _ptr(dv), _ptr(dsink), _ptr(delta), _ptr(lse), B, Hq, Hkv, T, Dk, Dv, float(scale),
                                 int(window), float(softcap), _ROUND[o_round])
     return dq, dk, dv, dsink, delta, lse
 

@@ -37,7 +37,12 @@
  *    the softmax sees (after scale and cap), the sink not included.
  *
  * Layouts: q, o, dO, dq are [B][Hq][T][D]; k, v, dk, dv are [B][Hkv][T][D];
- * lse and delta are [B][Hq][T]; all row-major, f64.
+ * lse and delta are [B][Hq][T]; all row-major, f64. The _ext functions take
+ * the key head dim Dk (q, k, dq, dk) and the value head dim Dv (v, o, dO, dv)
+ * separately: d_k != d_v is the decompressed form of multi-head latent
+ * attention (ARCHITECTURES.md "Vague 3" item 13 and the family table's DeepSeek
+ * V3 row: nope 128 + rope 64 = 192 for q.k, v 128), with the scale chosen by the
+ * caller (1/sqrt(192) there).
  */
 #include <math.h>
 #include <stdint.h>
@@ -130,7 +135,7 @@ static double sink_of(const double *sink, int hq) { return sink ? sink[hq] : -IN
  */
 void oracle_attn_fwd_ext(const double *q, const double *k, const double *v, const double *sink,
                          double *o, double *lse, double *max_logit, int B, int Hq, int Hkv, int T,
-                         int D, double scale, int window, double softcap) {
+                         int Dk, int Dv, double scale, int window, double softcap) {
     const int G = Hq / Hkv;
     double *rowmax = (double *)malloc(sizeof(double) * (size_t)B * Hq * T);
 #pragma omp parallel
@@ -142,16 +147,16 @@ void oracle_attn_fwd_ext(const double *q, const double *k, const double *v, cons
                 for (int i = 0; i < T; i++) {
                     const int hkv = hq / G;
                     const size_t qrow = ((size_t)(b * Hq + hq) * T + i);
-                    const double *qi = q + qrow * D;
-                    const double *K = k + (size_t)(b * Hkv + hkv) * T * D;
-                    const double *V = v + (size_t)(b * Hkv + hkv) * T * D;
+                    const double *qi = q + qrow * Dk;
+                    const double *K = k + (size_t)(b * Hkv + hkv) * T * Dk;
+                    const double *V = v + (size_t)(b * Hkv + hkv) * T * Dv;
                     const long lo = first_key(i, window);
-                    lse[qrow] = row_probs(qi, K, i, lo, D, scale, softcap, sink_of(sink, hq), p,
+                    lse[qrow] = row_probs(qi, K, i, lo, Dk, scale, softcap, sink_of(sink, hq), p,
                                           rowmax + qrow);
-                    double *oi = o + qrow * D;
-                    for (int d = 0; d < D; d++) oi[d] = 0.0;
+                    double *oi = o + qrow * Dv;
+                    for (int d = 0; d < Dv; d++) oi[d] = 0.0;
                     for (long j = lo; j <= i; j++)
-                        for (int d = 0; d < D; d++) oi[d] += p[j] * V[j * D + d];
+                        for (int d = 0; d < Dv; d++) oi[d] += p[j] * V[j * Dv + d];
                 }
         free(p);
     }
@@ -169,7 +174,7 @@ void oracle_attn_fwd_ext(const double *q, const double *k, const double *v, cons
 void oracle_attn_fwd(const double *q, const double *k, const double *v, double *o, double *lse,
                      int B, int Hq, int Hkv, int T, int D, double scale, int window,
                      double softcap) {
-    oracle_attn_fwd_ext(q, k, v, NULL, o, lse, NULL, B, Hq, Hkv, T, D, scale, window, softcap);
+    oracle_attn_fwd_ext(q, k, v, NULL, o, lse, NULL, B, Hq, Hkv, T, D, D, scale, window, softcap);
 }
 
 /*
@@ -197,8 +202,8 @@ void oracle_attn_fwd(const double *q, const double *k, const double *v, double *
  */
 void oracle_attn_bwd_ext(const double *q, const double *k, const double *v, const double *dO,
                          const double *sink, double *dq, double *dk, double *dv, double *dsink,
-                         double *delta, double *lse_out, int B, int Hq, int Hkv, int T, int D,
-                         double scale, int window, double softcap, int o_round) {
+                         double *delta, double *lse_out, int B, int Hq, int Hkv, int T, int Dk,
+                         int Dv, double scale, int window, double softcap, int o_round) {
     const int G = Hq / Hkv;
     const size_t nrows = (size_t)B * Hq * T;
     double *lse = (double *)malloc(sizeof(double) * nrows);
@@ -209,38 +214,38 @@ void oracle_attn_bwd_ext(const double *q, const double *k, const double *v, cons
     {
         double *p = (double *)malloc(sizeof(double) * (size_t)T);
         double *dp = (double *)malloc(sizeof(double) * (size_t)T);
-        double *oi = (double *)malloc(sizeof(double) * (size_t)D);
+        double *oi = (double *)malloc(sizeof(double) * (size_t)Dv);
 #pragma omp for collapse(3) schedule(dynamic, 8)
         for (int b = 0; b < B; b++)
             for (int hq = 0; hq < Hq; hq++)
                 for (int i = 0; i < T; i++) {
                     const int hkv = hq / G;
                     const size_t qrow = ((size_t)(b * Hq + hq) * T + i);
-                    const double *qi = q + qrow * D;
-                    const double *doi = dO + qrow * D;
-                    const double *K = k + (size_t)(b * Hkv + hkv) * T * D;
-                    const double *V = v + (size_t)(b * Hkv + hkv) * T * D;
+                    const double *qi = q + qrow * Dk;
+                    const double *doi = dO + qrow * Dv;
+                    const double *K = k + (size_t)(b * Hkv + hkv) * T * Dk;
+                    const double *V = v + (size_t)(b * Hkv + hkv) * T * Dv;
                     const long lo = first_key(i, window);
-                    lse[qrow] = row_probs(qi, K, i, lo, D, scale, softcap, sink_of(sink, hq), p, NULL);
+                    lse[qrow] = row_probs(qi, K, i, lo, Dk, scale, softcap, sink_of(sink, hq), p, NULL);
                     double dl = 0.0;
                     for (long j = lo; j <= i; j++) {
-                        dp[j] = dot(doi, V + j * D, D);
+                        dp[j] = dot(doi, V + j * Dv, Dv);
                         dl += p[j] * dp[j];
                     }
                     if (o_round != 0) {
-                        for (int d = 0; d < D; d++) oi[d] = 0.0;
+                        for (int d = 0; d < Dv; d++) oi[d] = 0.0;
                         for (long j = lo; j <= i; j++)
-                            for (int d = 0; d < D; d++) oi[d] += p[j] * V[j * D + d];
+                            for (int d = 0; d < Dv; d++) oi[d] += p[j] * V[j * Dv + d];
                         dl = 0.0;
-                        for (int d = 0; d < D; d++) dl += doi[d] * round_to(oi[d], o_round);
+                        for (int d = 0; d < Dv; d++) dl += doi[d] * round_to(oi[d], o_round);
                     }
                     dlt[qrow] = dl;
-                    double *dqi = dq + qrow * D;
-                    for (int d = 0; d < D; d++) dqi[d] = 0.0;
+                    double *dqi = dq + qrow * Dk;
+                    for (int d = 0; d < Dk; d++) dqi[d] = 0.0;
                     for (long j = lo; j <= i; j++) {
-                        const double s = raw_score(qi, K + j * D, D, scale);
+                        const double s = raw_score(qi, K + j * Dk, Dk, scale);
                         const double ds = p[j] * (dp[j] - dl) * cap_grad(s, softcap);
-                        for (int d = 0; d < D; d++) dqi[d] += scale * ds * K[j * D + d];
+                        for (int d = 0; d < Dk; d++) dqi[d] += scale * ds * K[j * Dk + d];
                     }
                 }
         free(p);
@@ -253,29 +258,28 @@ void oracle_attn_bwd_ext(const double *q, const double *k, const double *v, cons
     for (int b = 0; b < B; b++)
         for (int hkv = 0; hkv < Hkv; hkv++)
             for (int j = 0; j < T; j++) {
-                const double *K = k + (size_t)(b * Hkv + hkv) * T * D;
-                const double *V = v + (size_t)(b * Hkv + hkv) * T * D;
-                const double *kj = K + (size_t)j * D;
-                const double *vj = V + (size_t)j * D;
-                double *dkj = dk + ((size_t)(b * Hkv + hkv) * T + j) * D;
-                double *dvj = dv + ((size_t)(b * Hkv + hkv) * T + j) * D;
-                for (int d = 0; d < D; d++) dkj[d] = dvj[d] = 0.0;
+                const double *K = k + (size_t)(b * Hkv + hkv) * T * Dk;
+                const double *V = v + (size_t)(b * Hkv + hkv) * T * Dv;
+                const double *kj = K + (size_t)j * Dk;
+                const double *vj = V + (size_t)j * Dv;
+                double *dkj = dk + ((size_t)(b * Hkv + hkv) * T + j) * Dk;
+                double *dvj = dv + ((size_t)(b * Hkv + hkv) * T + j) * Dv;
+                for (int d = 0; d < Dk; d++) dkj[d] = 0.0;
+                for (int d = 0; d < Dv; d++) dvj[d] = 0.0;
                 long last = T - 1;
                 if (window > 0 && (long)j + window - 1 < last) last = (long)j + window - 1;
                 for (int g = 0; g < G; g++) {
                     const int hq = hkv * G + g;
                     for (long i = j; i <= last; i++) {
                         const size_t qrow = ((size_t)(b * Hq + hq) * T + i);
-                        const double *qi = q + qrow * D;
-                        const double *doi = dO + qrow * D;
-                        const double s = raw_score(qi, kj, D, scale);
+                        const double *qi = q + qrow * Dk;
+                        const double *doi = dO + qrow * Dv;
+                        const double s = raw_score(qi, kj, Dk, scale);
                         const double pij = exp(capped(s, softcap) - lse[qrow]);
-                        const double dpij = dot(doi, vj, D);
+                        const double dpij = dot(doi, vj, Dv);
                         const double ds = pij * (dpij - dlt[qrow]) * cap_grad(s, softcap);
-                        for (int d = 0; d < D; d++) {
-                            dvj[d] += pij * doi[d];
-                            dkj[d] += scale * ds * qi[d];
-                        }
+                        for (int d = 0; d < Dv; d++) dvj[d] += pij * doi[d];
+                        for (int d = 0; d < Dk; d++) dkj[d] += scale * ds * qi[d];
                     }
                 }
             }
@@ -303,7 +307,7 @@ void oracle_attn_bwd(const double *q, const double *k, const double *v, const do
                      double *dq, double *dk, double *dv, double *delta, double *lse_out,
                      int B, int Hq, int Hkv, int T, int D, double scale, int window,
                      double softcap, int o_round) {
-    oracle_attn_bwd_ext(q, k, v, dO, NULL, dq, dk, dv, NULL, delta, lse_out, B, Hq, Hkv, T, D,
+    oracle_attn_bwd_ext(q, k, v, dO, NULL, dq, dk, dv, NULL, delta, lse_out, B, Hq, Hkv, T, D, D,
                         scale, window, softcap, o_round);
 }
 

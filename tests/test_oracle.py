@@ -538,3 +538,48 @@ def test_decode_per_entry_lengths_and_cache_tail_ignored():
     # length 1 sees only position 0: o = v[0], lse = the one score
     np.testing.assert_allclose(o[1], np.repeat(vc[1, :, 0], Hq // Hkv, axis=0), rtol=1e-15)
     np.testing.assert_allclose(lse[1], scale * (q[1] @ kc[1, 0, 0]), rtol=1e-14)
+
+
+# ---------------------------------------------------------------- d_k != d_v
+# Decompressed multi-head latent attention: q.k over d_k = nope + rope, values of
+# d_v ("Vague 3" item 13; family table, DeepSeek V3 row).
+
+@pytest.mark.parametrize("B,Hq,Hkv,T,Dk,Dv,W,C", [
+    (1, 2, 2, 23, 12, 8, 0, 0.0),
+    (2, 4, 2, 31, 24, 16, 5, 0.0),
+    (1, 2, 1, 19, 8, 12, 0, 3.0),   # d_v > d_k too
+    (1, 3, 3, 27, 12, 8, 7, 2.0),
+])
+def test_dk_ne_dv_matches_torch_sdpa_autograd(B, Hq, Hkv, T, Dk, Dv, W, C):
+    sig = 2.0 if C else 1.0
+    q, k = rnd((B, Hq, T, Dk), 31, sig), rnd((B, Hkv, T, Dk), 32, sig)
+    v, dO = rnd((B, Hkv, T, Dv), 33), rnd((B, Hq, T, Dv), 34)
+    scale = 1.0 / math.sqrt(Dk)
+    o_ref, dq_ref, dk_ref, dv_ref = sdpa_grads(q, k, v, dO, scale, W, C)
+    o, lse, _ = oracle.attn_fwd_ext(q, k, v, scale, W, C)
+    assert o.shape == (B, Hq, T, Dv)
+    np.testing.assert_allclose(o, o_ref.numpy(), rtol=1e-12, atol=1e-12)
+    dq, dk, dv, _, _, lse2 = oracle.attn_bwd_ext(q, k, v, dO, scale, W, C)
+    np.testing.assert_allclose(dq, dq_ref.numpy(), rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(dk, dk_ref.numpy(), rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(dv, dv_ref.numpy(), rtol=1e-10, atol=1e-11)
+    np.testing.assert_array_equal(lse, lse2)
+
+
+def test_dk_ne_dv_value_columns_are_independent():
+    # o's value columns come from v's alone: cutting v (and dO) to its first
+    # columns gives the first columns of o and dv, and the same dq, dk when dO
+    # is zero on the columns cut
+    B, Hq, Hkv, T, Dk, Dv = 1, 2, 1, 17, 8, 12
+    q, k = rnd((B, Hq, T, Dk), 35), rnd((B, Hkv, T, Dk), 36)
+    v, dO = rnd((B, Hkv, T, Dv), 37), rnd((B, Hq, T, Dv), 38)
+    dO[..., 5:] = 0.0
+    o, lse, _ = oracle.attn_fwd_ext(q, k, v, 0.3)
+    o5, lse5, _ = oracle.attn_fwd_ext(q, k, v[..., :5], 0.3)
+    np.testing.assert_array_equal(o[..., :5], o5)
+    np.testing.assert_array_equal(lse, lse5)
+    g = oracle.attn_bwd_ext(q, k, v, dO, 0.3)
+    g5 = oracle.attn_bwd_ext(q, k, v[..., :5], dO[..., :5], 0.3)
+    np.testing.assert_allclose(g[0], g5[0], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(g[1], g5[1], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(g[2][..., :5], g5[2], rtol=1e-13, atol=1e-14)
