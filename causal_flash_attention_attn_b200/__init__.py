@@ -20,7 +20,8 @@ __all__ = [
     "FORGE_ERR_CUDA", "FORGE_ERR_TIMEOUT", "FORGE_DTYPE_F32", "FORGE_DTYPE_BF16", "ForgeError",
     "library", "library_path", "forge_attn_fwd", "forge_attn_bwd", "forge_attn_bwd_workspace_size",
     "forge_attn_bwd_noalloc", "forge_attn_fwd_ext", "forge_attn_bwd_ext", "forge_attn_decode",
-    "forge_attn_decode_workspace_size", "attention_decode",
+    "forge_attn_decode_workspace_size", "attention_decode", "forge_attn_fwd_dkv", "forge_attn_bwd_dkv",
+    "forge_attn_bwd_workspace_size_dkv",
     "forge_attn_bwd_preprocess", "forge_attn_bwd_main", "forge_attn_bwd_finalize", "forge_attn_check",
     "forge_attn_status_string", "forge_attn_selftest_timeout", "forge_attn_selftest_exp2", "forge_attn_last_cuda_error", "forge_attn_timeout_info", "forge_attn_version",
     "attention_fwd", "attention_bwd", "dtype_code",
@@ -73,6 +74,12 @@ def library():
     L.forge_attn_fwd_ext.restype = i
     L.forge_attn_bwd_ext.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, f, vp, vp, i, vp, st, vp]
     L.forge_attn_bwd_ext.restype = i
+    L.forge_attn_fwd_dkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, f, i, vp]
+    L.forge_attn_fwd_dkv.restype = i
+    L.forge_attn_bwd_workspace_size_dkv.argtypes = [i, i, i, i, i, i, i]
+    L.forge_attn_bwd_workspace_size_dkv.restype = st
+    L.forge_attn_bwd_dkv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, f, i, vp, st, vp]
+    L.forge_attn_bwd_dkv.restype = i
     L.forge_attn_decode_workspace_size.argtypes = [i, i, i, i, i]
     L.forge_attn_decode_workspace_size.restype = st
     L.forge_attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, f, vp, i, vp, st, vp]
@@ -160,6 +167,23 @@ def forge_attn_bwd_ext(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale,
                                         _ptr(dk), _ptr(dv), B, Hq, Hkv, T, D, float(scale), int(window),
                                         float(softcap), _ptr(sink), _ptr(dsink), int(dtype), _ptr(workspace),
                                         int(workspace_bytes), _stream(stream))
+
+
+def forge_attn_fwd_dkv(q, k, v, o, lse, B, Hq, Hkv, T, Dk, Dv, scale, window, softcap, dtype, stream=None) -> int:
+    return library().forge_attn_fwd_dkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, T, Dk, Dv,
+                                        float(scale), int(window), float(softcap), int(dtype), _stream(stream))
+
+
+def forge_attn_bwd_workspace_size_dkv(B, Hq, Hkv, T, Dk, Dv, dtype) -> int:
+    return int(library().forge_attn_bwd_workspace_size_dkv(B, Hq, Hkv, T, Dk, Dv, int(dtype)))
+
+
+def forge_attn_bwd_dkv(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, Dk, Dv, scale, window, softcap, dtype,
+                       workspace, workspace_bytes, stream=None) -> int:
+    return library().forge_attn_bwd_dkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
+                                        _ptr(dk), _ptr(dv), B, Hq, Hkv, T, Dk, Dv, float(scale), int(window),
+                                        float(softcap), int(dtype), _ptr(workspace), int(workspace_bytes),
+                                        _stream(stream))
 
 
 def forge_attn_decode_workspace_size(B, Hq, Hkv, T, D) -> int:

@@ -165,33 +165,33 @@ forge_status fwd_tc(const void *q, const void *k, const void *v, void *o, float 
     return launch_status();
 }
 
-template <typename T_, int D>
+template <typename T_, int DK, int DV = DK>
 forge_status fwd_simt(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv, int T,
                       float scale, int window, float softcap, const float *sink, float *max_logit, cudaStream_t st) {
-    const size_t sm = simt_fwd_smem<D>();
-    if (set_smem(simt_fwd<T_, D>, sm) != FORGE_OK) return FORGE_ERR_CUDA;
+    const size_t sm = simt_fwd_smem<DK, DV>();
+    if (set_smem(simt_fwd<T_, DK, DV>, sm) != FORGE_OK) return FORGE_ERR_CUDA;
     dim3 grid((T + kSimtRows - 1) / kSimtRows, B * Hq);
-    simt_fwd<T_, D><<<grid, kSimtThreads, sm, st>>>(static_cast<const T_ *>(q), static_cast<const T_ *>(k),
+    simt_fwd<T_, DK, DV><<<grid, kSimtThreads, sm, st>>>(static_cast<const T_ *>(q), static_cast<const T_ *>(k),
                                                      static_cast<const T_ *>(v), static_cast<T_ *>(o), lse, Hq, Hkv,
                                                      T, scale, window, softcap, sink, max_logit);
     return launch_status();
 }
 
-template <typename T_, int D>
+template <typename T_, int DK, int DV = DK>
 forge_status bwd_simt(const void *q, const void *k, const void *v, const float *lse, const void *dO,
                       const float *delta, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int T, float scale,
                       int window, float softcap, cudaStream_t st) {
-    const size_t sm1 = simt_bwd_dq_smem<D>(), sm2 = simt_bwd_dkdv_smem<D>();
-    if (set_smem(simt_bwd_dq<T_, D>, sm1) != FORGE_OK || set_smem(simt_bwd_dkdv<T_, D>, sm2) != FORGE_OK)
+    const size_t sm1 = simt_bwd_dq_smem<DK, DV>(), sm2 = simt_bwd_dkdv_smem<DK, DV>();
+    if (set_smem(simt_bwd_dq<T_, DK, DV>, sm1) != FORGE_OK || set_smem(simt_bwd_dkdv<T_, DK, DV>, sm2) != FORGE_OK)
         return FORGE_ERR_CUDA;
     dim3 g1((T + kSimtRows - 1) / kSimtRows, B * Hq);
-    simt_bwd_dq<T_, D><<<g1, kSimtThreads, sm1, st>>>(
+    simt_bwd_dq<T_, DK, DV><<<g1, kSimtThreads, sm1, st>>>(
         static_cast<const T_ *>(q), static_cast<const T_ *>(k), static_cast<const T_ *>(v), lse,
         static_cast<const T_ *>(dO), delta, static_cast<T_ *>(dq), Hq, Hkv, T, scale, window, softcap);
     forge_status s = launch_status();
     if (s != FORGE_OK) return s;
     dim3 g2((T + kSimtRows - 1) / kSimtRows, B * Hkv);
-    simt_bwd_dkdv<T_, D><<<g2, kSimtThreads, sm2, st>>>(
+    simt_bwd_dkdv<T_, DK, DV><<<g2, kSimtThreads, sm2, st>>>(
         static_cast<const T_ *>(q), static_cast<const T_ *>(k), static_cast<const T_ *>(v), lse,
         static_cast<const T_ *>(dO), delta, static_cast<T_ *>(dk), static_cast<T_ *>(dv), Hq, Hkv, T, scale, window,
         softcap);
@@ -526,6 +526,61 @@ forge_status forge_attn_bwd_noalloc(const void *q, const void *k, const void *v,
     // so whatever the previous call left in the array does not matter
     return forge_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale, window, softcap, dtype, scratch,
                           kNoAllocScratchBytes, stream);
+}
+
+// d_k != d_v: the f32 CUDA-core path at (d_k, d_v) = (192, 128), the decompressed
+// multi-head latent attention of the DeepSeek V3 family; the tensor-core kernels
+// keep d_k = d_v for now.
+static bool dkv_supported(int Dk, int Dv, forge_dtype dtype) {
+    return dtype == FORGE_DTYPE_F32 && Dk == 192 && Dv == 128;
+}
+
+size_t forge_attn_bwd_workspace_size_dkv(int B, int Hq, int Hkv, int T, int Dk, int Dv, forge_dtype dtype) {
+    if (Dk == Dv) return forge_attn_bwd_workspace_size(B, Hq, Hkv, T, Dk, dtype);
+    if (!dkv_supported(Dk, Dv, dtype) || check_sizes(B, Hq, Hkv, T, Dv, dtype) != FORGE_OK) return 0;
+    return delta_bytes(B, Hq, T);  // Delta only: the f32 path writes dq directly
+}
+
+forge_status forge_attn_fwd_dkv(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+                                int Hkv, int T, int Dk, int Dv, float scale, int window, float softcap,
+                                forge_dtype dtype, void *stream) {
+    if (Dk == Dv) return forge_attn_fwd(q, k, v, o, lse, B, Hq, Hkv, T, Dk, scale, window, softcap, dtype, stream);
+    forge_status s = check_sizes(B, Hq, Hkv, T, Dv, dtype);
+    if (s != FORGE_OK) return s;
+    if (!dkv_supported(Dk, Dv, dtype)) return FORGE_ERR_UNSUPPORTED;
+    if ((s = check_scalars(scale, window, softcap)) != FORGE_OK) return s;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return FORGE_ERR_INVALID_ARG;
+    window = effective_window(window, T);
+    return fwd_simt<float, 192, 128>(q, k, v, o, lse, B, Hq, Hkv, T, scale, window, softcap, nullptr, nullptr,
+                                     static_cast<cudaStream_t>(stream));
+}
+
+forge_status forge_attn_bwd_dkv(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                                const void *dO, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int T, int Dk,
+                                int Dv, float scale, int window, float softcap, forge_dtype dtype, void *workspace,
+                                size_t workspace_bytes, void *stream) {
+    if (Dk == Dv)
+        return forge_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, Dk, scale, window, softcap, dtype,
+                              workspace, workspace_bytes, stream);
+    forge_status s = check_sizes(B, Hq, Hkv, T, Dv, dtype);
+    if (s != FORGE_OK) return s;
+    if (!dkv_supported(Dk, Dv, dtype)) return FORGE_ERR_UNSUPPORTED;
+    if ((s = check_scalars(scale, window, softcap)) != FORGE_OK) return s;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dO) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return FORGE_ERR_INVALID_ARG;
+    if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+        workspace_bytes < forge_attn_bwd_workspace_size_dkv(B, Hq, Hkv, T, Dk, Dv, dtype))
+        return FORGE_ERR_WORKSPACE;
+    window = effective_window(window, T);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float *delta = static_cast<float *>(workspace);
+    const long rows = (long)B * Hq * T;
+    bwd_preprocess<float, 128><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
+        static_cast<const float *>(o), static_cast<const float *>(dO), delta, nullptr, rows, T, tpad_of(T));
+    if ((s = launch_status()) != FORGE_OK) return s;
+    return bwd_simt<float, 192, 128>(q, k, v, lse, dO, delta, dq, dk, dv, B, Hq, Hkv, T, scale, window, softcap, st);
 }
 
 size_t forge_attn_decode_workspace_size(int B, int Hq, int Hkv, int T, int D) {

@@ -63,12 +63,14 @@ __device__ __forceinline__ void load_rows(float *dst, int ld, const T *src, int 
     }
 }
 
-template <int D>
+// DK: head dim of q and k; DV: head dim of v and o (equal except for the
+// decompressed multi-head latent attention, d_k = 192, d_v = 128).
+template <int DK, int DV>
 constexpr size_t simt_fwd_smem() {
-    return sizeof(float) * (size_t)(kSimtRows * D + 2 * kSimtTile * (D + 1));
+    return sizeof(float) * (size_t)(kSimtRows * DK + kSimtTile * (DK + 1) + kSimtTile * (DV + 1));
 }
 
-template <typename T, int D>
+template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(kSimtThreads) simt_fwd(const T *__restrict__ q, const T *__restrict__ k,
                                                          const T *__restrict__ v, T *__restrict__ o,
                                                          float *__restrict__ lse, int Hq, int Hkv, int T_,
@@ -76,16 +78,16 @@ __global__ void __launch_bounds__(kSimtThreads) simt_fwd(const T *__restrict__ q
                                                          const float *__restrict__ sink, float *__restrict__ max_logit) {
     extern __shared__ float sm[];
     float *sQ = sm;
-    float *sK = sQ + kSimtRows * D;
-    float *sV = sK + kSimtTile * (D + 1);
-    constexpr int NT = D / 32;
+    float *sK = sQ + kSimtRows * DK;
+    float *sV = sK + kSimtTile * (DK + 1);
+    constexpr int NT = DV / 32;
     const int bh = blockIdx.y, b = bh / Hq, hq = bh % Hq, hkv = hq / (Hq / Hkv);
     const int r0 = blockIdx.x * kSimtRows;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const T *Qb = q + (size_t)bh * T_ * D;
-    const T *Kb = k + (size_t)(b * Hkv + hkv) * T_ * D;
-    const T *Vb = v + (size_t)(b * Hkv + hkv) * T_ * D;
-    load_rows<T, D>(sQ, D, Qb, r0, kSimtRows, T_);
+    const T *Qb = q + (size_t)bh * T_ * DK;
+    const T *Kb = k + (size_t)(b * Hkv + hkv) * T_ * DK;
+    const T *Vb = v + (size_t)(b * Hkv + hkv) * T_ * DV;
+    load_rows<T, DK>(sQ, DK, Qb, r0, kSimtRows, T_);
 
     // a sink (natural units) starts each row's (max, sum) at (sink, 1)
     float m[4], l[4], acc[4][NT], mraw[4];
@@ -102,8 +104,8 @@ __global__ void __launch_bounds__(kSimtThreads) simt_fwd(const T *__restrict__ q
     first = (first / kSimtTile) * kSimtTile;
     for (int k0 = first; k0 <= last; k0 += kSimtTile) {
         __syncthreads();
-        load_rows<T, D>(sK, D + 1, Kb, k0, kSimtTile, T_);
-        load_rows<T, D>(sV, D + 1, Vb, k0, kSimtTile, T_);
+        load_rows<T, DK>(sK, DK + 1, Kb, k0, kSimtTile, T_);
+        load_rows<T, DV>(sV, DV + 1, Vb, k0, kSimtTile, T_);
         __syncthreads();
 #pragma unroll
         for (int rr = 0; rr < 4; rr++) {
@@ -112,7 +114,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_fwd(const T *__restrict__ q
             const int kj = k0 + lane;
             float s = 0.0f;
 #pragma unroll 8
-            for (int d = 0; d < D; d++) s = fmaf(sQ[r * D + d], sK[lane * (D + 1) + d], s);
+            for (int d = 0; d < DK; d++) s = fmaf(sQ[r * DK + d], sK[lane * (DK + 1) + d], s);
             s = simt_capped(s * scale, softcap);
             const bool ok = visible(qi, kj, window) && kj < T_;
             s = ok ? s : -INFINITY;
@@ -128,7 +130,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_fwd(const T *__restrict__ q
             for (int j = 0; j < kSimtTile; j++) {
                 const float pj = __shfl_sync(0xffffffffu, p, j);
 #pragma unroll
-                for (int t = 0; t < NT; t++) acc[rr][t] = fmaf(pj, sV[j * (D + 1) + lane + 32 * t], acc[rr][t]);
+                for (int t = 0; t < NT; t++) acc[rr][t] = fmaf(pj, sV[j * (DV + 1) + lane + 32 * t], acc[rr][t]);
             }
             m[rr] = mnew;
         }
@@ -138,7 +140,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_fwd(const T *__restrict__ q
         const int qi = r0 + warp * 4 + rr;
         if (qi >= T_) continue;
         const float inv = 1.0f / l[rr];
-        T *orow = o + ((size_t)bh * T_ + qi) * D;
+        T *orow = o + ((size_t)bh * T_ + qi) * DV;
 #pragma unroll
         for (int t = 0; t < NT; t++) from_f32(orow + lane + 32 * t, acc[rr][t] * inv);
         if (lane == 0) lse[(size_t)bh * T_ + qi] = m[rr] + logf(l[rr]);
@@ -146,12 +148,12 @@ __global__ void __launch_bounds__(kSimtThreads) simt_fwd(const T *__restrict__ q
     }
 }
 
-template <int D>
+template <int DK, int DV>
 constexpr size_t simt_bwd_dq_smem() {
-    return sizeof(float) * (size_t)(2 * kSimtRows * D + 2 * kSimtTile * (D + 1));
+    return sizeof(float) * (size_t)(kSimtRows * (DK + DV) + kSimtTile * (DK + 1) + kSimtTile * (DV + 1));
 }
 
-template <typename T, int D>
+template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(kSimtThreads) simt_bwd_dq(const T *__restrict__ q, const T *__restrict__ k,
                                                             const T *__restrict__ v, const float *__restrict__ lse,
                                                             const T *__restrict__ dO, const float *__restrict__ delta,
@@ -159,17 +161,17 @@ __global__ void __launch_bounds__(kSimtThreads) simt_bwd_dq(const T *__restrict_
                                                             int window, float softcap) {
     extern __shared__ float sm[];
     float *sQ = sm;
-    float *sdO = sQ + kSimtRows * D;
-    float *sK = sdO + kSimtRows * D;
-    float *sV = sK + kSimtTile * (D + 1);
-    constexpr int NT = D / 32;
+    float *sdO = sQ + kSimtRows * DK;
+    float *sK = sdO + kSimtRows * DV;
+    float *sV = sK + kSimtTile * (DK + 1);
+    constexpr int NT = DK / 32;
     const int bh = blockIdx.y, b = bh / Hq, hq = bh % Hq, hkv = hq / (Hq / Hkv);
     const int r0 = blockIdx.x * kSimtRows;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const T *Kb = k + (size_t)(b * Hkv + hkv) * T_ * D;
-    const T *Vb = v + (size_t)(b * Hkv + hkv) * T_ * D;
-    load_rows<T, D>(sQ, D, q + (size_t)bh * T_ * D, r0, kSimtRows, T_);
-    load_rows<T, D>(sdO, D, dO + (size_t)bh * T_ * D, r0, kSimtRows, T_);
+    const T *Kb = k + (size_t)(b * Hkv + hkv) * T_ * DK;
+    const T *Vb = v + (size_t)(b * Hkv + hkv) * T_ * DV;
+    load_rows<T, DK>(sQ, DK, q + (size_t)bh * T_ * DK, r0, kSimtRows, T_);
+    load_rows<T, DV>(sdO, DV, dO + (size_t)bh * T_ * DV, r0, kSimtRows, T_);
     float acc[4][NT], L[4], Dl[4];
 #pragma unroll
     for (int rr = 0; rr < 4; rr++) {
@@ -184,8 +186,8 @@ __global__ void __launch_bounds__(kSimtThreads) simt_bwd_dq(const T *__restrict_
     first = (first / kSimtTile) * kSimtTile;
     for (int k0 = first; k0 <= last; k0 += kSimtTile) {
         __syncthreads();
-        load_rows<T, D>(sK, D + 1, Kb, k0, kSimtTile, T_);
-        load_rows<T, D>(sV, D + 1, Vb, k0, kSimtTile, T_);
+        load_rows<T, DK>(sK, DK + 1, Kb, k0, kSimtTile, T_);
+        load_rows<T, DV>(sV, DV + 1, Vb, k0, kSimtTile, T_);
         __syncthreads();
 #pragma unroll
         for (int rr = 0; rr < 4; rr++) {
@@ -194,10 +196,9 @@ __global__ void __launch_bounds__(kSimtThreads) simt_bwd_dq(const T *__restrict_
             const int kj = k0 + lane;
             float s = 0.0f, dp = 0.0f;
 #pragma unroll 8
-            for (int d = 0; d < D; d++) {
-                s = fmaf(sQ[r * D + d], sK[lane * (D + 1) + d], s);
-                dp = fmaf(sdO[r * D + d], sV[lane * (D + 1) + d], dp);
-            }
+            for (int d = 0; d < DK; d++) s = fmaf(sQ[r * DK + d], sK[lane * (DK + 1) + d], s);
+#pragma unroll 8
+            for (int d = 0; d < DV; d++) dp = fmaf(sdO[r * DV + d], sV[lane * (DV + 1) + d], dp);
             const float sc = simt_capped(s * scale, softcap);
             const bool ok = visible(qi, kj, window) && kj < T_;
             const float p = ok ? expf(sc - L[rr]) : 0.0f;
@@ -209,7 +210,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_bwd_dq(const T *__restrict_
             for (int j = 0; j < kSimtTile; j++) {
                 const float dsj = __shfl_sync(0xffffffffu, ds, j);
 #pragma unroll
-                for (int t = 0; t < NT; t++) acc[rr][t] = fmaf(dsj, sK[j * (D + 1) + lane + 32 * t], acc[rr][t]);
+                for (int t = 0; t < NT; t++) acc[rr][t] = fmaf(dsj, sK[j * (DK + 1) + lane + 32 * t], acc[rr][t]);
             }
         }
     }
@@ -217,18 +218,19 @@ __global__ void __launch_bounds__(kSimtThreads) simt_bwd_dq(const T *__restrict_
     for (int rr = 0; rr < 4; rr++) {
         const int qi = r0 + warp * 4 + rr;
         if (qi >= T_) continue;
-        T *row = dq + ((size_t)bh * T_ + qi) * D;
+        T *row = dq + ((size_t)bh * T_ + qi) * DK;
 #pragma unroll
         for (int t = 0; t < NT; t++) from_f32(row + lane + 32 * t, acc[rr][t] * scale);
     }
 }
 
-template <int D>
+template <int DK, int DV>
 constexpr size_t simt_bwd_dkdv_smem() {
-    return sizeof(float) * (size_t)(2 * kSimtRows * D + 2 * kSimtTile * (D + 1) + 2 * kSimtTile);
+    return sizeof(float) *
+           (size_t)(kSimtRows * (DK + DV) + kSimtTile * (DK + 1) + kSimtTile * (DV + 1) + 2 * kSimtTile);
 }
 
-template <typename T, int D>
+template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(kSimtThreads) simt_bwd_dkdv(const T *__restrict__ q, const T *__restrict__ k,
                                                               const T *__restrict__ v, const float *__restrict__ lse,
                                                               const T *__restrict__ dO,
@@ -236,24 +238,27 @@ __global__ void __launch_bounds__(kSimtThreads) simt_bwd_dkdv(const T *__restric
                                                               T *__restrict__ dv, int Hq, int Hkv, int T_,
                                                               float scale, int window, float softcap) {
     extern __shared__ float sm[];
-    float *sK = sm;                        // [16][D] key rows of this block
-    float *sV = sK + kSimtRows * D;        // [16][D]
-    float *sQ = sV + kSimtRows * D;        // [32][D+1] query tile
-    float *sdO = sQ + kSimtTile * (D + 1); // [32][D+1]
-    float *sL = sdO + kSimtTile * (D + 1); // [32]
-    float *sD = sL + kSimtTile;            // [32]
-    constexpr int NT = D / 32;
+    float *sK = sm;                          // [16][DK] key rows of this block
+    float *sV = sK + kSimtRows * DK;         // [16][DV]
+    float *sQ = sV + kSimtRows * DV;         // [32][DK+1] query tile
+    float *sdO = sQ + kSimtTile * (DK + 1);  // [32][DV+1]
+    float *sL = sdO + kSimtTile * (DV + 1);  // [32]
+    float *sD = sL + kSimtTile;              // [32]
+    constexpr int NK = DK / 32, NV = DV / 32;
     const int bkv = blockIdx.y, b = bkv / Hkv, hkv = bkv % Hkv;
     const int G = Hq / Hkv;
     const int r0 = blockIdx.x * kSimtRows;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    load_rows<T, D>(sK, D, k + (size_t)bkv * T_ * D, r0, kSimtRows, T_);
-    load_rows<T, D>(sV, D, v + (size_t)bkv * T_ * D, r0, kSimtRows, T_);
-    float adk[4][NT], adv[4][NT];
+    load_rows<T, DK>(sK, DK, k + (size_t)bkv * T_ * DK, r0, kSimtRows, T_);
+    load_rows<T, DV>(sV, DV, v + (size_t)bkv * T_ * DV, r0, kSimtRows, T_);
+    float adk[4][NK], adv[4][NV];
 #pragma unroll
-    for (int rr = 0; rr < 4; rr++)
+    for (int rr = 0; rr < 4; rr++) {
 #pragma unroll
-        for (int t = 0; t < NT; t++) adk[rr][t] = adv[rr][t] = 0.0f;
+        for (int t = 0; t < NK; t++) adk[rr][t] = 0.0f;
+#pragma unroll
+        for (int t = 0; t < NV; t++) adv[rr][t] = 0.0f;
+    }
     const int qfirst = (r0 / kSimtTile) * kSimtTile;
     int qlast = T_ - 1;
     if (window > 0) qlast = min(qlast, r0 + kSimtRows - 1 + window - 1);
@@ -261,8 +266,8 @@ __global__ void __launch_bounds__(kSimtThreads) simt_bwd_dkdv(const T *__restric
         const int bh = b * Hq + hkv * G + g;
         for (int q0 = qfirst; q0 <= qlast; q0 += kSimtTile) {
             __syncthreads();
-            load_rows<T, D>(sQ, D + 1, q + (size_t)bh * T_ * D, q0, kSimtTile, T_);
-            load_rows<T, D>(sdO, D + 1, dO + (size_t)bh * T_ * D, q0, kSimtTile, T_);
+            load_rows<T, DK>(sQ, DK + 1, q + (size_t)bh * T_ * DK, q0, kSimtTile, T_);
+            load_rows<T, DV>(sdO, DV + 1, dO + (size_t)bh * T_ * DV, q0, kSimtTile, T_);
             if (threadIdx.x < kSimtTile) {
                 const int qi = q0 + threadIdx.x;
                 sL[threadIdx.x] = qi < T_ ? lse[(size_t)bh * T_ + qi] : 0.0f;
@@ -276,10 +281,9 @@ __global__ void __launch_bounds__(kSimtThreads) simt_bwd_dkdv(const T *__restric
                 const int qi = q0 + lane;
                 float s = 0.0f, dp = 0.0f;
 #pragma unroll 8
-                for (int d = 0; d < D; d++) {
-                    s = fmaf(sK[r * D + d], sQ[lane * (D + 1) + d], s);
-                    dp = fmaf(sV[r * D + d], sdO[lane * (D + 1) + d], dp);
-                }
+                for (int d = 0; d < DK; d++) s = fmaf(sK[r * DK + d], sQ[lane * (DK + 1) + d], s);
+#pragma unroll 8
+                for (int d = 0; d < DV; d++) dp = fmaf(sV[r * DV + d], sdO[lane * (DV + 1) + d], dp);
                 const float sc = simt_capped(s * scale, softcap);
                 const bool ok = qi < T_ && visible(qi, kj, window);
                 const float p = ok ? expf(sc - sL[lane]) : 0.0f;
@@ -292,10 +296,9 @@ __global__ void __launch_bounds__(kSimtThreads) simt_bwd_dkdv(const T *__restric
                     const float pj = __shfl_sync(0xffffffffu, p, j);
                     const float dsj = __shfl_sync(0xffffffffu, ds, j);
 #pragma unroll
-                    for (int t = 0; t < NT; t++) {
-                        adv[rr][t] = fmaf(pj, sdO[j * (D + 1) + lane + 32 * t], adv[rr][t]);
-                        adk[rr][t] = fmaf(dsj, sQ[j * (D + 1) + lane + 32 * t], adk[rr][t]);
-                    }
+                    for (int t = 0; t < NV; t++) adv[rr][t] = fmaf(pj, sdO[j * (DV + 1) + lane + 32 * t], adv[rr][t]);
+#pragma unroll
+                    for (int t = 0; t < NK; t++) adk[rr][t] = fmaf(dsj, sQ[j * (DK + 1) + lane + 32 * t], adk[rr][t]);
                 }
             }
         }
@@ -304,13 +307,12 @@ __global__ void __launch_bounds__(kSimtThreads) simt_bwd_dkdv(const T *__restric
     for (int rr = 0; rr < 4; rr++) {
         const int kj = r0 + warp * 4 + rr;
         if (kj >= T_) continue;
-        T *krow = dk + ((size_t)bkv * T_ + kj) * D;
-        T *vrow = dv + ((size_t)bkv * T_ + kj) * D;
+        T *krow = dk + ((size_t)bkv * T_ + kj) * DK;
+        T *vrow = dv + ((size_t)bkv * T_ + kj) * DV;
 #pragma unroll
-        for (int t = 0; t < NT; t++) {
-            from_f32(krow + lane + 32 * t, adk[rr][t] * scale);
-            from_f32(vrow + lane + 32 * t, adv[rr][t]);
-        }
+        for (int t = 0; t < NK; t++) from_f32(krow + lane + 32 * t, adk[rr][t] * scale);
+#pragma unroll
+        for (int t = 0; t < NV; t++) from_f32(vrow + lane + 32 * t, adv[rr][t]);
     }
 }
 

@@ -176,6 +176,26 @@ forge_status forge_attn_bwd_finalize(void *dq, int B, int Hq, int Hkv, int T, in
                                      void *stream);
 
 /*
+ * Forward and backward with separate head dims for q, k (Dk) and v, o (Dv):
+ * decompressed multi-head latent attention (ARCHITECTURES.md "Vague 3" item 13;
+ * family table, DeepSeek V3 row: q.k over nope 128 + rope 64 = 192, values 128,
+ * scale 1/sqrt(192) chosen by the caller). Layouts as above with D = Dk for q,
+ * k, dq, dk and D = Dv for v, o, dO, dv. With Dk == Dv these are forge_attn_fwd /
+ * forge_attn_bwd. Otherwise only (Dk, Dv) = (192, 128) with FORGE_DTYPE_F32 is
+ * built (CUDA cores); anything else returns FORGE_ERR_UNSUPPORTED.
+ */
+forge_status forge_attn_fwd_dkv(const void *q, const void *k, const void *v, void *o, float *lse,
+                                int B, int Hq, int Hkv, int T, int Dk, int Dv, float scale, int window,
+                                float softcap, forge_dtype dtype, void *stream);
+size_t forge_attn_bwd_workspace_size_dkv(int B, int Hq, int Hkv, int T, int Dk, int Dv,
+                                         forge_dtype dtype);
+forge_status forge_attn_bwd_dkv(const void *q, const void *k, const void *v, const void *o,
+                                const float *lse, const void *dO, void *dq, void *dk, void *dv,
+                                int B, int Hq, int Hkv, int T, int Dk, int Dv, float scale,
+                                int window, float softcap, forge_dtype dtype, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
+/*
  * Decode: one new query per (batch entry, query head) against a KV cache
  * (INFERENCE_RESEARCH.md section 2: the cache is pre-allocated to the maximum
  * length, laid out [layer][head][seq][d], and decoding gets a dedicated kernel

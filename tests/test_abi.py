@@ -125,3 +125,15 @@ def test_ext_entry_points_reject_misaligned_extras():
     assert s == fa.FORGE_ERR_INVALID_ARG
     s = fa.forge_attn_fwd_ext(A, A, A, A, A, 1, 2, 2, 128, 64, 0.125, 0, 0.0, None, A + 1, fa.FORGE_DTYPE_BF16, 0)
     assert s == fa.FORGE_ERR_INVALID_ARG
+
+
+def test_dkv_entry_points_reject_unsupported_pairs_before_any_launch():
+    A = 0x10000
+    # bf16 with d_k != d_v has no tensor-core kernel yet
+    s = fa.forge_attn_fwd_dkv(A, A, A, A, A, 1, 2, 2, 128, 192, 128, 0.07, 0, 0.0, fa.FORGE_DTYPE_BF16, 0)
+    assert s == fa.FORGE_ERR_UNSUPPORTED
+    s = fa.forge_attn_fwd_dkv(A, A, A, A, A, 1, 2, 2, 128, 96, 64, 0.1, 0, 0.0, fa.FORGE_DTYPE_F32, 0)
+    assert s == fa.FORGE_ERR_UNSUPPORTED
+    assert fa.forge_attn_bwd_workspace_size_dkv(1, 2, 2, 128, 192, 128, fa.FORGE_DTYPE_BF16) == 0
+    # the f32 (192, 128) workspace holds Delta only
+    assert fa.forge_attn_bwd_workspace_size_dkv(1, 2, 2, 128, 192, 128, fa.FORGE_DTYPE_F32) >= 2 * 128 * 4

@@ -1,0 +1,44 @@
+"""GPU parity of d_k != d_v (decompressed multi-head latent attention: q.k over
+d_k = 192, values of d_v = 128; ARCHITECTURES.md "Vague 3" item 13) through the C
+ABI against the oracle, on the f32 CUDA-core path, with GQA, a window, a cap and
+ragged lengths. Tolerance: the f32 bar (1e-4 absolute)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import causal_flash_attention_attn_b200 as fa
+from parity_util import check_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,T,W,C", [(1, 4, 2, 150, 0, 0.0), (2, 2, 1, 97, 40, 0.0), (1, 2, 2, 130, 0, 20.0)])
+def test_dk192_dv128_matches_oracle(B, Hq, Hkv, T, W, C):
+    Dk, Dv = 192, 128
+    g = torch.Generator(device="cpu").manual_seed(T + W)
+    q = torch.randn(B, Hq, T, Dk, generator=g)
+    k = torch.randn(B, Hkv, T, Dk, generator=g)
+    v = torch.randn(B, Hkv, T, Dv, generator=g)
+    dO = torch.randn(B, Hq, T, Dv, generator=g)
+    dev = torch.device("cuda:0")
+    qd, kd, vd, dOd = (x.to(dev) for x in (q, k, v, dO))
+    sc = 1.0 / math.sqrt(Dk)
+    o = torch.full((B, Hq, T, Dv), float("nan"), device=dev)
+    lse = torch.full((B, Hq, T), float("nan"), device=dev)
+    s = fa.forge_attn_fwd_dkv(qd, kd, vd, o, lse, B, Hq, Hkv, T, Dk, Dv, sc, W, C, fa.FORGE_DTYPE_F32)
+    assert s == fa.FORGE_OK, fa.forge_attn_status_string(s)
+    nbytes = fa.forge_attn_bwd_workspace_size_dkv(B, Hq, Hkv, T, Dk, Dv, fa.FORGE_DTYPE_F32)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    dq, dk, dv = (torch.full_like(x, float("nan")) for x in (qd, kd, vd))
+    s = fa.forge_attn_bwd_dkv(qd, kd, vd, o, lse, dOd, dq, dk, dv, B, Hq, Hkv, T, Dk, Dv, sc, W, C,
+                              fa.FORGE_DTYPE_F32, ws, nbytes)
+    assert s == fa.FORGE_OK, fa.forge_attn_status_string(s)
+    torch.cuda.synchronize()
+    assert fa.forge_attn_check() == fa.FORGE_OK
+    ro, rl, _ = oracle.attn_fwd_ext(q, k, v, sc, W, C)
+    rdq, rdk, rdv, _, _, _ = oracle.attn_bwd_ext(q, k, v, dO, sc, W, C, o_round="f32")
+    for name, a, b in (("o", o, ro), ("lse", lse, rl), ("dq", dq, rdq), ("dk", dk, rdk), ("dv", dv, rdv)):
+        check_close(name, a.cpu(), b, "f32")
