@@ -534,6 +534,79 @@ def run_decode(args):
             "gpu_launches": 2 * args.steps, "clocks": clocks}
 
 
+# d_k != d_v (decompressed multi-head latent attention) on the f32 CUDA-core path
+DKV = {"workload": "mla_f32_b1_h16_t4096_dk192_dv128", "B": 1, "Hq": 16, "Hkv": 16, "T": 4096, "Dk": 192, "Dv": 128,
+       "dtype": "f32", "window": 0, "softcap": 0.0}
+# FP32 FMA peak of the CUDA cores: 148 SMs x 128 FMA lanes x 2 flops x 1.965 GHz
+F32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def run_dkv(args):
+    """--dkv: forward + backward with d_k = 192, d_v = 128 (f32, CUDA cores), FLOPs
+    counted per allowed pair as 2 (Dk + Dv) forward and 2 (3 Dk + 2 Dv) backward
+    (S recompute, dP, dV, dK, dQ), against the FP32 FMA peak."""
+    import torch
+    import causal_flash_attention_attn_b200 as fa
+
+    c = DKV
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    fa.library()
+    stream = torch.cuda.Stream(device=dev)
+    g = torch.Generator(device="cpu").manual_seed(6)
+    B, Hq, Hkv, T, Dk, Dv = c["B"], c["Hq"], c["Hkv"], c["T"], c["Dk"], c["Dv"]
+    q = torch.randn(B, Hq, T, Dk, generator=g).to(dev)
+    k = torch.randn(B, Hkv, T, Dk, generator=g).to(dev)
+    v = torch.randn(B, Hkv, T, Dv, generator=g).to(dev)
+    dO = torch.randn(B, Hq, T, Dv, generator=g).to(dev)
+    o = torch.empty(B, Hq, T, Dv, device=dev)
+    lse = torch.empty(B, Hq, T, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    nws = fa.forge_attn_bwd_workspace_size_dkv(B, Hq, Hkv, T, Dk, Dv, fa.FORGE_DTYPE_F32)
+    ws = torch.empty(nws, dtype=torch.uint8, device=dev)
+    sc = 1.0 / math.sqrt(Dk)
+    sh = stream.cuda_stream
+
+    def step():
+        s = fa.forge_attn_fwd_dkv(q, k, v, o, lse, B, Hq, Hkv, T, Dk, Dv, sc, 0, 0.0, fa.FORGE_DTYPE_F32, sh)
+        s |= fa.forge_attn_bwd_dkv(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, Dk, Dv, sc, 0, 0.0,
+                                   fa.FORGE_DTYPE_F32, ws, nws, sh)
+        if s != fa.FORGE_OK:
+            raise fa.ForgeError(s, "dkv")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    clk = ClockSampler(dev.index)
+    clk.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = clk.stop()
+    st = fa.forge_attn_check(sh)
+    if st != fa.FORGE_OK:
+        raise fa.ForgeError(st, "dkv timed run")
+    ms = e0.elapsed_time(e1) / args.steps
+    pairs = B * Hq * T * (T + 1) // 2
+    flops = pairs * (2 * (Dk + Dv) + 2 * (3 * Dk + 2 * Dv))
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"metric": "d_k != d_v attention fwd+bwd TFLOPS (f32 CUDA-core path)", "value": round(tf, 3),
+            "unit": "TFLOPS", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded N(0,1) q, k, v, dO)",
+            "config": dict(c, l2="not flushed: the per-step working set (about 0.2 GB) exceeds the 126 MB L2",
+                           flop_count="allowed pairs x (2 (Dk + Dv) forward + 2 (3 Dk + 2 Dv) backward)"),
+            "roofline": {"kernel": "simt_bwd_dkdv", "bound": "alu", "achieved": round(tf, 3),
+                         "peak": round(F32_FMA_TFLOPS, 1), "unit": "TFLOP/s", "frac": round(tf / F32_FMA_TFLOPS, 4),
+                         "traffic": None, "peak_source": "148 SMs x 128 FP32 FMA lanes x 2 x 1.965 GHz",
+                         "achieved_def": "all fwd+bwd flops / CUDA-event step time"},
+            "gpu_launches": 4 * args.steps, "clocks": clocks}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -545,6 +618,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--decode", action="store_true", help="time the KV-cache decode kernels instead")
+    ap.add_argument("--dkv", action="store_true", help="time the d_k != d_v (f32) path instead")
     args = ap.parse_args(argv)
     from causal_flash_attention_attn_b200 import inputs
     w = inputs.WORKLOADS[args.workload or inputs.HEADLINE]
@@ -552,6 +626,9 @@ def main(argv=None):
         args.warmup = 3
     if args.decode:
         print(json.dumps(run_decode(args)), flush=True)
+        return
+    if args.dkv:
+        print(json.dumps(run_dkv(args)), flush=True)
         return
     line = run_reference(args, w) if args.impl == "reference" else run_ours(args, w)
     if line is not None:
