@@ -165,6 +165,33 @@ forge_status fwd_tc(const void *q, const void *k, const void *v, void *o, float 
     return launch_status();
 }
 
+// Single-tile tensor-core forward with separate key and value head dims.
+template <int DK, int DV>
+forge_status fwd_tc_dkv(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv,
+                        int T, float scale, int window, float softcap, cudaStream_t st) {
+    using C = FwdTc<DK, DV>;
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, q, DK, T, (long long)B * Hq, 128) || !make_map(&mk, k, DK, T, (long long)B * Hkv, 128) ||
+        !make_map(&mv, v, DV, T, (long long)B * Hkv, 128)) {
+        t_last_cuda_error = "cuTensorMapEncodeTiled failed";
+        return FORGE_ERR_CUDA;
+    }
+    FwdParams p;
+    p.o = static_cast<__nv_bfloat16 *>(o);
+    p.lse = lse;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.T = T; p.window = window;
+    p.num_qt = (T + 127) / 128;
+    p.scale_log2 = scale * kLog2e;
+    p.softcap = softcap;
+    p.cap_in = softcap > 0.0f ? scale / softcap : 0.0f;
+    p.cap_out = softcap * kLog2e;
+    p.sink = nullptr;
+    p.max_logit = nullptr;
+    if (set_smem(fwd_tc_kernel<DK, DV>, C::SMEM) != FORGE_OK) return FORGE_ERR_CUDA;
+    fwd_tc_kernel<DK, DV><<<(unsigned)(p.num_qt * B * Hq), C::THREADS, C::SMEM, st>>>(mq, mk, mv, p);
+    return launch_status();
+}
+
 template <typename T_, int DK, int DV = DK>
 forge_status fwd_simt(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv, int T,
                       float scale, int window, float softcap, const float *sink, float *max_logit, cudaStream_t st) {
@@ -528,11 +555,14 @@ forge_status forge_attn_bwd_noalloc(const void *q, const void *k, const void *v,
                           kNoAllocScratchBytes, stream);
 }
 
-// d_k != d_v: the f32 CUDA-core path at (d_k, d_v) = (192, 128), the decompressed
-// multi-head latent attention of the DeepSeek V3 family; the tensor-core kernels
-// keep d_k = d_v for now.
+// d_k != d_v at (d_k, d_v) = (192, 128), the decompressed multi-head latent
+// attention of the DeepSeek V3 family: forward on the tensor cores (bf16) or the
+// CUDA cores (f32); backward on the CUDA cores (f32) only.
 static bool dkv_supported(int Dk, int Dv, forge_dtype dtype) {
     return dtype == FORGE_DTYPE_F32 && Dk == 192 && Dv == 128;
+}
+static bool dkv_fwd_supported(int Dk, int Dv, forge_dtype dtype) {
+    return (dtype == FORGE_DTYPE_F32 || dtype == FORGE_DTYPE_BF16) && Dk == 192 && Dv == 128;
 }
 
 size_t forge_attn_bwd_workspace_size_dkv(int B, int Hq, int Hkv, int T, int Dk, int Dv, forge_dtype dtype) {
@@ -547,13 +577,14 @@ forge_status forge_attn_fwd_dkv(const void *q, const void *k, const void *v, voi
     if (Dk == Dv) return forge_attn_fwd(q, k, v, o, lse, B, Hq, Hkv, T, Dk, scale, window, softcap, dtype, stream);
     forge_status s = check_sizes(B, Hq, Hkv, T, Dv, dtype);
     if (s != FORGE_OK) return s;
-    if (!dkv_supported(Dk, Dv, dtype)) return FORGE_ERR_UNSUPPORTED;
+    if (!dkv_fwd_supported(Dk, Dv, dtype)) return FORGE_ERR_UNSUPPORTED;
     if ((s = check_scalars(scale, window, softcap)) != FORGE_OK) return s;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return FORGE_ERR_INVALID_ARG;
     window = effective_window(window, T);
-    return fwd_simt<float, 192, 128>(q, k, v, o, lse, B, Hq, Hkv, T, scale, window, softcap, nullptr, nullptr,
-                                     static_cast<cudaStream_t>(stream));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dtype == FORGE_DTYPE_BF16) return fwd_tc_dkv<192, 128>(q, k, v, o, lse, B, Hq, Hkv, T, scale, window, softcap, st);
+    return fwd_simt<float, 192, 128>(q, k, v, o, lse, B, Hq, Hkv, T, scale, window, softcap, nullptr, nullptr, st);
 }
 
 forge_status forge_attn_bwd_dkv(const void *q, const void *k, const void *v, const void *o, const float *lse,

@@ -26,7 +26,9 @@
 
 namespace forge {
 
-template <int D>
+// DK: head dim of q and k; DV: head dim of v and o (DK = DV except for the
+// decompressed multi-head latent attention, 192 / 128).
+template <int DK, int DV = DK>
 struct FwdTc {
     static constexpr int BM = 128, BN = 128;
     // O += P V with P split into two bf16 terms, P = hi + lo (hi = bf16(P),
@@ -34,13 +36,15 @@ struct FwdTc {
     // instead of carrying the 2^-9 relative error of a single bf16 P. The
     // backward's Delta = rowsum(dO * O) inherits that accuracy; at head dim 256 a
     // single-term P moves Delta by up to ~0.2 on logits in the tanh regime.
-    static constexpr bool PSPLIT = (D == 256);
-    static constexpr int NCB = D / 64;                 // 64-column (128-byte) blocks
-    static constexpr uint32_t CB = 128 * 128;          // bytes of one column block of a 128-row tile
-    static constexpr uint32_t TILE = NCB * CB;         // one 128 x D bf16 tile
-    static constexpr int NSTAGE = D == 256 ? 2 : (D == 128 ? 4 : 6);
-    static constexpr uint32_t CTRL = 1024;             // barriers, TMEM slot, abort flag
-    static constexpr uint32_t SMEM = CTRL + TILE * (1 + NSTAGE) + 1024;
+    static constexpr bool PSPLIT = (DV == 256);
+    static constexpr int NCBK = DK / 64, NCBV = DV / 64;  // 64-column (128-byte) blocks
+    static constexpr uint32_t CB = 128 * 128;             // bytes of one column block of a 128-row tile
+    static constexpr uint32_t TILEK = NCBK * CB;          // one 128 x DK bf16 tile (Q, K)
+    static constexpr uint32_t TILEV = NCBV * CB;          // one 128 x DV bf16 tile (V)
+    static constexpr uint32_t SLOT = TILEK > TILEV ? TILEK : TILEV;  // a ring slot holds a K or a V tile
+    static constexpr int NSTAGE = DK == 256 ? 2 : (DK == 192 ? 3 : (DK == 128 ? 4 : 6));
+    static constexpr uint32_t CTRL = 1024;                // barriers, TMEM slot, abort flag
+    static constexpr uint32_t SMEM = CTRL + TILEK + SLOT * NSTAGE + 1024;
     static constexpr int THREADS = 192;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O = 256;
@@ -57,6 +61,7 @@ struct FwdTc {
     static constexpr uint32_t OFF_ABORT = 516;
     static_assert(NBAR * 8 <= 512, "control block");
     static_assert(SMEM <= 232448, "shared memory");
+    static_assert(256 + DV <= 512, "tensor memory");
 };
 
 // Row max of a 128-column tile held as 4 x 32 registers (8 independent chains).
@@ -122,16 +127,16 @@ struct FwdParams {
     float *max_logit;
 };
 
-template <int D>
+template <int DK, int DV = DK>
 __global__ void __launch_bounds__(192, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-    using C = FwdTc<D>;
+    using C = FwdTc<DK, DV>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = smem_u32(smem_raw);
     const uint32_t tiles = (sbase + C::CTRL + 1023u) & ~1023u;
     const uint32_t sQ = tiles;
-    const uint32_t sKV = tiles + C::TILE;
+    const uint32_t sKV = tiles + C::TILEK;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem_raw + C::OFF_ABORT);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + C::OFF_TMEM_SLOT);
     auto bar = [&](int i) -> uint32_t { return sbase + 8u * (uint32_t)i; };
@@ -179,17 +184,18 @@ __global__ void __launch_bounds__(192, 1)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             const uint64_t keep = policy_evict_last();
-            mbar_arrive_expect_tx(bar(C::B_Q), C::TILE);
-            for (int c = 0; c < C::NCB; c++) tma_load_3d(sQ + c * C::CB, &tmQ, bar(C::B_Q), c * 64, q0, bh);
+            mbar_arrive_expect_tx(bar(C::B_Q), C::TILEK);
+            for (int c = 0; c < C::NCBK; c++) tma_load_3d(sQ + c * C::CB, &tmQ, bar(C::B_Q), c * 64, q0, bh);
             int stage = 0;
             uint32_t ph = 0;
             int issued = 0;
             bool ok = true;
             auto load = [&](const CUtensorMap *m, int j) -> bool {
                 if (!mbar_wait(bar(C::B_KV_EMPTY + stage), ph ^ 1u, abort_flag)) return false;
-                mbar_arrive_expect_tx(bar(C::B_KV_FULL + stage), C::TILE);
-                for (int c = 0; c < C::NCB; c++)
-                    tma_load_3d_hint(sKV + stage * C::TILE + c * C::CB, m, bar(C::B_KV_FULL + stage), c * 64,
+                const bool is_v = (m == &tmV);
+                mbar_arrive_expect_tx(bar(C::B_KV_FULL + stage), is_v ? C::TILEV : C::TILEK);
+                for (int c = 0; c < (is_v ? C::NCBV : C::NCBK); c++)
+                    tma_load_3d_hint(sKV + stage * C::SLOT + c * C::CB, m, bar(C::B_KV_FULL + stage), c * 64,
                                      j * C::BN, bkv, keep);
                 issued++;
                 if (++stage == C::NSTAGE) {
@@ -218,7 +224,7 @@ __global__ void __launch_bounds__(192, 1)
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t ID_QK = idesc_bf16_f32(128, 128, false, false);
-            constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, false, true);
+            constexpr uint32_t ID_PV = idesc_bf16_f32(128, DV, false, true);
             int stage = 0;
             uint32_t ph = 0;
             auto next = [&]() {
@@ -230,10 +236,10 @@ __global__ void __launch_bounds__(192, 1)
             auto qk = [&](int buf) -> bool {
                 if (!mbar_wait(bar(C::B_KV_FULL + stage), ph, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t sK = sKV + stage * C::TILE;
+                const uint32_t sK = sKV + stage * C::SLOT;
                 const uint32_t dS = tmem + (buf ? C::COL_S1 : C::COL_S0);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; kk++) {
+                for (int kk = 0; kk < DK / 16; kk++) {
                     const uint32_t off = (kk >> 2) * C::CB + (kk & 3) * 32;
                     mma_ss(dS, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), ID_QK, kk > 0);
                 }
@@ -245,7 +251,7 @@ __global__ void __launch_bounds__(192, 1)
             auto pv = [&](int buf, bool acc) -> bool {
                 if (!mbar_wait(bar(C::B_KV_FULL + stage), ph, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t sV = sKV + stage * C::TILE;
+                const uint32_t sV = sKV + stage * C::SLOT;
                 const uint32_t aP = tmem + (buf ? C::COL_S1 : C::COL_S0);
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; kk++)
@@ -341,7 +347,7 @@ __global__ void __launch_bounds__(192, 1)
                 tc_fence_after();
                 const float f = (moved && u > 0) ? factor : 1.0f;
 #pragma unroll 1
-                for (int c0 = 0; c0 < D; c0 += 32) {
+                for (int c0 = 0; c0 < DV; c0 += 32) {
                     uint32_t o[32];
                     tmem_ld32(tmem + lane_base + C::COL_O + c0, o);
                     tmem_ld_wait(o);
@@ -382,9 +388,9 @@ __global__ void __launch_bounds__(192, 1)
         if (ok) {
             tc_fence_after();
             const float inv_l = 1.0f / l;
-            __nv_bfloat16 *orow = p.o + ((size_t)bh * p.T + (size_t)min(qi, p.T - 1)) * D;
+            __nv_bfloat16 *orow = p.o + ((size_t)bh * p.T + (size_t)min(qi, p.T - 1)) * DV;
 #pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 32) {
+            for (int c0 = 0; c0 < DV; c0 += 32) {
                 uint32_t o[32];
                 tmem_ld32(tmem + lane_base + C::COL_O + c0, o);
                 tmem_ld_wait(o);

@@ -181,8 +181,9 @@ forge_status forge_attn_bwd_finalize(void *dq, int B, int Hq, int Hkv, int T, in
  * family table, DeepSeek V3 row: q.k over nope 128 + rope 64 = 192, values 128,
  * scale 1/sqrt(192) chosen by the caller). Layouts as above with D = Dk for q,
  * k, dq, dk and D = Dv for v, o, dO, dv. With Dk == Dv these are forge_attn_fwd /
- * forge_attn_bwd. Otherwise only (Dk, Dv) = (192, 128) with FORGE_DTYPE_F32 is
- * built (CUDA cores); anything else returns FORGE_ERR_UNSUPPORTED.
+ * forge_attn_bwd. Otherwise only (Dk, Dv) = (192, 128) is built: the forward in
+ * bf16 (tensor cores) and f32 (CUDA cores), the backward in f32 (CUDA cores);
+ * anything else returns FORGE_ERR_UNSUPPORTED (the bf16 backward included).
  */
 forge_status forge_attn_fwd_dkv(const void *q, const void *k, const void *v, void *o, float *lse,
                                 int B, int Hq, int Hkv, int T, int Dk, int Dv, float scale, int window,

@@ -129,8 +129,9 @@ def test_ext_entry_points_reject_misaligned_extras():
 
 def test_dkv_entry_points_reject_unsupported_pairs_before_any_launch():
     A = 0x10000
-    # bf16 with d_k != d_v has no tensor-core kernel yet
-    s = fa.forge_attn_fwd_dkv(A, A, A, A, A, 1, 2, 2, 128, 192, 128, 0.07, 0, 0.0, fa.FORGE_DTYPE_BF16, 0)
+    # the bf16 backward with d_k != d_v has no tensor-core kernel yet
+    s = fa.forge_attn_bwd_dkv(A, A, A, A, A, A, A, A, A, 1, 2, 2, 128, 192, 128, 0.07, 0, 0.0, fa.FORGE_DTYPE_BF16,
+                              A, 1 << 20, 0)
     assert s == fa.FORGE_ERR_UNSUPPORTED
     s = fa.forge_attn_fwd_dkv(A, A, A, A, A, 1, 2, 2, 128, 96, 64, 0.1, 0, 0.0, fa.FORGE_DTYPE_F32, 0)
     assert s == fa.FORGE_ERR_UNSUPPORTED

@@ -42,3 +42,27 @@ def test_dk192_dv128_matches_oracle(B, Hq, Hkv, T, W, C):
     rdq, rdk, rdv, _, _, _ = oracle.attn_bwd_ext(q, k, v, dO, sc, W, C, o_round="f32")
     for name, a, b in (("o", o, ro), ("lse", lse, rl), ("dq", dq, rdq), ("dk", dk, rdk), ("dv", dv, rdv)):
         check_close(name, a.cpu(), b, "f32")
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,T,W,C", [(2, 4, 2, 300, 0, 0.0), (1, 2, 1, 257, 100, 0.0), (1, 4, 4, 200, 0, 20.0)])
+def test_dk192_dv128_bf16_forward_matches_oracle(B, Hq, Hkv, T, W, C):
+    """The tensor-core forward (single query tile per CTA, K/V ring slots sized
+    for d_k) at the bf16 bar."""
+    Dk, Dv = 192, 128
+    g = torch.Generator(device="cpu").manual_seed(1000 + T + W)
+    sig = 2.0 if C else 1.0
+    q = (torch.randn(B, Hq, T, Dk, generator=g) * sig).to(torch.bfloat16)
+    k = (torch.randn(B, Hkv, T, Dk, generator=g) * sig).to(torch.bfloat16)
+    v = torch.randn(B, Hkv, T, Dv, generator=g).to(torch.bfloat16)
+    dev = torch.device("cuda:0")
+    qd, kd, vd = (x.to(dev) for x in (q, k, v))
+    sc = 1.0 / math.sqrt(Dk)
+    o = torch.full((B, Hq, T, Dv), float("nan"), device=dev).to(torch.bfloat16)
+    lse = torch.full((B, Hq, T), float("nan"), device=dev)
+    s = fa.forge_attn_fwd_dkv(qd, kd, vd, o, lse, B, Hq, Hkv, T, Dk, Dv, sc, W, C, fa.FORGE_DTYPE_BF16)
+    assert s == fa.FORGE_OK, fa.forge_attn_status_string(s)
+    torch.cuda.synchronize()
+    assert fa.forge_attn_check() == fa.FORGE_OK
+    ro, rl, _ = oracle.attn_fwd_ext(q, k, v, sc, W, C)
+    check_close("o", o.cpu(), ro, "bf16")
+    check_close("lse", lse.cpu(), rl, "bf16")
