@@ -138,3 +138,22 @@ def test_dkv_entry_points_reject_unsupported_pairs_before_any_launch():
     assert fa.forge_attn_bwd_workspace_size_dkv(1, 2, 2, 128, 192, 128, fa.FORGE_DTYPE_BF16) == 0
     # the f32 (192, 128) workspace holds Delta only
     assert fa.forge_attn_bwd_workspace_size_dkv(1, 2, 2, 128, 192, 128, fa.FORGE_DTYPE_F32) >= 2 * 128 * 4
+
+
+def test_decode_validation_before_any_launch():
+    A = 0x10000
+    ws = fa.forge_attn_decode_workspace_size(2, 8, 2, 1000, 128)
+    assert ws > 0 and ws % 256 == 0
+    assert fa.forge_attn_decode_workspace_size(2, 8, 3, 1000, 128) == 0   # Hq % Hkv != 0
+    assert fa.forge_attn_decode_workspace_size(2, 8, 2, 1000, 96) == 0    # head dim not built
+    assert fa.forge_attn_decode_workspace_size(2, 8, 2, 4000, 128) >= ws  # grows with the cache length
+
+    def call(B=2, Hq=8, Hkv=2, T=1000, Tmax=1024, D=128, seq_lens=None, nbytes=None):
+        return fa.forge_attn_decode(A, A, A, A, None, seq_lens, B, Hq, Hkv, T, Tmax, D, 0.088, 0, 0.0, None,
+                                    fa.FORGE_DTYPE_BF16, A, ws if nbytes is None else nbytes, 0)
+
+    assert call(Hq=34, Hkv=2) == fa.FORGE_ERR_UNSUPPORTED            # 17 query heads per KV head
+    assert call(T=1025) == fa.FORGE_ERR_INVALID_ARG                   # T > Tmax
+    assert call(nbytes=ws - 256) == fa.FORGE_ERR_WORKSPACE            # workspace too small
+    assert call(seq_lens=A + 2) == fa.FORGE_ERR_INVALID_ARG           # misaligned lengths
+    assert call(D=80) == fa.FORGE_ERR_UNSUPPORTED
