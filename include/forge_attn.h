@@ -52,7 +52,7 @@ extern "C" {
 typedef enum {
     FORGE_OK = 0,
     FORGE_ERR_INVALID_ARG = 1, /* null or misaligned pointer, bad size, bad scalar */
-    FORGE_ERR_UNSUPPORTED = 2, /* valid but not built: head dim not in {64,128,256} */
+    FORGE_ERR_UNSUPPORTED = 2, /* valid but no kernel built for it (e.g. a head dim, a (d_k, d_v) pair, a decode group size) */
     FORGE_ERR_WORKSPACE = 3,   /* backward workspace missing, misaligned or too small */
     FORGE_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
     FORGE_ERR_TIMEOUT = 5      /* a bounded wait inside a kernel ran out */

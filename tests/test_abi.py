@@ -157,3 +157,42 @@ def test_decode_validation_before_any_launch():
     assert call(nbytes=ws - 256) == fa.FORGE_ERR_WORKSPACE            # workspace too small
     assert call(seq_lens=A + 2) == fa.FORGE_ERR_INVALID_ARG           # misaligned lengths
     assert call(D=80) == fa.FORGE_ERR_UNSUPPORTED
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "forge_attn.h"
+
+int main(void) {
+    void *fake = (void *)0x10000; /* never dereferenced: every call below fails validation first */
+    size_t ws = forge_attn_bwd_workspace_size(2, 28, 4, 4096, 128, FORGE_DTYPE_BF16);
+    forge_status bad_group = forge_attn_fwd(fake, fake, fake, fake, (float *)fake, 1, 4, 3, 128, 128,
+                                            0.1f, 0, 0.0f, FORGE_DTYPE_BF16, NULL);
+    forge_status bad_dim = forge_attn_fwd(fake, fake, fake, fake, (float *)fake, 1, 4, 2, 128, 96,
+                                          0.1f, 0, 0.0f, FORGE_DTYPE_BF16, NULL);
+    printf("%zu %d %d %s\n%s\n", ws, (int)bad_group, (int)bad_dim,
+           strstr(forge_attn_version(), "sm_100a") ? "sm_100a" : "?", forge_attn_status_string(FORGE_ERR_WORKSPACE));
+    return 0;
+}
+"""
+
+
+def test_header_compiles_as_c99_and_links(tmp_path):
+    # the boundary is a C ABI: a plain C99 client, warnings as errors, builds
+    # against the header and the shared library and gets the documented answers
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(fa.library_path)
+    libname = os.path.basename(fa.library_path)[3:-3]
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.dirname(HEADER),
+                    str(src), "-o", str(exe), "-L", libdir, "-l" + libname, "-Wl,-rpath," + libdir],
+                   check=True, capture_output=True, text=True)
+    line1, line2 = subprocess.run([str(exe)], check=True, capture_output=True, text=True,
+                                  timeout=60).stdout.splitlines()
+    out = line1.split()
+    assert int(out[0]) == fa.forge_attn_bwd_workspace_size(2, 28, 4, 4096, 128, fa.FORGE_DTYPE_BF16)
+    assert int(out[1]) == fa.FORGE_ERR_INVALID_ARG and int(out[2]) == fa.FORGE_ERR_UNSUPPORTED
+    assert out[3] == "sm_100a"
+    assert line2 == fa.forge_attn_status_string(fa.FORGE_ERR_WORKSPACE)
