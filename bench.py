@@ -607,6 +607,74 @@ def run_dkv(args):
             "gpu_launches": 4 * args.steps, "clocks": clocks}
 
 
+# the same shapes in bf16 on the tensor cores (forward only: the bf16 backward at
+# d_k != d_v is not built); B = 4 so the working set (330 MB) exceeds the L2
+DKV_BF16 = {"workload": "mla_bf16_b4_h16_t4096_dk192_dv128", "B": 4, "Hq": 16, "Hkv": 16, "T": 4096, "Dk": 192,
+            "Dv": 128, "dtype": "bf16", "window": 0, "softcap": 0.0}
+
+
+def run_dkv_bf16(args):
+    """--dkv --dkv-dtype bf16: the d_k != d_v forward on the tensor cores
+    (fwd_tc_kernel<192, 128>), FLOPs 2 (Dk + Dv) per allowed pair, against the
+    measured bf16 burst peak."""
+    import torch
+    import causal_flash_attention_attn_b200 as fa
+
+    c = DKV_BF16
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    fa.library()
+    stream = torch.cuda.Stream(device=dev)
+    g = torch.Generator(device="cpu").manual_seed(6)
+    B, Hq, Hkv, T, Dk, Dv = c["B"], c["Hq"], c["Hkv"], c["T"], c["Dk"], c["Dv"]
+    q = torch.randn(B, Hq, T, Dk, generator=g).to(torch.bfloat16).to(dev)
+    k = torch.randn(B, Hkv, T, Dk, generator=g).to(torch.bfloat16).to(dev)
+    v = torch.randn(B, Hkv, T, Dv, generator=g).to(torch.bfloat16).to(dev)
+    o = torch.empty(B, Hq, T, Dv, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, Hq, T, device=dev)
+    sc = 1.0 / math.sqrt(Dk)
+    sh = stream.cuda_stream
+
+    def step():
+        s = fa.forge_attn_fwd_dkv(q, k, v, o, lse, B, Hq, Hkv, T, Dk, Dv, sc, 0, 0.0, fa.FORGE_DTYPE_BF16, sh)
+        if s != fa.FORGE_OK:
+            raise fa.ForgeError(s, "dkv bf16")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    clk = ClockSampler(dev.index)
+    clk.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = clk.stop()
+    st = fa.forge_attn_check(sh)
+    if st != fa.FORGE_OK:
+        raise fa.ForgeError(st, "dkv bf16 timed run")
+    ms = e0.elapsed_time(e1) / args.steps
+    pairs = B * Hq * T * (T + 1) // 2
+    flops = pairs * 2 * (Dk + Dv)
+    tf = flops / (ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    return {"metric": "d_k != d_v attention forward TFLOPS (bf16 tensor cores)", "value": round(tf, 3),
+            "unit": "TFLOPS", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) q, k, v)",
+            "config": dict(c, l2="not flushed: the per-step working set (about 0.33 GB) exceeds the 126 MB L2",
+                           flop_count="allowed pairs x 2 (Dk + Dv)"),
+            "roofline": {"kernel": "fwd_tc_kernel<192,128>", "bound": "tensor", "achieved": round(tf, 3),
+                         "peak": peak, "unit": "TFLOP/s", "frac": round(tf / peak, 4), "traffic": None,
+                         "peak_source": f"{peak_src} bf16_tflops",
+                         "achieved_def": "forward flops / CUDA-event time of its one launch"},
+            "gpu_launches": args.steps, "clocks": clocks}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -618,7 +686,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--decode", action="store_true", help="time the KV-cache decode kernels instead")
-    ap.add_argument("--dkv", action="store_true", help="time the d_k != d_v (f32) path instead")
+    ap.add_argument("--dkv", action="store_true", help="time the d_k != d_v path instead")
+    ap.add_argument("--dkv-dtype", choices=["f32", "bf16"], default="f32",
+                    help="f32: forward + backward on the CUDA cores; bf16: the tensor-core forward")
     args = ap.parse_args(argv)
     from causal_flash_attention_attn_b200 import inputs
     w = inputs.WORKLOADS[args.workload or inputs.HEADLINE]
@@ -628,7 +698,7 @@ def main(argv=None):
         print(json.dumps(run_decode(args)), flush=True)
         return
     if args.dkv:
-        print(json.dumps(run_dkv(args)), flush=True)
+        print(json.dumps(run_dkv_bf16(args) if args.dkv_dtype == "bf16" else run_dkv(args)), flush=True)
         return
     line = run_reference(args, w) if args.impl == "reference" else run_ours(args, w)
     if line is not None:
