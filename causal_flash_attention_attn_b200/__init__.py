@@ -255,16 +255,51 @@ def forge_attn_version() -> str:
 
 
 # ---------------------------------------------------------- torch conveniences
+# The library reads raw pointers with the documented dense layouts, so these
+# helpers reject what it would misread: host tensors, strided views, mixed
+# dtypes or devices, and shapes that disagree.
+def _check(what, dtype, device, shapes, **tensors):
+    import torch
+    given = {name: t for name, t in tensors.items() if t is not None}
+    for name, t in given.items():
+        want = dtype.get(name)
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{what}: {name} must be a torch tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{what}: {name} must be contiguous")
+        if want is not None and t.dtype != want:
+            raise ValueError(f"{what}: {name} has dtype {t.dtype}, expected {want}")
+        if name in shapes and tuple(t.shape) != tuple(shapes[name]):
+            raise ValueError(f"{what}: {name} has shape {tuple(t.shape)}, expected {tuple(shapes[name])}")
+    for name, t in given.items():
+        if not t.is_cuda:
+            raise ValueError(f"{what}: {name} must be a CUDA tensor")
+        if t.device != device:
+            raise ValueError(f"{what}: {name} is on {t.device}, expected {device}")
+
+
 def _dims(q, k):
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError(f"q and k must be [B, H, T, D], got {tuple(q.shape)} and {tuple(k.shape)}")
     B, Hq, T, D = q.shape
     Hkv = k.shape[1]
+    return B, Hq, Hkv, T, D
+
+
+def _check_bhtd(what, q, k, **rest):
+    import torch
+    B, Hq, Hkv, T, D = _dims(q, k)
+    qs, kvs, rows = (B, Hq, T, D), (B, Hkv, T, D), (B, Hq, T)
+    shapes = dict(k=kvs, v=kvs, o=qs, dO=qs, lse=rows)
+    dt = dict(k=q.dtype, v=q.dtype, o=q.dtype, dO=q.dtype, lse=torch.float32)
+    _check(what, dt, q.device, shapes, q=q, k=k, **rest)
     return B, Hq, Hkv, T, D
 
 
 def attention_fwd(q, k, v, scale=None, window=0, softcap=0.0, stream=None):
     """Forward on device tensors [B,H,T,D] (bf16 or f32). Returns (o, lse)."""
     import torch
-    B, Hq, Hkv, T, D = _dims(q, k)
+    B, Hq, Hkv, T, D = _check_bhtd("attention_fwd", q, k, v=v)
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
@@ -279,8 +314,14 @@ def attention_decode(q, k_cache, v_cache, T=None, scale=None, window=0, softcap=
     """Decode on device tensors: q [B,Hq,D], caches [B,Hkv,Tmax,D]; T defaults to
     Tmax (or the largest of seq_lens, an int32 device tensor [B]). Returns (o, lse)."""
     import torch
+    if q.dim() != 3 or k_cache.dim() != 4:
+        raise ValueError(f"attention_decode: q must be [B, Hq, D] and the caches [B, Hkv, Tmax, D], got "
+                         f"{tuple(q.shape)} and {tuple(k_cache.shape)}")
     B, Hq, D = q.shape
     Hkv, Tmax = k_cache.shape[1], k_cache.shape[2]
+    _check("attention_decode", dict(k_cache=q.dtype, v_cache=q.dtype, sink=torch.float32, seq_lens=torch.int32),
+           q.device, dict(k_cache=(B, Hkv, Tmax, D), v_cache=(B, Hkv, Tmax, D), sink=(Hq,), seq_lens=(B,)),
+           q=q, k_cache=k_cache, v_cache=v_cache, sink=sink, seq_lens=seq_lens)
     if T is None:
         T = int(seq_lens.max().item()) if seq_lens is not None else Tmax
     scale = 1.0 / math.sqrt(D) if scale is None else scale
@@ -297,17 +338,17 @@ def attention_decode(q, k_cache, v_cache, T=None, scale=None, window=0, softcap=
 def attention_bwd(q, k, v, o, lse, dO, scale=None, window=0, softcap=0.0, workspace=None, stream=None):
     """Backward on device tensors. Returns (dq, dk, dv)."""
     import torch
-    B, Hq, Hkv, T, D = _dims(q, k)
+    B, Hq, Hkv, T, D = _check_bhtd("attention_bwd", q, k, v=v, o=o, lse=lse, dO=dO, workspace=workspace)
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     dt = dtype_code(q.dtype)
     nbytes = forge_attn_bwd_workspace_size(B, Hq, Hkv, T, D, dt)
-    if workspace is None or workspace.numel() < nbytes:
+    if workspace is None or workspace.numel() * workspace.element_size() < nbytes:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
     dq = torch.empty_like(q)
     dk = torch.empty_like(k)
     dv = torch.empty_like(v)
     s = forge_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale, window, softcap, dt,
-                       workspace, workspace.numel(), stream)
+                       workspace, workspace.numel() * workspace.element_size(), stream)
     if s != FORGE_OK:
         raise ForgeError(s, "forge_attn_bwd")
     return dq, dk, dv
