@@ -54,7 +54,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
     res = subprocess.run(cmd, capture_output=True, text=True)
     log = os.path.join(PKG, "build.log")
     with open(log, "w") as f:
-        f.write(" ".join(cmd) + "\n" + res.stdout + res.stderr)
+        # paths relative to the repository root, so the log reads the same on every machine
+        f.write((" ".join(cmd) + "\n" + res.stdout + res.stderr).replace(ROOT + os.sep, ""))
     if res.returncode != 0:
         sys.stderr.write(res.stderr[-20000:])
         raise RuntimeError(f"nvcc failed (see {log})")

@@ -1,5 +1,5 @@
 """Helpers shared by the GPU parity tests: run the CUDA path and the oracle on the
-same seeded inputs and compare with the tolerances of the spec contract:
+same seeded inputs and compare with the path's stated tolerances:
 max-abs 1e-4 on the f32 path (the Forge pages' own CPU-vs-GPU bar), and
 |gpu - ref| <= 2e-2 + 1e-2 * |ref| elementwise for bf16 inputs with f32
 accumulation."""
