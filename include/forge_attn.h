@@ -28,7 +28,13 @@
  *   FORGE_DTYPE_BF16 runs the tensor-core kernels (bf16 operands, f32
  *   accumulation, P and dS rounded to bf16 before their products);
  *   FORGE_DTYPE_F32 runs f32 CUDA-core kernels (f32 arithmetic throughout).
- *   Supported head dims: 64, 128, 256.
+ *   Supported head dims: 64, 128, 256 (d_k != d_v: forge_attn_fwd_dkv).
+ *
+ * Sizes (checked before any launch; FORGE_ERR_INVALID_ARG otherwise):
+ *   B, Hq, Hkv, T >= 1 (an empty problem is an error, not a no-op);
+ *   Hq % Hkv == 0; D even; B * Hq <= 2^24; T <= 2^30; B * Hq * T * D <= 2^40
+ *   elements; (T / 128 rounded up) * B * Hq < 2^31 (the grid). A D that passes
+ *   these but has no kernel returns FORGE_ERR_UNSUPPORTED.
  *
  * Ownership and behaviour:
  *   The caller allocates and frees every buffer, including the backward

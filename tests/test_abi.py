@@ -75,6 +75,25 @@ def test_fwd_rejects(kw, code):
     assert fwd(**kw) == code
 
 
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=1 << 12, Hq=1 << 12, Hkv=1 << 12, T=1), fa.FORGE_OK),               # B * Hq = 2^24: allowed
+    (dict(B=(1 << 12) + 1, Hq=1 << 12, Hkv=1 << 12, T=1), fa.FORGE_ERR_INVALID_ARG),
+    (dict(B=1, Hq=1, Hkv=1, T=1 << 30, D=64), fa.FORGE_OK),                     # 2^36 elements
+    (dict(B=1, Hq=1, Hkv=1, T=(1 << 30) + 1, D=64), fa.FORGE_ERR_INVALID_ARG),  # T > 2^30
+    (dict(B=1 << 6, Hq=1 << 8, Hkv=1 << 8, T=1 << 20, D=64), fa.FORGE_OK),      # 2^40 elements exactly
+    (dict(B=1 << 6, Hq=1 << 8, Hkv=1 << 8, T=1 << 20, D=128), fa.FORGE_ERR_INVALID_ARG),
+])
+def test_size_limits(kw, code):
+    # the index-arithmetic limits the header states; the workspace size is the
+    # host-side function that applies them without launching anything
+    a = dict(B=1, Hq=4, Hkv=2, T=128, D=128)
+    a.update(kw)
+    n = fa.forge_attn_bwd_workspace_size(a["B"], a["Hq"], a["Hkv"], a["T"], a["D"], fa.FORGE_DTYPE_BF16)
+    assert (n > 0) == (code == fa.FORGE_OK)
+    if code != fa.FORGE_OK:
+        assert fwd(**kw) == code
+
+
 def test_workspace_size_and_rejection():
     bf, f32 = fa.FORGE_DTYPE_BF16, fa.FORGE_DTYPE_F32
     n = fa.forge_attn_bwd_workspace_size(2, 28, 4, 4096, 128, bf)
