@@ -9,8 +9,8 @@
 //   dP^T = V dO^T           (tcgen05)
 //   P^T  = exp2(s*log2e - LSE*log2e), masked to 0   -> bf16 into TMEM (over S^T)
 //   dS^T = scale * P^T (dP^T - Delta) [* (1 - tanh^2)] -> bf16 into shared memory
-//          (the cap factor is the "exact tanh' chain": src/nn/attention.h
-//           commit log, Wave 2)
+//          (the cap's derivative taken exactly, as every backward on the pages
+//           does: src/nn/attention.h commit log, Wave 2)
 //   dV  += P^T dO           (A from TMEM)
 //   dK  += dS^T Q
 //   dQ   = dS K  (or its transpose K^T dS^T), drained from TMEM by four warps
@@ -148,7 +148,7 @@ struct BwdParams {
 //   phase A (needs S^T): P = exp2(s * scale * log2(e) - LSE * log2(e)), masked
 //            to 0, as bf16 pairs pk (P^T for dV += P^T dO), and the factor g of
 //            dS = g * (dP - Delta): g = P, or P (1 - tanh^2) under the cap
-//            (the "exact tanh' chain": src/nn/attention.h commit log, Wave 2);
+//            (the cap differentiated exactly: src/nn/attention.h commit log, Wave 2);
 //   phase B (needs dP^T): dS = g * (dP * scale - Delta * scale) as bf16 pairs.
 //   nl, nd: -LSE*log2(e) and -scale*Delta of the 32 columns (shared memory).
 // CAP and MASK are compile-time so each unrolled loop is one basic block; the

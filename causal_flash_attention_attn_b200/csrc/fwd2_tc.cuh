@@ -7,8 +7,8 @@
 // scores are in softmax, the tensor cores work on the other tile. Tile A sees
 // KV tiles [loA, tA], tile B [loB, tB] (tB = tA + 1); both ranges are the
 // causal/window ranges of their rows, so out-of-window KV tiles are never loaded
-// ("out-of-window KV blocks are skipped, so cost scales with the window":
-// src/nn/attention.h commit log, Wave 2).
+// (the pages' flash kernels skip KV blocks outside the window, which makes the
+// cost follow the window size: src/nn/attention.h commit log, Wave 2).
 //
 // Roles (384 threads): warps 0-3 softmax of tile A, warps 4-7 softmax of tile
 // B (one thread per query row / TMEM lane), warp 8 TMA producer, warp 9 MMA

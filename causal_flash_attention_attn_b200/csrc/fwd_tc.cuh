@@ -3,8 +3,8 @@
 // One CTA per (query tile of 128 rows, batch, query head), heaviest tiles
 // first. Only the KV tiles a tile can see are visited: j from
 // lo = (q0 - W + 1) / 128 (0 without a window) up to the diagonal tile, so the
-// cost scales with the window ("out-of-window KV blocks are skipped, so cost
-// scales with the window": src/nn/attention.h commit log, Wave 2).
+// cost follows the window size, as in the pages' flash kernels, which skip KV
+// blocks outside the window (src/nn/attention.h commit log, Wave 2).
 //
 // Roles (192 threads):
 //   warp 4   TMA producer: Q once, then K/V tiles through an NSTAGE ring in the

@@ -105,8 +105,8 @@ def layer_window(layer: int, window: int, global_every: int) -> int:
     ``sliding_global_every`` config pair (forge-studio RESEARCH.md section 2).
 
     Reading: layers are 0-based and layer l is global (window 0) when
-    global_every > 0 and (l + 1) % global_every == 0, so "5 local : 1 global"
-    (Gemma 3, ARCHITECTURES.md family table) is global_every = 6 and "alternating"
+    global_every > 0 and (l + 1) % global_every == 0, so five local layers per
+    global one (Gemma 3, ARCHITECTURES.md family table) is global_every = 6 and "alternating"
     (Gemma 2) is global_every = 2. With global_every = 0 every layer uses ``window``.
     """
     if global_every > 0 and (layer + 1) % global_every == 0:

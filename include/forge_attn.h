@@ -7,8 +7,9 @@
  * What the operation is (Forge pages):
  *   S_ij  = scale * (q_i . k_j)
  *   s_ij  = softcap * tanh(S_ij / softcap)      if softcap > 0, else S_ij
- *           ("cap*tanh on scores pre-softmax": src/nn/attention.h commit log,
- *            Wave 2 (attention kernels); ARCHITECTURES.md "Vague 2" item 9)
+ *           (the cap applies tanh to the scores before the softmax:
+ *            src/nn/attention.h commit log, Wave 2 (attention kernels);
+ *            ARCHITECTURES.md "Vague 2" item 9)
  *   key j is visible to query i iff  i - window < j <= i   (window = 0: j <= i)
  *           (ARCHITECTURES.md "Vague 2" item 8; sliding_window(0) default,
  *            forge-studio RESEARCH.md section 2)
@@ -17,7 +18,8 @@
  *   Query head hq reads KV head hq / (Hq / Hkv) (GQA; Hq % Hkv == 0 is the
  *   config rule n_heads % n_kv_heads == 0, RESEARCH.md section 2).
  *   The backward is the exact gradient of o with respect to q, k, v, including
- *   the tanh' factor of the cap ("exact tanh' chain in all backwards").
+ *   the tanh' factor of the cap (every backward on the pages differentiates
+ *   through the cap exactly).
  *   A per-layer pattern (sliding_global_every) is chosen by the caller: a global
  *   layer passes window = 0.
  *
@@ -81,8 +83,8 @@ forge_status forge_attn_fwd(const void *q, const void *k, const void *v, void *o
  * this is forge_attn_fwd):
  *  - sink [Hq] f32 (device): a learned logit per query head that joins every
  *    row's softmax denominator and has no value vector (attention sinks:
- *    ARCHITECTURES.md family table, GPT-OSS row, "biais par tête dans le
- *    dénominateur softmax"; "Vague 2" item 10, which starts the online softmax's
+ *    ARCHITECTURES.md family table, GPT-OSS row, a per-head bias added to the
+ *    softmax denominator; "Vague 2" item 10, which starts the online softmax's
  *    (max, sum) from it). In the units of the scores the softmax sees (after
  *    scale and cap; the sink itself is not capped). P_ij = exp(s_ij) /
  *    (exp(sink[hq]) + sum_j exp(s_ij)); lse includes it.

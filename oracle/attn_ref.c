@@ -16,7 +16,8 @@
  *    schema (forge-studio RESEARCH.md, section 2).
  *  - softcap: s -> cap * tanh(s / cap) on the pre-softmax scores, cap = 0 off.
  *    ARCHITECTURES.md "Vague 2" item 9; src/nn/attention.h commit log, "Wave 2
- *    (attention kernels)": attn_softcap, exact tanh' chain in all backwards.
+ *    (attention kernels)": attn_softcap, whose backward differentiates through
+ *    the tanh exactly.
  *  - GQA: n_heads % n_kv_heads == 0 (config schema validation, RESEARCH.md
  *    section 2). Reading: query head hq uses KV head hq / (Hq / Hkv), i.e. each
  *    KV head serves a contiguous group of query heads.
@@ -25,8 +26,8 @@
  *  - Reading: the scale multiplies q.k before the cap: s = cap*tanh(scale*q.k/cap).
  *  - Reading: LSE is the natural-log log-sum-exp of the (capped) scores of a row.
  *  - attention sinks: a learned logit per head that joins the softmax
- *    denominator and has no value vector ("biais par tête dans le dénominateur
- *    softmax": ARCHITECTURES.md family table, GPT-OSS row; "Vague 2" item 10,
+ *    denominator and has no value vector (a per-head bias in the softmax
+ *    denominator: ARCHITECTURES.md family table, GPT-OSS row; "Vague 2" item 10,
  *    which seeds the online softmax's (max, sum) with it; SMALL_MODELS_RESEARCH.md
  *    section 2.4). Readings: one logit sigma_h per query head, shared by every
  *    batch entry and row, in the units of the scores the softmax sees (it is

@@ -123,7 +123,7 @@ def test_selftest_rejects_bad_limit():
 
 def test_layer_window_pattern():
     from causal_flash_attention_attn_b200.inputs import layer_window
-    # Gemma 3-like 5 local : 1 global
+    # Gemma 3-like: five local layers, then one global
     assert [layer_window(l, 1024, 6) for l in range(12)] == [1024] * 5 + [0] + [1024] * 5 + [0]
     # alternating
     assert [layer_window(l, 4096, 2) for l in range(4)] == [4096, 0, 4096, 0]
