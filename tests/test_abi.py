@@ -215,3 +215,40 @@ def test_header_compiles_as_c99_and_links(tmp_path):
     assert int(out[1]) == fa.FORGE_ERR_INVALID_ARG and int(out[2]) == fa.FORGE_ERR_UNSUPPORTED
     assert out[3] == "sm_100a"
     assert line2 == fa.forge_attn_status_string(fa.FORGE_ERR_WORKSPACE)
+
+
+def _c_to_ctypes(decl):
+    """ctypes type the binding should use for one C parameter or return type."""
+    decl = " ".join(decl.replace("const ", "").split())
+    if "*" in decl:
+        return ctypes.c_char_p if decl.startswith("char") else ctypes.c_void_p
+    base = decl.split()[0] if decl.split()[0] != "unsigned" else "unsigned"
+    return {"int": ctypes.c_int, "float": ctypes.c_float, "size_t": ctypes.c_size_t, "unsigned": ctypes.c_uint,
+            "forge_dtype": ctypes.c_int, "forge_status": ctypes.c_int}[base]
+
+
+def header_prototypes():
+    text = re.sub(r"/\*.*?\*/", " ", open(HEADER).read(), flags=re.S)
+    protos = {}
+    for ret, name, params in re.findall(r"([\w][\w\s\*]*?)\s*\b(forge_attn_\w+)\s*\(([^)]*)\)\s*;", text):
+        params = " ".join(params.split())
+        plist = [] if params in ("", "void") else [p.strip() for p in params.split(",")]
+        # drop the parameter name, keep its type (pointer stars may sit on the name)
+        types = [re.sub(r"\b\w+$", "", p).strip() or p for p in plist]
+        protos[name] = (ret.strip(), types)
+    return protos
+
+
+def test_binding_signatures_match_the_header():
+    # every prototype's parameter count and kinds (pointer, int, float, size_t,
+    # unsigned) and its return kind equal the ctypes declarations the binding uses
+    protos = header_prototypes()
+    assert set(protos) == set(declared_functions())
+    L = fa.library()
+    for name, (ret, types) in protos.items():
+        fn = getattr(L, name)
+        want = [_c_to_ctypes(t) for t in types]
+        assert fn.argtypes is not None, name
+        assert list(fn.argtypes) == want, (name, fn.argtypes, want)
+        want_ret = _c_to_ctypes(ret)
+        assert fn.restype == want_ret, (name, fn.restype, want_ret)
