@@ -22,6 +22,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -104,31 +105,152 @@ def ncu_traffic(kernel, workload):
 
 
 # ------------------------------------------------------------------ clocks
-class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+REASON_NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, index):
+
+def parse_smi_lines(lines):
+    """(sm MHz samples, max MHz, reasons seen active) from nvidia-smi CSV lines of
+    ClockSampler.SMI_FIELDS (noheader, nounits)."""
+    sm, mx, reasons = [], None, set()
+    for line in lines:
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            sm.append(float(parts[1]))
+            mx = float(parts[2])
+        except ValueError:
+            continue
+        for n, v in zip(REASON_NAMES, parts[5:9]):
+            if v.lower() == "active":
+                reasons.add(n)
+    return sm, mx, reasons
+
+
+class ClockSampler:
+    """SM clock and clock-event reasons of the GPU a run uses, sampled while its
+    timed region runs (read-only: nothing here changes a GPU setting).
+
+    NVML first: a thread reads the clock and the reasons every `period_s`, the GPU
+    found by its UUID (then its PCI address) so that the sampled GPU is the one
+    CUDA runs on; only samples between begin() and end() -- host times that
+    bracket the timed region -- count. If NVML is unavailable, nvidia-smi polls
+    every 100 ms and every sample counts."""
+    SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index, period_s=0.002):
         self.index = index
+        self.period_s = period_s
         self.proc = None
         self.lines = []
+        self.samples = []          # (host time, sm MHz, reason mask) from NVML
+        self.t_begin = self.t_end = None
+        self.nvml = None
+        self.handle = None
+        self.max_mhz = None
+        self.bits = {}
+        self.stop_evt = threading.Event()
+        self.thread = None
+
+    def _uuid(self):
+        """NVML's name of the device ("GPU-" + 8-4-4-4-12 hex), or None."""
+        import torch
+        u = str(torch.cuda.get_device_properties(self.index).uuid)
+        return "GPU-" + u if re.fullmatch(r"[0-9a-fA-F]{8}(-[0-9a-fA-F]{4}){3}-[0-9a-fA-F]{12}", u) else None
+
+    # -- NVML
+    def _nvml_handle(self, nv):
+        import torch
+        uuid = self._uuid()
+        if uuid is not None:
+            try:
+                return nv.nvmlDeviceGetHandleByUUID(uuid)
+            except Exception:
+                pass
+        props = torch.cuda.get_device_properties(self.index)
+        bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+        return nv.nvmlDeviceGetHandleByPciBusId(bus)
+
+    def _start_nvml(self):
+        import pynvml as nv
+        nv.nvmlInit()
+        try:
+            self.handle = self._nvml_handle(nv)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM))
+            get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            for name, suffix in zip(REASON_NAMES, ("HwSlowdown", "HwThermalSlowdown", "SwThermalSlowdown",
+                                                   "SwPowerCap")):
+                self.bits[name] = getattr(nv, "nvmlClocksEventReason" + suffix,
+                                          getattr(nv, "nvmlClocksThrottleReason" + suffix, 0))
+            # one read before the thread starts, so a failing call falls back here
+            nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+            get(self.handle)
+        except Exception:
+            nv.nvmlShutdown()
+            raise
+        self.nvml = nv
+
+        def loop():
+            while not self.stop_evt.is_set():
+                t = time.perf_counter()
+                try:
+                    mhz = float(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM))
+                    mask = int(get(self.handle))
+                    self.samples.append((t, mhz, mask))
+                except Exception:
+                    pass
+                self.stop_evt.wait(self.period_s)
+
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
+
+    # -- nvidia-smi fallback
+    def _start_smi(self):
+        ident = str(self.index)
+        try:
+            ident = self._uuid() or ident
+        except Exception:
+            pass
+        self.proc = subprocess.Popen(
+            ["nvidia-smi", f"--id={ident}", f"--query-gpu={self.SMI_FIELDS}", "--format=csv,noheader,nounits",
+             "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+
+        def read():
+            for line in self.proc.stdout:
+                self.lines.append(line.strip())
+
+        self.thread = threading.Thread(target=read, daemon=True)
+        self.thread.start()
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
+            self._start_nvml()
+            return
+        except Exception:
+            self.nvml = None
+        try:
+            self._start_smi()
         except Exception:
             self.proc = None
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def begin(self):
+        self.t_begin = time.perf_counter()
+
+    def end(self):
+        self.t_end = time.perf_counter()
 
     def stop(self):
+        if self.nvml is not None:
+            self.stop_evt.set()
+            self.thread.join(timeout=2)
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
+            return self.summary_nvml()
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -137,24 +259,29 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.thread.join(timeout=2)
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
+        sm, mx, reasons = parse_smi_lines(self.lines)
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvidia-smi every 100 ms (before, during and after the timed region)"}
+
+    def summary_nvml(self):
+        lo = self.t_begin if self.t_begin is not None else float("-inf")
+        hi = self.t_end if self.t_end is not None else float("inf")
+        inside = [(mhz, mask) for t, mhz, mask in self.samples if lo <= t <= hi]
+        where = "inside the timed region"
+        if not inside:
+            # a region shorter than the period: the first sample after it began
+            after = [(mhz, mask) for t, mhz, mask in self.samples if t >= lo]
+            inside, where = after[:1], "first sample after the timed region began"
+        if not inside:
+            inside, where = [(mhz, mask) for _, mhz, mask in self.samples], "all samples (none after the region began)"
+        if not inside:
+            return None
+        reasons = sorted(n for n in REASON_NAMES if any(mask & self.bits.get(n, 0) for _, mask in inside))
+        return {"sm_mhz": statistics.median(m for m, _ in inside), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(inside),
+                "source": f"NVML every {self.period_s * 1e3:g} ms, {where}"}
 
 
 # ------------------------------------------------------------ distributed
@@ -297,11 +424,13 @@ def run_ours(args, w):
     time.sleep(0.3)
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
+    clk.begin()
     start.record(stream)
     for i in range(args.steps):
         step(evs[i])
     end.record(stream)
     torch.cuda.synchronize(dev)
+    clk.end()
     clocks = clk.stop()
     barrier(world, dev)
     st = fa.forge_attn_check(sh)
@@ -506,11 +635,13 @@ def run_decode(args):
     clk.start()
     time.sleep(0.3)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk.begin()
     e0.record(stream)
     for _ in range(args.steps):
         call()
     e1.record(stream)
     torch.cuda.synchronize(dev)
+    clk.end()
     clocks = clk.stop()
     st = fa.forge_attn_check(stream.cuda_stream)
     if st != fa.FORGE_OK:
@@ -581,11 +712,13 @@ def run_dkv(args):
     clk.start()
     time.sleep(0.3)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk.begin()
     e0.record(stream)
     for _ in range(args.steps):
         step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
+    clk.end()
     clocks = clk.stop()
     st = fa.forge_attn_check(sh)
     if st != fa.FORGE_OK:
@@ -647,11 +780,13 @@ def run_dkv_bf16(args):
     clk.start()
     time.sleep(0.3)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk.begin()
     e0.record(stream)
     for _ in range(args.steps):
         step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
+    clk.end()
     clocks = clk.stop()
     st = fa.forge_attn_check(sh)
     if st != fa.FORGE_OK:
