@@ -286,27 +286,50 @@ def _dims(q, k):
     return B, Hq, Hkv, T, D
 
 
-def _check_bhtd(what, q, k, **rest):
+def _check_bhtd(what, q, k, v, extras=False, **rest):
+    """Checks q, k, v and the rest; v (and o, dO) may have a head dim Dv of its own,
+    but then without the sink / max-logit extras. Returns (B, Hq, Hkv, T, D, Dv)."""
     import torch
     B, Hq, Hkv, T, D = _dims(q, k)
-    qs, kvs, rows = (B, Hq, T, D), (B, Hkv, T, D), (B, Hq, T)
-    shapes = dict(k=kvs, v=kvs, o=qs, dO=qs, lse=rows)
-    dt = dict(k=q.dtype, v=q.dtype, o=q.dtype, dO=q.dtype, lse=torch.float32)
-    _check(what, dt, q.device, shapes, q=q, k=k, **rest)
-    return B, Hq, Hkv, T, D
+    if v.dim() != 4:
+        raise ValueError(f"{what}: v must be [B, Hkv, T, Dv], got {tuple(v.shape)}")
+    Dv = v.shape[3]
+    if Dv != D and extras:
+        raise ValueError(f"{what}: sinks and the max logit are not offered with d_k != d_v")
+    qs, ks, vs, rows = (B, Hq, T, Dv), (B, Hkv, T, D), (B, Hkv, T, Dv), (B, Hq, T)
+    shapes = dict(k=ks, v=vs, o=qs, dO=qs, lse=rows, sink=(Hq,))
+    f = torch.float32
+    dt = dict(k=q.dtype, v=q.dtype, o=q.dtype, dO=q.dtype, lse=f, sink=f)
+    _check(what, dt, q.device, shapes, q=q, k=k, v=v, **rest)
+    return B, Hq, Hkv, T, D, Dv
 
 
-def attention_fwd(q, k, v, scale=None, window=0, softcap=0.0, stream=None):
-    """Forward on device tensors [B,H,T,D] (bf16 or f32). Returns (o, lse)."""
+def attention_fwd(q, k, v, scale=None, window=0, softcap=0.0, stream=None, *, sink=None, return_max_logit=False):
+    """Forward on device tensors q [B,Hq,T,D], k [B,Hkv,T,D], v [B,Hkv,T,Dv] (bf16
+    or f32). Returns (o, lse), or (o, lse, max_logit [B,Hq]) with
+    return_max_logit. sink: optional f32 [Hq] sink logits. Dv != D runs the
+    d_k != d_v entry point (no sink, no max logit there)."""
     import torch
-    B, Hq, Hkv, T, D = _check_bhtd("attention_fwd", q, k, v=v)
+    B, Hq, Hkv, T, D, Dv = _check_bhtd("attention_fwd", q, k, v, extras=sink is not None or return_max_logit,
+                                       sink=sink)
     scale = 1.0 / math.sqrt(D) if scale is None else scale
-    o = torch.empty_like(q)
+    dt = dtype_code(q.dtype)
+    o = torch.empty((B, Hq, T, Dv), dtype=q.dtype, device=q.device)
     lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
-    s = forge_attn_fwd(q, k, v, o, lse, B, Hq, Hkv, T, D, scale, window, softcap, dtype_code(q.dtype), stream)
+    ml = None
+    if Dv != D:
+        s, what = forge_attn_fwd_dkv(q, k, v, o, lse, B, Hq, Hkv, T, D, Dv, scale, window, softcap, dt,
+                                     stream), "forge_attn_fwd_dkv"
+    elif sink is not None or return_max_logit:
+        ml = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if return_max_logit else None
+        s, what = forge_attn_fwd_ext(q, k, v, o, lse, B, Hq, Hkv, T, D, scale, window, softcap, sink, ml, dt,
+                                     stream), "forge_attn_fwd_ext"
+    else:
+        s, what = forge_attn_fwd(q, k, v, o, lse, B, Hq, Hkv, T, D, scale, window, softcap, dt,
+                                 stream), "forge_attn_fwd"
     if s != FORGE_OK:
-        raise ForgeError(s, "forge_attn_fwd")
-    return o, lse
+        raise ForgeError(s, what)
+    return (o, lse, ml) if return_max_logit else (o, lse)
 
 
 def attention_decode(q, k_cache, v_cache, T=None, scale=None, window=0, softcap=0.0, seq_lens=None, sink=None,
@@ -335,20 +358,39 @@ def attention_decode(q, k_cache, v_cache, T=None, scale=None, window=0, softcap=
     return o, lse
 
 
-def attention_bwd(q, k, v, o, lse, dO, scale=None, window=0, softcap=0.0, workspace=None, stream=None):
-    """Backward on device tensors. Returns (dq, dk, dv)."""
+def attention_bwd(q, k, v, o, lse, dO, scale=None, window=0, softcap=0.0, workspace=None, stream=None, *,
+                  sink=None):
+    """Backward on device tensors (o and lse from the matching forward). Returns
+    (dq, dk, dv), or (dq, dk, dv, dsink [Hq]) when the forward had a sink. Dv != D
+    runs the d_k != d_v entry point."""
     import torch
-    B, Hq, Hkv, T, D = _check_bhtd("attention_bwd", q, k, v=v, o=o, lse=lse, dO=dO, workspace=workspace)
+    B, Hq, Hkv, T, D, Dv = _check_bhtd("attention_bwd", q, k, v, extras=sink is not None, o=o, lse=lse, dO=dO,
+                                       workspace=workspace, sink=sink)
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     dt = dtype_code(q.dtype)
-    nbytes = forge_attn_bwd_workspace_size(B, Hq, Hkv, T, D, dt)
+    if Dv != D:
+        nbytes = forge_attn_bwd_workspace_size_dkv(B, Hq, Hkv, T, D, Dv, dt)
+        if nbytes == 0:
+            raise ForgeError(FORGE_ERR_UNSUPPORTED, "forge_attn_bwd_dkv")
+    else:
+        nbytes = forge_attn_bwd_workspace_size(B, Hq, Hkv, T, D, dt)
     if workspace is None or workspace.numel() * workspace.element_size() < nbytes:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    wbytes = workspace.numel() * workspace.element_size()
     dq = torch.empty_like(q)
     dk = torch.empty_like(k)
     dv = torch.empty_like(v)
-    s = forge_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale, window, softcap, dt,
-                       workspace, workspace.numel() * workspace.element_size(), stream)
+    dsink = None
+    if Dv != D:
+        s, what = forge_attn_bwd_dkv(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, Dv, scale, window, softcap,
+                                     dt, workspace, wbytes, stream), "forge_attn_bwd_dkv"
+    elif sink is not None:
+        dsink = torch.empty((Hq,), dtype=torch.float32, device=q.device)
+        s, what = forge_attn_bwd_ext(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale, window, softcap,
+                                     sink, dsink, dt, workspace, wbytes, stream), "forge_attn_bwd_ext"
+    else:
+        s, what = forge_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, D, scale, window, softcap, dt,
+                                 workspace, wbytes, stream), "forge_attn_bwd"
     if s != FORGE_OK:
-        raise ForgeError(s, "forge_attn_bwd")
-    return dq, dk, dv
+        raise ForgeError(s, what)
+    return (dq, dk, dv, dsink) if sink is not None else (dq, dk, dv)

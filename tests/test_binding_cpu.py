@@ -47,8 +47,8 @@ def test_mixed_dtypes_are_rejected():
 
 
 def test_disagreeing_shapes_are_rejected():
-    with pytest.raises(ValueError, match=r"v has shape \(1, 2, 64, 16\)"):
-        fa.attention_fwd(Q, K, z(1, 2, 64, 16))
+    with pytest.raises(ValueError, match=r"v has shape \(1, 2, 63, 32\)"):
+        fa.attention_fwd(Q, K, z(1, 2, 63, 32))
     with pytest.raises(ValueError, match=r"k has shape"):
         fa.attention_fwd(Q, z(1, 2, 65, 32), z(1, 2, 65, 32))
     with pytest.raises(ValueError, match=r"o has shape"):
@@ -72,3 +72,33 @@ def test_workspace_must_be_contiguous():
     ws = torch.zeros(64, 64, dtype=torch.uint8).t()
     with pytest.raises(ValueError, match="workspace must be contiguous"):
         fa.attention_bwd(Q, K, K, Q, LSE, Q, workspace=ws)
+
+
+def test_extras_are_checked_like_the_rest():
+    with pytest.raises(ValueError, match="sink has dtype torch.bfloat16"):
+        fa.attention_fwd(Q, K, K, sink=z(4))
+    with pytest.raises(ValueError, match=r"sink has shape \(2,\)"):
+        fa.attention_fwd(Q, K, K, sink=z(2, dtype=torch.float32))
+    with pytest.raises(ValueError, match=r"sink has shape"):
+        fa.attention_bwd(Q, K, K, Q, LSE, Q, sink=z(3, dtype=torch.float32))
+    with pytest.raises(ValueError, match="q must be a CUDA tensor"):
+        fa.attention_fwd(Q, K, K, sink=z(4, dtype=torch.float32), return_max_logit=True)
+
+
+def test_dk_ne_dv_shapes_and_restrictions():
+    v48 = z(1, 2, 64, 48)          # d_v = 48 against d_k = 32
+    o48 = z(1, 4, 64, 48)
+    # o and dO take v's head dim
+    with pytest.raises(ValueError, match="q must be a CUDA tensor"):
+        fa.attention_fwd(Q, K, v48)
+    with pytest.raises(ValueError, match="q must be a CUDA tensor"):
+        fa.attention_bwd(Q, K, v48, o48, LSE, o48)
+    with pytest.raises(ValueError, match=r"o has shape \(1, 4, 64, 32\), expected \(1, 4, 64, 48\)"):
+        fa.attention_bwd(Q, K, v48, Q, LSE, o48)
+    # the extras are not offered with d_k != d_v
+    with pytest.raises(ValueError, match="not offered with d_k != d_v"):
+        fa.attention_fwd(Q, K, v48, sink=z(4, dtype=torch.float32))
+    with pytest.raises(ValueError, match="not offered with d_k != d_v"):
+        fa.attention_fwd(Q, K, v48, return_max_logit=True)
+    with pytest.raises(ValueError, match="not offered with d_k != d_v"):
+        fa.attention_bwd(Q, K, v48, o48, LSE, o48, sink=z(4, dtype=torch.float32))
