@@ -2,8 +2,9 @@
 
 The functions named ``forge_attn_*`` mirror the C ABI in include/forge_attn.h one
 to one (argument marshalling only: every pointer argument accepts a torch
-tensor or an integer device address). ``attention_fwd`` / ``attention_bwd``
-allocate outputs and workspace with torch and call them.
+tensor or an integer device address). ``attention_fwd`` / ``attention_bwd`` /
+``attention_decode`` allocate outputs and workspace with torch and call them;
+``attention`` wraps the first two in a torch.autograd.Function.
 
 PyTorch is used for device memory and streams only; all arithmetic runs in the
 library's CUDA kernels. There is no fallback: if the shared library is missing
@@ -24,7 +25,7 @@ __all__ = [
     "forge_attn_bwd_workspace_size_dkv",
     "forge_attn_bwd_preprocess", "forge_attn_bwd_main", "forge_attn_bwd_finalize", "forge_attn_check",
     "forge_attn_status_string", "forge_attn_selftest_timeout", "forge_attn_selftest_exp2", "forge_attn_last_cuda_error", "forge_attn_timeout_info", "forge_attn_version",
-    "attention_fwd", "attention_bwd", "dtype_code",
+    "attention_fwd", "attention_bwd", "attention", "dtype_code",
 ]
 
 FORGE_OK = 0
@@ -394,3 +395,40 @@ def attention_bwd(q, k, v, o, lse, dO, scale=None, window=0, softcap=0.0, worksp
     if s != FORGE_OK:
         raise ForgeError(s, what)
     return (dq, dk, dv, dsink) if sink is not None else (dq, dk, dv)
+
+
+# ------------------------------------------------------------------ autograd
+_attention_fn = None
+
+
+def _attention_function():
+    """The torch.autograd.Function over attention_fwd / attention_bwd (built on
+    first use, so that importing this module does not import torch)."""
+    global _attention_fn
+    if _attention_fn is None:
+        import torch
+
+        class ForgeAttention(torch.autograd.Function):
+            @staticmethod
+            def forward(ctx, q, k, v, sink, scale, window, softcap):
+                o, lse = attention_fwd(q, k, v, scale, window, softcap, sink=sink)
+                ctx.save_for_backward(q, k, v, o, lse, sink)
+                ctx.args = (scale, window, softcap)
+                return o
+
+            @staticmethod
+            def backward(ctx, dO):
+                q, k, v, o, lse, sink = ctx.saved_tensors
+                g = attention_bwd(q, k, v, o, lse, dO.contiguous(), *ctx.args, sink=sink)
+                return g[0], g[1], g[2], (g[3] if sink is not None else None), None, None, None
+
+        _attention_fn = ForgeAttention
+    return _attention_fn
+
+
+def attention(q, k, v, scale=None, window=0, softcap=0.0, sink=None):
+    """Causal attention with autograd: o = attention(q, k, v), gradients for q, k,
+    v (and sink) through the library's backward. Shapes, dtypes and options as
+    attention_fwd; scale defaults to 1/sqrt(head dim of q)."""
+    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else float(scale)
+    return _attention_function().apply(q, k, v, sink, scale, int(window), float(softcap))
