@@ -234,9 +234,13 @@ forge_status forge_attn_decode(const void *q, const void *k_cache, const void *v
                                size_t workspace_bytes, void *stream);
 
 /*
- * Synchronises `stream`, then reports (and clears) any error a kernel of this
- * library recorded on the current device since the last check: FORGE_OK,
- * FORGE_ERR_TIMEOUT, or FORGE_ERR_CUDA for an asynchronous CUDA error.
+ * Synchronises `stream`, then reports (and clears) the error a kernel of this
+ * library recorded on the current device since the last check, or FORGE_OK:
+ *   FORGE_ERR_TIMEOUT      a bounded wait inside a kernel ran out;
+ *   FORGE_ERR_INVALID_ARG  a decode length outside [1, T] (forge_attn_decode);
+ *   FORGE_ERR_UNSUPPORTED  the backward's shared-memory layout did not fit the
+ *                          dynamic shared-memory base it was given (nothing written);
+ *   FORGE_ERR_CUDA         an asynchronous CUDA error (forge_attn_last_cuda_error).
  */
 forge_status forge_attn_check(void *stream);
 
