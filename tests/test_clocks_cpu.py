@@ -79,7 +79,7 @@ def test_only_samples_inside_the_timed_region_count(fake):
     clk.begin()
     time.sleep(0.05)
     clk.end()
-    time.sleep(0.01)
+    time.sleep(0.1)                        # margin: a read that began before end() has finished
     nv.state.update(mhz=900.0, mask=0x8 | 0x40)  # after the region: must not count
     time.sleep(0.03)
     rec = clk.stop()
