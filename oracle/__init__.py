@@ -22,7 +22,6 @@ Every function takes and returns numpy float64 arrays in [B, H, T, D] layout.
 from __future__ import annotations
 
 import ctypes
-import os
 
 import numpy as np
 

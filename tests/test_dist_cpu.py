@@ -3,8 +3,6 @@ reduction, the barrier, the rank environment and the weak-scaling aggregate."""
 import os
 import socket
 
-import pytest
-import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 

@@ -4,7 +4,6 @@ ABI against the oracle, on the f32 CUDA-core path, with GQA, a window, a cap and
 ragged lengths. Tolerance: the f32 bar (1e-4 absolute)."""
 import math
 
-import numpy as np
 import pytest
 import torch
 

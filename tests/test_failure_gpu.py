@@ -1,7 +1,6 @@
 """Failure detection on the GPU without faulting it: a kernel waits on a barrier
 nothing completes, its bounded wait runs out after a short limit, it records
 FORGE_ERR_TIMEOUT and returns; the context stays usable."""
-import math
 
 import pytest
 import torch
