@@ -57,3 +57,40 @@ def test_single_process_paths_and_aggregate():
     one = bench.aggregate_tflops(1, 8.42e11, 1.4)
     assert abs(bench.aggregate_tflops(4, 8.42e11, 1.4) - 4 * one) < 1e-9
     assert abs(one - 8.42e11 / 1.4e-3 / 1e12) < 1e-9
+
+
+def _worker_one_dies(rank, world, port, out):
+    """Rank 1 leaves between steps (after the group formed, before the next
+    collective); rank 0's next collective must end with an error, not wait."""
+    import sys
+    import time
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    from datetime import timedelta
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=10))
+    import bench
+    bench.barrier(world)                      # both ranks reach the first step
+    if rank == 1:
+        os._exit(0)                            # leaves with nothing in flight
+    t0 = time.time()
+    try:
+        bench.max_over_ranks(1.0, world)
+        out.put(("no error", time.time() - t0))
+    except Exception as e:                     # gloo reports the lost peer
+        out.put((type(e).__name__, time.time() - t0))
+    os._exit(0)
+
+
+def test_a_rank_that_leaves_ends_the_next_collective_with_an_error():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_one_dies, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    kind, secs = q.get(timeout=120)
+    for p in procs:
+        p.join(timeout=60)
+    assert kind != "no error"
+    assert secs < 30.0                         # bounded by the group's 10 s timeout, not a hang
