@@ -65,5 +65,30 @@ def build(force: bool = False, verbose: bool = False) -> str:
     return LIB
 
 
+def resource_summary(log: str = os.path.join(PKG, "build.log")) -> str:
+    """Markdown table of ptxas's per-kernel resource lines in the build log:
+    registers a thread, spill stores / loads (bytes), static shared memory."""
+    import re
+    import shutil
+    text = open(log).read()
+    rows = []
+    for m in re.finditer(r"Compiling entry function '([^']+)'.*?(\d+) bytes stack frame, (\d+) bytes spill stores, "
+                         r"(\d+) bytes spill loads\s*\n[^\n]*Used (\d+) registers[^\n]*?(?:(\d+) bytes smem)?\n",
+                         text, flags=re.S):
+        rows.append(list(m.groups()))
+    names = [r[0] for r in rows]
+    if shutil.which("c++filt"):
+        out = subprocess.run(["c++filt"], input="\n".join(names), capture_output=True, text=True).stdout.split("\n")
+        names = [re.sub(r"\(anonymous namespace\)::", "", n) for n in out[:len(names)]]
+    lines = ["| kernel | registers | stack B | spill stores B | spill loads B | static smem B |",
+             "|---|---:|---:|---:|---:|---:|"]
+    for n, r in sorted(zip(names, rows)):
+        lines.append(f"| `{n}` | {r[4]} | {r[1]} | {r[2]} | {r[3]} | {r[5] or 0} |")
+    return "\n".join(lines) + "\n"
+
+
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    if "--resources" in sys.argv:
+        sys.stdout.write(resource_summary())
+    else:
+        print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))

@@ -361,14 +361,46 @@ __global__ void selftest_exp2_kernel(const float *x, float *y, float *y_ref, int
 // the whole device and forbids allocations outside it. forge_attn_bwd_noalloc
 // serves them with scratch that lives in this fixed-size device array instead
 // of a caller workspace. Every GPU that loads the library holds the array until
-// the process exits. Its device address is looked up once per device (on the
-// first call made with that device current) and cached.
+// the process exits. Its device address belongs to the device's current
+// context: it is looked up on the first call made with that device current and
+// cached together with the context's unique id, and looked up again when the
+// id has changed (a cudaDeviceReset ends the old context, and the module and
+// its array get a new address in the next one).
 namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mutex;
-void *g_noalloc_ptr[kNoAllocMaxDevices] = {};
+struct NoAllocEntry {
+    unsigned long long ctx_id;  // id of the context the address belongs to
+    void *ptr;
+};
+NoAllocEntry g_noalloc[kNoAllocMaxDevices] = {};
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+template <typename F>
+F driver_fn(const char *name) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &ptr, cudaEnableDefault, &q) == cudaSuccess && q == cudaDriverEntryPointSuccess)
+        return reinterpret_cast<F>(ptr);
+    return nullptr;
+}
+
+// Unique id of the calling thread's current context (never reused within the
+// process), or 0 when there is none or the driver cannot say.
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    if (get_current == nullptr || get_id == nullptr) return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+    if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
 
 forge_status noalloc_scratch_for_current_device(void **out) {
     int dev = -1;
@@ -376,13 +408,18 @@ forge_status noalloc_scratch_for_current_device(void **out) {
     if (s != FORGE_OK) return s;
     if (dev < 0 || dev >= kNoAllocMaxDevices) return FORGE_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (g_noalloc_ptr[dev] == nullptr) {
+    NoAllocEntry &e = g_noalloc[dev];
+    const unsigned long long id = current_context_id();
+    if (e.ptr == nullptr || id == 0 || id != e.ctx_id) {
+        // first call on this device, a context without a readable id (looked up
+        // every time then), or a new context since the last lookup
         void *p = nullptr;
         s = forge::cuda_status(cudaGetSymbolAddress(&p, g_noalloc_scratch));
         if (s != FORGE_OK) return s;
-        g_noalloc_ptr[dev] = p;
+        e.ptr = p;
+        e.ctx_id = current_context_id();  // the lookup may have created the context
     }
-    *out = g_noalloc_ptr[dev];
+    *out = e.ptr;
     return FORGE_OK;
 }
 }  // namespace

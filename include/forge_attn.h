@@ -149,8 +149,10 @@ forge_status forge_attn_bwd_ext(const void *q, const void *k, const void *v, con
  *    most 32 MiB (33554432 bytes); larger problems return FORGE_ERR_WORKSPACE
  *    (forge_attn_last_cuda_error says why) and launch nothing.
  *  - The array's device address is looked up the first time the entry point is
- *    called with a given device current; make that first call on each device
- *    before any stream capture.
+ *    called with a given device current, and again on the first call after the
+ *    device's context has changed (after a cudaDeviceReset, say), since the
+ *    array moves with the context; make the first call on each device, and the
+ *    first call after a reset, before any stream capture.
  *  - All calls share the one array per device. It keeps the previous call's
  *    contents; the call clears what must start at zero itself. Calls whose work
  *    overlaps on the GPU (other streams, other host threads) race on the array:

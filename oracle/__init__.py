@@ -48,6 +48,8 @@ def _load():
         lib.oracle_attn_probs.argtypes = [dp, dp, dp, i, i, i, i, i, d, i, d]
         lib.oracle_rowdot.argtypes = [dp, dp, dp, ctypes.c_long, i]
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_set_num_threads.argtypes = [i]
+        lib.oracle_set_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -78,6 +80,12 @@ def _dims_kv(q, k, v):
 
 def num_threads() -> int:
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> int:
+    """Threads the oracle's parallel loops use from now on; returns the count in
+    force. Timing only: the results do not depend on it."""
+    return int(_load().oracle_set_num_threads(int(n)))
 
 
 def attn_fwd(q, k, v, scale: float, window: int = 0, softcap: float = 0.0):

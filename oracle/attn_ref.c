@@ -373,3 +373,13 @@ int oracle_num_threads(void) {
     return 1;
 #endif
 }
+
+/* Threads the parallel loops use from now on (n >= 1), for timing the oracle on
+ * one core; returns the count in force afterwards. No effect on the results. */
+int oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    if (n >= 1) omp_set_num_threads(n);
+#endif
+    return oracle_num_threads();
+}
