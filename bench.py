@@ -77,12 +77,25 @@ def _strip_comments(text):
     return "".join(out)
 
 
-def kernel_source_hash():
-    """sha256 prefix of causal_flash_attention_attn_b200/csrc/* without comments,
-    whitespace runs collapsed (layout and comment edits leave it unchanged)."""
+# The sources each captured kernel is built from: its own header(s) and the
+# shared instruction wrappers. A traffic figure stands only while these are
+# unchanged (the launch configuration lives beside the kernel, in its traits).
+KERNEL_SOURCES = {
+    "bwd_tc_kernel": ("bwd_tc.cuh", "sm100.cuh"),
+    "fwd2_tc_kernel": ("fwd2_tc.cuh", "fwd_tc.cuh", "sm100.cuh"),
+    "fwd_tc_kernel": ("fwd_tc.cuh", "sm100.cuh"),
+    "decode_split": ("decode.cuh", "sm100.cuh"),
+}
+
+
+def kernel_source_hash(kernel=None):
+    """sha256 prefix of the kernel's sources (all of csrc/ when kernel is None or
+    unknown) without comments, whitespace runs collapsed (layout and comment edits
+    leave it unchanged)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "causal_flash_attention_attn_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    names = KERNEL_SOURCES.get(kernel) or sorted(os.listdir(csrc))
+    for name in sorted(names):
         with open(os.path.join(csrc, name), "r", encoding="utf-8") as f:
             h.update(name.encode())
             h.update(" ".join(_strip_comments(f.read()).split()).encode())
@@ -99,7 +112,7 @@ def ncu_traffic(kernel, workload):
     except Exception:
         return None
     e = d.get(f"{kernel}@{workload}")
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -320,6 +333,20 @@ def barrier(world: int, device=None):
 
 
 # ------------------------------------------------------------ CPU baseline
+def _oracle_groups(w, groups, q, k, v, dO):
+    """Seconds of the f64 oracle (fwd + bwd) over the listed (b, kv-head) groups."""
+    import oracle
+    G = w.G
+    t0 = time.perf_counter()
+    for b, h in groups:
+        hs = slice(h * G, (h + 1) * G)
+        ks, vs = k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1]
+        qs, ds = q[b:b + 1, hs], dO[b:b + 1, hs]
+        oracle.attn_fwd(qs, ks, vs, w.sm_scale, w.window, w.softcap)
+        oracle.attn_bwd(qs, ks, vs, ds, w.sm_scale, w.window, w.softcap)
+    return time.perf_counter() - t0
+
+
 def cpu_oracle_sample(w, budget_s=12.0, max_groups=None):
     """Time the f64 oracle (fwd + bwd) on whole KV groups of the workload, adding
     groups until ~budget_s of CPU work. Returns (tflops, seconds, description, cores)."""
@@ -327,33 +354,212 @@ def cpu_oracle_sample(w, budget_s=12.0, max_groups=None):
     from causal_flash_attention_attn_b200 import inputs
     from causal_flash_attention_attn_b200.inputs import allowed_pairs
     q, k, v, dO = inputs.make_inputs(w)
-    G = w.G
     groups = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
     if max_groups:
         groups = groups[:max_groups]
     done, secs, flops = 0, 0.0, 0.0
-    for b, h in groups:
-        hs = slice(h * G, (h + 1) * G)
-        ks, vs = k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1]
-        qs, ds = q[b:b + 1, hs], dO[b:b + 1, hs]
-        t0 = time.perf_counter()
-        oracle.attn_fwd(qs, ks, vs, w.sm_scale, w.window, w.softcap)
-        oracle.attn_bwd(qs, ks, vs, ds, w.sm_scale, w.window, w.softcap)
-        secs += time.perf_counter() - t0
-        flops += 14.0 * w.D * allowed_pairs(w.T, w.window) * G
+    for g in groups:
+        secs += _oracle_groups(w, [g], q, k, v, dO)
+        flops += 14.0 * w.D * allowed_pairs(w.T, w.window) * w.G
         done += 1
         if secs >= budget_s:
             break
     desc = (f"f64 oracle fwd+bwd on {done} of {w.B * w.Hkv} KV groups (b, kv-head) of {w.name}, "
-            f"each {G} query heads x T={w.T}")
+            f"each {w.G} query heads x T={w.T}")
     return flops / secs / 1e12, secs, desc, oracle.num_threads()
 
 
+def cpu_oracle_full(names=("f32_correctness", "forge_default")):
+    """The small workloads timed in full with the oracle's default threads, and the
+    f32 correctness workload on one thread as well. Pairs per second count the
+    allowed (query, key) pairs of the whole workload, forward and backward."""
+    import oracle
+    from causal_flash_attention_attn_b200 import inputs
+    from causal_flash_attention_attn_b200.inputs import allowed_pairs
+    out = {}
+    for name in names:
+        w = inputs.WORKLOADS[name]
+        q, k, v, dO = inputs.make_inputs(w)
+        groups = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+        pairs = allowed_pairs(w.T, w.window) * w.B * w.Hq
+        secs = _oracle_groups(w, groups, q, k, v, dO)
+        out[name] = {"seconds": round(secs, 4), "pairs_per_s": round(pairs / secs, 1),
+                     "tflops": round(14.0 * w.D * pairs / secs / 1e12, 6), "threads": oracle.num_threads()}
+    w = inputs.WORKLOADS["f32_correctness"]
+    q, k, v, dO = inputs.make_inputs(w)
+    before = oracle.num_threads()
+    oracle.set_num_threads(1)
+    try:
+        secs = _oracle_groups(w, [(b, h) for b in range(w.B) for h in range(w.Hkv)], q, k, v, dO)
+    finally:
+        oracle.set_num_threads(before)
+    pairs = allowed_pairs(w.T, w.window) * w.B * w.Hq
+    out["f32_correctness_single_thread"] = {"seconds": round(secs, 4), "pairs_per_s": round(pairs / secs, 1),
+                                            "tflops": round(14.0 * w.D * pairs / secs / 1e12, 6), "threads": 1}
+    return out
+
+
 # -------------------------------------------------------------------- ours
+def spread(xs):
+    """Median and spread of a list of per-step times (ms)."""
+    ys = sorted(xs)
+    n = len(ys)
+
+    def pct(p):
+        return ys[min(n - 1, max(0, int(round(p * (n - 1)))))]
+    return {"median": round(statistics.median(ys), 4), "min": round(ys[0], 4), "p10": round(pct(0.1), 4),
+            "p90": round(pct(0.9), 4), "max": round(ys[-1], 4), "n": n}
+
+
+class Runner:
+    """Device buffers and the timed step (forward, then the backward's three
+    stages) of one workload on one GPU, through the library's C ABI."""
+
+    def __init__(self, w, dev, stream, host_inputs=None):
+        import torch
+        import causal_flash_attention_attn_b200 as fa
+        from causal_flash_attention_attn_b200 import inputs
+        self.fa, self.w, self.dev, self.stream = fa, w, dev, stream
+        self.host = host_inputs if host_inputs is not None else inputs.make_inputs(w)
+        q, k, v, dO = self.host
+        B, Hq, Hkv, T, D = w.B, w.Hq, w.Hkv, w.T, w.D
+        self.dt = fa.dtype_code(inputs.torch_dtype(w.dtype))
+        self.qd, self.kd, self.vd, self.dOd = (x.to(dev) for x in (q, k, v, dO))
+        self.o = torch.empty_like(self.qd)
+        self.lse = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
+        self.dq, self.dk, self.dv = torch.empty_like(self.qd), torch.empty_like(self.kd), torch.empty_like(self.vd)
+        self.nws = fa.forge_attn_bwd_workspace_size(B, Hq, Hkv, T, D, self.dt)
+        self.ws = torch.empty(self.nws, dtype=torch.uint8, device=dev)
+        # Timing hygiene: when the per-step working set is not well above the L2
+        # size, every step first overwrites a 256 MB scratch buffer (outside the
+        # timed kernels) so that no step starts with the previous one's data in L2.
+        self.working_set = sum(x.numel() * x.element_size() for x in
+                               (self.qd, self.kd, self.vd, self.o, self.lse, self.dOd, self.dq, self.dk, self.dv,
+                                self.ws))
+        self.flush = self.working_set < 2 * L2_BYTES
+        self.scratch = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if self.flush else None
+
+    def step(self, ev=None):
+        import torch
+        fa, w, sh = self.fa, self.w, self.stream.cuda_stream
+        B, Hq, Hkv, T, D = w.B, w.Hq, w.Hkv, w.T, w.D
+        sc, W, C, dt, ws, nws = w.sm_scale, w.window, w.softcap, self.dt, self.ws, self.nws
+        if self.flush:
+            with torch.cuda.stream(self.stream):
+                self.scratch.fill_(1)
+        if ev:
+            ev[0].record(self.stream)
+        s = fa.forge_attn_fwd(self.qd, self.kd, self.vd, self.o, self.lse, B, Hq, Hkv, T, D, sc, W, C, dt, sh)
+        if ev:
+            ev[1].record(self.stream)
+        s |= fa.forge_attn_bwd_preprocess(self.o, self.dOd, B, Hq, Hkv, T, D, dt, ws, nws, sh)
+        if ev:
+            ev[2].record(self.stream)
+        s |= fa.forge_attn_bwd_main(self.qd, self.kd, self.vd, self.lse, self.dOd, self.dq, self.dk, self.dv, B, Hq,
+                                    Hkv, T, D, sc, W, C, dt, ws, nws, sh)
+        if ev:
+            ev[3].record(self.stream)
+        s |= fa.forge_attn_bwd_finalize(self.dq, B, Hq, Hkv, T, D, dt, ws, nws, sh)
+        if ev:
+            ev[4].record(self.stream)
+        if s != fa.FORGE_OK:
+            raise fa.ForgeError(s, "step")
+
+    def warm(self, n):
+        import torch
+        with torch.cuda.stream(self.stream):
+            for _ in range(n):
+                self.step()
+        torch.cuda.synchronize(self.dev)
+        st = self.fa.forge_attn_check(self.stream.cuda_stream)
+        if st != self.fa.FORGE_OK:
+            raise self.fa.ForgeError(st, "warmup")
+
+    @staticmethod
+    def per_kernel(evs):
+        per = {"fwd": [], "bwd_preprocess": [], "bwd_main": [], "bwd_finalize": [], "step": []}
+        for e in evs:
+            per["fwd"].append(e[0].elapsed_time(e[1]))
+            per["bwd_preprocess"].append(e[1].elapsed_time(e[2]))
+            per["bwd_main"].append(e[2].elapsed_time(e[3]))
+            per["bwd_finalize"].append(e[3].elapsed_time(e[4]))
+            per["step"].append(e[0].elapsed_time(e[4]))
+        return per
+
+    def timed(self, steps):
+        """Per-step CUDA-event times (ms) of each stage, steps back to back."""
+        import torch
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+        for i in range(steps):
+            self.step(evs[i])
+        torch.cuda.synchronize(self.dev)
+        st = self.fa.forge_attn_check(self.stream.cuda_stream)
+        if st != self.fa.FORGE_OK:
+            raise self.fa.ForgeError(st, "timed run")
+        return self.per_kernel(evs)
+
+
+def peak_for(kind, timed_s):
+    peaks, src = load_peaks()
+    key = kind + ("_sustained" if kind == "bf16_tflops" and timed_s > 2.0 else "")
+    return float(peaks.get(key, FALLBACK_PEAKS[key])), f"{src} {key}"
+
+
+def per_workload_block(args, dev, stream):
+    """Every bf16 layer type of the workloads timed on its own (W untimed, then
+    max(K, 30) timed steps; medians), plus the means the configurations pair the
+    layer types into: the 16K model's 6-layer period (five W = 1024 layers, one
+    global) and the Gemma-2-style 8K pair (one W = 4096 layer, one global)."""
+    import torch
+    from causal_flash_attention_attn_b200 import inputs
+    out, cache = {}, {}
+    steps = max(args.steps, 30)
+    for name, w in inputs.WORKLOADS.items():
+        if w.dtype != "bf16":
+            continue
+        key = (w.B, w.Hq, w.Hkv, w.T, w.D, w.seed, w.sigma_q, w.sigma_k, w.sigma_v, w.sigma_do)
+        if key not in cache:
+            cache.clear()
+            cache[key] = inputs.make_inputs(w)
+        r = Runner(w, dev, stream, host_inputs=cache[key])
+        r.warm(args.warmup)
+        with torch.cuda.stream(stream):
+            per = r.timed(steps)
+        fl_f, fl_b = flops_of(w)
+        med = {k_: statistics.median(v_) for k_, v_ in per.items()}
+        peak, _ = peak_for("bf16_tflops", sum(per["step"]) * 1e-3)
+        tf = (fl_f + fl_b) / (med["step"] * 1e-3) / 1e12
+        out[name] = {"ms_step": round(med["step"], 4), "ms_fwd": round(med["fwd"], 4),
+                     "ms_bwd_main": round(med["bwd_main"], 4),
+                     "ms_bwd_pre_fin": round(med["bwd_preprocess"] + med["bwd_finalize"], 4),
+                     "tflops": round(tf, 2), "frac": round(tf / peak, 4),
+                     "fwd_frac": round(fl_f / (med["fwd"] * 1e-3) / 1e12 / peak, 4),
+                     "bwd_main_frac": round(fl_b / (med["bwd_main"] * 1e-3) / 1e12 / peak, 4),
+                     "gflop": round((fl_f + fl_b) / 1e9, 2), "l2_flushed": r.flush, "steps": steps}
+        del r
+        torch.cuda.empty_cache()
+    peak, src = peak_for("bf16_tflops", 0.0)
+
+    def mean(parts):
+        ms = sum(n * out[k_]["ms_step"] for k_, n in parts)
+        gf = sum(n * out[k_]["gflop"] for k_, n in parts)
+        tf = gf / ms  # GFLOP / ms = TFLOP/s
+        return {"layers": {k_: n for k_, n in parts}, "ms": round(ms, 4), "tflops": round(tf, 2),
+                "frac": round(tf / peak, 4)}
+    means = {}
+    if "swa_w1024_16k" in out and "global_16k" in out:
+        means["sliding_16k_period6 (5 x W1024 + 1 global)"] = mean([("swa_w1024_16k", 5), ("global_16k", 1)])
+    if "softcap_w4096_8k" in out and "softcap_global_8k" in out:
+        means["softcap_8k_alternating (1 x W4096 + 1 global)"] = mean([("softcap_w4096_8k", 1),
+                                                                      ("softcap_global_8k", 1)])
+    return {"layer_types": out, "means": means, "peak": peak, "peak_source": src,
+            "timing": "per layer type: CUDA events around each stage, median of the timed steps; "
+                      "step = fwd + bwd preprocess + bwd main + bwd finalize"}
+
+
 def run_ours(args, w):
     import torch
     import causal_flash_attention_attn_b200 as fa
-    from causal_flash_attention_attn_b200 import inputs
 
     world, rank, local = dist_env()
     if world > 1:
@@ -368,53 +574,9 @@ def run_ours(args, w):
 
     # inputs: each rank its own batch of the workload (seed offset by rank)
     wr = w.with_(seed=w.seed + 1000 * rank) if rank else w
-    q, k, v, dO = inputs.make_inputs(wr)
-    B, Hq, Hkv, T, D = w.B, w.Hq, w.Hkv, w.T, w.D
-    dt = fa.dtype_code(inputs.torch_dtype(w.dtype))
-    qd, kd, vd, dOd = (x.to(dev) for x in (q, k, v, dO))
-    o = torch.empty_like(qd)
-    lse = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
-    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
-    nws = fa.forge_attn_bwd_workspace_size(B, Hq, Hkv, T, D, dt)
-    ws = torch.empty(nws, dtype=torch.uint8, device=dev)
-    sc, W, C = w.sm_scale, w.window, w.softcap
-    sh = stream.cuda_stream
-    # Timing hygiene: when the per-step working set is not well above the L2
-    # size, every step first overwrites a 256 MB scratch buffer (outside the
-    # timed kernels) so that no step starts with the previous one's data in L2.
-    working_set = sum(x.numel() * x.element_size() for x in (qd, kd, vd, o, lse, dOd, dq, dk, dv, ws))
-    flush = working_set < 2 * L2_BYTES
-    scratch = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush else None
-
-    def step(ev=None):
-        if flush:
-            with torch.cuda.stream(stream):
-                scratch.fill_(1)
-        if ev:
-            ev[0].record(stream)
-        s = fa.forge_attn_fwd(qd, kd, vd, o, lse, B, Hq, Hkv, T, D, sc, W, C, dt, sh)
-        if ev:
-            ev[1].record(stream)
-        s |= fa.forge_attn_bwd_preprocess(o, dOd, B, Hq, Hkv, T, D, dt, ws, nws, sh)
-        if ev:
-            ev[2].record(stream)
-        s |= fa.forge_attn_bwd_main(qd, kd, vd, lse, dOd, dq, dk, dv, B, Hq, Hkv, T, D, sc, W, C, dt, ws, nws, sh)
-        if ev:
-            ev[3].record(stream)
-        s |= fa.forge_attn_bwd_finalize(dq, B, Hq, Hkv, T, D, dt, ws, nws, sh)
-        if ev:
-            ev[4].record(stream)
-        if s != fa.FORGE_OK:
-            raise fa.ForgeError(s, "step")
-
+    r = Runner(wr, dev, stream)
     launches_per_step = 4
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            step()
-    torch.cuda.synchronize(dev)
-    st = fa.forge_attn_check(sh)
-    if st != fa.FORGE_OK:
-        raise fa.ForgeError(st, "warmup")
+    r.warm(args.warmup)
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     clk = ClockSampler(dev.index)
@@ -425,43 +587,40 @@ def run_ours(args, w):
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     clk.begin()
-    start.record(stream)
-    for i in range(args.steps):
-        step(evs[i])
-    end.record(stream)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for i in range(args.steps):
+            r.step(evs[i])
+        end.record(stream)
     torch.cuda.synchronize(dev)
     clk.end()
     clocks = clk.stop()
     barrier(world, dev)
-    st = fa.forge_attn_check(sh)
+    st = fa.forge_attn_check(stream.cuda_stream)
     if st != fa.FORGE_OK:
         raise fa.ForgeError(st, "timed run")
     ms_local = start.elapsed_time(end)
-    if flush:
+    if r.flush:
         # the flushes sit between the timed kernels: time the kernels only
         ms_local = sum(e[0].elapsed_time(e[4]) for e in evs)
     ms = max_over_ranks(ms_local, world, dev)
-    per = {"fwd": [], "bwd_preprocess": [], "bwd_main": [], "bwd_finalize": []}
-    for e in evs:
-        per["fwd"].append(e[0].elapsed_time(e[1]))
-        per["bwd_preprocess"].append(e[1].elapsed_time(e[2]))
-        per["bwd_main"].append(e[2].elapsed_time(e[3]))
-        per["bwd_finalize"].append(e[3].elapsed_time(e[4]))
-    avg = {kname: sum(v) / len(v) for kname, v in per.items()}
+    per = Runner.per_kernel(evs)
+    avg = {kname: sum(v) / len(v) for kname, v in per.items() if kname != "step"}
 
     # end to end through the same C ABI from pinned host buffers
     e2e = None
     if not args.no_e2e:
+        q, k, v, dO = r.host
         hq_, hk_, hv_, hdo = (x.pin_memory() for x in (q, k, v, dO))
-        hdq, hdk, hdv = (torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in (qd, kd, vd))
+        hdq, hdk, hdv = (torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in (r.qd, r.kd, r.vd))
         h2d = sum(x.numel() * x.element_size() for x in (hq_, hk_, hv_, hdo))
         d2h = sum(x.numel() * x.element_size() for x in (hdq, hdk, hdv))
 
         def e2e_step():
-            for dst, src in ((qd, hq_), (kd, hk_), (vd, hv_), (dOd, hdo)):
+            for dst, src in ((r.qd, hq_), (r.kd, hk_), (r.vd, hv_), (r.dOd, hdo)):
                 dst.copy_(src, non_blocking=True)
-            step()
-            for dst, src in ((hdq, dq), (hdk, dk), (hdv, dv)):
+            r.step()
+            for dst, src in ((hdq, r.dq), (hdk, r.dk), (hdv, r.dv)):
                 dst.copy_(src, non_blocking=True)
 
         with torch.cuda.stream(stream):
@@ -491,10 +650,7 @@ def run_ours(args, w):
     fl_f, fl_b = flops_of(w)
     ms_step = ms / args.steps
     tflops = aggregate_tflops(world, fl_f + fl_b, ms_step)
-    peaks, peak_src = load_peaks()
-    timed_s = ms * 1e-3
-    peak_key = "bf16_tflops_sustained" if timed_s > 2.0 else "bf16_tflops"
-    peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
+    peak, peak_src = peak_for("bf16_tflops", ms * 1e-3)
     # dominant kernel: the larger of forward and backward-main by time
     dom = "bwd_main" if avg["bwd_main"] >= avg["fwd"] else "fwd"
     dom_flops = fl_b if dom == "bwd_main" else fl_f
@@ -520,25 +676,35 @@ def run_ours(args, w):
                    "flops_per_step_per_gpu": fl_f + fl_b,
                    "flop_count": "only causal/in-window pairs; fwd 4*D*pairs, bwd 10*D*pairs",
                    "l2": ("flushed: a 256 MB buffer is written before each step (working set "
-                          f"{working_set / 1e6:.0f} MB); step time = sum of the kernels' CUDA-event times") if flush
-                         else (f"not flushed: per-step working set (q,k,v,o,dO,dq,dk,dv,lse + workspace) "
-                               f"{working_set / 1e6:.0f} MB exceeds twice the 126 MB L2")},
+                          f"{r.working_set / 1e6:.0f} MB); step time = sum of the kernels' CUDA-event times")
+                   if r.flush else
+                   (f"not flushed: per-step working set (q,k,v,o,dO,dq,dk,dv,lse + workspace) "
+                    f"{r.working_set / 1e6:.0f} MB exceeds twice the 126 MB L2")},
         "pct_of_bf16_peak": round(100.0 * tflops / world / peak, 2),
         "kernels_ms": {k_: round(v_, 4) for k_, v_ in avg.items()},
+        "step_ms": spread(per["step"]),
+        "kernels_ms_spread": {k_: spread(v_) for k_, v_ in per.items() if k_ != "step"},
         "roofline": {"kernel": kname, "bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "peak_source": f"{peak_src} {peak_key}",
+                     "peak_source": peak_src,
                      "achieved_def": f"{'10' if dom == 'bwd_main' else '4'}*D*pairs per launch / "
-                                     "CUDA-event launch time"},
+                                     "CUDA-event launch time (mean over the timed steps)"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
     if e2e:
         line["e2e"] = e2e
+    del r
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_per_workload:
+        line["per_workload"] = per_workload_block(args, dev, stream)
     if world == 1 and not args.no_cpu:
         v_, secs, desc, cores = cpu_oracle_sample(w, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": round(v_, 6), "unit": "TFLOPS", "cores": cores, "kind": "oracle",
-                                "sample": desc, "seconds": round(secs, 2)}
+                                "sample": desc, "seconds": round(secs, 2),
+                                "os_cpu_count": os.cpu_count(),
+                                "OMP_NUM_THREADS": os.environ.get("OMP_NUM_THREADS"),
+                                "full": cpu_oracle_full()}
     return line
 
 
@@ -740,16 +906,18 @@ def run_dkv(args):
             "gpu_launches": 4 * args.steps, "clocks": clocks}
 
 
-# the same shapes in bf16 on the tensor cores (forward only: the bf16 backward at
-# d_k != d_v is not built); B = 4 so the working set (330 MB) exceeds the L2
+# the same shapes in bf16 on the tensor cores; B = 4 so the working set (about
+# 0.45 GB) exceeds the L2
 DKV_BF16 = {"workload": "mla_bf16_b4_h16_t4096_dk192_dv128", "B": 4, "Hq": 16, "Hkv": 16, "T": 4096, "Dk": 192,
             "Dv": 128, "dtype": "bf16", "window": 0, "softcap": 0.0}
 
 
 def run_dkv_bf16(args):
-    """--dkv --dkv-dtype bf16: the d_k != d_v forward on the tensor cores
-    (fwd_tc_kernel<192, 128>), FLOPs 2 (Dk + Dv) per allowed pair, against the
-    measured bf16 burst peak."""
+    """--dkv --dkv-dtype bf16: forward (fwd_tc_kernel<192, 128>) and backward
+    (preprocess, bwd_dkdv_tc_kernel, bwd_dq_tc_kernel) on the tensor cores.
+    FLOPs per allowed pair: 2 (Dk + Dv) forward, 2 (3 Dk + 2 Dv) backward (the
+    algorithmic count; the two backward kernels recompute S and dP, which is not
+    counted). Against the measured bf16 burst peak."""
     import torch
     import causal_flash_attention_attn_b200 as fa
 
@@ -763,67 +931,84 @@ def run_dkv_bf16(args):
     q = torch.randn(B, Hq, T, Dk, generator=g).to(torch.bfloat16).to(dev)
     k = torch.randn(B, Hkv, T, Dk, generator=g).to(torch.bfloat16).to(dev)
     v = torch.randn(B, Hkv, T, Dv, generator=g).to(torch.bfloat16).to(dev)
+    dO = torch.randn(B, Hq, T, Dv, generator=g).to(torch.bfloat16).to(dev)
     o = torch.empty(B, Hq, T, Dv, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(B, Hq, T, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    nws = fa.forge_attn_bwd_workspace_size_dkv(B, Hq, Hkv, T, Dk, Dv, fa.FORGE_DTYPE_BF16)
+    ws = torch.empty(nws, dtype=torch.uint8, device=dev)
     sc = 1.0 / math.sqrt(Dk)
     sh = stream.cuda_stream
 
-    def step():
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
         s = fa.forge_attn_fwd_dkv(q, k, v, o, lse, B, Hq, Hkv, T, Dk, Dv, sc, 0, 0.0, fa.FORGE_DTYPE_BF16, sh)
+        if ev:
+            ev[1].record(stream)
+        s |= fa.forge_attn_bwd_dkv(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, T, Dk, Dv, sc, 0, 0.0,
+                                   fa.FORGE_DTYPE_BF16, ws, nws, sh)
+        if ev:
+            ev[2].record(stream)
         if s != fa.FORGE_OK:
             raise fa.ForgeError(s, "dkv bf16")
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     clk = ClockSampler(dev.index)
     clk.start()
     time.sleep(0.3)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clk.begin()
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
     torch.cuda.synchronize(dev)
     clk.end()
     clocks = clk.stop()
     st = fa.forge_attn_check(sh)
     if st != fa.FORGE_OK:
         raise fa.ForgeError(st, "dkv bf16 timed run")
-    ms = e0.elapsed_time(e1) / args.steps
+    fwd = [e[0].elapsed_time(e[1]) for e in evs]
+    bwd = [e[1].elapsed_time(e[2]) for e in evs]
+    ms = statistics.median(e[0].elapsed_time(e[2]) for e in evs)
     pairs = B * Hq * T * (T + 1) // 2
-    flops = pairs * 2 * (Dk + Dv)
-    tf = flops / (ms * 1e-3) / 1e12
-    peaks, peak_src = load_peaks()
-    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    return {"metric": "d_k != d_v attention forward TFLOPS (bf16 tensor cores)", "value": round(tf, 3),
+    fl_f, fl_b = pairs * 2 * (Dk + Dv), pairs * 2 * (3 * Dk + 2 * Dv)
+    tf = (fl_f + fl_b) / (ms * 1e-3) / 1e12
+    peak, peak_src = peak_for("bf16_tflops", 0.0)
+    bwd_tf = fl_b / (statistics.median(bwd) * 1e-3) / 1e12
+    return {"metric": "d_k != d_v attention fwd+bwd TFLOPS (bf16 tensor cores)", "value": round(tf, 3),
             "unit": "TFLOPS", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "step_ms": spread([e[0].elapsed_time(e[2]) for e in evs]),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded N(0,1) q, k, v)",
-            "config": dict(c, l2="not flushed: the per-step working set (about 0.33 GB) exceeds the 126 MB L2",
-                           flop_count="allowed pairs x 2 (Dk + Dv)"),
-            "roofline": {"kernel": "fwd_tc_kernel<192,128>", "bound": "tensor", "achieved": round(tf, 3),
-                         "peak": peak, "unit": "TFLOP/s", "frac": round(tf / peak, 4), "traffic": None,
-                         "peak_source": f"{peak_src} bf16_tflops",
-                         "achieved_def": "forward flops / CUDA-event time of its one launch"},
-            "gpu_launches": args.steps, "clocks": clocks}
+            "data": "synthetic (seeded N(0,1) q, k, v, dO)",
+            "config": dict(c, l2="not flushed: the per-step working set (about 0.45 GB) exceeds the 126 MB L2",
+                           flop_count="allowed pairs x (2 (Dk + Dv) forward + 2 (3 Dk + 2 Dv) backward)"),
+            "kernels_ms": {"fwd": round(statistics.median(fwd), 4), "bwd": round(statistics.median(bwd), 4)},
+            "pct_of_bf16_peak": round(100 * tf / peak, 2),
+            "roofline": {"kernel": "bwd (preprocess + bwd_dkdv_tc_kernel + bwd_dq_tc_kernel)", "bound": "tensor",
+                         "achieved": round(bwd_tf, 3), "peak": peak, "unit": "TFLOP/s", "frac": round(bwd_tf / peak, 4),
+                         "traffic": None, "peak_source": peak_src,
+                         "achieved_def": "2 (3 Dk + 2 Dv) flops per allowed pair / CUDA-event time of the backward call"},
+            "gpu_launches": 4 * args.steps, "clocks": clocks}
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=None)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the per-layer-type block (every bf16 workload timed on its own)")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--decode", action="store_true", help="time the KV-cache decode kernels instead")
     ap.add_argument("--dkv", action="store_true", help="time the d_k != d_v path instead")
     ap.add_argument("--dkv-dtype", choices=["f32", "bf16"], default="f32",
-                    help="f32: forward + backward on the CUDA cores; bf16: the tensor-core forward")
+                    help="f32: forward + backward on the CUDA cores; bf16: forward + backward on the tensor cores")
     args = ap.parse_args(argv)
     from causal_flash_attention_attn_b200 import inputs
     w = inputs.WORKLOADS[args.workload or inputs.HEADLINE]

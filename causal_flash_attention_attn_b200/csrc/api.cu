@@ -13,6 +13,7 @@
 #include "forge_attn.h"
 
 #include "bwd_aux.cuh"
+#include "bwd_dkv.cuh"
 #include "bwd_tc.cuh"
 #include "decode.cuh"
 #include "fwd2_tc.cuh"
@@ -116,6 +117,19 @@ forge_status cuda_status(cudaError_t e) {
 
 forge_status launch_status() { return cuda_status(cudaGetLastError()); }
 
+// SM count of the current device (cached per device), for persistent grids.
+int sm_count() {
+    static int cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
 template <typename K>
 forge_status set_smem(K kernel, size_t bytes) {
     if (bytes <= 48 * 1024) return FORGE_OK;
@@ -159,7 +173,9 @@ forge_status fwd_tc(const void *q, const void *k, const void *v, void *o, float 
             return FORGE_ERR_CUDA;
         }
         if (set_smem(fwd2_tc_kernel<D>, C2::SMEM) != FORGE_OK) return FORGE_ERR_CUDA;
-        const unsigned grid = (unsigned)(((p.num_qt + 1) / 2) * B * Hq);
+        // persistent: one CTA per SM (shared memory and TMEM allow no more)
+        const long long items = (long long)((p.num_qt + 1) / 2) * B * Hq;
+        const unsigned grid = (unsigned)(items < sm_count() ? items : sm_count());
         fwd2_tc_kernel<D><<<grid, C2::THREADS, C2::SMEM, st>>>(mq, mk, mv, mo, p);
     }
     return launch_status();
@@ -251,8 +267,57 @@ forge_status bwd_tc(const void *q, const void *k, const void *v, const float *ls
     p.cap_in = softcap > 0.0f ? scale / softcap : 0.0f;
     p.cap_out = softcap * kLog2e;
     if (set_smem(bwd_tc_kernel<D>, C::SMEM) != FORGE_OK) return FORGE_ERR_CUDA;
-    const unsigned grid = (unsigned)(p.num_kt * B * Hkv * C::NSPLIT);
+    // persistent: one CTA per SM (the kernel's shared memory and TMEM allow no
+    // more), each walking its share of the work items
+    const long long items = (long long)p.num_kt * B * Hkv * C::NSPLIT;
+    const unsigned grid = (unsigned)(items < sm_count() ? items : sm_count());
     bwd_tc_kernel<D><<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, mdo, macc, p);
+    return launch_status();
+}
+
+// bf16 backward with separate key and value head dims: the dK/dV kernel (one CTA
+// per key tile and KV head), then the dQ kernel (one CTA per query tile and
+// query head). Both read Delta from the workspace and write their outputs.
+template <int DK, int DV>
+forge_status bwd_tc_dkv(const void *q, const void *k, const void *v, const float *lse, const void *dO,
+                        const float *delta, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int T, float scale,
+                        int window, float softcap, cudaStream_t st) {
+    using CA = BwdKvTc<DK, DV>;
+    using CQ = BwdQTc<DK, DV>;
+    CUtensorMap mq, mk, mv, mdo, mk64, mv64;
+    if (!make_map(&mq, q, DK, T, (long long)B * Hq, 128) || !make_map(&mk, k, DK, T, (long long)B * Hkv, 128) ||
+        !make_map(&mv, v, DV, T, (long long)B * Hkv, 128) || !make_map(&mdo, dO, DV, T, (long long)B * Hq, 128) ||
+        !make_map(&mk64, k, DK, T, (long long)B * Hkv, CQ::BN) || !make_map(&mv64, v, DV, T, (long long)B * Hkv, CQ::BN)) {
+        t_last_cuda_error = "cuTensorMapEncodeTiled failed";
+        return FORGE_ERR_CUDA;
+    }
+    BwdParams p;
+    p.lse = lse;
+    p.delta = delta;
+    p.dq_acc = nullptr;
+    p.dk = static_cast<__nv_bfloat16 *>(dk);
+    p.dv = static_cast<__nv_bfloat16 *>(dv);
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.T = T; p.Tpad = tpad_of(T); p.window = window;
+    p.num_kt = (T + 127) / 128;
+    p.scale = scale;
+    p.scale_log2 = scale * kLog2e;
+    p.softcap = softcap;
+    p.cap_in = softcap > 0.0f ? scale / softcap : 0.0f;
+    p.cap_out = softcap * kLog2e;
+    if (set_smem(bwd_dkdv_tc_kernel<DK, DV>, CA::SMEM) != FORGE_OK) return FORGE_ERR_CUDA;
+    bwd_dkdv_tc_kernel<DK, DV><<<(unsigned)(p.num_kt * B * Hkv), CA::THREADS, CA::SMEM, st>>>(mq, mk, mv, mdo, p);
+    forge_status s = launch_status();
+    if (s != FORGE_OK) return s;
+    BwdQParams pq;
+    pq.lse = lse;
+    pq.delta = delta;
+    pq.dq = static_cast<__nv_bfloat16 *>(dq);
+    pq.B = B; pq.Hq = Hq; pq.Hkv = Hkv; pq.T = T; pq.window = window;
+    pq.num_qt = (T + 127) / 128;
+    pq.scale = p.scale; pq.scale_log2 = p.scale_log2; pq.softcap = p.softcap; pq.cap_in = p.cap_in;
+    pq.cap_out = p.cap_out;
+    if (set_smem(bwd_dq_tc_kernel<DK, DV>, CQ::SMEM) != FORGE_OK) return FORGE_ERR_CUDA;
+    bwd_dq_tc_kernel<DK, DV><<<(unsigned)(pq.num_qt * B * Hq), CQ::THREADS, CQ::SMEM, st>>>(mq, mk64, mv64, mdo, pq);
     return launch_status();
 }
 
@@ -593,19 +658,17 @@ forge_status forge_attn_bwd_noalloc(const void *q, const void *k, const void *v,
 }
 
 // d_k != d_v at (d_k, d_v) = (192, 128), the decompressed multi-head latent
-// attention of the DeepSeek V3 family: forward on the tensor cores (bf16) or the
-// CUDA cores (f32); backward on the CUDA cores (f32) only.
+// attention of the DeepSeek V3 family: on the tensor cores (bf16) or the CUDA
+// cores (f32), forward and backward.
 static bool dkv_supported(int Dk, int Dv, forge_dtype dtype) {
-    return dtype == FORGE_DTYPE_F32 && Dk == 192 && Dv == 128;
-}
-static bool dkv_fwd_supported(int Dk, int Dv, forge_dtype dtype) {
     return (dtype == FORGE_DTYPE_F32 || dtype == FORGE_DTYPE_BF16) && Dk == 192 && Dv == 128;
 }
+static bool dkv_fwd_supported(int Dk, int Dv, forge_dtype dtype) { return dkv_supported(Dk, Dv, dtype); }
 
 size_t forge_attn_bwd_workspace_size_dkv(int B, int Hq, int Hkv, int T, int Dk, int Dv, forge_dtype dtype) {
     if (Dk == Dv) return forge_attn_bwd_workspace_size(B, Hq, Hkv, T, Dk, dtype);
     if (!dkv_supported(Dk, Dv, dtype) || check_sizes(B, Hq, Hkv, T, Dv, dtype) != FORGE_OK) return 0;
-    return delta_bytes(B, Hq, T);  // Delta only: the f32 path writes dq directly
+    return delta_bytes(B, Hq, T);  // Delta only: both paths write dq directly
 }
 
 forge_status forge_attn_fwd_dkv(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
@@ -645,6 +708,13 @@ forge_status forge_attn_bwd_dkv(const void *q, const void *k, const void *v, con
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     float *delta = static_cast<float *>(workspace);
     const long rows = (long)B * Hq * T;
+    if (dtype == FORGE_DTYPE_BF16) {
+        bwd_preprocess<__nv_bfloat16, 128><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
+            static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dO), delta, nullptr, rows, T,
+            tpad_of(T));
+        if ((s = launch_status()) != FORGE_OK) return s;
+        return bwd_tc_dkv<192, 128>(q, k, v, lse, dO, delta, dq, dk, dv, B, Hq, Hkv, T, scale, window, softcap, st);
+    }
     bwd_preprocess<float, 128><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
         static_cast<const float *>(o), static_cast<const float *>(dO), delta, nullptr, rows, T, tpad_of(T));
     if ((s = launch_status()) != FORGE_OK) return s;

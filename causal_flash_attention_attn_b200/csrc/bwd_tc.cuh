@@ -70,11 +70,15 @@ struct BwdTc {
     static constexpr uint32_t TK = NCB * CBK;            // K (or V) tile bytes
     static constexpr uint32_t TQ = NCB * CBQ;            // Q (or dO) tile bytes
     static constexpr uint32_t TS = (BM / 64) * CBK;      // dS^T tile bytes
-    static constexpr uint32_t OFF_K = 0, OFF_V = TK, OFF_Q = 2 * TK;
+    // K/V buffers: two at head dim 64, so that the next work item's K and V load
+    // while the current one finishes; one where shared memory has no room
+    static constexpr int NKV = D == 64 ? 2 : 1;
+    static constexpr uint32_t KVB = 2 * TK;              // one K + V buffer
+    static constexpr uint32_t OFF_K = 0, OFF_V = TK, OFF_Q = NKV * KVB;
     static constexpr uint32_t OFF_DO = OFF_Q + QST * TQ;
     static constexpr uint32_t OFF_DS = OFF_DO + QST * TQ;
     static constexpr bool BULK_DQ = D == 64;             // staged TMA reduce-add of dQ
-    static constexpr int NSTG = D == 64 ? 2 : 1;         // dQ staging tiles
+    static constexpr int NSTG = 1;                       // dQ staging tiles
     static constexpr uint32_t STG = BM * DH * 4;         // one f32 dQ staging tile
     static constexpr uint32_t OFF_STG = OFF_DS + TS;
     static constexpr uint32_t TILES = OFF_STG + (BULK_DQ ? NSTG * STG : 0);
@@ -115,8 +119,9 @@ struct BwdTc {
     static_assert(!DQT || DH == 128, "transposed dQ needs M = 128");
     static_assert(SMEM <= 232448, "shared memory");
     // barriers
-    static constexpr int B_KV = 0;
-    static constexpr int B_Q_FULL = 1;                   // [QST]
+    static constexpr int B_KV_FULL = 0;                  // [NKV]
+    static constexpr int B_KV_EMPTY = NKV;               // [NKV]
+    static constexpr int B_Q_FULL = 2 * NKV;             // [QST]
     static constexpr int B_Q_EMPTY = B_Q_FULL + QST;     // [QST]
     static constexpr int B_S_FULL = B_Q_EMPTY + QST;
     static constexpr int B_DS_EMPTY = B_S_FULL + 1;
@@ -125,9 +130,17 @@ struct BwdTc {
     static constexpr int B_DP_FULL = B_DS_FULL + 1;
     static constexpr int B_DQ_FULL = B_DP_FULL + 1;
     static constexpr int B_DQ_FREE = B_DQ_FULL + 1;
-    static constexpr int B_KDONE = B_DQ_FREE + 1;
-    static constexpr int NBAR = B_KDONE + 1;
+    static constexpr int B_KDONE = B_DQ_FREE + 1;        // a work item's dK, dV complete in TMEM
+    static constexpr int B_EPI_DONE = B_KDONE + 1;       // ... and read out (8 compute + 4 drain warps)
+    static constexpr int NBAR = B_EPI_DONE + 1;
     static_assert(NBAR * 8 <= (int)OFF_TMEM_SLOT, "control block");
+};
+
+// A work item: (key tile n, batch b, KV head, head-dim half h), heaviest (n = 0)
+// first. Its steps walk the query tiles m_lo .. m_lo + nm - 1 of each of the G
+// heads of the group.
+struct BwdItem {
+    int h, bkv, b, hkv, k0, m_lo, nm, steps;
 };
 
 struct BwdParams {
@@ -234,6 +247,77 @@ __device__ __forceinline__ void bwd_store_ds(const uint32_t (&dk)[16], int c0, i
     }
 }
 
+// The MMA issuer's products, operands passed by value (shared-memory addresses
+// of the operand tiles, TMEM address of the accumulator).
+// S^T = K Q^T (or dP^T = V dO^T) over the full head dim.
+template <class C>
+__device__ __forceinline__ void bwd_mma_kq(uint32_t d_tmem, uint32_t sA, uint32_t sB) {
+    constexpr uint32_t ID = idesc_bf16_f32(128, C::BM, false, false);
+#pragma unroll
+    for (int kk = 0; kk < C::D / 16; kk++) {
+        const uint32_t oa = (kk >> 2) * C::CBK + (kk & 3) * 32;
+        const uint32_t ob = (kk >> 2) * C::CBQ + (kk & 3) * 32;
+        mma_ss(d_tmem, sdesc_sw128(opaque_u32(sA) + oa, 16, 1024), sdesc_sw128(opaque_u32(sB) + ob, 16, 1024), ID, kk > 0);
+    }
+}
+// dV += P^T dO (A = P^T from TMEM; dO MN-major from the half's column blocks)
+template <class C>
+__device__ __forceinline__ void bwd_mma_dv(uint32_t tmem, uint32_t sdO_h, bool first) {
+    constexpr uint32_t ID = idesc_bf16_f32(128, C::DH, false, true);
+#pragma unroll
+    for (int kk = 0; kk < C::BM / 16; kk++)
+        mma_ts(tmem + C::COL_DV, tmem + C::col_p(kk), sdesc_sw128(opaque_u32(sdO_h) + kk * 2048, C::CBQ, 1024), ID,
+               (!first || kk > 0) ? 1u : 0u);
+}
+// dK += dS^T Q (A = dS^T from shared memory; Q MN-major from the half's column blocks)
+template <class C>
+__device__ __forceinline__ void bwd_mma_dk(uint32_t tmem, uint32_t sdS, uint32_t sQ_h, bool first) {
+    constexpr uint32_t ID = idesc_bf16_f32(128, C::DH, false, true);
+#pragma unroll
+    for (int kk = 0; kk < C::BM / 16; kk++) {
+        const uint32_t oa = (kk >> 2) * C::CBK + (kk & 3) * 32;
+        mma_ss(tmem + C::COL_DK, sdesc_sw128(opaque_u32(sdS) + oa, 16, 1024), sdesc_sw128(opaque_u32(sQ_h) + kk * 2048, C::CBQ, 1024), ID,
+               (!first || kk > 0) ? 1u : 0u);
+    }
+}
+// dQ = dS K, or its transpose K^T dS^T (K's half from the column blocks at sK_h)
+template <class C>
+__device__ __forceinline__ void bwd_mma_dq(uint32_t tmem, uint32_t sdS, uint32_t sK, uint32_t sK_h) {
+    constexpr uint32_t ID =
+        C::DQT ? idesc_bf16_f32(128, C::BM, true, true) : idesc_bf16_f32(128, C::D, true, true);
+#pragma unroll
+    for (int kk = 0; kk < C::BN / 16; kk++) {
+        if constexpr (C::DQT) {
+            mma_ss(tmem + C::COL_DQ, sdesc_sw128(opaque_u32(sK_h) + kk * 2048, C::CBK, 1024),
+                   sdesc_sw128(opaque_u32(sdS) + kk * 2048, C::CBK, 1024), ID, kk > 0);
+        } else {
+            mma_ss(tmem + C::COL_DQ, sdesc_sw128(opaque_u32(sdS) + kk * 2048, C::CBK, 1024),
+                   sdesc_sw128(opaque_u32(sK) + kk * 2048, C::CBK, 1024), ID, kk > 0);
+        }
+    }
+}
+
+template <class C, class P>
+__device__ __forceinline__ BwdItem bwd_item(int w, const P &p) {
+    BwdItem it;
+    const int per_n = p.B * p.Hkv * C::NSPLIT;
+    const int n = w / per_n;
+    const int rest = w % per_n;
+    it.h = rest % C::NSPLIT;
+    it.bkv = rest / C::NSPLIT;  // b * Hkv + hkv
+    it.b = it.bkv / p.Hkv;
+    it.hkv = it.bkv % p.Hkv;
+    it.k0 = n * C::BN;
+    it.m_lo = it.k0 / C::BM;
+    const int q_last = p.window > 0 ? min(p.T - 1, it.k0 + C::BN - 1 + p.window - 1) : p.T - 1;
+    it.nm = q_last / C::BM - it.m_lo + 1;
+    it.steps = (p.Hq / p.Hkv) * it.nm;
+    return it;
+}
+
+// Persistent: gridDim.x CTAs walk the work items in the snake order above. Every
+// barrier's phase counts steps (or items) over the CTA's whole run, so the
+// pipeline carries on from one item into the next; TMEM is allocated once.
 template <int D>
 __global__ void __launch_bounds__(512, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -245,7 +329,7 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t tiles = (sbase + 1023u) & ~1023u;
     const uint32_t ctrl = tiles + C::TILES;
     uint8_t *const ctrl_p = smem_raw + (ctrl - sbase);
-    const uint32_t sK = tiles + C::OFF_K, sV = tiles + C::OFF_V, sQ0 = tiles + C::OFF_Q;
+    const uint32_t sK0 = tiles + C::OFF_K, sQ0 = tiles + C::OFF_Q;
     const uint32_t sdO0 = tiles + C::OFF_DO, sdS = tiles + C::OFF_DS, sStg = tiles + C::OFF_STG;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl_p + C::OFF_ABORT);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ctrl_p + C::OFF_TMEM_SLOT);
@@ -259,25 +343,16 @@ __global__ void __launch_bounds__(512, 1)
     }
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    // work item: key tile n (heaviest = smallest n first), batch b, KV head, half h
-    const int per_n = p.B * p.Hkv * C::NSPLIT;
-    const int n = blockIdx.x / per_n;
-    int rest = blockIdx.x % per_n;
-    const int h = rest % C::NSPLIT;
-    rest /= C::NSPLIT;
-    const int bkv = rest;  // b * Hkv + hkv
-    const int b = bkv / p.Hkv, hkv = bkv % p.Hkv;
+    const int nitems = p.num_kt * p.B * p.Hkv * C::NSPLIT;
     const int G = p.Hq / p.Hkv;
-    const int k0 = n * C::BN;
     const int W = p.window;
-    const int m_lo = k0 / C::BM;
-    const int q_last = W > 0 ? min(p.T - 1, k0 + C::BN - 1 + W - 1) : p.T - 1;
-    const int m_hi = q_last / C::BM;
-    const int nm = m_hi - m_lo + 1;
-    const int steps = G * nm;
+    auto item_of = [&](int pass) -> int { return snake_item(pass, (int)blockIdx.x, (int)gridDim.x); };
 
     if (threadIdx.x == 0) {
-        mbar_init(bar(C::B_KV), 1);
+        for (int s = 0; s < C::NKV; s++) {
+            mbar_init(bar(C::B_KV_FULL + s), 1);
+            mbar_init(bar(C::B_KV_EMPTY + s), 1);
+        }
         for (int s = 0; s < C::QST; s++) {
             mbar_init(bar(C::B_Q_FULL + s), 33);
             mbar_init(bar(C::B_Q_EMPTY + s), 1);
@@ -290,6 +365,7 @@ __global__ void __launch_bounds__(512, 1)
         mbar_init(bar(C::B_DQ_FULL), 1);
         mbar_init(bar(C::B_DQ_FREE), 4);
         mbar_init(bar(C::B_KDONE), 1);
+        mbar_init(bar(C::B_EPI_DONE), 12);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -313,53 +389,72 @@ __global__ void __launch_bounds__(512, 1)
         setmaxnreg_dec<C::REG_CTRL>();
         if (warp == C::W_LOAD) {
             // -------------------------------------------------------- producer
-            int issued = 0;
+            int issued = 0, kv_issued = 0;  // Q/dO and K/V loads issued (for the abort drain)
             bool ok = true;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::TK);
-                for (int c = 0; c < C::NCB; c++) {
-                    tma_load_3d(sK + c * C::CBK, &tmK, bar(C::B_KV), c * 64, k0, bkv);
-                    tma_load_3d(sV + c * C::CBK, &tmV, bar(C::B_KV), c * 64, k0, bkv);
-                }
-            }
-            for (int i = 0; i < steps; i++) {
-                const int st = i % C::QST;
-                const uint32_t ph = (uint32_t)((i / C::QST) & 1);
-                const int g = i / nm, m = m_lo + i % nm;
-                const int bhq = b * p.Hq + hkv * G + g;
-                // this step's LSE and Delta into registers first: their global-load
-                // latency overlaps the wait for a free stage
-                float lv[C::BM / 32], dv[C::BM / 32];
-#pragma unroll
-                for (int r = 0; r < C::BM / 32; r++) {
-                    const int q = m * C::BM + lane + 32 * r;
-                    const size_t idx = (size_t)bhq * p.T + (size_t)min(q, p.T - 1);
-                    lv[r] = q < p.T ? p.lse[idx] * kLog2e : INFINITY;
-                    dv[r] = q < p.T ? p.delta[idx] * p.scale : 0.0f;
-                }
-                if (!mbar_wait_warp(bar(C::B_Q_EMPTY + st), ph ^ 1u, abort_flag)) {
+            int gs = 0;  // step count over all of this CTA's items
+            for (int pass = 0; ok; pass++) {
+                const int w = item_of(pass);
+                if (w >= nitems) break;
+                const BwdItem I = bwd_item<C>(w, p);
+                // K, V of the item into buffer pass % NKV once the item that used it
+                // NKV items ago has no product left reading it
+                const int kvs = pass % C::NKV;
+                if (!mbar_wait_warp(bar(C::B_KV_EMPTY + kvs), (uint32_t)(((pass / C::NKV) & 1) ^ 1), abort_flag)) {
                     ok = false;
                     break;
                 }
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(bar(C::B_Q_FULL + st), 2 * C::TQ);
+                    const uint32_t sK = sK0 + (uint32_t)kvs * C::KVB, sV = sK + C::TK;
+                    mbar_arrive_expect_tx(bar(C::B_KV_FULL + kvs), 2 * C::TK);
                     for (int c = 0; c < C::NCB; c++) {
-                        tma_load_3d(sQ0 + st * C::TQ + c * C::CBQ, &tmQ, bar(C::B_Q_FULL + st), c * 64, m * C::BM,
-                                    bhq);
-                        tma_load_3d(sdO0 + st * C::TQ + c * C::CBQ, &tmdO, bar(C::B_Q_FULL + st), c * 64,
-                                    m * C::BM, bhq);
+                        tma_load_3d(sK + c * C::CBK, &tmK, bar(C::B_KV_FULL + kvs), c * 64, I.k0, I.bkv);
+                        tma_load_3d(sV + c * C::CBK, &tmV, bar(C::B_KV_FULL + kvs), c * 64, I.k0, I.bkv);
                     }
                 }
-                issued++;
+                kv_issued++;
+                for (int i = 0; i < I.steps; i++, gs++) {
+                    const int st = gs % C::QST;
+                    const uint32_t ph = (uint32_t)((gs / C::QST) & 1);
+                    const int g = i / I.nm, m = I.m_lo + i % I.nm;
+                    const int bhq = I.b * p.Hq + I.hkv * G + g;
+                    // this step's LSE and Delta into registers first: their global-load
+                    // latency overlaps the wait for a free stage
+                    float lv[C::BM / 32], dv[C::BM / 32];
 #pragma unroll
-                for (int r = 0; r < C::BM / 32; r++) {
-                    sLSE[st * C::BM + lane + 32 * r] = -lv[r];
-                    sDLT[st * C::BM + lane + 32 * r] = -dv[r];
+                    for (int r = 0; r < C::BM / 32; r++) {
+                        const int q = m * C::BM + lane + 32 * r;
+                        const size_t idx = (size_t)bhq * p.T + (size_t)min(q, p.T - 1);
+                        lv[r] = q < p.T ? p.lse[idx] * kLog2e : INFINITY;
+                        dv[r] = q < p.T ? p.delta[idx] * p.scale : 0.0f;
+                    }
+                    if (!mbar_wait_warp(bar(C::B_Q_EMPTY + st), ph ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(bar(C::B_Q_FULL + st), 2 * C::TQ);
+                        for (int c = 0; c < C::NCB; c++) {
+                            tma_load_3d(sQ0 + st * C::TQ + c * C::CBQ, &tmQ, bar(C::B_Q_FULL + st), c * 64,
+                                        m * C::BM, bhq);
+                            tma_load_3d(sdO0 + st * C::TQ + c * C::CBQ, &tmdO, bar(C::B_Q_FULL + st), c * 64,
+                                        m * C::BM, bhq);
+                        }
+                    }
+                    issued++;
+#pragma unroll
+                    for (int r = 0; r < C::BM / 32; r++) {
+                        sLSE[st * C::BM + lane + 32 * r] = -lv[r];
+                        sDLT[st * C::BM + lane + 32 * r] = -dv[r];
+                    }
+                    mbar_arrive(bar(C::B_Q_FULL + st));
                 }
-                mbar_arrive(bar(C::B_Q_FULL + st));
             }
             if (!ok && lane == 0) {
-                mbar_wait_drain(bar(C::B_KV), 0, 200000000ull);
+                // let the copies already issued land before the CTA exits
+                for (int back = 1; back <= min(kv_issued, C::NKV); back++) {
+                    const int L = kv_issued - back;
+                    mbar_wait_drain(bar(C::B_KV_FULL + L % C::NKV), (uint32_t)((L / C::NKV) & 1), 200000000ull);
+                }
                 for (int back = 1; back <= min(issued, C::QST); back++) {
                     const int L = issued - back;
                     mbar_wait_drain(bar(C::B_Q_FULL + L % C::QST), (uint32_t)((L / C::QST) & 1), 200000000ull);
@@ -367,179 +462,196 @@ __global__ void __launch_bounds__(512, 1)
             }
         } else if (warp == C::W_MMA && lane == 0) {
             // ------------------------------------------------------ MMA issuer
-            constexpr uint32_t ID_S = idesc_bf16_f32(128, C::BM, false, false);
-            constexpr uint32_t ID_ACC = idesc_bf16_f32(128, C::DH, false, true);
-            constexpr uint32_t ID_DQ =
-                C::DQT ? idesc_bf16_f32(128, C::BM, true, true) : idesc_bf16_f32(128, C::D, true, true);
-            const uint32_t h_q = (uint32_t)h * (C::DH / 64) * C::CBQ;  // column-block offset of half h
-            const uint32_t h_k = (uint32_t)h * (C::DH / 64) * C::CBK;
-            // S^T(j) = K Q(j)^T, over the full head dim
-            auto issue_s = [&](int j) -> bool {
-                const int st = j % C::QST;
-                if (!mbar_wait(bar(C::B_Q_FULL + st), (uint32_t)((j / C::QST) & 1), abort_flag)) return false;
+            // S^T(j) = K Q(j)^T once stage j % QST holds Q(j) (j counts steps over all items)
+            auto wait_q = [&](int j) -> bool {
+                if (!mbar_wait(bar(C::B_Q_FULL + j % C::QST), (uint32_t)((j / C::QST) & 1), abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t sQ = sQ0 + st * C::TQ;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; kk++) {
-                    const uint32_t ok_ = (kk >> 2) * C::CBK + (kk & 3) * 32;
-                    const uint32_t oq = (kk >> 2) * C::CBQ + (kk & 3) * 32;
-                    mma_ss(tmem + C::COL_S, sdesc_sw128(sK + ok_, 16, 1024), sdesc_sw128(sQ + oq, 16, 1024), ID_S,
-                           kk > 0);
-                }
-                tc_commit(bar(C::B_S_FULL));
                 return true;
             };
-            // dP^T(j) = V dO(j)^T (the stage of j is already known to be full)
-            auto issue_dp = [&](int j) {
-                const uint32_t sdO = sdO0 + (j % C::QST) * C::TQ;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; kk++) {
-                    const uint32_t ok_ = (kk >> 2) * C::CBK + (kk & 3) * 32;
-                    const uint32_t oq = (kk >> 2) * C::CBQ + (kk & 3) * 32;
-                    mma_ss(tmem + C::COL_DP, sdesc_sw128(sV + ok_, 16, 1024), sdesc_sw128(sdO + oq, 16, 1024),
-                           ID_S, kk > 0);
-                }
-                tc_commit(bar(C::B_DP_FULL));
-            };
-            bool ok = mbar_wait(bar(C::B_KV), 0, abort_flag);
-            if (ok && (ok = issue_s(0))) issue_dp(0);
-            for (int i = 0; ok && i < steps; i++) {
-                const int st = i % C::QST;
-                const uint32_t sQ = sQ0 + st * C::TQ, sdO = sdO0 + st * C::TQ;
-                const bool more = i + 1 < steps;
-                // dV += P^T dO, P^T from TMEM (phase A of step i)
-                if (!(ok = mbar_wait(bar(C::B_P_FULL), (uint32_t)(i & 1), abort_flag))) break;
+            constexpr bool EARLY_S = C::QST > 1;   // S^T(j + 1) issued before dS(j) is formed
+            constexpr bool DQ_FIRST = C::QST > 1;  // dQ(j) issued before dK(j)
+            bool ok = true;
+            int gs = 0, pass = 0;
+            for (; ok; pass++) {
+                const int w = item_of(pass);
+                if (w >= nitems) break;
+                const BwdItem I = bwd_item<C>(w, p);
+                const int kvs = pass % C::NKV;
+                const uint32_t sK = sK0 + (uint32_t)kvs * C::KVB, sV = sK + C::TK;
+                const uint32_t h_q = (uint32_t)I.h * (C::DH / 64) * C::CBQ;  // column-block offset of half h
+                const uint32_t h_k = (uint32_t)I.h * (C::DH / 64) * C::CBK;
+                if (!(ok = mbar_wait(bar(C::B_KV_FULL + kvs), (uint32_t)((pass / C::NKV) & 1), abort_flag))) break;
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < C::BM / 16; kk++)
-                    mma_ts(tmem + C::COL_DV, tmem + C::col_p(kk), sdesc_sw128(sdO + h_q + kk * 2048, C::CBQ, 1024),
-                           ID_ACC, (i > 0 || kk > 0) ? 1u : 0u);
-                // S^T(i + 1) over S^T(i) / P^T(i): phase A has read S^T(i), and dV(i)
-                // is ahead of it on the tensor cores. It runs while the compute warps
-                // form dS of step i. With a single Q/dO stage Q(i + 1) can only be
-                // loaded once dK(i) has read Q(i), so S^T(i + 1) then comes after dQ(i).
-                constexpr bool EARLY_S = C::QST > 1;
-                if (EARLY_S && more && !(ok = issue_s(i + 1))) break;
-                // dK += dS^T Q, dQ (phase B of step i)
-                if (!(ok = mbar_wait(bar(C::B_DS_FULL), (uint32_t)(i & 1), abort_flag))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < C::BM / 16; kk++) {
-                    const uint32_t oa = (kk >> 2) * C::CBK + (kk & 3) * 32;
-                    mma_ss(tmem + C::COL_DK, sdesc_sw128(sdS + oa, 16, 1024),
-                           sdesc_sw128(sQ + h_q + kk * 2048, C::CBQ, 1024), ID_ACC, (i > 0 || kk > 0) ? 1u : 0u);
-                }
-                tc_commit(bar(C::B_Q_EMPTY + st));  // Q(i), dO(i) read by every product issued so far
-                // dQ (the drain warps must have emptied the previous one; in the
-                // aliased layout they did so before dP^T(i) was issued)
-                if (!C::DQ_ALIAS && i > 0) {
-                    if (!(ok = mbar_wait(bar(C::B_DQ_FREE), (uint32_t)((i - 1) & 1), abort_flag))) break;
+                if (!(ok = wait_q(gs))) break;
+                bwd_mma_kq<C>(tmem + C::COL_S, sK, sQ0 + (gs % C::QST) * C::TQ);
+                tc_commit(bar(C::B_S_FULL));
+                // in the aliased layout dP^T overwrites the previous dQ^T: wait for its drain
+                if (C::DQ_ALIAS && gs > 0) {
+                    if (!(ok = mbar_wait(bar(C::B_DQ_FREE), (uint32_t)((gs - 1) & 1), abort_flag))) break;
                     tc_fence_after();
                 }
-#pragma unroll
-                for (int kk = 0; kk < C::BN / 16; kk++) {
-                    if constexpr (C::DQT) {
-                        mma_ss(tmem + C::COL_DQ, sdesc_sw128(sK + h_k + kk * 2048, C::CBK, 1024),
-                               sdesc_sw128(sdS + kk * 2048, C::CBK, 1024), ID_DQ, kk > 0);
-                    } else {
-                        mma_ss(tmem + C::COL_DQ, sdesc_sw128(sdS + kk * 2048, C::CBK, 1024),
-                               sdesc_sw128(sK + kk * 2048, C::CBK, 1024), ID_DQ, kk > 0);
-                    }
-                }
-                tc_commit(bar(C::B_DQ_FULL));
-                tc_commit(bar(C::B_DS_EMPTY));
-                if (!EARLY_S && more && !(ok = issue_s(i + 1))) break;
-                if (more) {
-                    // dP^T(i + 1): phase B has read dP^T(i); in the aliased layout it
-                    // also overwrites dQ^T(i), so wait for the drain warps
-                    if (C::DQ_ALIAS) {
-                        if (!(ok = mbar_wait(bar(C::B_DQ_FREE), (uint32_t)(i & 1), abort_flag))) break;
+                bwd_mma_kq<C>(tmem + C::COL_DP, sV, sdO0 + (gs % C::QST) * C::TQ);
+                tc_commit(bar(C::B_DP_FULL));
+                for (int i = 0; i < I.steps; i++, gs++) {
+                    const int st = gs % C::QST;
+                    const uint32_t sQ = sQ0 + st * C::TQ, sdO = sdO0 + st * C::TQ;
+                    const bool more = i + 1 < I.steps;
+                    // dV += P^T dO, P^T from TMEM (phase A of step gs)
+                    if (!(ok = mbar_wait(bar(C::B_P_FULL), (uint32_t)(gs & 1), abort_flag))) break;
+                    tc_fence_after();
+                    // the first dV and dK of an item overwrite the accumulators: the
+                    // previous item's must have been read out
+                    if (i == 0 && pass > 0) {
+                        if (!(ok = mbar_wait(bar(C::B_EPI_DONE), (uint32_t)((pass - 1) & 1), abort_flag))) break;
                         tc_fence_after();
                     }
-                    issue_dp(i + 1);
+                    bwd_mma_dv<C>(tmem, sdO + h_q, i == 0);
+                    // S^T(gs + 1) over S^T(gs) / P^T(gs): phase A has read S^T(gs), and
+                    // dV(gs) is ahead of it on the tensor cores. It runs while the compute
+                    // warps form dS of step gs. With a single Q/dO stage Q(gs + 1) can
+                    // only be loaded once dK(gs) has read Q(gs), so S^T(gs + 1) then comes
+                    // after dQ(gs).
+                    if (EARLY_S && more) {
+                        if (!(ok = wait_q(gs + 1))) break;
+                        bwd_mma_kq<C>(tmem + C::COL_S, sK, sQ0 + ((gs + 1) % C::QST) * C::TQ);
+                        tc_commit(bar(C::B_S_FULL));
+                    }
+                    // dQ and dK += dS^T Q (phase B of step gs). With two Q/dO stages dQ
+                    // goes first: the drain warps copy it out while dK runs, so dK is
+                    // off the path dS(gs) -> dQ(gs) -> copy-out -> dP^T(gs + 1) -> dS(gs + 1).
+                    // With one stage dK goes first, since Q(gs + 1) can only be loaded
+                    // once the products that read Q(gs) (dK(gs)) have completed.
+                    if (!(ok = mbar_wait(bar(C::B_DS_FULL), (uint32_t)(gs & 1), abort_flag))) break;
+                    tc_fence_after();
+                    if (!DQ_FIRST) {
+                        bwd_mma_dk<C>(tmem, sdS, sQ + h_q, i == 0);
+                        tc_commit(bar(C::B_Q_EMPTY + st));  // Q, dO of this step read by every product issued
+                    }
+                    // the drain warps must have emptied the previous dQ (in the aliased
+                    // layout they did so before dP^T(gs) was issued)
+                    if (!C::DQ_ALIAS && gs > 0) {
+                        if (!(ok = mbar_wait(bar(C::B_DQ_FREE), (uint32_t)((gs - 1) & 1), abort_flag))) break;
+                        tc_fence_after();
+                    }
+                    bwd_mma_dq<C>(tmem, sdS, sK, sK + h_k);
+                    tc_commit(bar(C::B_DQ_FULL));
+                    if (DQ_FIRST) {
+                        bwd_mma_dk<C>(tmem, sdS, sQ + h_q, i == 0);
+                        tc_commit(bar(C::B_Q_EMPTY + st));
+                    }
+                    tc_commit(bar(C::B_DS_EMPTY));
+                    if (!EARLY_S && more) {
+                        if (!(ok = wait_q(gs + 1))) break;
+                        bwd_mma_kq<C>(tmem + C::COL_S, sK, sQ0 + ((gs + 1) % C::QST) * C::TQ);
+                        tc_commit(bar(C::B_S_FULL));
+                    }
+                    if (more) {
+                        // dP^T(gs + 1): phase B has read dP^T(gs); in the aliased layout it
+                        // also overwrites dQ^T(gs), so wait for the drain warps
+                        if (C::DQ_ALIAS) {
+                            if (!(ok = mbar_wait(bar(C::B_DQ_FREE), (uint32_t)(gs & 1), abort_flag))) break;
+                            tc_fence_after();
+                        }
+                        bwd_mma_kq<C>(tmem + C::COL_DP, sV, sdO0 + ((gs + 1) % C::QST) * C::TQ);
+                        tc_commit(bar(C::B_DP_FULL));
+                    }
                 }
+                if (!ok) break;
+                tc_commit(bar(C::B_KV_EMPTY + kvs));  // K, V of this item read by every product issued
+                tc_commit(bar(C::B_KDONE));           // dK, dV of this item final
             }
-            tc_commit(bar(C::B_KDONE));
-            if (!ok) mbar_wait_drain(bar(C::B_KDONE), 0, 200000000ull);
+            if (!ok) {
+                // let every product issued finish before TMEM is released
+                tc_commit(bar(C::B_KDONE));
+                mbar_wait_drain(bar(C::B_KDONE), (uint32_t)(pass & 1), 200000000ull);
+            }
         }
     } else if (warp < C::W_DRAIN) {
         setmaxnreg_inc<C::REG_COMPUTE>();
         // ------------------------------- compute (key rows = TMEM lanes, row halves)
         const int hc = warp / 4;             // query-row half of the step
         const int kr = (warp % 4) * 32 + lane;  // key row within the tile
-        const int kj = k0 + kr;
         const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
         const bool cap = p.softcap > 0.0f;
         bool ok = true;
-        for (int i = 0; i < steps; i++) {
-            const int st = i % C::QST;
-            const int m = m_lo + i % nm;
-            const int qb = m * C::BM;
-            // phase A: S^T -> P^T (TMEM) and the dS factors g (registers)
-            if (!(ok = mbar_wait_warp(bar(C::B_Q_FULL + st), (uint32_t)((i / C::QST) & 1), abort_flag))) break;
-            if (!(ok = mbar_wait_warp(bar(C::B_S_FULL), (uint32_t)(i & 1), abort_flag))) break;
-            tc_fence_after();
-            const float *nls = sLSE + st * C::BM;
-            const float *nds = sDLT + st * C::BM;
-            const bool mask = (k0 + C::BN - 1 > qb) || (W > 0 && k0 <= qb + C::BM - 1 - W);
-            float g[C::HALF / 32][32];
+        int gs = 0;
+        for (int pass = 0; ok; pass++) {
+            const int w = item_of(pass);
+            if (w >= nitems) break;
+            const BwdItem I = bwd_item<C>(w, p);
+            const int kj = I.k0 + kr;
+            for (int i = 0; i < I.steps; i++, gs++) {
+                const int st = gs % C::QST;
+                const int m = I.m_lo + i % I.nm;
+                const int qb = m * C::BM;
+                // phase A: S^T -> P^T (TMEM) and the dS factors g (registers)
+                if (!(ok = mbar_wait_warp(bar(C::B_Q_FULL + st), (uint32_t)((gs / C::QST) & 1), abort_flag))) break;
+                if (!(ok = mbar_wait_warp(bar(C::B_S_FULL), (uint32_t)(gs & 1), abort_flag))) break;
+                tc_fence_after();
+                const float *nls = sLSE + st * C::BM;
+                const float *nds = sDLT + st * C::BM;
+                const bool mask = (I.k0 + C::BN - 1 > qb) || (W > 0 && I.k0 <= qb + C::BM - 1 - W);
+                float g[C::HALF / 32][32];
 #pragma unroll
-            for (int c = 0; c < C::HALF / 32; c++) {
-                const int c0 = hc * C::HALF + 32 * c;
-                uint32_t sc[32], pk[16];
-                tmem_ld32(tmem + lane_base + C::COL_S + c0, sc);
-                tmem_ld_wait(sc);
-                if (cap) {
-                    if (mask) bwd_p32<true, true>(sc, nls + c0, p, kj, qb + c0, W, pk, g[c]);
-                    else bwd_p32<true, false>(sc, nls + c0, p, kj, qb + c0, W, pk, g[c]);
-                } else {
-                    if (mask) bwd_p32<false, true>(sc, nls + c0, p, kj, qb + c0, W, pk, g[c]);
-                    else bwd_p32<false, false>(sc, nls + c0, p, kj, qb + c0, W, pk, g[c]);
+                for (int c = 0; c < C::HALF / 32; c++) {
+                    const int c0 = hc * C::HALF + 32 * c;
+                    uint32_t sc[32], pk[16];
+                    tmem_ld32(tmem + lane_base + C::COL_S + c0, sc);
+                    tmem_ld_wait(sc);
+                    if (cap) {
+                        if (mask) bwd_p32<true, true>(sc, nls + c0, p, kj, qb + c0, W, pk, g[c]);
+                        else bwd_p32<true, false>(sc, nls + c0, p, kj, qb + c0, W, pk, g[c]);
+                    } else {
+                        if (mask) bwd_p32<false, true>(sc, nls + c0, p, kj, qb + c0, W, pk, g[c]);
+                        else bwd_p32<false, false>(sc, nls + c0, p, kj, qb + c0, W, pk, g[c]);
+                    }
+                    tmem_st16(tmem + lane_base + C::COL_S + hc * C::HALF + 16 * c, pk);
                 }
-                tmem_st16(tmem + lane_base + C::COL_S + hc * C::HALF + 16 * c, pk);
-            }
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::B_P_FULL));
-            // phase B: dP^T -> dS^T (shared memory); the dS^T tile was last read
-            // by the dK/dQ products of step i - 1
-            if (!(ok = mbar_wait_warp(bar(C::B_DP_FULL), (uint32_t)(i & 1), abort_flag))) break;
-            if (i > 0 && !(ok = mbar_wait_warp(bar(C::B_DS_EMPTY), (uint32_t)((i - 1) & 1), abort_flag))) break;
-            tc_fence_after();
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::B_P_FULL));
+                // phase B: dP^T -> dS^T (shared memory); the dS^T tile was last read
+                // by the dK/dQ products of the previous step
+                if (!(ok = mbar_wait_warp(bar(C::B_DP_FULL), (uint32_t)(gs & 1), abort_flag))) break;
+                if (gs > 0 && !(ok = mbar_wait_warp(bar(C::B_DS_EMPTY), (uint32_t)((gs - 1) & 1), abort_flag))) break;
+                tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < C::HALF / 32; c++) {
-                const int c0 = hc * C::HALF + 32 * c;
-                uint32_t dc[32], dk[16];
-                tmem_ld32(tmem + lane_base + C::COL_DP + c0, dc);
-                tmem_ld_wait(dc);
-                bwd_ds32(dc, g[c], nds + c0, p, dk);
-                bwd_store_ds<D>(dk, c0, kr, sdS);
+                for (int c = 0; c < C::HALF / 32; c++) {
+                    const int c0 = hc * C::HALF + 32 * c;
+                    uint32_t dc[32], dk[16];
+                    tmem_ld32(tmem + lane_base + C::COL_DP + c0, dc);
+                    tmem_ld_wait(dc);
+                    bwd_ds32(dc, g[c], nds + c0, p, dk);
+                    bwd_store_ds<D>(dk, c0, kr, sdS);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::B_DS_FULL));
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::B_DS_FULL));
-        }
-        // epilogue: dV rows, this warp's half of the columns
-        if (ok) ok = mbar_wait_warp(bar(C::B_KDONE), 0, abort_flag);
-        if (ok) {
+            if (!ok) break;
+            // epilogue of the item: dV rows, this warp's half of the columns
+            if (!(ok = mbar_wait_warp(bar(C::B_KDONE), (uint32_t)(pass & 1), abort_flag))) break;
             tc_fence_after();
-            __nv_bfloat16 *row = p.dv + ((size_t)bkv * p.T + (size_t)min(kj, p.T - 1)) * D + h * C::DH;
+            __nv_bfloat16 *row = p.dv + ((size_t)I.bkv * p.T + (size_t)min(kj, p.T - 1)) * D + I.h * C::DH;
 #pragma unroll 1
             for (int c0 = hc * (C::DH / 2); c0 < (hc + 1) * (C::DH / 2); c0 += 32) {
                 uint32_t o[32];
                 tmem_ld32(tmem + lane_base + C::COL_DV + c0, o);
                 tmem_ld_wait(o);
-                uint32_t w[16];
+                uint32_t w16[16];
 #pragma unroll
-                for (int i = 0; i < 16; i++) w[i] = pack_bf16x2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1]));
+                for (int e = 0; e < 16; e++) w16[e] = pack_bf16x2(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1]));
                 if (kj < p.T) {
                     uint4 *dst = reinterpret_cast<uint4 *>(row + c0);
 #pragma unroll
-                    for (int i = 0; i < 4; i++) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                    for (int e = 0; e < 4; e++) dst[e] = make_uint4(w16[4 * e], w16[4 * e + 1], w16[4 * e + 2], w16[4 * e + 3]);
                 }
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_EPI_DONE));
         }
     } else {
         setmaxnreg_inc<C::REG_DRAIN>();
@@ -547,86 +659,95 @@ __global__ void __launch_bounds__(512, 1)
         const int t = threadIdx.x - 32 * C::W_DRAIN;  // TMEM lane of this thread
         const uint32_t lane_base = (uint32_t)((warp - C::W_DRAIN) * 32) << 16;
         bool ok = true;
-        for (int i = 0; i < steps; i++) {
-            const int g = i / nm, m = m_lo + i % nm;
-            const int bhq = b * p.Hq + hkv * G + g;
-            if (!(ok = mbar_wait_warp(bar(C::B_DQ_FULL), (uint32_t)(i & 1), abort_flag))) break;
-            tc_fence_after();
-            // this thread's dQ values: a query row's DH columns, or (transposed)
-            // a head-dim column's BM rows, in 32-column TMEM loads
-            constexpr int NQC = (C::DQT ? C::BM : C::DH) / 32;
-            uint32_t v[NQC][32];
+        int gs = 0;
+        for (int pass = 0; ok; pass++) {
+            const int w = item_of(pass);
+            if (w >= nitems) break;
+            const BwdItem I = bwd_item<C>(w, p);
+            for (int i = 0; i < I.steps; i++, gs++) {
+                const int g = i / I.nm, m = I.m_lo + i % I.nm;
+                const int bhq = I.b * p.Hq + I.hkv * G + g;
+                if (!(ok = mbar_wait_warp(bar(C::B_DQ_FULL), (uint32_t)(gs & 1), abort_flag))) break;
+                tc_fence_after();
+                // this thread's dQ values: a query row's DH columns, or (transposed)
+                // a head-dim column's BM rows, in 32-column TMEM loads
+                constexpr int NQC = (C::DQT ? C::BM : C::DH) / 32;
+                uint32_t v[NQC][32];
 #pragma unroll
-            for (int j = 0; j < NQC; j++) tmem_ld32(tmem + lane_base + C::COL_DQ + 32 * j, v[j]);
+                for (int j = 0; j < NQC; j++) tmem_ld32(tmem + lane_base + C::COL_DQ + 32 * j, v[j]);
 #pragma unroll
-            for (int j = 0; j < NQC; j++) tmem_ld_wait(v[j]);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::B_DQ_FREE));
-            if constexpr (C::BULK_DQ) {
-                static_assert(!C::BULK_DQ || NQC == 2, "staging covers 64 dQ values a thread");
-                const uint32_t(&v0)[32] = v[0];
-                const uint32_t(&v1)[32] = v[1 % NQC];
-                // Staging tile [BM rows][DH cols] f32, stored as DH/32 column blocks of
-                // [BM][32] with the 128-byte swizzle (16-byte chunk ^ row % 8), the
-                // layout of a TMA box {32, BM, 1}. The tile is reused once the reduce
-                // that last read it (NSTG steps ago) has read its source.
-                const uint32_t stg = sStg + (uint32_t)(i % C::NSTG) * C::STG;
-                if (t == 0) bulk_wait_read<C::NSTG - 1>();
-                named_barrier_sync(1, 128);
-                // thread t = query row t; v = the 64 head-dim values of that row
-                const uint32_t row = stg + (uint32_t)t * 128u;
+                for (int j = 0; j < NQC; j++) tmem_ld_wait(v[j]);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::B_DQ_FREE));
+                if constexpr (C::BULK_DQ) {
+                    static_assert(!C::BULK_DQ || NQC == 2, "staging covers 64 dQ values a thread");
+                    const uint32_t(&v0)[32] = v[0];
+                    const uint32_t(&v1)[32] = v[1 % NQC];
+                    // Staging tile [BM rows][DH cols] f32, stored as DH/32 column blocks of
+                    // [BM][32] with the 128-byte swizzle (16-byte chunk ^ row % 8), the
+                    // layout of a TMA box {32, BM, 1}. The tile is reused once the reduce
+                    // that last read it (NSTG steps ago) has read its source.
+                    const uint32_t stg = sStg + (uint32_t)(gs % C::NSTG) * C::STG;
+                    if (t == 0) bulk_wait_read<C::NSTG - 1>();
+                    named_barrier_sync(1, 128);
+                    // thread t = query row t; v = the 64 head-dim values of that row
+                    const uint32_t row = stg + (uint32_t)t * 128u;
 #pragma unroll
-                for (int c4 = 0; c4 < 8; c4++) {
-                    const uint32_t sw = (((uint32_t)c4 ^ ((uint32_t)t & 7u)) << 4);
-                    st_shared_v4(row + sw, v0[4 * c4], v0[4 * c4 + 1], v0[4 * c4 + 2], v0[4 * c4 + 3]);
-                    st_shared_v4(row + (uint32_t)(C::BM * 128) + sw, v1[4 * c4], v1[4 * c4 + 1], v1[4 * c4 + 2],
-                                 v1[4 * c4 + 3]);
-                }
-                fence_proxy_async_smem();
-                named_barrier_sync(1, 128);
-                if (t == 0) {
+                    for (int c4 = 0; c4 < 8; c4++) {
+                        const uint32_t sw = (((uint32_t)c4 ^ ((uint32_t)t & 7u)) << 4);
+                        st_shared_v4(row + sw, v0[4 * c4], v0[4 * c4 + 1], v0[4 * c4 + 2], v0[4 * c4 + 3]);
+                        st_shared_v4(row + (uint32_t)(C::BM * 128) + sw, v1[4 * c4], v1[4 * c4 + 1], v1[4 * c4 + 2],
+                                     v1[4 * c4 + 3]);
+                    }
+                    fence_proxy_async_smem();
+                    named_barrier_sync(1, 128);
+                    if (t == 0) {
 #pragma unroll
-                    for (int cb = 0; cb < C::DH / 32; cb++)
-                        tma_reduce_add_3d(&tmAcc, stg + (uint32_t)cb * (uint32_t)(C::BM * 128), h * C::DH + 32 * cb,
-                                          m * C::BM, bhq);
-                    bulk_commit();
-                }
-            } else {
-                // lane = head-dim column h*DH + t, BM query rows: each warp-wide
-                // reduction covers 32 consecutive floats of one dQ row
-                static_assert(C::BULK_DQ || C::DQT, "per-element reduction expects the transposed dQ");
+                        for (int cb = 0; cb < C::DH / 32; cb++)
+                            tma_reduce_add_3d(&tmAcc, stg + (uint32_t)cb * (uint32_t)(C::BM * 128), I.h * C::DH + 32 * cb,
+                                              m * C::BM, bhq);
+                        bulk_commit();
+                    }
+                } else {
+                    // lane = head-dim column h*DH + t, BM query rows: each warp-wide
+                    // reduction covers 32 consecutive floats of one dQ row
+                    static_assert(C::BULK_DQ || C::DQT, "per-element reduction expects the transposed dQ");
 
-                float *base = p.dq_acc + ((size_t)bhq * p.Tpad + (size_t)m * C::BM) * D + h * C::DH + t;
+                    float *base = p.dq_acc + ((size_t)bhq * p.Tpad + (size_t)m * C::BM) * D + I.h * C::DH + t;
 #pragma unroll
-                for (int j = 0; j < NQC; j++) {
+                    for (int j = 0; j < NQC; j++) {
 #pragma unroll
-                    for (int c = 0; c < 32; c++) atomicAdd(base + (size_t)(32 * j + c) * D, __uint_as_float(v[j][c]));
+                        for (int c = 0; c < 32; c++) atomicAdd(base + (size_t)(32 * j + c) * D, __uint_as_float(v[j][c]));
+                    }
                 }
             }
-        }
-        if constexpr (C::BULK_DQ) {
-            if (t == 0) bulk_wait<0>();  // reductions complete before the CTA retires
-        }
-        if (ok) ok = mbar_wait_warp(bar(C::B_KDONE), 0, abort_flag);
-        if (ok) {
+            if (!ok) break;
+            // epilogue of the item: dK rows
+            if (!(ok = mbar_wait_warp(bar(C::B_KDONE), (uint32_t)(pass & 1), abort_flag))) break;
             tc_fence_after();
-            const int kj = k0 + t;
-            __nv_bfloat16 *row = p.dk + ((size_t)bkv * p.T + (size_t)min(kj, p.T - 1)) * D + h * C::DH;
+            const int kj = I.k0 + t;
+            __nv_bfloat16 *row = p.dk + ((size_t)I.bkv * p.T + (size_t)min(kj, p.T - 1)) * D + I.h * C::DH;
 #pragma unroll 1
             for (int c0 = 0; c0 < C::DH; c0 += 32) {
                 uint32_t o[32];
                 tmem_ld32(tmem + lane_base + C::COL_DK + c0, o);
                 tmem_ld_wait(o);
-                uint32_t w[16];
+                uint32_t w16[16];
 #pragma unroll
-                for (int i = 0; i < 16; i++) w[i] = pack_bf16x2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1]));
+                for (int e = 0; e < 16; e++) w16[e] = pack_bf16x2(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1]));
                 if (kj < p.T) {
                     uint4 *dst = reinterpret_cast<uint4 *>(row + c0);
 #pragma unroll
-                    for (int i = 0; i < 4; i++) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                    for (int e = 0; e < 4; e++) dst[e] = make_uint4(w16[4 * e], w16[4 * e + 1], w16[4 * e + 2], w16[4 * e + 3]);
                 }
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_EPI_DONE));
+        }
+        if constexpr (C::BULK_DQ) {
+            if (t == 0) bulk_wait<0>();  // reductions complete before the CTA retires
         }
     }
 

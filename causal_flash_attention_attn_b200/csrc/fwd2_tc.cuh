@@ -1,8 +1,9 @@
 // fwd2_tc.cuh -- tensor-core forward with two query tiles per CTA (head dims 64
 // and 128; head dim 256 uses fwd_tc.cuh, whose single tile fills TMEM).
 //
-// One CTA per (pair of consecutive 128-row query tiles A, B of one head), so the
-// CTA streams each K/V tile once for 256 query rows and runs two softmax streams
+// Work item: a pair of consecutive 128-row query tiles A, B of one head; one
+// persistent CTA per SM walks its items (snake order over the heaviest-first
+// list). The CTA streams each K/V tile once for 256 query rows and runs two softmax streams
 // side by side (8 softmax warps, two per SM sub-partition): while one tile's
 // scores are in softmax, the tensor cores work on the other tile. Tile A sees
 // KV tiles [loA, tA], tile B [loB, tB] (tB = tA + 1); both ranges are the
@@ -33,33 +34,68 @@ struct Fwd2Tc {
     static constexpr uint32_t CB = 128 * 128;          // column block of a 128-row tile
     static constexpr uint32_t TILE = NCB * CB;         // one 128 x D bf16 tile
     static constexpr int NSTAGE = D == 128 ? 4 : 8;
+    // Q buffers (tiles A and B each): two at head dim 64, so that the next work
+    // item's queries load while the current item runs; one at head dim 128,
+    // where shared memory has no room for a second
+    static constexpr int NQB = D == 64 ? 2 : 1;
     static constexpr uint32_t CTRL = 1024;
-    static constexpr uint32_t SMEM = CTRL + TILE * (2 + NSTAGE) + 1024;
+    static constexpr uint32_t SMEM = CTRL + TILE * (2 * NQB + NSTAGE) + 1024;
     // warpgroups 0, 1: softmax of tiles A, B; warpgroup 2: producer (warp 8),
     // MMA issuer (warp 9), two idle warps. Launched at 168 registers a thread
     // (three warps per SM sub-partition); warpgroup 2 gives back down to
     // REG_CTRL so the softmax warpgroups can grow to REG_SOFTMAX:
     // 4 * (168 - REG_CTRL) = 8 * (REG_SOFTMAX - 168).
     static constexpr int THREADS = 384;
-    static constexpr int REG_LAUNCH = 168, REG_CTRL = 56, REG_SOFTMAX = 224;
+    static constexpr int REG_LAUNCH = 168, REG_CTRL = 72, REG_SOFTMAX = 216;
     static_assert(4 * (REG_LAUNCH - REG_CTRL) >= 8 * (REG_SOFTMAX - REG_LAUNCH), "register split");
     static_assert((2 * REG_SOFTMAX + REG_CTRL) * 32 <= 16384, "registers of one SM sub-partition");
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t col_s(int x) { return (uint32_t)(x * 128); }
     static constexpr uint32_t col_o(int x) { return (uint32_t)(256 + x * D); }
-    static constexpr int B_Q = 0;
-    static constexpr int B_KV_FULL = 1;
-    static constexpr int B_KV_EMPTY = 1 + NSTAGE;
-    static constexpr int B_S_FULL = 1 + 2 * NSTAGE;   // [2]
-    static constexpr int B_P_FULL = 3 + 2 * NSTAGE;   // [2]
-    static constexpr int B_O_FINAL = 5 + 2 * NSTAGE;  // [2]
-    static constexpr int NBAR = 7 + 2 * NSTAGE;
+    static constexpr int B_Q_FULL = 0;                  // [NQB]
+    static constexpr int B_Q_EMPTY = NQB;               // [NQB] both tiles' O stores have read the buffer
+    static constexpr int B_KV_FULL = 2 * NQB;           // [NSTAGE]
+    static constexpr int B_KV_EMPTY = B_KV_FULL + NSTAGE;
+    static constexpr int B_S_FULL = B_KV_EMPTY + NSTAGE;  // [2]
+    static constexpr int B_P_FULL = B_S_FULL + 2;         // [2]
+    static constexpr int B_O_FINAL = B_P_FULL + 2;        // [2]
+    static constexpr int B_O_EMPTY = B_O_FINAL + 2;       // [2] O_x read out of TMEM
+    static constexpr int NBAR = B_O_EMPTY + 2;
     static constexpr uint32_t OFF_TMEM_SLOT = 512, OFF_ABORT = 516;
     static constexpr int EMU_MASK = 7;                 // pairs with (c & 7) == 7 use the FMA-pipe exp2
     static_assert(NBAR * 8 <= 512, "control block");
     static_assert(SMEM <= 232448, "shared memory");
     static_assert(256 + 2 * D <= 512, "tensor memory");
 };
+
+// A work item of the forward: query tiles tA = 2 pr and tB = 2 pr + 1 of head bh
+// (pairs heaviest first); tile A sees KV tiles [loA, tA], tile B [loB, tB].
+struct Fwd2Item {
+    int bh, hq, bkv, tA, tB, qA0, qB0, loA, loB, lo, hi;
+    bool hasB;
+};
+
+template <class C>
+__device__ __forceinline__ Fwd2Item fwd2_item(int w, const FwdParams &p) {
+    Fwd2Item I;
+    const int nbh = p.B * p.Hq;
+    const int npairs = (p.num_qt + 1) / 2;
+    const int pr = npairs - 1 - w / nbh;
+    I.bh = w % nbh;
+    const int b = I.bh / p.Hq;
+    I.hq = I.bh % p.Hq;
+    I.bkv = b * p.Hkv + I.hq / (p.Hq / p.Hkv);
+    I.tA = 2 * pr;
+    I.tB = 2 * pr + 1;
+    I.hasB = I.tB < p.num_qt;
+    I.qA0 = I.tA * C::BM;
+    I.qB0 = I.tB * C::BM;
+    I.loA = p.window > 0 ? max(0, I.qA0 - p.window + 1) / C::BN : 0;
+    I.loB = p.window > 0 ? max(0, I.qB0 - p.window + 1) / C::BN : 0;
+    I.lo = I.loA;
+    I.hi = I.hasB ? I.tB : I.tA;
+    return I;
+}
 
 // Row max over 128 scores with three-input maxima (4 chains).
 __device__ __forceinline__ float row_max128(const uint32_t (&s)[4][32]) {
@@ -103,6 +139,9 @@ __device__ __forceinline__ void exp_chunk32(const uint32_t (&s)[32], uint64_t sl
     }
 }
 
+// Persistent: gridDim.x CTAs walk the work items (pairs of query tiles of one
+// head, heaviest first) in the snake order of snake_item; barrier phases count
+// KV tiles (or items) over the CTA's whole run and TMEM is allocated once.
 template <int D>
 __global__ void __launch_bounds__(384, 1)
     fwd2_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -112,30 +151,22 @@ __global__ void __launch_bounds__(384, 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = smem_u32(smem_raw);
     const uint32_t tiles = (sbase + C::CTRL + 1023u) & ~1023u;
-    const uint32_t sQ = tiles;                  // Q_A then Q_B
-    const uint32_t sKV = tiles + 2 * C::TILE;   // NSTAGE K/V tiles
+    const uint32_t sQ0 = tiles;                          // NQB x (Q_A, Q_B)
+    const uint32_t sKV = tiles + 2 * C::NQB * C::TILE;  // NSTAGE K/V tiles
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem_raw + C::OFF_ABORT);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + C::OFF_TMEM_SLOT);
     auto bar = [&](int i) -> uint32_t { return sbase + 8u * (uint32_t)i; };
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int nbh = p.B * p.Hq;
-    const int npairs = (p.num_qt + 1) / 2;
-    const int pr = npairs - 1 - (int)(blockIdx.x / nbh);
-    const int bh = blockIdx.x % nbh;
-    const int b = bh / p.Hq, hq = bh % p.Hq;
-    const int bkv = b * p.Hkv + hq / (p.Hq / p.Hkv);
     const int W = p.window;
-    const int tA = 2 * pr, tB = 2 * pr + 1;
-    const bool hasB = tB < p.num_qt;
-    const int qA0 = tA * C::BM, qB0 = tB * C::BM;
-    const int loA = W > 0 ? max(0, qA0 - W + 1) / C::BN : 0;
-    const int loB = W > 0 ? max(0, qB0 - W + 1) / C::BN : 0;
-    const int lo = loA, hi = hasB ? tB : tA;
-    auto active = [&](int x, int j) -> bool { return x == 0 ? (j >= loA && j <= tA) : (hasB && j >= loB && j <= tB); };
+    const int nitems = ((p.num_qt + 1) / 2) * p.B * p.Hq;
+    auto item_of = [&](int pass) -> int { return snake_item(pass, (int)blockIdx.x, (int)gridDim.x); };
 
     if (threadIdx.x == 0) {
-        mbar_init(bar(C::B_Q), 1);
+        for (int s = 0; s < C::NQB; s++) {
+            mbar_init(bar(C::B_Q_FULL + s), 1);
+            mbar_init(bar(C::B_Q_EMPTY + s), 2);
+        }
         for (int s = 0; s < C::NSTAGE; s++) {
             mbar_init(bar(C::B_KV_FULL + s), 1);
             mbar_init(bar(C::B_KV_EMPTY + s), 1);
@@ -144,6 +175,7 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(bar(C::B_S_FULL + x), 1);
             mbar_init(bar(C::B_P_FULL + x), 4);
             mbar_init(bar(C::B_O_FINAL + x), 1);
+            mbar_init(bar(C::B_O_EMPTY + x), 4);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -169,31 +201,48 @@ __global__ void __launch_bounds__(384, 1)
             // ------------------------------------------------------------ producer
             if (lane == 0) {
                 const uint64_t keep = policy_evict_last();
-                mbar_arrive_expect_tx(bar(C::B_Q), hasB ? 2 * C::TILE : C::TILE);
-                for (int c = 0; c < C::NCB; c++) {
-                    tma_load_3d(sQ + c * C::CB, &tmQ, bar(C::B_Q), c * 64, qA0, bh);
-                    if (hasB) tma_load_3d(sQ + C::TILE + c * C::CB, &tmQ, bar(C::B_Q), c * 64, qB0, bh);
-                }
-                // ring slots in order K(lo), V(lo), K(lo+1), V(lo+1), ...
-                int issued = 0;
+                int issued = 0, q_issued = 0;  // ring slots and Q buffers loaded (for the abort drain)
                 bool ok = true;
-                for (int j = lo; ok && j <= hi; j++) {
-                    for (int kv = 0; kv < 2 && ok; kv++) {
-                        const int st = issued % C::NSTAGE;
-                        const uint32_t ph = (uint32_t)((issued / C::NSTAGE) & 1);
-                        if (!mbar_wait(bar(C::B_KV_EMPTY + st), ph ^ 1u, abort_flag)) {
-                            ok = false;
-                            break;
+                for (int pass = 0; ok; pass++) {
+                    const int w = item_of(pass);
+                    if (w >= nitems) break;
+                    const Fwd2Item I = fwd2_item<C>(w, p);
+                    // the item's queries once both O stores of the item that used this
+                    // buffer NQB items ago have read it
+                    const int qb = pass % C::NQB;
+                    if (!mbar_wait(bar(C::B_Q_EMPTY + qb), (uint32_t)(((pass / C::NQB) & 1) ^ 1), abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t sQ = sQ0 + (uint32_t)qb * 2 * C::TILE;
+                    mbar_arrive_expect_tx(bar(C::B_Q_FULL + qb), I.hasB ? 2 * C::TILE : C::TILE);
+                    for (int c = 0; c < C::NCB; c++) {
+                        tma_load_3d(sQ + c * C::CB, &tmQ, bar(C::B_Q_FULL + qb), c * 64, I.qA0, I.bh);
+                        if (I.hasB) tma_load_3d(sQ + C::TILE + c * C::CB, &tmQ, bar(C::B_Q_FULL + qb), c * 64, I.qB0, I.bh);
+                    }
+                    q_issued++;
+                    // ring slots in order K(lo), V(lo), K(lo+1), V(lo+1), ...
+                    for (int j = I.lo; ok && j <= I.hi; j++) {
+                        for (int kv = 0; kv < 2 && ok; kv++) {
+                            const int st = issued % C::NSTAGE;
+                            const uint32_t ph = (uint32_t)((issued / C::NSTAGE) & 1);
+                            if (!mbar_wait(bar(C::B_KV_EMPTY + st), ph ^ 1u, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            mbar_arrive_expect_tx(bar(C::B_KV_FULL + st), C::TILE);
+                            for (int c = 0; c < C::NCB; c++)
+                                tma_load_3d_hint(sKV + st * C::TILE + c * C::CB, kv ? &tmV : &tmK,
+                                                 bar(C::B_KV_FULL + st), c * 64, j * C::BN, I.bkv, keep);
+                            issued++;
                         }
-                        mbar_arrive_expect_tx(bar(C::B_KV_FULL + st), C::TILE);
-                        for (int c = 0; c < C::NCB; c++)
-                            tma_load_3d_hint(sKV + st * C::TILE + c * C::CB, kv ? &tmV : &tmK, bar(C::B_KV_FULL + st),
-                                             c * 64, j * C::BN, bkv, keep);
-                        issued++;
                     }
                 }
                 if (!ok) {
-                    mbar_wait_drain(bar(C::B_Q), 0, 200000000ull);
+                    for (int back = 1; back <= min(q_issued, C::NQB); back++) {
+                        const int L = q_issued - back;
+                        mbar_wait_drain(bar(C::B_Q_FULL + L % C::NQB), (uint32_t)((L / C::NQB) & 1), 200000000ull);
+                    }
                     for (int back = 1; back <= min(issued, C::NSTAGE); back++) {
                         const int L = issued - back;
                         mbar_wait_drain(bar(C::B_KV_FULL + L % C::NSTAGE), (uint32_t)((L / C::NSTAGE) & 1), 200000000ull);
@@ -209,61 +258,86 @@ __global__ void __launch_bounds__(384, 1)
                     return mbar_wait(bar(C::B_KV_FULL + slot % C::NSTAGE), (uint32_t)((slot / C::NSTAGE) & 1), abort_flag);
                 };
                 auto release = [&](int slot) { tc_commit(bar(C::B_KV_EMPTY + slot % C::NSTAGE)); };
-                auto issue_qk = [&](int x, int slot) {
-                    const uint32_t sK = sKV + (slot % C::NSTAGE) * C::TILE;
-                    const uint32_t sQx = sQ + (uint32_t)x * C::TILE;
-    #pragma unroll
-                    for (int kk = 0; kk < D / 16; kk++) {
-                        const uint32_t off = (kk >> 2) * C::CB + (kk & 3) * 32;
-                        mma_ss(tmem + C::col_s(x), sdesc_sw128(sQx + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), ID_QK,
-                               kk > 0);
-                    }
-                    tc_commit(bar(C::B_S_FULL + x));
-                };
-                auto issue_pv = [&](int x, int slot, bool acc) {
-                    const uint32_t sV = sKV + (slot % C::NSTAGE) * C::TILE;
-    #pragma unroll
-                    for (int kk = 0; kk < C::BN / 16; kk++)
-                        mma_ts(tmem + C::col_o(x), tmem + C::col_s(x) + kk * 8, sdesc_sw128(sV + kk * 2048, C::CB, 1024),
-                               ID_PV, (acc || kk > 0) ? 1u : 0u);
-                };
-                bool ok = mbar_wait(bar(C::B_Q), 0, abort_flag);
-                if (ok) ok = wait_full(0);
-                if (ok) {
+                int slot0 = 0;          // ring slot of the current item's K(lo)
+                int cnt[2] = {0, 0};    // PVs issued per tile over the whole run (P_FULL phases)
+                bool ok = true;
+                int pass = 0;
+                for (; ok; pass++) {
+                    const int w = item_of(pass);
+                    if (w >= nitems) break;
+                    const Fwd2Item I = fwd2_item<C>(w, p);
+                    const int qb = pass % C::NQB;
+                    const uint32_t sQ = sQ0 + (uint32_t)qb * 2 * C::TILE;
+                    auto active = [&](int x, int j) -> bool {
+                        return x == 0 ? (j >= I.loA && j <= I.tA) : (I.hasB && j >= I.loB && j <= I.tB);
+                    };
+                    auto issue_qk = [&](int x, int slot) {
+                        const uint32_t sK = sKV + (slot % C::NSTAGE) * C::TILE;
+                        const uint32_t sQx = sQ + (uint32_t)x * C::TILE;
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; kk++) {
+                            const uint32_t off = (kk >> 2) * C::CB + (kk & 3) * 32;
+                            mma_ss(tmem + C::col_s(x), sdesc_sw128(opaque_u32(sQx) + off, 16, 1024),
+                                   sdesc_sw128(opaque_u32(sK) + off, 16, 1024), ID_QK, kk > 0);
+                        }
+                        tc_commit(bar(C::B_S_FULL + x));
+                    };
+                    auto issue_pv = [&](int x, int slot, bool acc) {
+                        const uint32_t sV = sKV + (slot % C::NSTAGE) * C::TILE;
+#pragma unroll
+                        for (int kk = 0; kk < C::BN / 16; kk++)
+                            mma_ts(tmem + C::col_o(x), tmem + C::col_s(x) + kk * 8,
+                                   sdesc_sw128(opaque_u32(sV) + kk * 2048, C::CB, 1024), ID_PV, (acc || kk > 0) ? 1u : 0u);
+                    };
+                    if (!(ok = mbar_wait(bar(C::B_Q_FULL + qb), (uint32_t)((pass / C::NQB) & 1), abort_flag))) break;
+                    if (!(ok = wait_full(slot0))) break;
                     tc_fence_after();
-                    if (active(0, lo)) issue_qk(0, 0);
-                    if (active(1, lo)) issue_qk(1, 0);
-                    release(0);
-                }
-                int cnt[2] = {0, 0};
-                for (int j = lo; ok && j <= hi; j++) {
-                    const int slotV = 2 * (j - lo) + 1, slotK = slotV + 1;
-                    if (!(ok = wait_full(slotV))) break;
-                    bool k_ready = false;
-                    for (int x = 0; x < 2 && ok; x++) {
-                        if (active(x, j)) {
-                            if (!(ok = mbar_wait(bar(C::B_P_FULL + x), (uint32_t)(cnt[x] & 1), abort_flag))) break;
-                            tc_fence_after();
-                            issue_pv(x, slotV, cnt[x] > 0);
-                            cnt[x]++;
-                        }
-                        if (j < hi && active(x, j + 1)) {
-                            if (!k_ready) {
-                                if (!(ok = wait_full(slotK))) break;
+                    if (active(0, I.lo)) issue_qk(0, slot0);
+                    if (active(1, I.lo)) issue_qk(1, slot0);
+                    release(slot0);
+                    bool first[2] = {true, true};
+                    for (int j = I.lo; ok && j <= I.hi; j++) {
+                        const int slotV = slot0 + 2 * (j - I.lo) + 1, slotK = slotV + 1;
+                        if (!(ok = wait_full(slotV))) break;
+                        bool k_ready = false;
+                        for (int x = 0; x < 2 && ok; x++) {
+                            if (active(x, j)) {
+                                if (!(ok = mbar_wait(bar(C::B_P_FULL + x), (uint32_t)(cnt[x] & 1), abort_flag))) break;
                                 tc_fence_after();
-                                k_ready = true;
+                                // the first PV of an item overwrites O_x: the previous
+                                // item's O_x must have been read out
+                                if (first[x] && pass > 0) {
+                                    if (!(ok = mbar_wait(bar(C::B_O_EMPTY + x), (uint32_t)((pass - 1) & 1), abort_flag)))
+                                        break;
+                                    tc_fence_after();
+                                }
+                                issue_pv(x, slotV, !first[x]);
+                                first[x] = false;
+                                cnt[x]++;
                             }
-                            issue_qk(x, slotK);
+                            if (j < I.hi && active(x, j + 1)) {
+                                if (!k_ready) {
+                                    if (!(ok = wait_full(slotK))) break;
+                                    tc_fence_after();
+                                    k_ready = true;
+                                }
+                                issue_qk(x, slotK);
+                            }
                         }
+                        if (!ok) break;
+                        release(slotV);
+                        if (j < I.hi) release(slotK);
                     }
                     if (!ok) break;
-                    release(slotV);
-                    if (j < hi) release(slotK);
+                    slot0 += 2 * (I.hi - I.lo + 1);
+                    // O_FINAL fires once every MMA of the item (and before) has completed
+                    tc_commit(bar(C::B_O_FINAL + 0));
+                    tc_commit(bar(C::B_O_FINAL + 1));
                 }
-                // O_FINAL fires once every MMA issued so far has completed
-                tc_commit(bar(C::B_O_FINAL + 0));
-                tc_commit(bar(C::B_O_FINAL + 1));
-                if (!ok) mbar_wait_drain(bar(C::B_O_FINAL + 0), 0, 200000000ull);
+                if (!ok) {
+                    tc_commit(bar(C::B_O_FINAL + 0));
+                    mbar_wait_drain(bar(C::B_O_FINAL + 0), (uint32_t)(pass & 1), 200000000ull);
+                }
             }
         }
     } else {
@@ -274,18 +348,23 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
         const uint32_t tS = tmem + lane_base + C::col_s(x);
         const uint32_t tO = tmem + lane_base + C::col_o(x);
-        const int q0 = x ? qB0 : qA0;
-        const int lox = x ? loB : loA, hix = x ? tB : tA;
-        const int qi = q0 + row;
-        const int r0 = q0 + 32 * (warp % 4);
         const bool cap = p.softcap > 0.0f;
         const uint64_t sl2x2 = f2_make(p.scale_log2, p.scale_log2);
-        float m = p.sink ? p.sink[hq] * kLog2e : -INFINITY, l = p.sink ? 1.0f : 0.0f;
-        float mraw = -INFINITY;  // row max of the (log2-unit) scores, the sink excluded
-        bool ok = (x == 0) || hasB;
-        if (ok) {
-            int cnt = 0;
-            for (int j = lox; j <= hix; j++, cnt++) {
+        int cnt = 0;  // KV tiles of this tile slot over the whole run (S_FULL phases)
+        bool ok = true;
+        for (int pass = 0; ok; pass++) {
+            const int w = item_of(pass);
+            if (w >= nitems) break;
+            const Fwd2Item I = fwd2_item<C>(w, p);
+            const int qb = pass % C::NQB;
+            const bool has = (x == 0) || I.hasB;
+            const int q0 = x ? I.qB0 : I.qA0;
+            const int lox = x ? I.loB : I.loA, hix = x ? I.tB : I.tA;
+            const int qi = q0 + row;
+            const int r0 = q0 + 32 * (warp % 4);
+            float m = p.sink ? p.sink[I.hq] * kLog2e : -INFINITY, l = p.sink ? 1.0f : 0.0f;
+            float mraw = -INFINITY;  // row max of the (log2-unit) scores, the sink excluded
+            for (int j = lox; has && j <= hix; j++, cnt++) {
                 const int k0 = j * C::BN;
                 if (!(ok = mbar_wait_warp(bar(C::B_S_FULL + x), (uint32_t)(cnt & 1), abort_flag))) break;
                 tc_fence_after();
@@ -333,9 +412,10 @@ __global__ void __launch_bounds__(384, 1)
                 const float m_new = (mx > m + 8.0f) ? mx : m;
                 const bool moved = (m_new != m);
                 const float factor = moved ? ex2_approx(m - m_new) : 1.0f;
-                if (__any_sync(0xffffffffu, moved && cnt > 0)) {
+                const bool later = j > lox;  // O_x holds PVs of this item
+                if (__any_sync(0xffffffffu, moved && later)) {
                     // O_x already holds every PV of this tile's earlier KV tiles
-                    const float f = (moved && cnt > 0) ? factor : 1.0f;
+                    const float f = (moved && later) ? factor : 1.0f;
                     const uint64_t f2 = f2_make(f, f);
 #pragma unroll 1
                     for (int c0 = 0; c0 < D; c0 += 32) {
@@ -392,53 +472,62 @@ __global__ void __launch_bounds__(384, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(C::B_P_FULL + x));
-                float r0, r1, r2, r3;
-                f2_split(rs[0], r0, r1);
+                float r0_, r1, r2, r3;
+                f2_split(rs[0], r0_, r1);
                 f2_split(rs[1], r2, r3);
-                l = l * factor + ((r0 + r1) + (r2 + r3));
+                l = l * factor + ((r0_ + r1) + (r2 + r3));
             }
-        }
-        if (ok) ok = mbar_wait_warp(bar(C::B_O_FINAL + x), 0, abort_flag);
-        if (ok && ((x == 0) || hasB)) {
+            if (!ok) break;
+            if (!(ok = mbar_wait_warp(bar(C::B_O_FINAL + x), (uint32_t)(pass & 1), abort_flag))) break;
             tc_fence_after();
-            const float inv_l = 1.0f / l;
-            const uint64_t inv2 = f2_make(inv_l, inv_l);
-            // Stage this tile's O (bf16) in its Q buffer, which every MMA has
-            // finished reading once O_FINAL fired, in the 128-byte-swizzled
-            // layout of the O tensor map, then store it with TMA (rows >= T
-            // are clipped by the map).
-            const uint32_t sO = sQ + (uint32_t)x * C::TILE;
+            // Stage this tile's O (bf16) in its Q buffer, which every MMA of the
+            // item has finished reading once O_FINAL fired, in the 128-byte-swizzled
+            // layout of the O tensor map, then store it with TMA (rows >= T are
+            // clipped by the map).
+            const uint32_t sO = sQ0 + (uint32_t)qb * 2 * C::TILE + (uint32_t)x * C::TILE;
+            if (has) {
+                const float inv_l = 1.0f / l;
+                const uint64_t inv2 = f2_make(inv_l, inv_l);
 #pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 32) {
-                uint32_t o[32];
-                tmem_ld32(tO + c0, o);
-                tmem_ld_wait(o);
-                uint32_t w[16];
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + c0, o);
+                    tmem_ld_wait(o);
+                    uint32_t w16[16];
 #pragma unroll
-                for (int i = 0; i < 16; i++) {
-                    float a, bb;
-                    f2_split(f2_mul(f2_make(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), inv2), a, bb);
-                    w[i] = pack_bf16x2(a, bb);
+                    for (int i = 0; i < 16; i++) {
+                        float a, bb;
+                        f2_split(f2_mul(f2_make(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), inv2), a, bb);
+                        w16[i] = pack_bf16x2(a, bb);
+                    }
+                    const uint32_t rowaddr = sO + (uint32_t)(c0 / 64) * C::CB + (uint32_t)row * 128u;
+                    const uint32_t ch0 = (uint32_t)((c0 % 64) / 8);
+#pragma unroll
+                    for (int i = 0; i < 4; i++)
+                        st_shared_v4(rowaddr + ((((ch0 + i) ^ (uint32_t)(row & 7))) << 4), w16[4 * i], w16[4 * i + 1],
+                                     w16[4 * i + 2], w16[4 * i + 3]);
                 }
-                const uint32_t rowaddr = sO + (uint32_t)(c0 / 64) * C::CB + (uint32_t)row * 128u;
-                const uint32_t ch0 = (uint32_t)((c0 % 64) / 8);
-#pragma unroll
-                for (int i = 0; i < 4; i++)
-                    st_shared_v4(rowaddr + ((((ch0 + i) ^ (uint32_t)(row & 7))) << 4), w[4 * i], w[4 * i + 1],
-                                 w[4 * i + 2], w[4 * i + 3]);
             }
-            fence_proxy_async_smem();
-            named_barrier_sync(1 + x, 128);
-            if (row == 0) {
-                for (int cb = 0; cb < C::NCB; cb++) tma_store_3d(&tmO, sO + cb * C::CB, cb * 64, q0, bh);
-                bulk_commit();
-                bulk_wait_read<0>();
+            // O_x is in registers / shared memory: the next item's PVs may overwrite it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_O_EMPTY + x));
+            if (has) {
+                fence_proxy_async_smem();
+                named_barrier_sync(1 + x, 128);
+                if (row == 0) {
+                    for (int cb = 0; cb < C::NCB; cb++) tma_store_3d(&tmO, sO + cb * C::CB, cb * 64, q0, I.bh);
+                    bulk_commit();
+                    bulk_wait_read<0>();
+                }
+                if (qi < p.T) p.lse[(size_t)I.bh * p.T + qi] = (m + __log2f(l)) * kLn2;
+                if (p.max_logit) {
+                    const float r = warp_max_f32(qi < p.T ? mraw * kLn2 : -INFINITY);
+                    if (lane == 0) atomic_max_f32(p.max_logit + I.bh, r);
+                }
             }
-            if (qi < p.T) p.lse[(size_t)bh * p.T + qi] = (m + __log2f(l)) * kLn2;
-            if (p.max_logit) {
-                const float r = warp_max_f32(qi < p.T ? mraw * kLn2 : -INFINITY);
-                if (lane == 0) atomic_max_f32(p.max_logit + bh, r);
-            }
+            // the Q buffer is free for the item NQB ahead once both tiles' stores read it
+            if (row == 0) mbar_arrive(bar(C::B_Q_EMPTY + qb));
         }
     }
 

@@ -332,6 +332,25 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, b
            (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// An operand base the compiler must treat as unknown at each use: without it the
+// descriptors of every unrolled MMA, loop-invariant over the steps, are
+// precomputed and held in registers (two 64-bit words per MMA), more than the
+// issuing warpgroup's register budget, and spill.
+__device__ __forceinline__ uint32_t opaque_u32(uint32_t x) {
+    asm volatile("" : "+r"(x));
+    return x;
+}
+
+// ------------------------------------------------------------- work schedule
+// Work items of CTA `cta` in a persistent grid of `grid` CTAs, the items listed
+// heaviest first: pass k takes item k * grid + cta on even passes and
+// k * grid + grid - 1 - cta on odd ones (a snake, so that a CTA given a heavy
+// item early gets a light one next). With grid = number of items there is one
+// pass and CTA c takes item c.
+__device__ __forceinline__ int snake_item(int pass, int cta, int grid) {
+    return pass * grid + ((pass & 1) ? grid - 1 - cta : cta);
+}
+
 // ---------------------------------------------------------------- float helpers
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;

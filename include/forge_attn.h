@@ -191,9 +191,12 @@ forge_status forge_attn_bwd_finalize(void *dq, int B, int Hq, int Hkv, int T, in
  * family table, DeepSeek V3 row: q.k over nope 128 + rope 64 = 192, values 128,
  * scale 1/sqrt(192) chosen by the caller). Layouts as above with D = Dk for q,
  * k, dq, dk and D = Dv for v, o, dO, dv. With Dk == Dv these are forge_attn_fwd /
- * forge_attn_bwd. Otherwise only (Dk, Dv) = (192, 128) is built: the forward in
- * bf16 (tensor cores) and f32 (CUDA cores), the backward in f32 (CUDA cores);
- * anything else returns FORGE_ERR_UNSUPPORTED (the bf16 backward included).
+ * forge_attn_bwd. Otherwise only (Dk, Dv) = (192, 128) is built, forward and
+ * backward, in bf16 (tensor cores) and f32 (CUDA cores); any other pair returns
+ * FORGE_ERR_UNSUPPORTED. The workspace of the backward holds Delta only
+ * (forge_attn_bwd_workspace_size_dkv bytes): both dtypes write dq directly. The
+ * bf16 backward runs a dK/dV kernel (one CTA per key tile and KV head) and a dQ
+ * kernel (one CTA per query tile and query head), each recomputing P.
  */
 forge_status forge_attn_fwd_dkv(const void *q, const void *k, const void *v, void *o, float *lse,
                                 int B, int Hq, int Hkv, int T, int Dk, int Dv, float scale, int window,

@@ -148,15 +148,22 @@ def test_ext_entry_points_reject_misaligned_extras():
 
 def test_dkv_entry_points_reject_unsupported_pairs_before_any_launch():
     A = 0x10000
-    # the bf16 backward with d_k != d_v has no tensor-core kernel yet
-    s = fa.forge_attn_bwd_dkv(A, A, A, A, A, A, A, A, A, 1, 2, 2, 128, 192, 128, 0.07, 0, 0.0, fa.FORGE_DTYPE_BF16,
-                              A, 1 << 20, 0)
-    assert s == fa.FORGE_ERR_UNSUPPORTED
+    # only (192, 128) is built; other pairs are refused in both dtypes
+    for dt in (fa.FORGE_DTYPE_BF16, fa.FORGE_DTYPE_F32):
+        s = fa.forge_attn_bwd_dkv(A, A, A, A, A, A, A, A, A, 1, 2, 2, 128, 128, 64, 0.07, 0, 0.0, dt, A, 1 << 20, 0)
+        assert s == fa.FORGE_ERR_UNSUPPORTED
+        assert fa.forge_attn_bwd_workspace_size_dkv(1, 2, 2, 128, 256, 128, dt) == 0
     s = fa.forge_attn_fwd_dkv(A, A, A, A, A, 1, 2, 2, 128, 96, 64, 0.1, 0, 0.0, fa.FORGE_DTYPE_F32, 0)
     assert s == fa.FORGE_ERR_UNSUPPORTED
-    assert fa.forge_attn_bwd_workspace_size_dkv(1, 2, 2, 128, 192, 128, fa.FORGE_DTYPE_BF16) == 0
-    # the f32 (192, 128) workspace holds Delta only
-    assert fa.forge_attn_bwd_workspace_size_dkv(1, 2, 2, 128, 192, 128, fa.FORGE_DTYPE_F32) >= 2 * 128 * 4
+    # the (192, 128) workspace holds Delta only, in both dtypes
+    for dt in (fa.FORGE_DTYPE_BF16, fa.FORGE_DTYPE_F32):
+        n = fa.forge_attn_bwd_workspace_size_dkv(1, 2, 2, 128, 192, 128, dt)
+        assert 2 * 128 * 4 <= n < 4096, n
+    # a workspace one byte short is refused before any launch
+    n = fa.forge_attn_bwd_workspace_size_dkv(1, 2, 2, 128, 192, 128, fa.FORGE_DTYPE_BF16)
+    s = fa.forge_attn_bwd_dkv(A, A, A, A, A, A, A, A, A, 1, 2, 2, 128, 192, 128, 0.07, 0, 0.0, fa.FORGE_DTYPE_BF16,
+                              A, n - 1, 0)
+    assert s == fa.FORGE_ERR_WORKSPACE
 
 
 def test_decode_validation_before_any_launch():

@@ -1,7 +1,7 @@
 """The N > 1 host path of bench.py on CPU: two gloo ranks, the max-over-ranks timing
 reduction, the barrier, the rank environment and the weak-scaling aggregate."""
 import os
-import socket
+import tempfile
 
 import torch.distributed as dist
 import torch.multiprocessing as mp
@@ -9,19 +9,20 @@ import torch.multiprocessing as mp
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _free_port():
-    with socket.socket() as s:
-        s.bind(("127.0.0.1", 0))
-        return s.getsockname()[1]
+def _rendezvous():
+    """A fresh file for the ranks to meet through (no TCP port to race for)."""
+    fd, path = tempfile.mkstemp(prefix="gloo_rdzv_")
+    os.close(fd)
+    os.unlink(path)
+    return "file://" + path
 
 
-def _worker(rank, world, port, out):
+def _worker(rank, world, init, out):
     import sys
     sys.path.insert(0, ROOT)
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
-                      LOCAL_RANK=str(rank))
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
     from datetime import timedelta
-    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    dist.init_process_group("gloo", init_method=init, rank=rank, world_size=world, timeout=timedelta(seconds=60))
     import bench
     w, r, l = bench.dist_env()
     t = bench.max_over_ranks(10.0 + 5.0 * rank, w)
@@ -33,8 +34,8 @@ def _worker(rank, world, port, out):
 def test_two_gloo_ranks_reduce_max_and_agree():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    init = _rendezvous()
+    procs = [ctx.Process(target=_worker, args=(r, 2, init, q)) for r in range(2)]
     for p in procs:
         p.start()
     res = sorted(q.get(timeout=120) for _ in procs)
@@ -59,16 +60,15 @@ def test_single_process_paths_and_aggregate():
     assert abs(one - 8.42e11 / 1.4e-3 / 1e12) < 1e-9
 
 
-def _worker_one_dies(rank, world, port, out):
+def _worker_one_dies(rank, world, init, out):
     """Rank 1 leaves between steps (after the group formed, before the next
     collective); rank 0's next collective must end with an error, not wait."""
     import sys
     import time
     sys.path.insert(0, ROOT)
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
-                      LOCAL_RANK=str(rank))
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
     from datetime import timedelta
-    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=10))
+    dist.init_process_group("gloo", init_method=init, rank=rank, world_size=world, timeout=timedelta(seconds=10))
     import bench
     bench.barrier(world)                      # both ranks reach the first step
     if rank == 1:
@@ -85,8 +85,8 @@ def _worker_one_dies(rank, world, port, out):
 def test_a_rank_that_leaves_ends_the_next_collective_with_an_error():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    port = _free_port()
-    procs = [ctx.Process(target=_worker_one_dies, args=(r, 2, port, q)) for r in range(2)]
+    init = _rendezvous()
+    procs = [ctx.Process(target=_worker_one_dies, args=(r, 2, init, q)) for r in range(2)]
     for p in procs:
         p.start()
     kind, secs = q.get(timeout=120)
