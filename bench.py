@@ -440,6 +440,9 @@ class Runner:
         self.scratch = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if self.flush else None
 
     def step(self, ev=None):
+        """One forward + backward. ev: None, 2 events (the step's bounds only, so
+        that consecutive kernels may overlap their launch) or 5 (between every
+        stage, for the per-kernel breakdown)."""
         import torch
         fa, w, sh = self.fa, self.w, self.stream.cuda_stream
         B, Hq, Hkv, T, D = w.B, w.Hq, w.Hkv, w.T, w.D
@@ -447,21 +450,22 @@ class Runner:
         if self.flush:
             with torch.cuda.stream(self.stream):
                 self.scratch.fill_(1)
+        full = ev is not None and len(ev) == 5
         if ev:
             ev[0].record(self.stream)
         s = fa.forge_attn_fwd(self.qd, self.kd, self.vd, self.o, self.lse, B, Hq, Hkv, T, D, sc, W, C, dt, sh)
-        if ev:
+        if full:
             ev[1].record(self.stream)
         s |= fa.forge_attn_bwd_preprocess(self.o, self.dOd, B, Hq, Hkv, T, D, dt, ws, nws, sh)
-        if ev:
+        if full:
             ev[2].record(self.stream)
         s |= fa.forge_attn_bwd_main(self.qd, self.kd, self.vd, self.lse, self.dOd, self.dq, self.dk, self.dv, B, Hq,
                                     Hkv, T, D, sc, W, C, dt, ws, nws, sh)
-        if ev:
+        if full:
             ev[3].record(self.stream)
         s |= fa.forge_attn_bwd_finalize(self.dq, B, Hq, Hkv, T, D, dt, ws, nws, sh)
         if ev:
-            ev[4].record(self.stream)
+            ev[-1].record(self.stream)
         if s != fa.FORGE_OK:
             raise fa.ForgeError(s, "step")
 
@@ -486,17 +490,21 @@ class Runner:
             per["step"].append(e[0].elapsed_time(e[4]))
         return per
 
-    def timed(self, steps):
-        """Per-step CUDA-event times (ms) of each stage, steps back to back."""
+    def timed(self, steps, per_kernel=True):
+        """Per-step CUDA-event times (ms), steps back to back: of each stage
+        (per_kernel) or of the whole step only ({"step": [...]})."""
         import torch
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+        n = 5 if per_kernel else 2
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n)] for _ in range(steps)]
         for i in range(steps):
             self.step(evs[i])
         torch.cuda.synchronize(self.dev)
         st = self.fa.forge_attn_check(self.stream.cuda_stream)
         if st != self.fa.FORGE_OK:
             raise self.fa.ForgeError(st, "timed run")
-        return self.per_kernel(evs)
+        if per_kernel:
+            return self.per_kernel(evs)
+        return {"step": [e[0].elapsed_time(e[1]) for e in evs]}
 
 
 def peak_for(kind, timed_s):
@@ -524,12 +532,15 @@ def per_workload_block(args, dev, stream):
         r = Runner(w, dev, stream, host_inputs=cache[key])
         r.warm(args.warmup)
         with torch.cuda.stream(stream):
-            per = r.timed(steps)
+            whole = r.timed(steps, per_kernel=False)  # step times, nothing between the kernels
+            per = r.timed(steps)                       # the per-stage breakdown
         fl_f, fl_b = flops_of(w)
         med = {k_: statistics.median(v_) for k_, v_ in per.items()}
-        peak, _ = peak_for("bf16_tflops", sum(per["step"]) * 1e-3)
+        med["step"] = statistics.median(whole["step"])
+        peak, _ = peak_for("bf16_tflops", sum(whole["step"]) * 1e-3)
         tf = (fl_f + fl_b) / (med["step"] * 1e-3) / 1e12
-        out[name] = {"ms_step": round(med["step"], 4), "ms_fwd": round(med["fwd"], 4),
+        out[name] = {"ms_step": round(med["step"], 4), "ms_step_sum_of_stages": round(statistics.median(per["step"]), 4),
+                     "ms_fwd": round(med["fwd"], 4),
                      "ms_bwd_main": round(med["bwd_main"], 4),
                      "ms_bwd_pre_fin": round(med["bwd_preprocess"] + med["bwd_finalize"], 4),
                      "tflops": round(tf, 2), "frac": round(tf / peak, 4),
@@ -578,7 +589,9 @@ def run_ours(args, w):
     launches_per_step = 4
     r.warm(args.warmup)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    # the timed steps carry events at their bounds only (nothing between the
+    # kernels of a step); the per-kernel breakdown is taken on K more steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     clk = ClockSampler(dev.index)
     barrier(world, dev)
     torch.cuda.synchronize(dev)
@@ -602,9 +615,11 @@ def run_ours(args, w):
     ms_local = start.elapsed_time(end)
     if r.flush:
         # the flushes sit between the timed kernels: time the kernels only
-        ms_local = sum(e[0].elapsed_time(e[4]) for e in evs)
+        ms_local = sum(e[0].elapsed_time(e[1]) for e in evs)
     ms = max_over_ranks(ms_local, world, dev)
-    per = Runner.per_kernel(evs)
+    step_times = [e[0].elapsed_time(e[1]) for e in evs]
+    with torch.cuda.stream(stream):
+        per = r.timed(args.steps)
     avg = {kname: sum(v) / len(v) for kname, v in per.items() if kname != "step"}
 
     # end to end through the same C ABI from pinned host buffers
@@ -682,7 +697,7 @@ def run_ours(args, w):
                     f"{r.working_set / 1e6:.0f} MB exceeds twice the 126 MB L2")},
         "pct_of_bf16_peak": round(100.0 * tflops / world / peak, 2),
         "kernels_ms": {k_: round(v_, 4) for k_, v_ in avg.items()},
-        "step_ms": spread(per["step"]),
+        "step_ms": spread(step_times),
         "kernels_ms_spread": {k_: spread(v_) for k_, v_ in per.items() if k_ != "step"},
         "roofline": {"kernel": kname, "bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,

@@ -58,6 +58,14 @@ int tpad_of(int T) { return (T + 127) / 128 * 128; }
 size_t delta_bytes(int B, int Hq, int T) { return round256(sizeof(float) * (size_t)B * Hq * T); }
 size_t acc_bytes(int B, int Hq, int T, int D) { return round256(sizeof(float) * (size_t)B * Hq * tpad_of(T) * D); }
 
+// Blocks of bwd_preprocess for `rows` rows of head dim D: 8 warps a block, each
+// warp 32 / min(32, D / 8) rows.
+unsigned preprocess_grid(long rows, int D) {
+    const int lpr = D / 8 < 32 ? D / 8 : 32;
+    const long per_block = 8L * (32 / lpr);
+    return (unsigned)((rows + per_block - 1) / per_block);
+}
+
 // ----------------------------------------------------------------- tensor maps
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -130,6 +138,26 @@ int sm_count() {
     return cache[dev];
 }
 
+// Launch with programmatic stream serialization: the kernel may start while the
+// previous kernel on the stream finishes (its prologue overlaps that kernel's
+// tail); the kernels launched this way call griddep_wait before touching global
+// memory, so the stream order of all memory effects is kept.
+template <typename... KArgs, typename... Args>
+forge_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                        Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...));
+}
+
 template <typename K>
 forge_status set_smem(K kernel, size_t bytes) {
     if (bytes <= 48 * 1024) return FORGE_OK;
@@ -176,7 +204,7 @@ forge_status fwd_tc(const void *q, const void *k, const void *v, void *o, float 
         // persistent: one CTA per SM (shared memory and TMEM allow no more)
         const long long items = (long long)((p.num_qt + 1) / 2) * B * Hq;
         const unsigned grid = (unsigned)(items < sm_count() ? items : sm_count());
-        fwd2_tc_kernel<D><<<grid, C2::THREADS, C2::SMEM, st>>>(mq, mk, mv, mo, p);
+        return launch_pdl(fwd2_tc_kernel<D>, dim3(grid), dim3(C2::THREADS), C2::SMEM, st, mq, mk, mv, mo, p);
     }
     return launch_status();
 }
@@ -271,8 +299,7 @@ forge_status bwd_tc(const void *q, const void *k, const void *v, const float *ls
     // more), each walking its share of the work items
     const long long items = (long long)p.num_kt * B * Hkv * C::NSPLIT;
     const unsigned grid = (unsigned)(items < sm_count() ? items : sm_count());
-    bwd_tc_kernel<D><<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, mdo, macc, p);
-    return launch_status();
+    return launch_pdl(bwd_tc_kernel<D>, dim3(grid), dim3(C::THREADS), C::SMEM, st, mq, mk, mv, mdo, macc, p);
 }
 
 // bf16 backward with separate key and value head dims: the dK/dV kernel (one CTA
@@ -549,19 +576,19 @@ forge_status forge_attn_bwd_preprocess(const void *o, const void *dO, int B, int
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     float *delta = static_cast<float *>(workspace);
     const long rows = (long)B * Hq * T;
-    const unsigned grid = (unsigned)((rows + 7) / 8);
+    const unsigned grid = preprocess_grid(rows, D);
     if (dtype == FORGE_DTYPE_BF16) {
         // the dq accumulator receives reductions: zero it in the same pass
         float *acc = reinterpret_cast<float *>(static_cast<char *>(workspace) + delta_bytes(B, Hq, T));
-        FORGE_DISPATCH_D(D, bwd_preprocess<__nv_bfloat16, kD><<<grid, 256, 0, st>>>(
-                                static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dO), delta,
-                                acc, rows, T, tpad_of(T));)
-        return launch_status();
+        FORGE_DISPATCH_D(D, return launch_pdl(bwd_preprocess<__nv_bfloat16, kD>, dim3(grid), dim3(256), 0, st,
+                                              static_cast<const __nv_bfloat16 *>(o),
+                                              static_cast<const __nv_bfloat16 *>(dO), delta, acc, rows, T,
+                                              tpad_of(T));)
     }
-    FORGE_DISPATCH_D(D, bwd_preprocess<float, kD><<<grid, 256, 0, st>>>(static_cast<const float *>(o),
-                                                                          static_cast<const float *>(dO), delta,
-                                                                          nullptr, rows, T, tpad_of(T));)
-    return launch_status();
+    FORGE_DISPATCH_D(D, return launch_pdl(bwd_preprocess<float, kD>, dim3(grid), dim3(256), 0, st,
+                                          static_cast<const float *>(o), static_cast<const float *>(dO), delta,
+                                          static_cast<float *>(nullptr), rows, T, tpad_of(T));)
+    return FORGE_ERR_UNSUPPORTED;
 }
 
 forge_status forge_attn_bwd_main(const void *q, const void *k, const void *v, const float *lse, const void *dO,
@@ -599,9 +626,9 @@ forge_status forge_attn_bwd_finalize(void *dq, int B, int Hq, int Hkv, int T, in
     const float *acc = reinterpret_cast<const float *>(static_cast<char *>(workspace) + delta_bytes(B, Hq, T));
     const long long total = (long long)B * Hq * T * (D / 8);
     const unsigned grid = (unsigned)((total + 255) / 256);
-    FORGE_DISPATCH_D(D, bwd_finalize_dq<kD><<<grid, 256, 0, st>>>(acc, static_cast<__nv_bfloat16 *>(dq),
-                                                                  (long)B * Hq, T, tpad_of(T));)
-    return launch_status();
+    FORGE_DISPATCH_D(D, return launch_pdl(bwd_finalize_dq<kD>, dim3(grid), dim3(256), 0, st, acc,
+                                          static_cast<__nv_bfloat16 *>(dq), (long)B * Hq, T, tpad_of(T));)
+    return FORGE_ERR_UNSUPPORTED;
 }
 
 forge_status forge_attn_bwd_ext(const void *q, const void *k, const void *v, const void *o, const float *lse,
@@ -709,13 +736,13 @@ forge_status forge_attn_bwd_dkv(const void *q, const void *k, const void *v, con
     float *delta = static_cast<float *>(workspace);
     const long rows = (long)B * Hq * T;
     if (dtype == FORGE_DTYPE_BF16) {
-        bwd_preprocess<__nv_bfloat16, 128><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
+        bwd_preprocess<__nv_bfloat16, 128><<<preprocess_grid(rows, 128), 256, 0, st>>>(
             static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dO), delta, nullptr, rows, T,
             tpad_of(T));
         if ((s = launch_status()) != FORGE_OK) return s;
         return bwd_tc_dkv<192, 128>(q, k, v, lse, dO, delta, dq, dk, dv, B, Hq, Hkv, T, scale, window, softcap, st);
     }
-    bwd_preprocess<float, 128><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
+    bwd_preprocess<float, 128><<<preprocess_grid(rows, 128), 256, 0, st>>>(
         static_cast<const float *>(o), static_cast<const float *>(dO), delta, nullptr, rows, T, tpad_of(T));
     if ((s = launch_status()) != FORGE_OK) return s;
     return bwd_simt<float, 192, 128>(q, k, v, lse, dO, delta, dq, dk, dv, B, Hq, Hkv, T, scale, window, softcap, st);

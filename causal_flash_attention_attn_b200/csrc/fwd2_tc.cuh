@@ -44,9 +44,11 @@ struct Fwd2Tc {
     // MMA issuer (warp 9), two idle warps. Launched at 168 registers a thread
     // (three warps per SM sub-partition); warpgroup 2 gives back down to
     // REG_CTRL so the softmax warpgroups can grow to REG_SOFTMAX:
-    // 4 * (168 - REG_CTRL) = 8 * (REG_SOFTMAX - 168).
+    // 4 * (168 - REG_CTRL) >= 8 * (REG_SOFTMAX - 168). The work-item loop needs
+    // REG_CTRL >= 64 (72 at head dim 64) for the producer and MMA warps to run
+    // without spills.
     static constexpr int THREADS = 384;
-    static constexpr int REG_LAUNCH = 168, REG_CTRL = 72, REG_SOFTMAX = 216;
+    static constexpr int REG_LAUNCH = 168, REG_CTRL = D == 64 ? 72 : 64, REG_SOFTMAX = 216;
     static_assert(4 * (REG_LAUNCH - REG_CTRL) >= 8 * (REG_SOFTMAX - REG_LAUNCH), "register split");
     static_assert((2 * REG_SOFTMAX + REG_CTRL) * 32 <= 16384, "registers of one SM sub-partition");
     static constexpr uint32_t TMEM_COLS = 512;
@@ -194,6 +196,7 @@ __global__ void __launch_bounds__(384, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    griddep_wait();  // the previous kernel's writes (q, k, v, max_logit) are visible
 
     if (warp >= 8) {
         setmaxnreg_dec<C::REG_CTRL>();
@@ -207,6 +210,8 @@ __global__ void __launch_bounds__(384, 1)
                     const int w = item_of(pass);
                     if (w >= nitems) break;
                     const Fwd2Item I = fwd2_item<C>(w, p);
+                    // this CTA's last item: the next kernel may start launching
+                    if (item_of(pass + 1) >= nitems) griddep_launch_dependents();
                     // the item's queries once both O stores of the item that used this
                     // buffer NQB items ago have read it
                     const int qb = pass % C::NQB;
@@ -259,7 +264,7 @@ __global__ void __launch_bounds__(384, 1)
                 };
                 auto release = [&](int slot) { tc_commit(bar(C::B_KV_EMPTY + slot % C::NSTAGE)); };
                 int slot0 = 0;          // ring slot of the current item's K(lo)
-                int cnt[2] = {0, 0};    // PVs issued per tile over the whole run (P_FULL phases)
+                int cnt0 = 0, cnt1 = 0;  // PVs issued per tile over the whole run (P_FULL phases)
                 bool ok = true;
                 int pass = 0;
                 for (; ok; pass++) {
@@ -268,54 +273,56 @@ __global__ void __launch_bounds__(384, 1)
                     const Fwd2Item I = fwd2_item<C>(w, p);
                     const int qb = pass % C::NQB;
                     const uint32_t sQ = sQ0 + (uint32_t)qb * 2 * C::TILE;
-                    auto active = [&](int x, int j) -> bool {
-                        return x == 0 ? (j >= I.loA && j <= I.tA) : (I.hasB && j >= I.loB && j <= I.tB);
-                    };
+                    // KV range of each tile ([lo_x, hi_x]; empty for a missing tile B)
+                    const int lo0 = I.loA, hi0 = I.tA, lo1 = I.loB, hi1 = I.hasB ? I.tB : -1;
                     auto issue_qk = [&](int x, int slot) {
-                        const uint32_t sK = sKV + (slot % C::NSTAGE) * C::TILE;
-                        const uint32_t sQx = sQ + (uint32_t)x * C::TILE;
+                        const uint64_t dq = sdesc_sw128(opaque_u32(sQ + (uint32_t)x * C::TILE), 16, 1024);
+                        const uint64_t dk = sdesc_sw128(opaque_u32(sKV + (slot % C::NSTAGE) * C::TILE), 16, 1024);
 #pragma unroll
                         for (int kk = 0; kk < D / 16; kk++) {
                             const uint32_t off = (kk >> 2) * C::CB + (kk & 3) * 32;
-                            mma_ss(tmem + C::col_s(x), sdesc_sw128(opaque_u32(sQx) + off, 16, 1024),
-                                   sdesc_sw128(opaque_u32(sK) + off, 16, 1024), ID_QK, kk > 0);
+                            mma_ss(tmem + C::col_s(x), sdesc_step(dq, off), sdesc_step(dk, off), ID_QK, kk > 0);
                         }
                         tc_commit(bar(C::B_S_FULL + x));
                     };
                     auto issue_pv = [&](int x, int slot, bool acc) {
-                        const uint32_t sV = sKV + (slot % C::NSTAGE) * C::TILE;
+                        const uint64_t dv = sdesc_sw128(opaque_u32(sKV + (slot % C::NSTAGE) * C::TILE), C::CB, 1024);
 #pragma unroll
                         for (int kk = 0; kk < C::BN / 16; kk++)
-                            mma_ts(tmem + C::col_o(x), tmem + C::col_s(x) + kk * 8,
-                                   sdesc_sw128(opaque_u32(sV) + kk * 2048, C::CB, 1024), ID_PV, (acc || kk > 0) ? 1u : 0u);
+                            mma_ts(tmem + C::col_o(x), tmem + C::col_s(x) + kk * 8, sdesc_step(dv, kk * 2048), ID_PV,
+                                   (acc || kk > 0) ? 1u : 0u);
                     };
                     if (!(ok = mbar_wait(bar(C::B_Q_FULL + qb), (uint32_t)((pass / C::NQB) & 1), abort_flag))) break;
                     if (!(ok = wait_full(slot0))) break;
                     tc_fence_after();
-                    if (active(0, I.lo)) issue_qk(0, slot0);
-                    if (active(1, I.lo)) issue_qk(1, slot0);
+                    if (I.lo >= lo0 && I.lo <= hi0) issue_qk(0, slot0);
+                    if (I.lo >= lo1 && I.lo <= hi1) issue_qk(1, slot0);
                     release(slot0);
-                    bool first[2] = {true, true};
+                    bool first0 = true, first1 = true;
                     for (int j = I.lo; ok && j <= I.hi; j++) {
                         const int slotV = slot0 + 2 * (j - I.lo) + 1, slotK = slotV + 1;
                         if (!(ok = wait_full(slotV))) break;
                         bool k_ready = false;
-                        for (int x = 0; x < 2 && ok; x++) {
-                            if (active(x, j)) {
-                                if (!(ok = mbar_wait(bar(C::B_P_FULL + x), (uint32_t)(cnt[x] & 1), abort_flag))) break;
+#pragma unroll
+                        for (int x = 0; x < 2; x++) {
+                            const int lox = x ? lo1 : lo0, hix = x ? hi1 : hi0;
+                            bool &first = x ? first1 : first0;
+                            int &cx = x ? cnt1 : cnt0;
+                            if (ok && j >= lox && j <= hix) {
+                                if (!(ok = mbar_wait(bar(C::B_P_FULL + x), (uint32_t)(cx & 1), abort_flag))) break;
                                 tc_fence_after();
                                 // the first PV of an item overwrites O_x: the previous
                                 // item's O_x must have been read out
-                                if (first[x] && pass > 0) {
+                                if (first && pass > 0) {
                                     if (!(ok = mbar_wait(bar(C::B_O_EMPTY + x), (uint32_t)((pass - 1) & 1), abort_flag)))
                                         break;
                                     tc_fence_after();
                                 }
-                                issue_pv(x, slotV, !first[x]);
-                                first[x] = false;
-                                cnt[x]++;
+                                issue_pv(x, slotV, !first);
+                                first = false;
+                                cx++;
                             }
-                            if (j < I.hi && active(x, j + 1)) {
+                            if (ok && j < I.hi && j + 1 >= lox && j + 1 <= hix) {
                                 if (!k_ready) {
                                     if (!(ok = wait_full(slotK))) break;
                                     tc_fence_after();

@@ -341,6 +341,22 @@ __device__ __forceinline__ uint32_t opaque_u32(uint32_t x) {
     return x;
 }
 
+// ------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while the
+// kernel before it on the stream is finishing. griddep_wait blocks until that
+// kernel has completed and its memory operations are visible: every such kernel
+// calls it before its first global-memory access (read or write). Before it,
+// only shared memory, TMEM and the kernel parameters may be touched.
+// griddep_launch_dependents tells the hardware that the next kernel of the
+// stream may begin launching once every CTA of this grid has said so (or exited).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+// Descriptor of the operand `bytes` further on: the start-address field holds
+// address >> 4 in 14 bits and shared-memory addresses stay below 2^18, so the
+// field never carries into its neighbour and a plain 64-bit add is exact.
+__device__ __forceinline__ uint64_t sdesc_step(uint64_t desc, uint32_t bytes) { return desc + (uint64_t)(bytes >> 4); }
+
 // ------------------------------------------------------------- work schedule
 // Work items of CTA `cta` in a persistent grid of `grid` CTAs, the items listed
 // heaviest first: pass k takes item k * grid + cta on even passes and

@@ -60,9 +60,11 @@ def test_single_process_paths_and_aggregate():
     assert abs(one - 8.42e11 / 1.4e-3 / 1e12) < 1e-9
 
 
-def _worker_one_dies(rank, world, init, out):
+def _worker_one_dies(rank, world, init, out, passed):
     """Rank 1 leaves between steps (after the group formed, before the next
-    collective); rank 0's next collective must end with an error, not wait."""
+    collective); rank 0's next collective must end with an error, not wait.
+    Rank 1 leaves only once rank 0 has come out of the barrier (`passed`), so
+    that the collective that meets the missing rank is the next one."""
     import sys
     import time
     sys.path.insert(0, ROOT)
@@ -72,13 +74,19 @@ def _worker_one_dies(rank, world, init, out):
     import bench
     bench.barrier(world)                      # both ranks reach the first step
     if rank == 1:
+        passed.wait(60)
         os._exit(0)                            # leaves with nothing in flight
+    passed.set()
+    time.sleep(0.5)                            # rank 1 is gone before the next collective
     t0 = time.time()
     try:
         bench.max_over_ranks(1.0, world)
         out.put(("no error", time.time() - t0))
     except Exception as e:                     # gloo reports the lost peer
         out.put((type(e).__name__, time.time() - t0))
+    # a queue hands its items to a feeder thread: flush it before the hard exit
+    out.close()
+    out.join_thread()
     os._exit(0)
 
 
@@ -86,7 +94,8 @@ def test_a_rank_that_leaves_ends_the_next_collective_with_an_error():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     init = _rendezvous()
-    procs = [ctx.Process(target=_worker_one_dies, args=(r, 2, init, q)) for r in range(2)]
+    passed = ctx.Event()
+    procs = [ctx.Process(target=_worker_one_dies, args=(r, 2, init, q, passed)) for r in range(2)]
     for p in procs:
         p.start()
     kind, secs = q.get(timeout=120)
