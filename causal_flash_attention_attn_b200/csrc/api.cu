@@ -201,9 +201,15 @@ forge_status fwd_tc(const void *q, const void *k, const void *v, void *o, float 
             return FORGE_ERR_CUDA;
         }
         if (set_smem(fwd2_tc_kernel<D>, C2::SMEM) != FORGE_OK) return FORGE_ERR_CUDA;
-        // persistent: one CTA per SM (shared memory and TMEM allow no more)
+        // Persistent (one CTA per SM, the most shared memory and TMEM allow) for
+        // short sequences, whose items are too light to amortise a CTA's start;
+        // one CTA per item otherwise, where the hardware's dynamic placement
+        // balances the uneven items better than a static order (measured forward
+        // times: 16K global layer 2.57 ms persistent against 2.40 ms one CTA per
+        // item; T = 512, head dim 64: 0.039 ms persistent against 0.045 ms).
         const long long items = (long long)((p.num_qt + 1) / 2) * B * Hq;
-        const unsigned grid = (unsigned)(items < sm_count() ? items : sm_count());
+        const bool persistent = p.num_qt <= 8;
+        const unsigned grid = (unsigned)(persistent && items > sm_count() ? sm_count() : items);
         return launch_pdl(fwd2_tc_kernel<D>, dim3(grid), dim3(C2::THREADS), C2::SMEM, st, mq, mk, mv, mo, p);
     }
     return launch_status();

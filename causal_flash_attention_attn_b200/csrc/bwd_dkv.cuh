@@ -21,8 +21,9 @@
 //
 // bwd_dq_tc_kernel -- one CTA per (query tile of 128 rows, batch, query head),
 //   Q and dO resident, dQ in TMEM over the key tiles the rows see (64 keys a
-//   tile, K through a three-slot ring since dQ(j) reads K(j) after S(j), V
-//   through a two-slot ring). Two softmax warpgroups take alternate key tiles,
+//   tile, K through a four-slot ring since dQ(j) reads K(j) after S(j), V
+//   through a two-slot ring, each ring with its own producer warp). Two softmax
+//   warpgroups take alternate key tiles,
 //   each with its own 64 TMEM columns:
 //     S  = Q K^T   -> buffer;  P, the dS factor g in registers
 //     dP = dO V^T  -> buffer (over S)
@@ -38,6 +39,25 @@
 #include "sm100.cuh"
 
 namespace forge {
+
+// Block b of a grid of ntile x nhead blocks -> (tile index heaviest first, head),
+// the heads taken in groups of kHeadGroup: all tiles of a group's heads before
+// the next group, so the operands a head shares across its tiles (K and V in
+// the dQ kernel, Q and dO in the dK/dV kernel) are read while still in L2.
+constexpr int kHeadGroup = 8;
+__device__ __forceinline__ void grouped_block(int blk, int ntile, int nhead, int &tile_from_heavy, int &head) {
+    const int full = nhead / kHeadGroup;
+    const int per = ntile * kHeadGroup;
+    if (blk < full * per) {
+        const int g = blk / per, r = blk % per;
+        tile_from_heavy = r / kHeadGroup;
+        head = g * kHeadGroup + r % kHeadGroup;
+    } else {
+        const int r = blk - full * per, gs = nhead - full * kHeadGroup;
+        tile_from_heavy = r / gs;
+        head = full * kHeadGroup + r % gs;
+    }
+}
 
 // ------------------------------------------------------------ dK / dV kernel
 template <int DK, int DV>
@@ -93,9 +113,8 @@ __global__ void __launch_bounds__(384, 1)
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     // work item: key tile n (heaviest = smallest n first), batch b, KV head
-    const int per_n = p.B * p.Hkv;
-    const int n = blockIdx.x / per_n;
-    const int bkv = blockIdx.x % per_n;
+    int n, bkv;
+    grouped_block((int)blockIdx.x, p.num_kt, p.B * p.Hkv, n, bkv);
     const int b = bkv / p.Hkv, hkv = bkv % p.Hkv;
     const int G = p.Hq / p.Hkv;
     const int k0 = n * C::BN;
@@ -369,16 +388,18 @@ struct BwdQTc {
     static constexpr uint32_t CBN = 64 * 128;             // column block of a 64-row tile
     static constexpr uint32_t TQ = NCBK * CBQ, TDO = NCBV * CBQ;
     static constexpr uint32_t TKT = NCBK * CBN, TVT = NCBV * CBN;
-    static constexpr int KST = 3, VST = 2;                // ring slots
+    static constexpr int KST = 4, VST = 2;                // ring slots
     static constexpr uint32_t OFF_Q = 0, OFF_DO = TQ, OFF_K = TQ + TDO, OFF_V = OFF_K + KST * TKT;
     static constexpr uint32_t TILES = OFF_V + VST * TVT;
     static constexpr uint32_t OFF_TMEM_SLOT = 240, OFF_ABORT = 244;
     static constexpr uint32_t CTRL = 256;
     static constexpr uint32_t SMEM = 1024 + TILES + CTRL;
     // warps 0-3 softmax of the even key tiles, 4-7 of the odd ones (one query
-    // row a thread), warp 8 loads, warp 9 issues MMAs and owns TMEM
+    // row a thread), warp 8 loads Q, dO and the K ring, warp 9 issues MMAs and
+    // owns TMEM, warp 10 loads the V ring (so that a V load never waits behind a
+    // K load held up by a ring slot that a later dQ product frees)
     static constexpr int THREADS = 384;
-    static constexpr int W_LOAD = 8, W_MMA = 9;
+    static constexpr int W_LOAD = 8, W_MMA = 9, W_LOAD_V = 10;
     static constexpr uint32_t COL_DQ = 128;
     static constexpr uint32_t col_buf(int x) { return (uint32_t)(x * 64); }
     static constexpr uint32_t TMEM_COLS = 512;
@@ -408,9 +429,9 @@ __global__ void __launch_bounds__(384, 1)
     auto bar = [&](int i) -> uint32_t { return ctrl + 8u * (uint32_t)i; };
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int nbh = p.B * p.Hq;
-    const int qt = p.num_qt - 1 - (int)(blockIdx.x / nbh);  // heaviest tiles first
-    const int bh = blockIdx.x % nbh;
+    int qt, bh;
+    grouped_block((int)blockIdx.x, p.num_qt, p.B * p.Hq, qt, bh);
+    qt = p.num_qt - 1 - qt;  // heaviest tiles first
     const int b = bh / p.Hq, hq = bh % p.Hq;
     const int bkv = b * p.Hkv + hq / (p.Hq / p.Hkv);
     const int W = p.window;
@@ -454,52 +475,39 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == C::W_LOAD) {
-        // ------------------------------------------------------------ producer
+    if (warp == C::W_LOAD || warp == C::W_LOAD_V) {
+        // ------------------------------------------------------------ producers
         if (lane == 0) {
             const uint64_t keep = policy_evict_last();
-            mbar_arrive_expect_tx(bar(C::B_QD), C::TQ + C::TDO);
-            for (int c = 0; c < C::NCBK; c++) tma_load_3d(sQ + c * C::CBQ, &tmQ, bar(C::B_QD), c * 64, q0, bh);
-            for (int c = 0; c < C::NCBV; c++) tma_load_3d(sdO + c * C::CBQ, &tmdO, bar(C::B_QD), c * 64, q0, bh);
-            // K(u) and V(u) in the order of first use: K0 K1 V0 K2 V1 K3 V2 ...
-            // (K(u + 1) is needed before V(u): S(u + 1) is issued early)
-            int nk = 0, nv = 0;
+            const bool kq = warp == C::W_LOAD;  // Q, dO and K; else V
+            if (kq) {
+                mbar_arrive_expect_tx(bar(C::B_QD), C::TQ + C::TDO);
+                for (int c = 0; c < C::NCBK; c++) tma_load_3d(sQ + c * C::CBQ, &tmQ, bar(C::B_QD), c * 64, q0, bh);
+                for (int c = 0; c < C::NCBV; c++) tma_load_3d(sdO + c * C::CBQ, &tmdO, bar(C::B_QD), c * 64, q0, bh);
+            }
+            // K(u) (or V(u)) for u = 0 .. n-1, each ring slot reused once the
+            // product that last read it has completed
+            const int nst = kq ? C::KST : C::VST;
+            const int B_FULL = kq ? C::B_K_FULL : C::B_V_FULL, B_EMPTY = kq ? C::B_K_EMPTY : C::B_V_EMPTY;
+            const uint32_t base = kq ? sK0 : sV0, tile = kq ? C::TKT : C::TVT;
+            const int ncb = kq ? C::NCBK : C::NCBV;
+            const CUtensorMap *map = kq ? &tmK : &tmV;
+            int issued = 0;
             bool ok = true;
-            auto load_k = [&]() -> bool {
-                const int s = nk % C::KST;
-                if (!mbar_wait(bar(C::B_K_EMPTY + s), (uint32_t)(((nk / C::KST) & 1) ^ 1), abort_flag)) return false;
-                mbar_arrive_expect_tx(bar(C::B_K_FULL + s), C::TKT);
-                for (int c = 0; c < C::NCBK; c++)
-                    tma_load_3d_hint(sK0 + s * C::TKT + c * C::CBN, &tmK, bar(C::B_K_FULL + s), c * 64,
-                                     (lo + nk) * C::BN, bkv, keep);
-                nk++;
-                return true;
-            };
-            auto load_v = [&]() -> bool {
-                const int s = nv % C::VST;
-                if (!mbar_wait(bar(C::B_V_EMPTY + s), (uint32_t)(((nv / C::VST) & 1) ^ 1), abort_flag)) return false;
-                mbar_arrive_expect_tx(bar(C::B_V_FULL + s), C::TVT);
-                for (int c = 0; c < C::NCBV; c++)
-                    tma_load_3d_hint(sV0 + s * C::TVT + c * C::CBN, &tmV, bar(C::B_V_FULL + s), c * 64,
-                                     (lo + nv) * C::BN, bkv, keep);
-                nv++;
-                return true;
-            };
-            ok = load_k();
-            if (ok && n > 1) ok = load_k();
-            for (int u = 0; ok && u < n; u++) {
-                ok = load_v();
-                if (ok && u + 2 < n) ok = load_k();
+            for (int u = 0; u < n; u++) {
+                const int s = u % nst;
+                if (!(ok = mbar_wait(bar(B_EMPTY + s), (uint32_t)(((u / nst) & 1) ^ 1), abort_flag))) break;
+                mbar_arrive_expect_tx(bar(B_FULL + s), tile);
+                for (int c = 0; c < ncb; c++)
+                    tma_load_3d_hint(base + s * tile + c * C::CBN, map, bar(B_FULL + s), c * 64, (lo + u) * C::BN, bkv,
+                                     keep);
+                issued++;
             }
             if (!ok) {
-                mbar_wait_drain(bar(C::B_QD), 0, 200000000ull);
-                for (int back = 1; back <= min(nk, C::KST); back++) {
-                    const int L = nk - back;
-                    mbar_wait_drain(bar(C::B_K_FULL + L % C::KST), (uint32_t)((L / C::KST) & 1), 200000000ull);
-                }
-                for (int back = 1; back <= min(nv, C::VST); back++) {
-                    const int L = nv - back;
-                    mbar_wait_drain(bar(C::B_V_FULL + L % C::VST), (uint32_t)((L / C::VST) & 1), 200000000ull);
+                if (kq) mbar_wait_drain(bar(C::B_QD), 0, 200000000ull);
+                for (int back = 1; back <= min(issued, nst); back++) {
+                    const int L = issued - back;
+                    mbar_wait_drain(bar(B_FULL + L % nst), (uint32_t)((L / nst) & 1), 200000000ull);
                 }
             }
         }
