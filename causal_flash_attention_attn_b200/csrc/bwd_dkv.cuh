@@ -556,25 +556,44 @@ __global__ void __launch_bounds__(384, 1)
                            ID_DQ, (u > 0 || kk > 0) ? 1u : 0u);
                 tc_commit(bar(C::B_K_EMPTY + s));
             };
-            auto wait_ds = [&](int u) -> bool {
-                if (!mbar_wait(bar(C::B_DS + (u & 1)), (uint32_t)((u >> 1) & 1), abort_flag)) return false;
-                tc_fence_after();
-                return true;
-            };
+            // Issue whichever product is ready, each kind in its own order:
+            //   S(ns)  once K(ns) has landed and dQ(ns - 2) (the last reader of
+            //          buffer ns % 2) has been issued;
+            //   dP(np) once S(np) is issued, phase A of tile np is done and V(np)
+            //          has landed;
+            //   dQ(nq) once dP(nq) is issued and phase B of tile nq is done.
+            // The two softmax warpgroups then never wait for each other's pace.
             bool ok = mbar_wait(bar(C::B_QD), 0, abort_flag);
-            if (ok) ok = issue_s(0);
-            if (ok && n > 1) ok = issue_s(1);
-            for (int u = 0; ok && u < n; u++) {
-                if (!(ok = mbar_wait(bar(C::B_PA + (u & 1)), (uint32_t)((u >> 1) & 1), abort_flag))) break;
-                tc_fence_after();
-                if (!(ok = issue_dp(u))) break;
-                if (u >= 1) {
-                    if (!(ok = wait_ds(u - 1))) break;
-                    issue_dq(u - 1);
-                    if (u + 1 < n && !(ok = issue_s(u + 1))) break;
+            int ns = 0, np = 0, nq = 0;
+            uint64_t t_last = globaltimer_ns();
+            while (ok && nq < n) {
+                bool progress = false;
+                if (nq < np && mbar_try_wait(bar(C::B_DS + (nq & 1)), (uint32_t)((nq >> 1) & 1))) {
+                    tc_fence_after();
+                    issue_dq(nq++);
+                    progress = true;
+                }
+                if (np < ns && mbar_try_wait(bar(C::B_PA + (np & 1)), (uint32_t)((np >> 1) & 1)) &&
+                    mbar_try_wait(bar(C::B_V_FULL + np % C::VST), (uint32_t)((np / C::VST) & 1))) {
+                    tc_fence_after();
+                    ok = issue_dp(np++);  // its V wait returns at once
+                    progress = true;
+                }
+                if (ok && ns < n && nq >= ns - 1 &&
+                    mbar_try_wait(bar(C::B_K_FULL + ns % C::KST), (uint32_t)((ns / C::KST) & 1))) {
+                    ok = issue_s(ns++);   // its K wait returns at once
+                    progress = true;
+                }
+                if (progress) {
+                    t_last = globaltimer_ns();
+                } else if (*abort_flag) {
+                    ok = false;
+                } else if (globaltimer_ns() - t_last > kWaitLimitNs) {
+                    record_status(kStatusTimeout);
+                    *abort_flag = 1;
+                    ok = false;
                 }
             }
-            if (ok && (ok = wait_ds(n - 1))) issue_dq(n - 1);
             // DQ_DONE fires once every MMA issued so far has completed
             tc_commit(bar(C::B_DQ_DONE));
             if (!ok) mbar_wait_drain(bar(C::B_DQ_DONE), 0, 200000000ull);

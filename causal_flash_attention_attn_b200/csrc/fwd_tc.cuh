@@ -6,14 +6,18 @@
 // cost follows the window size, as in the pages' flash kernels, which skip KV
 // blocks outside the window (src/nn/attention.h commit log, Wave 2).
 //
-// Roles (192 threads):
-//   warp 4   TMA producer: Q once, then K/V tiles through an NSTAGE ring in the
+// Roles (320 threads):
+//   warp 8   TMA producer: Q once, then K/V tiles through an NSTAGE ring in the
 //            order the MMA warp consumes them: K0 K1 | V0 K2 | V1 K3 | ...
-//   warp 5   MMA issuer (one thread) and TMEM owner (512 columns):
+//   warp 9   MMA issuer (one thread) and TMEM owner (512 columns):
 //            S_b = Q K_j^T into S buffer b = j % 2 (128 columns each), then
 //            O += P_j V_j with P read from tensor memory (it overwrites S_b).
 //            Two S buffers let QK^T of tile j+1 run while tile j is in softmax.
-//   warps 0-3 softmax + epilogue, one thread per query row (TMEM lane):
+//   warps 0-7 softmax + epilogue: warps w and w + 4 share the TMEM lanes (query
+//            rows) 32 (w % 4).. and split each row's 128 scores into halves w / 4,
+//            so two warps per SM sub-partition share the exponential (and tanh)
+//            work; they exchange only the row max of each tile (shared memory,
+//            one named barrier per pair) and add their row sums at the end.
 //            s = scale*S (or cap*tanh(scale*S/cap)), masked only on tiles that
 //            straddle the diagonal or the window edge; online softmax in base 2.
 //            The running max is only moved when a row max exceeds it by more
@@ -44,8 +48,12 @@ struct FwdTc {
     static constexpr uint32_t SLOT = TILEK > TILEV ? TILEK : TILEV;  // a ring slot holds a K or a V tile
     static constexpr int NSTAGE = DK == 256 ? 2 : (DK == 192 ? 3 : (DK == 128 ? 4 : 6));
     static constexpr uint32_t CTRL = 1024;                // barriers, TMEM slot, abort flag
-    static constexpr uint32_t SMEM = CTRL + TILEK + SLOT * NSTAGE + 1024;
-    static constexpr int THREADS = 192;
+    // after the tiles: the row-max exchange of the two column halves,
+    // [2 tile parities][2 halves][128 rows] f32, and the halves' row sums [2][128]
+    static constexpr uint32_t XCH = 2 * 2 * 128 * 4 + 2 * 128 * 4;
+    static constexpr uint32_t SMEM = CTRL + TILEK + SLOT * NSTAGE + 1024 + XCH;
+    static constexpr int THREADS = 320;
+    static constexpr int W_LOAD = 8, W_MMA = 9;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O = 256;
     // barrier indices
@@ -109,6 +117,37 @@ __device__ __forceinline__ float fwd_exp_tile(uint32_t (&s)[4][32], uint32_t (&p
     return (rs[0] + rs[1]) + (rs[2] + rs[3]);
 }
 
+// The same for one half of a tile row (64 columns held as 2 x 32 registers);
+// PSPLIT residuals are left in s. Returns the half's row sum of p.
+template <bool CAP, bool EMU, bool PSPLIT>
+__device__ __forceinline__ float fwd_exp_half(uint32_t (&s)[2][32], uint32_t (&pk)[32], float sl2, float msub) {
+    float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int c = 0; c < 32; c++) {
+        const float x0 = __uint_as_float(s[(2 * c) >> 5][(2 * c) & 31]);
+        const float x1 = __uint_as_float(s[(2 * c + 1) >> 5][(2 * c + 1) & 31]);
+        const float y0 = CAP ? x0 - msub : fmaf(x0, sl2, -msub);
+        const float y1 = CAP ? x1 - msub : fmaf(x1, sl2, -msub);
+        float p0, p1;
+        if (EMU && (c & 3) == 3) {
+            p0 = exp2_poly(y0);
+            p1 = exp2_poly(y1);
+        } else {
+            p0 = ex2_approx(y0);
+            p1 = ex2_approx(y1);
+        }
+        rs[c & 3] += p0 + p1;
+        pk[c] = pack_bf16x2(p0, p1);
+        if constexpr (PSPLIT) {
+            const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(&pk[c]);
+            const float2 hf = __bfloat1622float2(hi);
+            s[(2 * c) >> 5][(2 * c) & 31] = __float_as_uint(p0 - hf.x);
+            s[(2 * c + 1) >> 5][(2 * c + 1) & 31] = __float_as_uint(p1 - hf.y);
+        }
+    }
+    return (rs[0] + rs[1]) + (rs[2] + rs[3]);
+}
+
 struct FwdParams {
     __nv_bfloat16 *o;
     float *lse;
@@ -128,7 +167,7 @@ struct FwdParams {
 };
 
 template <int DK, int DV = DK>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
     using C = FwdTc<DK, DV>;
@@ -137,6 +176,8 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t tiles = (sbase + C::CTRL + 1023u) & ~1023u;
     const uint32_t sQ = tiles;
     const uint32_t sKV = tiles + C::TILEK;
+    float *xmax = reinterpret_cast<float *>(smem_raw + (tiles - sbase) + C::TILEK + C::SLOT * C::NSTAGE);  // [2][2][128]
+    float *xsum = xmax + 2 * 2 * 128;                                                                     // [2][128]
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem_raw + C::OFF_ABORT);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + C::OFF_TMEM_SLOT);
     auto bar = [&](int i) -> uint32_t { return sbase + 8u * (uint32_t)i; };
@@ -159,19 +200,19 @@ __global__ void __launch_bounds__(192, 1)
         }
         for (int s = 0; s < 2; s++) {
             mbar_init(bar(C::B_S_FULL + s), 1);
-            mbar_init(bar(C::B_P_FULL + s), 4);
+            mbar_init(bar(C::B_P_FULL + s), 8);
         }
         mbar_init(bar(C::B_O_READY), 1);
         mbar_init(bar(C::B_O_FINAL), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == C::W_LOAD && lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
     }
-    if (warp == 5) {
+    if (warp == C::W_MMA) {
         tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -180,7 +221,7 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp == C::W_LOAD) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             const uint64_t keep = policy_evict_last();
@@ -220,7 +261,7 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == C::W_MMA) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t ID_QK = idesc_bf16_f32(128, 128, false, false);
@@ -285,61 +326,70 @@ __global__ void __launch_bounds__(192, 1)
             tc_commit(bar(C::B_O_FINAL));
             if (!ok) mbar_wait_drain(bar(C::B_O_FINAL), 0, 200000000ull);
         }
-    } else {
-        // ---------------------------------------------- softmax (warps 0..3)
-        const int row = threadIdx.x;
+    } else if (warp < 8) {
+        // ------------------------------------- softmax (warps 0..7, two column halves)
+        const int quad = warp % 4;          // TMEM lanes 32 quad .. (query rows)
+        const int hf = warp / 4;            // column half of every tile
+        const int row = quad * 32 + lane;
         const int qi = q0 + row;
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+        const uint32_t pair_bar = 1 + (uint32_t)quad;  // named barrier of warps quad, quad + 4
         const int W = p.window;
-        float m = p.sink ? p.sink[hq] * kLog2e : -INFINITY, l = p.sink ? 1.0f : 0.0f;
+        float m = p.sink ? p.sink[hq] * kLog2e : -INFINITY;
+        // the sink's 1 in the sum is counted once, by half 0
+        float l = (p.sink && hf == 0) ? 1.0f : 0.0f;
         float mraw = -INFINITY;  // row max of the (log2-unit) scores, the sink excluded
         bool ok = true;
         for (int u = 0; u < n; u++) {
             const int buf = u & 1;
-            const int k0 = (lo + u) * C::BN;
+            const int k0 = (lo + u) * C::BN + hf * 64;  // first key of this half
             if (!mbar_wait_warp(bar(C::B_S_FULL + buf), (uint32_t)((u >> 1) & 1), abort_flag)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             const uint32_t tS = tmem + lane_base + (buf ? C::COL_S1 : C::COL_S0);
-            uint32_t s[4][32];
-            tmem_ld32(tS + 0, s[0]);
-            tmem_ld32(tS + 32, s[1]);
-            tmem_ld32(tS + 64, s[2]);
-            tmem_ld32(tS + 96, s[3]);
+            uint32_t s[2][32];
+            tmem_ld32(tS + hf * 64, s[0]);
+            tmem_ld32(tS + hf * 64 + 32, s[1]);
             tmem_ld_wait(s[0]);
             tmem_ld_wait(s[1]);
-            tmem_ld_wait(s[2]);
-            tmem_ld_wait(s[3]);
             // capped scores are turned into log2 units here; plain ones stay raw
             // (the scale is folded into the exponent's FMA, and max commutes
             // with a positive scale)
             const bool cap = p.softcap > 0.0f;
             if (cap) {
 #pragma unroll
-                for (int c = 0; c < 128; c++) {
+                for (int c = 0; c < 64; c++) {
                     const float x = __uint_as_float(s[c >> 5][c & 31]);
                     s[c >> 5][c & 31] = __float_as_uint(p.cap_out * tanh_via_ex2(x * p.cap_in));
                 }
             }
-            const bool need_mask = (k0 + C::BN - 1 > q0) || (W > 0 && k0 <= q0 + C::BM - 1 - W);
+            const int kt0 = (lo + u) * C::BN;
+            const bool need_mask = (kt0 + C::BN - 1 > q0) || (W > 0 && kt0 <= q0 + C::BM - 1 - W);
             if (need_mask) {
 #pragma unroll
-                for (int c = 0; c < 128; c++) {
+                for (int c = 0; c < 64; c++) {
                     const int kj = k0 + c;
                     const bool vis = kj <= qi && (W == 0 || kj > qi - W);
                     if (!vis) s[c >> 5][c & 31] = __float_as_uint(-INFINITY);
                 }
             }
-            float mx = fwd_row_max(s);
+            float mh = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 64; c++) mh = fmaxf(mh, __uint_as_float(s[c >> 5][c & 31]));
+            // the row max over both halves: exchange through shared memory (both
+            // halves have read all their scores, so P may go over S after this)
+            xmax[(buf * 2 + hf) * 128 + row] = mh;
+            named_barrier_sync(pair_bar, 64);
+            float mx = fmaxf(mh, xmax[(buf * 2 + (hf ^ 1)) * 128 + row]);
             if (!cap) mx *= p.scale_log2;
             mraw = fmaxf(mraw, mx);
             const float m_new = (mx > m + 8.0f) ? mx : m;
             const bool moved = (m_new != m);
             const float factor = moved ? ex2_approx(m - m_new) : 1.0f;
             if (__any_sync(0xffffffffu, moved && u > 0)) {
-                // rescale O (row-wise) once PV of the previous tile has landed
+                // rescale this half's O columns once PV of the previous tile has landed
                 if (!mbar_wait_warp(bar(C::B_O_READY), (uint32_t)((u - 1) & 1), abort_flag)) {
                     ok = false;
                     break;
@@ -347,7 +397,7 @@ __global__ void __launch_bounds__(192, 1)
                 tc_fence_after();
                 const float f = (moved && u > 0) ? factor : 1.0f;
 #pragma unroll 1
-                for (int c0 = 0; c0 < DV; c0 += 32) {
+                for (int c0 = hf * (DV / 2); c0 < (hf + 1) * (DV / 2); c0 += 32) {
                     uint32_t o[32];
                     tmem_ld32(tmem + lane_base + C::COL_O + c0, o);
                     tmem_ld_wait(o);
@@ -359,24 +409,24 @@ __global__ void __launch_bounds__(192, 1)
             }
             m = m_new;
             const float msub = (m == -INFINITY) ? 0.0f : m;
-            uint32_t pk[2][32];
+            uint32_t pk[32];
             float rs;
             if (cap) {
-                rs = need_mask ? fwd_exp_tile<true, false, C::PSPLIT>(s, pk, p.scale_log2, msub)
-                               : fwd_exp_tile<true, true, C::PSPLIT>(s, pk, p.scale_log2, msub);
+                rs = need_mask ? fwd_exp_half<true, false, C::PSPLIT>(s, pk, p.scale_log2, msub)
+                               : fwd_exp_half<true, true, C::PSPLIT>(s, pk, p.scale_log2, msub);
             } else {
-                rs = need_mask ? fwd_exp_tile<false, false, C::PSPLIT>(s, pk, p.scale_log2, msub)
-                               : fwd_exp_tile<false, true, C::PSPLIT>(s, pk, p.scale_log2, msub);
+                rs = need_mask ? fwd_exp_half<false, false, C::PSPLIT>(s, pk, p.scale_log2, msub)
+                               : fwd_exp_half<false, true, C::PSPLIT>(s, pk, p.scale_log2, msub);
             }
-            tmem_st32(tS + 0, pk[0]);
-            tmem_st32(tS + 32, pk[1]);
+            // P (bf16 pairs) of this half's 64 keys: columns [32 hf, 32 hf + 32) of S
+            tmem_st32(tS + hf * 32, pk);
             if constexpr (C::PSPLIT) {
+                // low parts in columns [64 + 32 hf, 64 + 32 hf + 32)
 #pragma unroll
-                for (int c = 0; c < 64; c++)
-                    pk[c >> 5][c & 31] = pack_bf16x2(__uint_as_float(s[(2 * c) >> 5][(2 * c) & 31]),
-                                                     __uint_as_float(s[(2 * c + 1) >> 5][(2 * c + 1) & 31]));
-                tmem_st32(tS + 64, pk[0]);
-                tmem_st32(tS + 96, pk[1]);
+                for (int c = 0; c < 32; c++)
+                    pk[c] = pack_bf16x2(__uint_as_float(s[(2 * c) >> 5][(2 * c) & 31]),
+                                        __uint_as_float(s[(2 * c + 1) >> 5][(2 * c + 1) & 31]));
+                tmem_st32(tS + 64 + hf * 32, pk);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -387,10 +437,14 @@ __global__ void __launch_bounds__(192, 1)
         if (ok) ok = mbar_wait_warp(bar(C::B_O_FINAL), 0, abort_flag);
         if (ok) {
             tc_fence_after();
-            const float inv_l = 1.0f / l;
+            // both halves' row sums
+            xsum[hf * 128 + row] = l;
+            named_barrier_sync(pair_bar, 64);
+            const float lt = l + xsum[(hf ^ 1) * 128 + row];
+            const float inv_l = 1.0f / lt;
             __nv_bfloat16 *orow = p.o + ((size_t)bh * p.T + (size_t)min(qi, p.T - 1)) * DV;
 #pragma unroll 1
-            for (int c0 = 0; c0 < DV; c0 += 32) {
+            for (int c0 = hf * (DV / 2); c0 < (hf + 1) * (DV / 2); c0 += 32) {
                 uint32_t o[32];
                 tmem_ld32(tmem + lane_base + C::COL_O + c0, o);
                 tmem_ld_wait(o);
@@ -404,17 +458,19 @@ __global__ void __launch_bounds__(192, 1)
                     for (int i = 0; i < 4; i++) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
                 }
             }
-            if (qi < p.T) p.lse[(size_t)bh * p.T + qi] = (m + __log2f(l)) * kLn2;
-            if (p.max_logit) {
-                const float r = warp_max_f32(qi < p.T ? mraw * kLn2 : -INFINITY);
-                if ((threadIdx.x & 31) == 0) atomic_max_f32(p.max_logit + bh, r);
+            if (hf == 0) {
+                if (qi < p.T) p.lse[(size_t)bh * p.T + qi] = (m + __log2f(lt)) * kLn2;
+                if (p.max_logit) {
+                    const float r = warp_max_f32(qi < p.T ? mraw * kLn2 : -INFINITY);
+                    if (lane == 0) atomic_max_f32(p.max_logit + bh, r);
+                }
             }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == C::W_MMA) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
