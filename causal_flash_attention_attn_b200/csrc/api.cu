@@ -200,7 +200,9 @@ forge_status fwd_tc(const void *q, const void *k, const void *v, void *o, float 
             t_last_cuda_error = "cuTensorMapEncodeTiled failed";
             return FORGE_ERR_CUDA;
         }
-        if (set_smem(fwd2_tc_kernel<D>, C2::SMEM) != FORGE_OK) return FORGE_ERR_CUDA;
+        if (set_smem(fwd2_tc_kernel<D, true>, C2::SMEM) != FORGE_OK ||
+            set_smem(fwd2_tc_kernel<D, false>, C2::SMEM) != FORGE_OK)
+            return FORGE_ERR_CUDA;
         // Persistent (one CTA per SM, the most shared memory and TMEM allow) for
         // short sequences, whose items are too light to amortise a CTA's start;
         // one CTA per item otherwise, where the hardware's dynamic placement
@@ -210,7 +212,11 @@ forge_status fwd_tc(const void *q, const void *k, const void *v, void *o, float 
         const long long items = (long long)((p.num_qt + 1) / 2) * B * Hq;
         const bool persistent = p.num_qt <= 8;
         const unsigned grid = (unsigned)(persistent && items > sm_count() ? sm_count() : items);
-        return launch_pdl(fwd2_tc_kernel<D>, dim3(grid), dim3(C2::THREADS), C2::SMEM, st, mq, mk, mv, mo, p);
+        // (the persistent form with grid = items takes the same items; the flag
+        // only removes the work-item loop from the one-item-per-CTA code)
+        if (persistent)
+            return launch_pdl(fwd2_tc_kernel<D, true>, dim3(grid), dim3(C2::THREADS), C2::SMEM, st, mq, mk, mv, mo, p);
+        return launch_pdl(fwd2_tc_kernel<D, false>, dim3(grid), dim3(C2::THREADS), C2::SMEM, st, mq, mk, mv, mo, p);
     }
     return launch_status();
 }

@@ -49,6 +49,9 @@ struct Fwd2Tc {
     // without spills.
     static constexpr int THREADS = 384;
     static constexpr int REG_LAUNCH = 168, REG_CTRL = D == 64 ? 72 : 64, REG_SOFTMAX = 216;
+    // one item per CTA (no work-item loop): the control warps fit in 56
+    static constexpr int REG_CTRL_ONE = 56, REG_SOFTMAX_ONE = 224;
+    static_assert(4 * (REG_LAUNCH - REG_CTRL_ONE) >= 8 * (REG_SOFTMAX_ONE - REG_LAUNCH), "register split");
     static_assert(4 * (REG_LAUNCH - REG_CTRL) >= 8 * (REG_SOFTMAX - REG_LAUNCH), "register split");
     static_assert((2 * REG_SOFTMAX + REG_CTRL) * 32 <= 16384, "registers of one SM sub-partition");
     static constexpr uint32_t TMEM_COLS = 512;
@@ -144,7 +147,9 @@ __device__ __forceinline__ void exp_chunk32(const uint32_t (&s)[32], uint64_t sl
 // Persistent: gridDim.x CTAs walk the work items (pairs of query tiles of one
 // head, heaviest first) in the snake order of snake_item; barrier phases count
 // KV tiles (or items) over the CTA's whole run and TMEM is allocated once.
-template <int D>
+// PERSIST = false: one CTA per item (grid = number of items), compiled without
+// the work-item loop.
+template <int D, bool PERSIST>
 __global__ void __launch_bounds__(384, 1)
     fwd2_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -162,7 +167,9 @@ __global__ void __launch_bounds__(384, 1)
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int W = p.window;
     const int nitems = ((p.num_qt + 1) / 2) * p.B * p.Hq;
-    auto item_of = [&](int pass) -> int { return snake_item(pass, (int)blockIdx.x, (int)gridDim.x); };
+    auto item_of = [&](int pass) -> int {
+        return PERSIST ? snake_item(pass, (int)blockIdx.x, (int)gridDim.x) : (pass == 0 ? (int)blockIdx.x : nitems);
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::NQB; s++) {
@@ -199,14 +206,14 @@ __global__ void __launch_bounds__(384, 1)
     griddep_wait();  // the previous kernel's writes (q, k, v, max_logit) are visible
 
     if (warp >= 8) {
-        setmaxnreg_dec<C::REG_CTRL>();
+        setmaxnreg_dec<PERSIST ? C::REG_CTRL : C::REG_CTRL_ONE>();
         if (warp == 8) {
             // ------------------------------------------------------------ producer
             if (lane == 0) {
                 const uint64_t keep = policy_evict_last();
                 int issued = 0, q_issued = 0;  // ring slots and Q buffers loaded (for the abort drain)
                 bool ok = true;
-                for (int pass = 0; ok; pass++) {
+                for (int pass = 0; ok && (PERSIST || pass == 0); pass++) {
                     const int w = item_of(pass);
                     if (w >= nitems) break;
                     const Fwd2Item I = fwd2_item<C>(w, p);
@@ -267,7 +274,7 @@ __global__ void __launch_bounds__(384, 1)
                 int cnt0 = 0, cnt1 = 0;  // PVs issued per tile over the whole run (P_FULL phases)
                 bool ok = true;
                 int pass = 0;
-                for (; ok; pass++) {
+                for (; ok && (PERSIST || pass == 0); pass++) {
                     const int w = item_of(pass);
                     if (w >= nitems) break;
                     const Fwd2Item I = fwd2_item<C>(w, p);
@@ -348,7 +355,7 @@ __global__ void __launch_bounds__(384, 1)
             }
         }
     } else {
-        setmaxnreg_inc<C::REG_SOFTMAX>();
+        setmaxnreg_inc<PERSIST ? C::REG_SOFTMAX : C::REG_SOFTMAX_ONE>();
         // ---------------------------------------- softmax: warps 0-3 tile A, 4-7 tile B
         const int x = warp / 4;
         const int row = threadIdx.x % 128;
@@ -359,7 +366,7 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t sl2x2 = f2_make(p.scale_log2, p.scale_log2);
         int cnt = 0;  // KV tiles of this tile slot over the whole run (S_FULL phases)
         bool ok = true;
-        for (int pass = 0; ok; pass++) {
+        for (int pass = 0; ok && (PERSIST || pass == 0); pass++) {
             const int w = item_of(pass);
             if (w >= nitems) break;
             const Fwd2Item I = fwd2_item<C>(w, p);
