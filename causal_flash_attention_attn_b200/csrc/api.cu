@@ -138,6 +138,19 @@ int sm_count() {
     return cache[dev];
 }
 
+// L2 size of the current device in bytes (cached per device)
+long long l2_bytes() {
+    static long long cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 126LL << 20;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrL2CacheSize, dev) != cudaSuccess || n < 1) n = 126 << 20;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
 // Launch with programmatic stream serialization: the kernel may start while the
 // previous kernel on the stream finishes (its prologue overlaps that kernel's
 // tail); the kernels launched this way call griddep_wait before touching global
@@ -306,6 +319,11 @@ forge_status bwd_tc(const void *q, const void *k, const void *v, const float *ls
     p.softcap = softcap;
     p.cap_in = softcap > 0.0f ? scale / softcap : 0.0f;
     p.cap_out = softcap * kLog2e;
+    // descending query tiles where it measured faster: global causal attention at
+    // head dim <= 128, T <= 8192, with Q, dO and the f32 dq accumulator larger
+    // than L2 (bwd_step in bwd_tc.cuh)
+    const double operand_bytes = (double)B * Hq * T * D * (2 + 2 + 4);
+    p.q_desc = window == 0 && D <= 128 && T <= 8192 && operand_bytes > (double)l2_bytes() ? 1 : 0;
     if (set_smem(bwd_tc_kernel<D>, C::SMEM) != FORGE_OK) return FORGE_ERR_CUDA;
     // persistent: one CTA per SM (the kernel's shared memory and TMEM allow no
     // more), each walking its share of the work items
@@ -343,6 +361,7 @@ forge_status bwd_tc_dkv(const void *q, const void *k, const void *v, const float
     p.softcap = softcap;
     p.cap_in = softcap > 0.0f ? scale / softcap : 0.0f;
     p.cap_out = softcap * kLog2e;
+    p.q_desc = 0;
     if (set_smem(bwd_dkdv_tc_kernel<DK, DV>, CA::SMEM) != FORGE_OK) return FORGE_ERR_CUDA;
     bwd_dkdv_tc_kernel<DK, DV><<<(unsigned)(p.num_kt * B * Hkv), CA::THREADS, CA::SMEM, st>>>(mq, mk, mv, mdo, p);
     forge_status s = launch_status();

@@ -154,6 +154,32 @@ struct BwdParams {
     float softcap;         // 0 = off
     float cap_in;          // scale / softcap
     float cap_out;         // softcap * log2(e)
+    int q_desc;            // step order: 0 = head by head, query tiles ascending;
+                           // 1 = query tiles descending from T - 1, every head per tile
+};
+
+// An item's steps in order: (query head g of the group, query tile m). Head by head,
+// each CTA sweeps its own range of query tiles, so concurrent CTAs touch
+// different Q, dO and dq-accumulator tiles. Descending with the heads innermost,
+// the CTAs of a group that start together stay on the same query tile (every
+// range ends at T - 1), so those tiles are fetched from DRAM about once and
+// reused from L2 (measured on the 4K GQA layer: DRAM 1064 -> 705 MB a launch,
+// 0.686 -> 0.652 ms); it was slower where the operands already fit in L2 or
+// the ranges are short (windows, T = 512), and at head dim 256 and 16K.
+struct BwdStep {
+    int g, m;
+    __device__ __forceinline__ BwdStep(const BwdItem &I, int q_desc) : g(0), m(q_desc ? I.m_lo + I.nm - 1 : I.m_lo) {}
+    __device__ __forceinline__ void next(const BwdItem &I, int G, int q_desc) {
+        if (q_desc) {
+            if (++g == G) {
+                g = 0;
+                m--;
+            }
+        } else if (++m == I.m_lo + I.nm) {
+            m = I.m_lo;
+            g++;
+        }
+    }
 };
 
 // The two phases of one key row's P / dS work (this thread's TMEM lane), 32
@@ -421,10 +447,11 @@ __global__ void __launch_bounds__(512, 1)
                     }
                 }
                 kv_issued++;
-                for (int i = 0; i < I.steps; i++, gs++) {
+                BwdStep sp(I, p.q_desc);
+                for (int i = 0; i < I.steps; i++, gs++, sp.next(I, G, p.q_desc)) {
                     const int st = gs % C::QST;
                     const uint32_t ph = (uint32_t)((gs / C::QST) & 1);
-                    const int g = i / I.nm, m = I.m_lo + i % I.nm;
+                    const int g = sp.g, m = sp.m;
                     const int bhq = I.b * p.Hq + I.hkv * G + g;
                     // this step's LSE and Delta into registers first: their global-load
                     // latency overlaps the wait for a free stage
@@ -582,9 +609,10 @@ __global__ void __launch_bounds__(512, 1)
             if (w >= nitems) break;
             const BwdItem I = bwd_item<C>(w, p);
             const int kj = I.k0 + kr;
-            for (int i = 0; i < I.steps; i++, gs++) {
+            BwdStep sp(I, p.q_desc);
+            for (int i = 0; i < I.steps; i++, gs++, sp.next(I, G, p.q_desc)) {
                 const int st = gs % C::QST;
-                const int m = I.m_lo + i % I.nm;
+                const int m = sp.m;
                 const int qb = m * C::BM;
                 // phase A: S^T -> P^T (TMEM) and the dS factors g (registers)
                 if (!(ok = mbar_wait_warp(bar(C::B_Q_FULL + st), (uint32_t)((gs / C::QST) & 1), abort_flag))) break;
@@ -666,8 +694,9 @@ __global__ void __launch_bounds__(512, 1)
             const int w = item_of(pass);
             if (w >= nitems) break;
             const BwdItem I = bwd_item<C>(w, p);
-            for (int i = 0; i < I.steps; i++, gs++) {
-                const int g = i / I.nm, m = I.m_lo + i % I.nm;
+            BwdStep sp(I, p.q_desc);
+            for (int i = 0; i < I.steps; i++, gs++, sp.next(I, G, p.q_desc)) {
+                const int g = sp.g, m = sp.m;
                 const int bhq = I.b * p.Hq + I.hkv * G + g;
                 if (!(ok = mbar_wait_warp(bar(C::B_DQ_FULL), (uint32_t)(gs & 1), abort_flag))) break;
                 tc_fence_after();

@@ -187,33 +187,50 @@ __global__ void __launch_bounds__(kDecThreads) decode_split(const T_ *__restrict
 #pragma unroll
                 for (int e = 0; e < 8; e++) k1[d + e] = f[e];
             }
-            for (int g = 0; g < G; g++) {
-                const float4 *qg = reinterpret_cast<const float4 *>(q_s + (g * C::SQ + sl) * C::QP);
-                float a0 = 0.0f, a1 = 0.0f;
+            // all heads' dot products first (independent chains), then their
+            // slice reductions interleaved
+            float a0[MG], a1[MG];
 #pragma unroll
-                for (int d4 = 0; d4 < C::SL / 4; d4++) {
-                    const float4 qv = qg[d4];
-                    a0 = fmaf(qv.x, k0[4 * d4], a0);
-                    a1 = fmaf(qv.x, k1[4 * d4], a1);
-                    a0 = fmaf(qv.y, k0[4 * d4 + 1], a0);
-                    a1 = fmaf(qv.y, k1[4 * d4 + 1], a1);
-                    a0 = fmaf(qv.z, k0[4 * d4 + 2], a0);
-                    a1 = fmaf(qv.z, k1[4 * d4 + 2], a1);
-                    a0 = fmaf(qv.w, k0[4 * d4 + 3], a0);
-                    a1 = fmaf(qv.w, k1[4 * d4 + 3], a1);
-                }
+            for (int g = 0; g < MG; g++) {
+                a0[g] = a1[g] = 0.0f;
+                if (g < G) {
+                    const float4 *qg = reinterpret_cast<const float4 *>(q_s + (g * C::SQ + sl) * C::QP);
 #pragma unroll
-                for (int o = C::SQ / 2; o > 0; o >>= 1) {
-                    a0 += __shfl_xor_sync(0xffffffffu, a0, o);
-                    a1 += __shfl_xor_sync(0xffffffffu, a1, o);
-                }
-                if (sl == 0) {
-                    if (p.cap_out > 0.0f) {
-                        a0 = p.cap_out * tanhf(a0);
-                        a1 = p.cap_out * tanhf(a1);
+                    for (int d4 = 0; d4 < C::SL / 4; d4++) {
+                        const float4 qv = qg[d4];
+                        a0[g] = fmaf(qv.x, k0[4 * d4], a0[g]);
+                        a1[g] = fmaf(qv.x, k1[4 * d4], a1[g]);
+                        a0[g] = fmaf(qv.y, k0[4 * d4 + 1], a0[g]);
+                        a1[g] = fmaf(qv.y, k1[4 * d4 + 1], a1[g]);
+                        a0[g] = fmaf(qv.z, k0[4 * d4 + 2], a0[g]);
+                        a1[g] = fmaf(qv.z, k1[4 * d4 + 2], a1[g]);
+                        a0[g] = fmaf(qv.w, k0[4 * d4 + 3], a0[g]);
+                        a1[g] = fmaf(qv.w, k1[4 * d4 + 3], a1[g]);
                     }
-                    p_s[g * C::KT + j0] = j0 < nk ? a0 : -INFINITY;
-                    p_s[g * C::KT + j0 + 1] = j0 + 1 < nk ? a1 : -INFINITY;
+                }
+            }
+#pragma unroll
+            for (int o = C::SQ / 2; o > 0; o >>= 1) {
+#pragma unroll
+                for (int g = 0; g < MG; g++) {
+                    if (g < G) {
+                        a0[g] += __shfl_xor_sync(0xffffffffu, a0[g], o);
+                        a1[g] += __shfl_xor_sync(0xffffffffu, a1[g], o);
+                    }
+                }
+            }
+            if (sl == 0) {
+#pragma unroll
+                for (int g = 0; g < MG; g++) {
+                    if (g < G) {
+                        float s0 = a0[g], s1 = a1[g];
+                        if (p.cap_out > 0.0f) {
+                            s0 = p.cap_out * tanhf(s0);
+                            s1 = p.cap_out * tanhf(s1);
+                        }
+                        p_s[g * C::KT + j0] = j0 < nk ? s0 : -INFINITY;
+                        p_s[g * C::KT + j0 + 1] = j0 + 1 < nk ? s1 : -INFINITY;
+                    }
                 }
             }
         }
