@@ -85,6 +85,7 @@ KERNEL_SOURCES = {
     "fwd2_tc_kernel": ("fwd2_tc.cuh", "fwd_tc.cuh", "sm100.cuh"),
     "fwd_tc_kernel": ("fwd_tc.cuh", "sm100.cuh"),
     "decode_split": ("decode.cuh", "sm100.cuh"),
+    "decode_split_warp": ("decode.cuh", "sm100.cuh"),
 }
 
 
@@ -838,9 +839,9 @@ def run_decode(args):
             "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic (seeded N(0,1) q and caches)",
             "config": dict(c, l2="not flushed: the 1.07 GB cache exceeds the 126 MB L2"),
-            "roofline": {"kernel": "decode_split", "bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
+            "roofline": {"kernel": "decode_split_warp", "bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
                          "unit": "GB/s", "frac": round(gbs / peak, 4),
-                         "traffic": ncu_traffic("decode_split", c["workload"]),
+                         "traffic": ncu_traffic("decode_split_warp", c["workload"]),
                          "peak_source": f"{peak_src} hbm_gbs",
                          "achieved_def": "K+V cache bytes + q, o, lse bytes per call / CUDA-event time of both kernels"},
             "gpu_launches": 2 * args.steps, "clocks": clocks}

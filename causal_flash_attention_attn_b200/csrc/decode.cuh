@@ -313,6 +313,305 @@ __global__ void __launch_bounds__(kDecThreads) decode_split(const T_ *__restrict
     }
 }
 
+// ---------------------------------------------------------------------------
+// decode_split_warp: the same (key chunk, batch entry, KV head) work per CTA,
+// with every warp an independent pipeline over its share of the chunk (steps
+// w, w + NW, w + 2 NW, ... of KW keys), for groups with MG * D <= 1024 and rows
+// of at most 256 * MG bytes. Per warp: its own ring of NST stages filled by
+// bulk copies (one for the step's K rows, one for its V rows, completing on the
+// stage's mbarrier), the G queries in registers (lane L holds head dims
+// L*DL .. L*DL + DL - 1 of every head), its own running max, sum and output.
+// Per step, each lane forms partial dot products over its DL dims for the
+// KW * MG = 32 (key, head) slots; a transposed shuffle reduction (at each level a
+// lane keeps one half of its slots and adds its partner's copy of that half)
+// leaves lane L with the full score of slot L (key L / MG, head L % MG), so the
+// softmax of the step needs one score per lane and the per-head maximum only
+// log2(KW) shuffles. The running max moves only when a step's maximum exceeds
+// it by more than 8 (log2 units), so most steps skip the rescale of o. P.V: each
+// lane accumulates its DL dims of every head from the V rows and the step's
+// probabilities (through shared memory, read as broadcasts). No CTA barrier
+// runs until the warps merge their (max, sum, o) at the end.
+constexpr int kDecWarps = 4;
+constexpr int kDecWRing = 8192;  // bytes of K/V ring per warp (about)
+
+template <typename T_, int D, int MG>
+struct DecWCfg {
+    static constexpr int DL = D / 32;                  // head dims per lane
+    static constexpr int KW = 32 / MG;                 // keys per step: 32 (key, head) slots
+    static constexpr int ROWB = D * (int)sizeof(T_);   // bytes of one cache row
+    static constexpr int SEGB = DL * (int)sizeof(T_);  // bytes of a lane's part of a row
+    static constexpr int STEPB = KW * ROWB;            // K (or V) bytes of one step
+    static constexpr int STAGEB = 2 * STEPB;
+    static constexpr int NST = kDecWRing / STAGEB < 2 ? 2 : (kDecWRing / STAGEB > 8 ? 8 : kDecWRing / STAGEB);
+    static constexpr int RING = kDecWarps * NST * STAGEB;
+    // after the ring: mbarriers [NW][NST], p [NW][32] as (p, p) pairs,
+    // correction [NW][MG], max and sum [NW][MG] each, the abort flag
+    static constexpr int OFF_BAR = RING;
+    static constexpr int OFF_P = OFF_BAR + kDecWarps * NST * 8;
+    static constexpr int OFF_C = OFF_P + kDecWarps * 32 * 8;
+    static constexpr int OFF_M = OFF_C + kDecWarps * MG * 4;
+    static constexpr int OFF_L = OFF_M + kDecWarps * MG * 4;
+    static constexpr int OFF_ABORT = OFF_L + kDecWarps * MG * 4;
+    static constexpr int SMEM = OFF_ABORT + 16;
+    static_assert(MG * D <= 1024 && STEPB <= 8192, "shape served by decode_split");
+    static_assert((size_t)kDecWarps * MG * D * 4 <= (size_t)RING, "merge space");
+    static_assert(SMEM <= 232448, "shared memory");
+    static_assert(ROWB % 16 == 0 && SEGB % 4 == 0 && (MG & (MG - 1)) == 0 && DL % 2 == 0, "shape");
+};
+
+// A lane's DL elements of a row as DL / 2 packed f32 pairs (element 2i in the
+// low half): bf16 -> f32 is a 16-bit shift (low element) or a mask (high one).
+template <typename T_, int DL>
+__device__ __forceinline__ void load_seg2(const uint8_t *p, uint64_t (&f)[DL / 2]) {
+    if constexpr (sizeof(T_) == 2) {
+        uint32_t w[DL / 2];
+        if constexpr (DL == 2) {
+            w[0] = *reinterpret_cast<const uint32_t *>(p);
+        } else if constexpr (DL == 4) {
+            const uint2 u = *reinterpret_cast<const uint2 *>(p);
+            w[0] = u.x; w[1] = u.y;
+        } else {
+            const uint4 u = *reinterpret_cast<const uint4 *>(p);
+            w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
+        }
+#pragma unroll
+        for (int i = 0; i < DL / 2; i++) f[i] = f2_make(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
+    } else {
+#pragma unroll
+        for (int i = 0; i < DL / 2; i++) f[i] = *reinterpret_cast<const uint64_t *>(p + 8 * i);
+    }
+}
+
+// v[r] (32 partial sums per lane) -> the warp-wide sum of slot `lane`. Slot
+// e = key * MG + head; register r of lane L holds slot r ^ (L & ~(MG - 1)) (the
+// caller reads key rows in that lane-permuted order), so at the levels that
+// reduce over key bits (offsets 16 .. MG) every lane keeps its lower half of
+// registers and sends the upper half, with no per-lane selection; the levels
+// over head bits (offsets MG / 2 .. 1) pick the half by the lane's bit.
+template <int MG>
+__device__ __forceinline__ float warp_transpose_sum32(float (&v)[32], int lane) {
+#pragma unroll
+    for (int o = 16; o >= MG; o >>= 1) {
+#pragma unroll
+        for (int i = 0; i < o; i++) v[i] += __shfl_xor_sync(0xffffffffu, v[i + o], o);
+    }
+#pragma unroll
+    for (int o = MG / 2; o > 0; o >>= 1) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < o; i++) {
+            const float send = up ? v[i] : v[i + o];
+            const float keep = up ? v[i + o] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+    return v[0];
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+template <typename T_, int D, int MG>
+__global__ void __launch_bounds__(kDecWarps * 32) decode_split_warp(const T_ *__restrict__ q,
+                                                                    const T_ *__restrict__ kc,
+                                                                    const T_ *__restrict__ vc, const DecParams p) {
+    using C = DecWCfg<T_, D, MG>;
+    extern __shared__ __align__(128) uint8_t dsm[];
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int bkv = blockIdx.y, b = bkv / p.Hkv, hkv = bkv % p.Hkv, split = blockIdx.x;
+    const int G = p.Hq / p.Hkv;
+    const uint32_t ring = smem_u32(dsm) + (uint32_t)(warp * C::NST * C::STAGEB);
+    const uint32_t bars = smem_u32(dsm + C::OFF_BAR) + (uint32_t)(warp * C::NST * 8);
+    float *pw = reinterpret_cast<float *>(dsm + C::OFF_P) + warp * 64;  // (p, p) per slot
+    float *cw = reinterpret_cast<float *>(dsm + C::OFF_C) + warp * MG;
+    float *m_s = reinterpret_cast<float *>(dsm + C::OFF_M);
+    float *l_s = reinterpret_cast<float *>(dsm + C::OFF_L);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(dsm + C::OFF_ABORT);
+
+    int len = p.seq_lens ? p.seq_lens[b] : p.T;
+    if (len < 1 || len > p.T) {
+        if (tid == 0) record_status(kStatusInvalidArg);
+        len = 0;
+    }
+    const int lo = p.window > 0 ? max(0, len - p.window) : 0;
+    const int c0 = max(lo, split * p.chunk), c1 = min(len, (split + 1) * p.chunk);
+    const size_t hstride = (size_t)p.nsplit * (D + 2);
+    float *part = p.part + ((size_t)(b * p.Hq + hkv * G) * p.nsplit + split) * (D + 2);
+    if (c0 >= c1) {
+        for (int idx = tid; idx < G * (D + 2); idx += kDecWarps * 32) {
+            const int g = idx / (D + 2), e = idx % (D + 2);
+            part[g * hstride + e] = e == 0 ? -INFINITY : 0.0f;
+        }
+        return;
+    }
+    const uint8_t *Kb = reinterpret_cast<const uint8_t *>(kc + (size_t)bkv * p.Tmax * D);
+    const uint8_t *Vb = reinterpret_cast<const uint8_t *>(vc + (size_t)bkv * p.Tmax * D);
+    const int nsteps = (c1 - c0 + C::KW - 1) / C::KW;
+    // this warp's steps: w + j * NW for j = 0, 1, ...
+    const int nj = warp < nsteps ? (nsteps - warp + kDecWarps - 1) / kDecWarps : 0;
+    auto issue = [&](int j) {  // lane 0: step j of this warp into stage j % NST
+        const int k0 = c0 + (warp + j * kDecWarps) * C::KW;
+        const uint32_t bytes = (uint32_t)(min(C::KW, c1 - k0) * C::ROWB);
+        const uint32_t st = ring + (uint32_t)((j % C::NST) * C::STAGEB), bar = bars + (uint32_t)((j % C::NST) * 8);
+        mbar_arrive_expect_tx(bar, 2 * bytes);
+        bulk_load(st, Kb + (size_t)k0 * C::ROWB, bytes, bar);
+        bulk_load(st + C::STEPB, Vb + (size_t)k0 * C::ROWB, bytes, bar);
+    };
+    if (tid == 0) *abort_flag = 0;
+    if (lane == 0) {
+        for (int s = 0; s < C::NST; s++) mbar_init(bars + 8 * s, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();  // the abort flag and every warp's barriers are initialised
+    if (lane == 0) {
+        for (int j = 0; j < C::NST && j < nj; j++) issue(j);
+    }
+    // the queries of the group (pre-scaled), this lane's head dims
+    // (packed f32 pairs of consecutive head dims)
+    uint64_t q2[MG][C::DL / 2], acc2[MG][C::DL / 2];
+#pragma unroll
+    for (int g = 0; g < MG; g++) {
+#pragma unroll
+        for (int i = 0; i < C::DL / 2; i++) {
+            const T_ *qg = q + (size_t)(b * p.Hq + hkv * G + g) * D + lane * C::DL + 2 * i;
+            q2[g][i] = g < G ? f2_make(to_f32(qg[0]) * p.qscale, to_f32(qg[1]) * p.qscale) : f2_make(0.0f, 0.0f);
+            acc2[g][i] = f2_make(0.0f, 0.0f);
+        }
+    }
+    // this lane's slot: key lane / MG of a step, head lane % MG
+    const int key_l = lane / MG, g_l = lane % MG;
+    float m_run = -INFINITY, l_run = 0.0f;  // the slot's head: running max (log2 units), this lane's sum
+    bool ok = true;
+    int j = 0;
+    for (; j < nj; j++) {
+        const uint32_t st = ring + (uint32_t)((j % C::NST) * C::STAGEB);
+        if (!(ok = mbar_wait_warp(bars + (uint32_t)((j % C::NST) * 8), (uint32_t)((j / C::NST) & 1), abort_flag)))
+            break;
+        const int k0 = c0 + (warp + j * kDecWarps) * C::KW;
+        const int nk = min(C::KW, c1 - k0);
+        const uint8_t *kt = dsm + (st - smem_u32(dsm)), *vt = kt + C::STEPB;
+        // partial scores over this lane's dims: register k * MG + g takes key row
+        // k ^ key_l (the order warp_transpose_sum32 expects). Rows past nk hold
+        // stale data; their slots are masked below.
+        float sc[32];
+#pragma unroll
+        for (int k = 0; k < C::KW; k++) {
+            uint64_t k2[C::DL / 2];
+            load_seg2<T_, C::DL>(kt + (k ^ key_l) * C::ROWB + lane * C::SEGB, k2);
+#pragma unroll
+            for (int g = 0; g < MG; g++) {
+                uint64_t a2 = f2_mul(q2[g][0], k2[0]);
+#pragma unroll
+                for (int i = 1; i < C::DL / 2; i++) a2 = f2_fma(q2[g][i], k2[i], a2);
+                float x, y;
+                f2_split(a2, x, y);
+                sc[k * MG + g] = x + y;
+            }
+        }
+        float s = warp_transpose_sum32<MG>(sc, lane);
+        if (p.cap_out > 0.0f) s = p.cap_out * tanhf(s);
+        s = key_l < nk ? s : -INFINITY;
+        float mx = s;
+#pragma unroll
+        for (int o = MG; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float m_new = mx > m_run + 8.0f ? mx : m_run;  // finite: the step has a key
+        const float corr = exp2f(m_run - m_new);
+        const float pr = exp2f(s - m_new);
+        l_run = fmaf(l_run, corr, pr);
+        const bool rescale = __any_sync(0xffffffffu, m_new != m_run);
+        m_run = m_new;
+        *reinterpret_cast<float2 *>(pw + 2 * lane) = make_float2(pr, pr);
+        if (rescale && lane < MG) cw[lane] = corr;
+        __syncwarp();
+        if (rescale) {
+#pragma unroll
+            for (int g = 0; g < MG; g++) {
+                const float cg = cw[g];
+                const uint64_t c2 = f2_make(cg, cg);
+#pragma unroll
+                for (int i = 0; i < C::DL / 2; i++) acc2[g][i] = f2_mul(acc2[g][i], c2);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < C::KW; k++) {
+            if (k < nk) {
+                uint64_t v2[C::DL / 2];
+                load_seg2<T_, C::DL>(vt + k * C::ROWB + lane * C::SEGB, v2);
+                // (p, p) of every head for key k (slots k * MG ..)
+                uint64_t p2[MG];
+                if constexpr (MG >= 2) {
+#pragma unroll
+                    for (int g = 0; g < MG; g += 2) {
+                        const uint4 t = *reinterpret_cast<const uint4 *>(pw + 2 * (k * MG + g));
+                        p2[g] = (uint64_t)t.x | ((uint64_t)t.y << 32);
+                        p2[g + 1] = (uint64_t)t.z | ((uint64_t)t.w << 32);
+                    }
+                } else {
+                    p2[0] = *reinterpret_cast<const uint64_t *>(pw + 2 * k);
+                }
+#pragma unroll
+                for (int g = 0; g < MG; g++) {
+#pragma unroll
+                    for (int i = 0; i < C::DL / 2; i++) acc2[g][i] = f2_fma(p2[g], v2[i], acc2[g][i]);
+                }
+            }
+        }
+        __syncwarp();  // every lane is done with the stage and the probabilities
+        if (lane == 0 && j + C::NST < nj) {
+            fence_proxy_async_smem();
+            issue(j + C::NST);
+        }
+    }
+    if (!ok) {
+        // let this warp's copies in flight land before the CTA's memory is released
+        if (lane == 0) {
+            for (int jj = j; jj < nj && jj < j + C::NST; jj++)
+                mbar_wait_drain(bars + (uint32_t)((jj % C::NST) * 8), (uint32_t)((jj / C::NST) & 1), 100000000ull);
+        }
+        __syncwarp();
+    }
+    // the warp's sum per head (lanes of one head hold parts of it), then the merge
+#pragma unroll
+    for (int o = MG; o < 32; o <<= 1) l_run += __shfl_xor_sync(0xffffffffu, l_run, o);
+    if (key_l == 0) {
+        m_s[warp * MG + g_l] = m_run;
+        l_s[warp * MG + g_l] = l_run;
+    }
+    __syncthreads();  // every warp is out of its loop: the ring is free
+    float *red = reinterpret_cast<float *>(dsm);  // [NW][MG][D]
+#pragma unroll
+    for (int g = 0; g < MG; g++) {
+#pragma unroll
+        for (int i = 0; i < C::DL / 2; i++)
+            *reinterpret_cast<uint64_t *>(red + ((size_t)warp * MG + g) * D + lane * C::DL + 2 * i) = acc2[g][i];
+    }
+    __syncthreads();
+    if (*abort_flag) return;
+    for (int idx = tid; idx < G * D; idx += kDecWarps * 32) {
+        const int g = idx / D, d = idx % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kDecWarps; w++) M = fmaxf(M, m_s[w * MG + g]);
+        float o = 0.0f, L = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kDecWarps; w++) {
+            const float mw = m_s[w * MG + g];
+            if (mw == -INFINITY) continue;  // a warp with no step
+            const float f = exp2f(mw - M);
+            o = fmaf(red[((size_t)w * MG + g) * D + d], f, o);
+            L = fmaf(l_s[w * MG + g], f, L);
+        }
+        part[g * hstride + 2 + d] = o;
+        if (d == 0) {
+            part[g * hstride + 0] = M;
+            part[g * hstride + 1] = L;
+        }
+    }
+}
+
 // One CTA (D threads) per (batch entry, query head): merge the chunks, then the
 // sink: M = max of the chunk maxima (and the sink), L = sum l 2^(m - M), o = sum
 // o 2^(m - M) / L, lse = (M + log2 L) ln 2.

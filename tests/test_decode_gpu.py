@@ -1,7 +1,9 @@
 """GPU parity of the KV-cache decode (one query per entry and head against the
 cache, INFERENCE_RESEARCH.md section 2) through the C ABI against the oracle, on
 the three head dims, bf16 and f32, GQA, windows, caps, sinks and per-entry
-lengths. Tolerances are those of the other parity tests."""
+lengths, through both split kernels (the warp-pipelined one for groups whose
+queries fit a lane's registers, the CTA-wide one for the others). Tolerances
+are those of the other parity tests."""
 import math
 
 import numpy as np
@@ -23,6 +25,12 @@ CASES = [
     ("bf16_d128_g16_lens_win", "bf16", 2, 16, 1, 2048, 2048, 128, 100, 0.0, True, [2048, 129]),
     ("f32_d128", "f32", 2, 4, 2, 333, 400, 128, 0, 0.0, False, None),
     ("f32_d256_win_lens", "f32", 2, 2, 1, 260, 300, 256, 50, 0.0, False, [260, 10]),
+    # groups of 4 query heads at head dims 128 and 256 (the warp-pipelined kernel),
+    # ragged lengths; 8 heads at 256 (the CTA-wide kernel)
+    ("bf16_d128_g4_lens", "bf16", 3, 16, 4, 1500, 1536, 128, 0, 0.0, False, [1500, 3, 1029]),
+    ("bf16_d256_g4_cap_sink", "bf16", 2, 8, 2, 700, 768, 256, 0, 25.0, True, None),
+    ("bf16_d256_g8_win", "bf16", 1, 8, 1, 800, 800, 256, 300, 0.0, False, None),
+    ("f32_d64_mha_lens", "f32", 2, 3, 3, 450, 512, 64, 0, 0.0, False, [450, 33]),
 ]
 
 
