@@ -86,8 +86,8 @@ KERNEL_SOURCES = {
     "fwd_tc_kernel": ("fwd_tc.cuh", "sm100.cuh"),
     "decode_split": ("decode.cuh", "sm100.cuh"),
     "decode_split_warp": ("decode.cuh", "sm100.cuh"),
-    "bwd_dkdv_tc_kernel": ("bwd_dkv.cuh", "sm100.cuh"),
-    "bwd_dq_tc_kernel": ("bwd_dkv.cuh", "sm100.cuh"),
+    "bwd_dkdv_tc_kernel": ("bwd_dkv.cuh", "bwd_tc.cuh", "fwd_tc.cuh", "sm100.cuh"),
+    "bwd_dq_tc_kernel": ("bwd_dkv.cuh", "bwd_tc.cuh", "fwd_tc.cuh", "sm100.cuh"),
 }
 
 

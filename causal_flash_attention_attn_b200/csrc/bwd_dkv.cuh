@@ -36,28 +36,10 @@
 #pragma once
 
 #include "bwd_tc.cuh"
+#include "fwd_tc.cuh"
 #include "sm100.cuh"
 
 namespace forge {
-
-// Block b of a grid of ntile x nhead blocks -> (tile index heaviest first, head),
-// the heads taken in groups of kHeadGroup: all tiles of a group's heads before
-// the next group, so the operands a head shares across its tiles (K and V in
-// the dQ kernel, Q and dO in the dK/dV kernel) are read while still in L2.
-constexpr int kHeadGroup = 8;
-__device__ __forceinline__ void grouped_block(int blk, int ntile, int nhead, int &tile_from_heavy, int &head) {
-    const int full = nhead / kHeadGroup;
-    const int per = ntile * kHeadGroup;
-    if (blk < full * per) {
-        const int g = blk / per, r = blk % per;
-        tile_from_heavy = r / kHeadGroup;
-        head = g * kHeadGroup + r % kHeadGroup;
-    } else {
-        const int r = blk - full * per, gs = nhead - full * kHeadGroup;
-        tile_from_heavy = r / gs;
-        head = full * kHeadGroup + r % gs;
-    }
-}
 
 // ------------------------------------------------------------ dK / dV kernel
 template <int DK, int DV>

@@ -30,6 +30,26 @@
 
 namespace forge {
 
+// Block b of a grid of ntile x nhead blocks -> (tile index heaviest first, head),
+// the heads taken in groups of kHeadGroup: all tiles of a group's heads before
+// the next group, so the operands a head shares across its tiles (K and V in
+// the forward and the dQ kernel, Q and dO in the dK/dV kernel) are read while
+// still in L2.
+constexpr int kHeadGroup = 8;
+__device__ __forceinline__ void grouped_block(int blk, int ntile, int nhead, int &tile_from_heavy, int &head) {
+    const int full = nhead / kHeadGroup;
+    const int per = ntile * kHeadGroup;
+    if (blk < full * per) {
+        const int g = blk / per, r = blk % per;
+        tile_from_heavy = r / kHeadGroup;
+        head = g * kHeadGroup + r % kHeadGroup;
+    } else {
+        const int r = blk - full * per, gs = nhead - full * kHeadGroup;
+        tile_from_heavy = r / gs;
+        head = full * kHeadGroup + r % gs;
+    }
+}
+
 // DK: head dim of q and k; DV: head dim of v and o (DK = DV except for the
 // decompressed multi-head latent attention, 192 / 128).
 template <int DK, int DV = DK>
@@ -183,9 +203,9 @@ __global__ void __launch_bounds__(320, 1)
     auto bar = [&](int i) -> uint32_t { return sbase + 8u * (uint32_t)i; };
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int nbh = p.B * p.Hq;
-    const int qt = p.num_qt - 1 - (int)(blockIdx.x / nbh);
-    const int bh = blockIdx.x % nbh;
+    int qt_heavy, bh;
+    grouped_block((int)blockIdx.x, p.num_qt, p.B * p.Hq, qt_heavy, bh);
+    const int qt = p.num_qt - 1 - qt_heavy;
     const int b = bh / p.Hq, hq = bh % p.Hq;
     const int bkv = b * p.Hkv + hq / (p.Hq / p.Hkv);
     const int q0 = qt * C::BM;
