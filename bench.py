@@ -625,7 +625,11 @@ def run_ours(args, w):
         per = r.timed(args.steps)
     avg = {kname: sum(v) / len(v) for kname, v in per.items() if kname != "step"}
 
-    # end to end through the same C ABI from pinned host buffers
+    # end to end through the same C ABI from pinned host buffers: every step copies
+    # its inputs host -> device and its gradients device -> host. The copies run on
+    # their own streams into two alternating device buffer sets, so step k's
+    # uploads overlap step k - 1's compute and downloads (PCIe carries both
+    # directions at once); events order each buffer set's reuse.
     e2e = None
     if not args.no_e2e:
         q, k, v, dO = r.host
@@ -633,31 +637,60 @@ def run_ours(args, w):
         hdq, hdk, hdv = (torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in (r.qd, r.kd, r.vd))
         h2d = sum(x.numel() * x.element_size() for x in (hq_, hk_, hv_, hdo))
         d2h = sum(x.numel() * x.element_size() for x in (hdq, hdk, hdv))
+        bufs = [r, Runner(w, dev, stream, host_inputs=r.host)]
+        up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        ev = lambda: torch.cuda.Event()
+        up_done, comp_done, down_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+        used = [False, False]
 
-        def e2e_step():
-            for dst, src in ((r.qd, hq_), (r.kd, hk_), (r.vd, hv_), (r.dOd, hdo)):
-                dst.copy_(src, non_blocking=True)
-            r.step()
-            for dst, src in ((hdq, r.dq), (hdk, r.dk), (hdv, r.dv)):
-                dst.copy_(src, non_blocking=True)
+        def e2e_step(i):
+            j, b = i % 2, bufs[i % 2]
+            if used[j]:
+                up.wait_event(comp_done[j])      # step i - 2 has read this set's inputs
+            with torch.cuda.stream(up):
+                for dst, src in ((b.qd, hq_), (b.kd, hk_), (b.vd, hv_), (b.dOd, hdo)):
+                    dst.copy_(src, non_blocking=True)
+                up_done[j].record(up)
+            stream.wait_event(up_done[j])
+            if used[j]:
+                stream.wait_event(down_done[j])  # step i - 2's gradients are on the host
+            with torch.cuda.stream(stream):
+                b.step()
+                comp_done[j].record(stream)
+            down.wait_event(comp_done[j])
+            with torch.cuda.stream(down):
+                for dst, src in ((hdq, b.dq), (hdk, b.dk), (hdv, b.dv)):
+                    dst.copy_(src, non_blocking=True)
+                down_done[j].record(down)
+            used[j] = True
 
-        with torch.cuda.stream(stream):
-            for _ in range(2):
-                e2e_step()
+        def e2e_run(n, s0=None, s1=None):
+            if s0 is not None:
+                s0.record(stream)
+                up.wait_event(s0)
+            for i in range(n):
+                e2e_step(i)
+            for j in range(2):
+                if used[j]:
+                    stream.wait_event(down_done[j])
+            if s1 is not None:
+                s1.record(stream)
+
+        e2e_run(2)
         torch.cuda.synchronize(dev)
         barrier(world, dev)
         s0 = torch.cuda.Event(enable_timing=True)
         s1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            s0.record(stream)
-            for _ in range(args.steps):
-                e2e_step()
-            s1.record(stream)
+        e2e_run(args.steps, s0, s1)
         torch.cuda.synchronize(dev)
+        st = fa.forge_attn_check(stream.cuda_stream)
+        if st != fa.FORGE_OK:
+            raise fa.ForgeError(st, "end-to-end run")
         e2e_ms = max_over_ranks(s0.elapsed_time(s1), world, dev) / args.steps
         fl_f, fl_b = flops_of(w)
         e2e = {"value": round(aggregate_tflops(world, fl_f + fl_b, e2e_ms), 3), "unit": "TFLOPS",
-               "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "copies": "pinned host, own H2D and D2H streams, two device buffer sets, overlapping compute"}
 
     if world > 1:
         import torch.distributed as dist
