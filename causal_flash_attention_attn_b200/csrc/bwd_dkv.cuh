@@ -364,26 +364,28 @@ struct BwdQParams {
 
 template <int DK, int DV>
 struct BwdQTc {
-    static constexpr int BM = 128, BN = 64;               // query rows per CTA, keys per tile
+    // query rows per CTA, keys per tile, keys per softmax warpgroup (half a tile)
+    static constexpr int BM = 128, BN = 128, HB = 64;
     static constexpr int NCBK = DK / 64, NCBV = DV / 64;
-    static constexpr uint32_t CBQ = 128 * 128;            // column block of a 128-row tile
-    static constexpr uint32_t CBN = 64 * 128;             // column block of a 64-row tile
-    static constexpr uint32_t TQ = NCBK * CBQ, TDO = NCBV * CBQ;
-    static constexpr uint32_t TKT = NCBK * CBN, TVT = NCBV * CBN;
-    static constexpr int KST = 4, VST = 2;                // ring slots
+    static constexpr uint32_t CB = 128 * 128;             // column block (64 dims) of a 128-row tile
+    static constexpr uint32_t TQ = NCBK * CB, TDO = NCBV * CB;
+    static constexpr uint32_t TKT = NCBK * CB, TVT = NCBV * CB;
+    static constexpr int KST = 2, VST = 1;                // ring slots
     static constexpr uint32_t OFF_Q = 0, OFF_DO = TQ, OFF_K = TQ + TDO, OFF_V = OFF_K + KST * TKT;
     static constexpr uint32_t TILES = OFF_V + VST * TVT;
     static constexpr uint32_t OFF_TMEM_SLOT = 240, OFF_ABORT = 244;
     static constexpr uint32_t CTRL = 256;
     static constexpr uint32_t SMEM = 1024 + TILES + CTRL;
-    // warps 0-3 softmax of the even key tiles, 4-7 of the odd ones (one query
-    // row a thread), warp 8 loads Q, dO and the K ring, warp 9 issues MMAs and
-    // owns TMEM, warp 10 loads the V ring (so that a V load never waits behind a
-    // K load held up by a ring slot that a later dQ product frees)
+    // warps 0-3 softmax of keys 0-63 of every tile, 4-7 of keys 64-127 (one
+    // query row a thread), warp 8 loads Q, dO and the K ring, warp 9 issues MMAs
+    // and owns TMEM, warp 10 loads the V ring (so that a V load never waits
+    // behind a K load held up by a ring slot that a later dQ product frees).
+    // TMEM: two 128-column buffers (S of tile u, then dP over it, then each
+    // half's dS over its first 32 columns) for tiles u % 2, and dQ.
     static constexpr int THREADS = 384;
     static constexpr int W_LOAD = 8, W_MMA = 9, W_LOAD_V = 10;
-    static constexpr uint32_t COL_DQ = 128;
-    static constexpr uint32_t col_buf(int x) { return (uint32_t)(x * 64); }
+    static constexpr uint32_t COL_DQ = 256;
+    static constexpr uint32_t col_buf(int x) { return (uint32_t)(x * BN); }
     static constexpr uint32_t TMEM_COLS = 512;
     static_assert(COL_DQ + DK <= TMEM_COLS, "tensor memory");
     static_assert(SMEM <= 232448, "shared memory");
@@ -434,9 +436,9 @@ __global__ void __launch_bounds__(384, 1)
         }
         for (int x = 0; x < 2; x++) {
             mbar_init(bar(C::B_S_FULL + x), 1);
-            mbar_init(bar(C::B_PA + x), 4);
+            mbar_init(bar(C::B_PA + x), 8);
             mbar_init(bar(C::B_DP_FULL + x), 1);
-            mbar_init(bar(C::B_DS + x), 4);
+            mbar_init(bar(C::B_DS + x), 8);
         }
         mbar_init(bar(C::B_DQ_DONE), 1);
         *abort_flag = 0;
@@ -464,8 +466,8 @@ __global__ void __launch_bounds__(384, 1)
             const bool kq = warp == C::W_LOAD;  // Q, dO and K; else V
             if (kq) {
                 mbar_arrive_expect_tx(bar(C::B_QD), C::TQ + C::TDO);
-                for (int c = 0; c < C::NCBK; c++) tma_load_3d(sQ + c * C::CBQ, &tmQ, bar(C::B_QD), c * 64, q0, bh);
-                for (int c = 0; c < C::NCBV; c++) tma_load_3d(sdO + c * C::CBQ, &tmdO, bar(C::B_QD), c * 64, q0, bh);
+                for (int c = 0; c < C::NCBK; c++) tma_load_3d(sQ + c * C::CB, &tmQ, bar(C::B_QD), c * 64, q0, bh);
+                for (int c = 0; c < C::NCBV; c++) tma_load_3d(sdO + c * C::CB, &tmdO, bar(C::B_QD), c * 64, q0, bh);
             }
             // K(u) (or V(u)) for u = 0 .. n-1, each ring slot reused once the
             // product that last read it has completed
@@ -481,7 +483,7 @@ __global__ void __launch_bounds__(384, 1)
                 if (!(ok = mbar_wait(bar(B_EMPTY + s), (uint32_t)(((u / nst) & 1) ^ 1), abort_flag))) break;
                 mbar_arrive_expect_tx(bar(B_FULL + s), tile);
                 for (int c = 0; c < ncb; c++)
-                    tma_load_3d_hint(base + s * tile + c * C::CBN, map, bar(B_FULL + s), c * 64, (lo + u) * C::BN, bkv,
+                    tma_load_3d_hint(base + s * tile + c * C::CB, map, bar(B_FULL + s), c * 64, (lo + u) * C::BN, bkv,
                                      keep);
                 issued++;
             }
@@ -498,8 +500,7 @@ __global__ void __launch_bounds__(384, 1)
         if (lane == 0) {
             constexpr uint32_t ID_S = idesc_bf16_f32(128, C::BN, false, false);
             constexpr uint32_t ID_DQ = idesc_bf16_f32(128, DK, false, true);
-            auto offq = [](int kk) -> uint32_t { return (uint32_t)((kk >> 2) * C::CBQ + (kk & 3) * 32); };
-            auto offn = [](int kk) -> uint32_t { return (uint32_t)((kk >> 2) * C::CBN + (kk & 3) * 32); };
+            auto offk = [](int kk) -> uint32_t { return (uint32_t)((kk >> 2) * C::CB + (kk & 3) * 32); };
             // S(u) = Q K(u)^T into buffer u % 2
             auto issue_s = [&](int u) -> bool {
                 const int s = u % C::KST;
@@ -508,8 +509,8 @@ __global__ void __launch_bounds__(384, 1)
                 const uint32_t sK = sK0 + s * C::TKT;
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; kk++)
-                    mma_ss(tmem + C::col_buf(u & 1), sdesc_sw128(sQ + offq(kk), 16, 1024),
-                           sdesc_sw128(sK + offn(kk), 16, 1024), ID_S, kk > 0);
+                    mma_ss(tmem + C::col_buf(u & 1), sdesc_sw128(sQ + offk(kk), 16, 1024),
+                           sdesc_sw128(sK + offk(kk), 16, 1024), ID_S, kk > 0);
                 tc_commit(bar(C::B_S_FULL + (u & 1)));
                 return true;
             };
@@ -521,21 +522,26 @@ __global__ void __launch_bounds__(384, 1)
                 const uint32_t sV = sV0 + s * C::TVT;
 #pragma unroll
                 for (int kk = 0; kk < DV / 16; kk++)
-                    mma_ss(tmem + C::col_buf(u & 1), sdesc_sw128(sdO + offq(kk), 16, 1024),
-                           sdesc_sw128(sV + offn(kk), 16, 1024), ID_S, kk > 0);
+                    mma_ss(tmem + C::col_buf(u & 1), sdesc_sw128(sdO + offk(kk), 16, 1024),
+                           sdesc_sw128(sV + offk(kk), 16, 1024), ID_S, kk > 0);
                 tc_commit(bar(C::B_DP_FULL + (u & 1)));
                 tc_commit(bar(C::B_V_EMPTY + s));
                 return true;
             };
-            // dQ += dS(u) K(u): dS from the first 32 columns of buffer u % 2, K
-            // MN-major (N = the key head dim)
+            // dQ += dS(u) K(u), one half of the keys at a time: dS of half h from
+            // the first 32 columns of its 64 in buffer u % 2, K rows 64 h .. MN-major
+            // (N = the key head dim)
             auto issue_dq = [&](int u) {
                 const int s = u % C::KST;
                 const uint32_t sK = sK0 + s * C::TKT;
 #pragma unroll
-                for (int kk = 0; kk < C::BN / 16; kk++)
-                    mma_ts(tmem + C::COL_DQ, tmem + C::col_buf(u & 1) + 8 * kk, sdesc_sw128(sK + kk * 2048, C::CBN, 1024),
-                           ID_DQ, (u > 0 || kk > 0) ? 1u : 0u);
+                for (int h = 0; h < 2; h++) {
+#pragma unroll
+                    for (int kk = 0; kk < C::HB / 16; kk++)
+                        mma_ts(tmem + C::COL_DQ, tmem + C::col_buf(u & 1) + C::HB * h + 8 * kk,
+                               sdesc_sw128(sK + (h * (C::HB / 16) + kk) * 2048, C::CB, 1024), ID_DQ,
+                               (u > 0 || h > 0 || kk > 0) ? 1u : 0u);
+                }
                 tc_commit(bar(C::B_K_EMPTY + s));
             };
             // Issue whichever product is ready, each kind in its own order:
@@ -544,7 +550,7 @@ __global__ void __launch_bounds__(384, 1)
             //   dP(np) once S(np) is issued, phase A of tile np is done and V(np)
             //          has landed;
             //   dQ(nq) once dP(nq) is issued and phase B of tile nq is done.
-            // The two softmax warpgroups then never wait for each other's pace.
+            // S(ns + 1) runs while the softmax warpgroups work on tile ns.
             bool ok = mbar_wait(bar(C::B_QD), 0, abort_flag);
             int ns = 0, np = 0, nq = 0;
             uint64_t t_last = globaltimer_ns();
@@ -581,22 +587,22 @@ __global__ void __launch_bounds__(384, 1)
             if (!ok) mbar_wait_drain(bar(C::B_DQ_DONE), 0, 200000000ull);
         }
     } else if (warp < 8) {
-        // ------------------------------ softmax (one query row a thread), tiles x, x+2, ...
+        // --------------- softmax (one query row a thread), keys 64 x .. 64 x + 63 of every tile
         const int x = warp / 4;
         const int row = threadIdx.x % 128;
         const int qi = q0 + row;
         const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
-        const uint32_t tB = tmem + lane_base + C::col_buf(x);
         const bool cap = p.softcap > 0.0f;
         const size_t ridx = (size_t)bh * p.T + (size_t)min(qi, p.T - 1);
         // rows past T: P = 0 (and dS = 0) through nl = -inf
         const float nl = qi < p.T ? -p.lse[ridx] * kLog2e : -INFINITY;
         const float nd = qi < p.T ? -p.delta[ridx] * p.scale : 0.0f;
         bool ok = true;
-        int cnt = 0;
-        for (int u = x; u < n; u += 2, cnt++) {
-            const int k0 = (lo + u) * C::BN;
-            if (!(ok = mbar_wait_warp(bar(C::B_S_FULL + x), (uint32_t)(cnt & 1), abort_flag))) break;
+        for (int u = 0; u < n; u++) {
+            const int k0 = (lo + u) * C::BN + C::HB * x;
+            const uint32_t tB = tmem + lane_base + C::col_buf(u & 1) + C::HB * x;
+            const uint32_t ph = (uint32_t)((u >> 1) & 1);  // phase of buffer u % 2's barriers
+            if (!(ok = mbar_wait_warp(bar(C::B_S_FULL + (u & 1)), ph, abort_flag))) break;
             tc_fence_after();
             uint32_t s[2][32];
             tmem_ld32(tB, s[0]);
@@ -605,7 +611,7 @@ __global__ void __launch_bounds__(384, 1)
             tmem_ld_wait(s[1]);
             // warp-uniform: does any key of the tile fall outside some row's range?
             const int r0 = q0 + 32 * (warp % 4);
-            const bool mask = (k0 + C::BN - 1 > r0) || (W > 0 && k0 <= r0 + 31 - W);
+            const bool mask = (k0 + C::HB - 1 > r0) || (W > 0 && k0 <= r0 + 31 - W);
             float g[2][32];
 #pragma unroll
             for (int h = 0; h < 2; h++) {
@@ -631,9 +637,9 @@ __global__ void __launch_bounds__(384, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::B_PA + x));
+            if (lane == 0) mbar_arrive(bar(C::B_PA + (u & 1)));
             // phase B: dP -> dS (bf16) into the buffer's first 32 columns
-            if (!(ok = mbar_wait_warp(bar(C::B_DP_FULL + x), (uint32_t)(cnt & 1), abort_flag))) break;
+            if (!(ok = mbar_wait_warp(bar(C::B_DP_FULL + (u & 1)), ph, abort_flag))) break;
             tc_fence_after();
             uint32_t d[2][32];
             tmem_ld32(tB, d[0]);
@@ -652,7 +658,7 @@ __global__ void __launch_bounds__(384, 1)
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::B_DS + x));
+            if (lane == 0) mbar_arrive(bar(C::B_DS + (u & 1)));
         }
         // epilogue: warpgroup x writes its half of the dQ columns of its rows
         if (ok) ok = mbar_wait_warp(bar(C::B_DQ_DONE), 0, abort_flag);

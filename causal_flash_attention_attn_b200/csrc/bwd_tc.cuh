@@ -279,7 +279,6 @@ __device__ __forceinline__ void bwd_store_ds(const uint32_t (&dk)[16], int c0, i
 template <class C>
 __device__ __forceinline__ void bwd_mma_kq(uint32_t d_tmem, uint32_t sA, uint32_t sB) {
     constexpr uint32_t ID = idesc_bf16_f32(128, C::BM, false, false);
-#pragma unroll
     const uint64_t da = sdesc_sw128(opaque_u32(sA), 16, 1024), db = sdesc_sw128(opaque_u32(sB), 16, 1024);
 #pragma unroll
     for (int kk = 0; kk < C::D / 16; kk++) {
@@ -292,7 +291,6 @@ __device__ __forceinline__ void bwd_mma_kq(uint32_t d_tmem, uint32_t sA, uint32_
 template <class C>
 __device__ __forceinline__ void bwd_mma_dv(uint32_t tmem, uint32_t sdO_h, bool first) {
     constexpr uint32_t ID = idesc_bf16_f32(128, C::DH, false, true);
-#pragma unroll
     const uint64_t db = sdesc_sw128(opaque_u32(sdO_h), C::CBQ, 1024);
 #pragma unroll
     for (int kk = 0; kk < C::BM / 16; kk++)
@@ -303,7 +301,6 @@ __device__ __forceinline__ void bwd_mma_dv(uint32_t tmem, uint32_t sdO_h, bool f
 template <class C>
 __device__ __forceinline__ void bwd_mma_dk(uint32_t tmem, uint32_t sdS, uint32_t sQ_h, bool first) {
     constexpr uint32_t ID = idesc_bf16_f32(128, C::DH, false, true);
-#pragma unroll
     const uint64_t da = sdesc_sw128(opaque_u32(sdS), 16, 1024), db = sdesc_sw128(opaque_u32(sQ_h), C::CBQ, 1024);
 #pragma unroll
     for (int kk = 0; kk < C::BM / 16; kk++) {

@@ -419,7 +419,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_split_warp(const T_ *__
                                                                     const T_ *__restrict__ kc,
                                                                     const T_ *__restrict__ vc, const DecParams p) {
     using C = DecWCfg<T_, D, MG>;
-    extern __shared__ __align__(128) uint8_t dsm[];
+    extern __shared__ __align__(16) uint8_t dsm[];
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int bkv = blockIdx.y, b = bkv / p.Hkv, hkv = bkv % p.Hkv, split = blockIdx.x;
     const int G = p.Hq / p.Hkv;
