@@ -96,7 +96,9 @@ def test_sink_and_max_logit_match_oracle(case):
 @pytest.mark.parametrize("case", [CASES[0], CASES[3], CASES[4]], ids=["bf16_d128", "bf16_d256", "f32_d64"])
 def test_without_sink_equals_plain_entry_points_bitwise(case):
     """sink = NULL with a max-logit request computes o and lse exactly as
-    forge_attn_fwd, and forge_attn_bwd_ext with NULLs exactly as forge_attn_bwd."""
+    forge_attn_fwd, and forge_attn_bwd_ext with NULLs exactly as forge_attn_bwd
+    (dk, dv bit for bit; dq is summed over key tiles with f32 atomics, so the
+    order of those additions may move its bf16 rounding by one unit)."""
     name, dtype, B, Hq, Hkv, T, D, W, C = case
     w = _workload(name, dtype, B, Hq, Hkv, T, D, W, C, seed=43)
     (q, k, v, dO), (o, lse, ml, dq, dk, dv, _) = _run_ext(w, None)
@@ -106,8 +108,10 @@ def test_without_sink_equals_plain_entry_points_bitwise(case):
     o2, lse2 = fa.attention_fwd(qd, kd, vd, sc, W, C)
     dq2, dk2, dv2 = fa.attention_bwd(qd, kd, vd, o2, lse2, dOd, sc, W, C)
     torch.cuda.synchronize()
-    for a, b in ((o, o2), (lse, lse2), (dq, dq2), (dk, dk2), (dv, dv2)):
+    for a, b in ((o, o2), (lse, lse2), (dk, dk2), (dv, dv2)):
         assert torch.equal(a, b.cpu())
+    tol = 2.0 ** -7 if dtype == "bf16" else 1e-6
+    assert torch.allclose(dq.float(), dq2.cpu().float(), rtol=tol, atol=1e-6)
     _, _, rml = oracle.attn_fwd_ext(q, k, v, sc, W, C)
     check_close("max_logit", ml, rml, dtype)
 

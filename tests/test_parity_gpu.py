@@ -28,6 +28,11 @@ SMALL = [
     (2, 8, 1, 257, 64, 0, 0.0, "bf16"),
     (1, 2, 1, 1000, 128, 0, 0.0, "bf16"),
     (1, 2, 2, 384, 256, 0, 0.0, "bf16"),
+    # few KV groups at head dim 128: the heaviest key tiles run as two work items
+    # whose dK, dV are summed (split items)
+    (1, 16, 1, 1024, 128, 0, 0.0, "bf16"),
+    (1, 6, 1, 777, 128, 0, 0.0, "bf16"),
+    (2, 14, 2, 640, 128, 0, 3.0, "bf16"),
     (1, 2, 1, 200, 256, 0, 50.0, "bf16"),
     # windows
     (1, 2, 1, 300, 128, 1, 0.0, "bf16"),
