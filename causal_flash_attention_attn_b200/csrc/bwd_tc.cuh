@@ -182,6 +182,11 @@ struct BwdStep {
     }
 };
 
+// f32 reduction into global memory with an L2 cache-policy hint
+__device__ __forceinline__ void red_add_f32_hint(float *addr, float v, uint64_t policy) {
+    asm volatile("red.global.add.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(addr), "f"(v), "l"(policy) : "memory");
+}
+
 // The two phases of one key row's P / dS work (this thread's TMEM lane), 32
 // query columns at a time:
 //   phase A (needs S^T): P = exp2(s * scale * log2(e) - LSE * log2(e)), masked
@@ -742,11 +747,14 @@ __global__ void __launch_bounds__(512, 1)
                     // reduction covers 32 consecutive floats of one dQ row
                     static_assert(C::BULK_DQ || C::DQT, "per-element reduction expects the transposed dQ");
 
+                    // evict-last: the accumulator lines are reduced into again by the
+                    // other key tiles' CTAs soon, and read by the finalize
                     float *base = p.dq_acc + ((size_t)bhq * p.Tpad + (size_t)m * C::BM) * D + I.h * C::DH + t;
+                    const uint64_t keep = policy_evict_last();
 #pragma unroll
                     for (int j = 0; j < NQC; j++) {
 #pragma unroll
-                        for (int c = 0; c < 32; c++) atomicAdd(base + (size_t)(32 * j + c) * D, __uint_as_float(v[j][c]));
+                        for (int c = 0; c < 32; c++) red_add_f32_hint(base + (size_t)(32 * j + c) * D, __uint_as_float(v[j][c]), keep);
                     }
                 }
             }
