@@ -20,15 +20,15 @@
 //   while the compute warps form P of step i + 1, dV(i) while they form dS(i).
 //
 // bwd_dq_tc_kernel -- one CTA per (query tile of 128 rows, batch, query head),
-//   Q and dO resident, dQ in TMEM over the key tiles the rows see (64 keys a
-//   tile, K through a four-slot ring since dQ(j) reads K(j) after S(j), V
-//   through a two-slot ring, each ring with its own producer warp). Two softmax
-//   warpgroups take alternate key tiles,
-//   each with its own 64 TMEM columns:
+//   Q and dO resident, dQ in TMEM over the key tiles the rows see (128 keys a
+//   tile, K through a two-slot ring since dQ(j) reads K(j) after S(j), V through
+//   a one-slot ring, each ring with its own producer warp). The two softmax
+//   warpgroups split every tile's keys (64 each) and alternate 128-column TMEM
+//   buffers by tile:
 //     S  = Q K^T   -> buffer;  P, the dS factor g in registers
 //     dP = dO V^T  -> buffer (over S)
-//     dS = g (dP - Delta) * scale -> bf16 into the buffer's first 32 columns
-//     dQ += dS K   (A = dS from TMEM)
+//     dS = g (dP - Delta) * scale -> bf16 into the first 32 columns of each half
+//     dQ += dS K   (A = dS from TMEM, one K = 64 product per half)
 //   Every dQ row is complete in its CTA: no f32 accumulator, no atomics.
 //
 // Both recompute S and dP: 2 (DK + DV + DV + DK) + 2 (DK + DV + DK) flops per

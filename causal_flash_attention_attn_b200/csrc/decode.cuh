@@ -5,8 +5,12 @@
 // one layer's [B][Hkv][Tmax][D] here), and decoding gets a dedicated kernel: one
 // query, split-K along the cache for long contexts; GQA is the largest saving of
 // KV bandwidth. The work is HBM-bound (each cache byte is read once and feeds
-// 2*G flops per element), so it runs on the CUDA cores with coalesced, pipelined
-// cp.async loads rather than on the tensor cores.
+// 2*G flops per element), so it runs on the CUDA cores with pipelined
+// asynchronous loads rather than on the tensor cores.
+//
+// Two split kernels share the (key chunk, batch entry, KV head) decomposition:
+// decode_split_warp (below; every warp an independent pipeline) where the
+// group's queries fit a lane's registers, decode_split otherwise.
 //
 // decode_split: one CTA per (key chunk, batch entry, KV head), all G query heads
 // of the group at once, so every K/V byte is read once for the G heads. K/V
