@@ -81,15 +81,22 @@ struct BwdTc {
     static constexpr int NSTG = 1;                       // dQ staging tiles
     static constexpr uint32_t STG = BM * DH * 4;         // one f32 dQ staging tile
     static constexpr uint32_t OFF_STG = OFF_DS + TS;
-    static constexpr uint32_t TILES = OFF_STG + (BULK_DQ ? NSTG * STG : 0);
+    // head dim 256 (one Q/dO stage): this CTA's half of Q again, for dK, so that the
+    // stage is free for the next step's Q and dO once dV has read it
+    static constexpr bool QSHADOW = D == 256;
+    static constexpr uint32_t OFF_QSH = OFF_STG + (BULK_DQ ? NSTG * STG : 0);
+    static constexpr uint32_t TQSH = (DH / 64) * CBQ;
+    static constexpr uint32_t TILES = OFF_QSH + (QSHADOW ? TQSH : 0);
     // control block after the tiles: barriers, TMEM slot, abort flag, per-stage
     // LSE/Delta rows. The tiles need 1024-byte alignment (128-byte swizzle); the
     // dynamic shared memory base is 1024-aligned in practice, and SLACK covers
     // a base that is not wherever the budget leaves room (the kernel checks).
     static constexpr uint32_t OFF_TMEM_SLOT = 240, OFF_ABORT = 244;
-    static constexpr uint32_t OFF_LSE = 256;                        // [QST][BM] f32, -LSE * log2(e)
-    static constexpr uint32_t OFF_DLT = OFF_LSE + QST * BM * 4;     // [QST][BM] f32, -scale * Delta
-    static constexpr uint32_t CTRL = OFF_DLT + QST * BM * 4;
+    // LSE and Delta rows of a step, in slot (step % 2): with one Q/dO stage the
+    // next step's rows arrive while phase B still reads this step's Delta
+    static constexpr uint32_t OFF_LSE = 256;                        // [2][BM] f32, -LSE * log2(e)
+    static constexpr uint32_t OFF_DLT = OFF_LSE + 2 * BM * 4;       // [2][BM] f32, -scale * Delta
+    static constexpr uint32_t CTRL = OFF_DLT + 2 * BM * 4;
     static constexpr uint32_t SLACK = (TILES + CTRL + 1024 <= 232448) ? 1024 : 0;
     static constexpr uint32_t SMEM = SLACK + TILES + CTRL;
     // Roles: warps 0-7 compute (warp w: TMEM lanes 32 (w % 4).., query-row half
@@ -132,7 +139,9 @@ struct BwdTc {
     static constexpr int B_DQ_FREE = B_DQ_FULL + 1;
     static constexpr int B_KDONE = B_DQ_FREE + 1;        // a work item's dK, dV complete in TMEM
     static constexpr int B_EPI_DONE = B_KDONE + 1;       // ... and read out (8 compute + 4 drain warps)
-    static constexpr int NBAR = B_EPI_DONE + 1;
+    static constexpr int B_QSH_FULL = B_EPI_DONE + 1;    // the Q half for dK has landed (QSHADOW)
+    static constexpr int B_QSH_EMPTY = B_QSH_FULL + 1;   // ... and dK has read it
+    static constexpr int NBAR = B_QSH_EMPTY + 1;
     static_assert(NBAR * 8 <= (int)OFF_TMEM_SLOT, "control block");
 };
 
@@ -365,6 +374,7 @@ __global__ void __launch_bounds__(512, 1)
     uint8_t *const ctrl_p = smem_raw + (ctrl - sbase);
     const uint32_t sK0 = tiles + C::OFF_K, sQ0 = tiles + C::OFF_Q;
     const uint32_t sdO0 = tiles + C::OFF_DO, sdS = tiles + C::OFF_DS, sStg = tiles + C::OFF_STG;
+    const uint32_t sQsh = tiles + C::OFF_QSH;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl_p + C::OFF_ABORT);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ctrl_p + C::OFF_TMEM_SLOT);
     float *sLSE = reinterpret_cast<float *>(ctrl_p + C::OFF_LSE);
@@ -400,6 +410,8 @@ __global__ void __launch_bounds__(512, 1)
         mbar_init(bar(C::B_DQ_FREE), 4);
         mbar_init(bar(C::B_KDONE), 1);
         mbar_init(bar(C::B_EPI_DONE), 12);
+        mbar_init(bar(C::B_QSH_FULL), 1);
+        mbar_init(bar(C::B_QSH_EMPTY), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -424,7 +436,7 @@ __global__ void __launch_bounds__(512, 1)
         setmaxnreg_dec<C::REG_CTRL>();
         if (warp == C::W_LOAD) {
             // -------------------------------------------------------- producer
-            int issued = 0, kv_issued = 0;  // Q/dO and K/V loads issued (for the abort drain)
+            int issued = 0, kv_issued = 0, qsh_issued = 0;  // loads issued (for the abort drain)
             bool ok = true;
             int gs = 0;  // step count over all of this CTA's items
             for (int pass = 0; ok; pass++) {
@@ -481,10 +493,25 @@ __global__ void __launch_bounds__(512, 1)
                     issued++;
 #pragma unroll
                     for (int r = 0; r < C::BM / 32; r++) {
-                        sLSE[st * C::BM + lane + 32 * r] = -lv[r];
-                        sDLT[st * C::BM + lane + 32 * r] = -dv[r];
+                        sLSE[(gs & 1) * C::BM + lane + 32 * r] = -lv[r];
+                        sDLT[(gs & 1) * C::BM + lane + 32 * r] = -dv[r];
                     }
                     mbar_arrive(bar(C::B_Q_FULL + st));
+                    if constexpr (C::QSHADOW) {
+                        // this CTA's half of Q(gs) again, for dK(gs), once dK(gs - 1) has
+                        // read the previous one
+                        if (!mbar_wait_warp(bar(C::B_QSH_EMPTY), (uint32_t)(gs & 1) ^ 1u, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(bar(C::B_QSH_FULL), C::TQSH);
+                            for (int c = 0; c < C::DH / 64; c++)
+                                tma_load_3d(sQsh + c * C::CBQ, &tmQ, bar(C::B_QSH_FULL), (I.h * (C::DH / 64) + c) * 64,
+                                            m * C::BM, bhq);
+                        }
+                        qsh_issued++;
+                    }
                 }
             }
             if (!ok && lane == 0) {
@@ -497,6 +524,8 @@ __global__ void __launch_bounds__(512, 1)
                     const int L = issued - back;
                     mbar_wait_drain(bar(C::B_Q_FULL + L % C::QST), (uint32_t)((L / C::QST) & 1), 200000000ull);
                 }
+                if (C::QSHADOW && qsh_issued > 0)
+                    mbar_wait_drain(bar(C::B_QSH_FULL), (uint32_t)((qsh_issued - 1) & 1), 200000000ull);
             }
         } else if (warp == C::W_MMA && lane == 0) {
             // ------------------------------------------------------ MMA issuer
@@ -543,6 +572,8 @@ __global__ void __launch_bounds__(512, 1)
                         tc_fence_after();
                     }
                     bwd_mma_dv<C>(tmem, sdO + h_q, i == 0);
+                    // with the Q shadow, dV(gs) is the stage's last reader
+                    if constexpr (C::QSHADOW) tc_commit(bar(C::B_Q_EMPTY + st));
                     // S^T(gs + 1) over S^T(gs) / P^T(gs): phase A has read S^T(gs), and
                     // dV(gs) is ahead of it on the tensor cores. It runs while the compute
                     // warps form dS of step gs. With a single Q/dO stage Q(gs + 1) can
@@ -560,8 +591,15 @@ __global__ void __launch_bounds__(512, 1)
                     // layer.)
                     if (!(ok = mbar_wait(bar(C::B_DS_FULL), (uint32_t)(gs & 1), abort_flag))) break;
                     tc_fence_after();
-                    bwd_mma_dk<C>(tmem, sdS, sQ + h_q, i == 0);
-                    tc_commit(bar(C::B_Q_EMPTY + st));  // Q, dO of this step read by every product issued
+                    if constexpr (C::QSHADOW) {
+                        if (!(ok = mbar_wait(bar(C::B_QSH_FULL), (uint32_t)(gs & 1), abort_flag))) break;
+                        tc_fence_after();
+                        bwd_mma_dk<C>(tmem, sdS, sQsh, i == 0);
+                        tc_commit(bar(C::B_QSH_EMPTY));
+                    } else {
+                        bwd_mma_dk<C>(tmem, sdS, sQ + h_q, i == 0);
+                        tc_commit(bar(C::B_Q_EMPTY + st));  // Q, dO of this step read by every product issued
+                    }
                     // the drain warps must have emptied the previous dQ (in the aliased
                     // layout they did so before dP^T(gs) was issued)
                     if (!C::DQ_ALIAS && gs > 0) {
@@ -620,8 +658,8 @@ __global__ void __launch_bounds__(512, 1)
                 if (!(ok = mbar_wait_warp(bar(C::B_Q_FULL + st), (uint32_t)((gs / C::QST) & 1), abort_flag))) break;
                 if (!(ok = mbar_wait_warp(bar(C::B_S_FULL), (uint32_t)(gs & 1), abort_flag))) break;
                 tc_fence_after();
-                const float *nls = sLSE + st * C::BM;
-                const float *nds = sDLT + st * C::BM;
+                const float *nls = sLSE + (gs & 1) * C::BM;
+                const float *nds = sDLT + (gs & 1) * C::BM;
                 const bool mask = (I.k0 + C::BN - 1 > qb) || (W > 0 && I.k0 <= qb + C::BM - 1 - W);
                 float g[C::HALF / 32][32];
 #pragma unroll
