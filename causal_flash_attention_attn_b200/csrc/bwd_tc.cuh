@@ -84,6 +84,10 @@ struct BwdTc {
     // head dim 256 (one Q/dO stage): this CTA's half of Q again, for dK, so that the
     // stage is free for the next step's Q and dO once dV has read it
     static constexpr bool QSHADOW = D == 256;
+    // head dim 64: the drain warps, whose dQ leaves by TMA, also write the item's
+    // dV rows, so the compute warps go straight on to the next item's first step
+    // (elsewhere the compute warps write dV while the drain warps write dK)
+    static constexpr bool DV_BY_DRAIN = D == 64;
     static constexpr uint32_t OFF_QSH = OFF_STG + (BULK_DQ ? NSTG * STG : 0);
     static constexpr uint32_t TQSH = (DH / 64) * CBQ;
     static constexpr uint32_t TILES = OFF_QSH + (QSHADOW ? TQSH : 0);
@@ -100,11 +104,11 @@ struct BwdTc {
     static constexpr uint32_t SLACK = (TILES + CTRL + 1024 <= 232448) ? 1024 : 0;
     static constexpr uint32_t SMEM = SLACK + TILES + CTRL;
     // Roles: warps 0-7 compute (warp w: TMEM lanes 32 (w % 4).., query-row half
-    // w / 4 of the step), 8-11 dQ drain and dK epilogue, 12 loads, 13 MMA issue
-    // and TMEM owner, 14-15 idle (they complete the fourth warpgroup). Launched
-    // at 128 registers a thread; the fourth warpgroup gives back down to
-    // REG_CTRL, the compute warpgroups grow to REG_COMPUTE, the drain
-    // warpgroup to REG_DRAIN.
+    // w / 4 of the step), 8-11 dQ drain and dK (head dim 64: and dV) epilogue,
+    // 12 loads, 13 MMA issue and TMEM owner, 14-15 idle (they complete the fourth
+    // warpgroup). Launched at 128 registers a thread; the fourth warpgroup gives
+    // back down to REG_CTRL, the compute warpgroups grow to REG_COMPUTE, the
+    // drain warpgroup to REG_DRAIN.
     static constexpr int THREADS = 512;
     static constexpr int W_DRAIN = 8, W_LOAD = 12, W_MMA = 13;
     static constexpr int REG_LAUNCH = 128, REG_CTRL = 80, REG_COMPUTE = 144, REG_DRAIN = 144;
@@ -138,7 +142,8 @@ struct BwdTc {
     static constexpr int B_DQ_FULL = B_DP_FULL + 1;
     static constexpr int B_DQ_FREE = B_DQ_FULL + 1;
     static constexpr int B_KDONE = B_DQ_FREE + 1;        // a work item's dK, dV complete in TMEM
-    static constexpr int B_EPI_DONE = B_KDONE + 1;       // ... and read out (8 compute + 4 drain warps)
+    static constexpr int B_EPI_DONE = B_KDONE + 1;       // ... and read out (4 drain warps, + 8 compute
+                                                          // warps unless DV_BY_DRAIN)
     static constexpr int B_QSH_FULL = B_EPI_DONE + 1;    // the Q half for dK has landed (QSHADOW)
     static constexpr int B_QSH_EMPTY = B_QSH_FULL + 1;   // ... and dK has read it
     static constexpr int NBAR = B_QSH_EMPTY + 1;
@@ -190,6 +195,26 @@ struct BwdStep {
         }
     }
 };
+
+// Epilogue of a work item: columns [c_lo, c_hi) of this thread's TMEM lane (one
+// key row of dK or dV, f32, from TMEM address `taddr`) as bf16 to `row`; the
+// stores are skipped for a row past the sequence end
+__device__ __forceinline__ void bwd_row_out(uint32_t taddr, __nv_bfloat16 *row, int c_lo, int c_hi, bool valid) {
+#pragma unroll 1
+    for (int c0 = c_lo; c0 < c_hi; c0 += 32) {
+        uint32_t o[32];
+        tmem_ld32(taddr + (uint32_t)c0, o);
+        tmem_ld_wait(o);
+        uint32_t w16[16];
+#pragma unroll
+        for (int e = 0; e < 16; e++) w16[e] = pack_bf16x2(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1]));
+        if (valid) {
+            uint4 *dst = reinterpret_cast<uint4 *>(row + c0);
+#pragma unroll
+            for (int e = 0; e < 4; e++) dst[e] = make_uint4(w16[4 * e], w16[4 * e + 1], w16[4 * e + 2], w16[4 * e + 3]);
+        }
+    }
+}
 
 // f32 reduction into global memory with an L2 cache-policy hint
 __device__ __forceinline__ void red_add_f32_hint(float *addr, float v, uint64_t policy) {
@@ -409,7 +434,7 @@ __global__ void __launch_bounds__(512, 1)
         mbar_init(bar(C::B_DQ_FULL), 1);
         mbar_init(bar(C::B_DQ_FREE), 4);
         mbar_init(bar(C::B_KDONE), 1);
-        mbar_init(bar(C::B_EPI_DONE), 12);
+        mbar_init(bar(C::B_EPI_DONE), C::DV_BY_DRAIN ? 4 : 12);
         mbar_init(bar(C::B_QSH_FULL), 1);
         mbar_init(bar(C::B_QSH_EMPTY), 1);
         *abort_flag = 0;
@@ -701,31 +726,20 @@ __global__ void __launch_bounds__(512, 1)
                 if (lane == 0) mbar_arrive(bar(C::B_DS_FULL));
             }
             if (!ok) break;
-            // epilogue of the item: dV rows, this warp's half of the columns
-            if (!(ok = mbar_wait_warp(bar(C::B_KDONE), (uint32_t)(pass & 1), abort_flag))) break;
-            tc_fence_after();
-            __nv_bfloat16 *row = p.dv + ((size_t)I.bkv * p.T + (size_t)min(kj, p.T - 1)) * D + I.h * C::DH;
-#pragma unroll 1
-            for (int c0 = hc * (C::DH / 2); c0 < (hc + 1) * (C::DH / 2); c0 += 32) {
-                uint32_t o[32];
-                tmem_ld32(tmem + lane_base + C::COL_DV + c0, o);
-                tmem_ld_wait(o);
-                uint32_t w16[16];
-#pragma unroll
-                for (int e = 0; e < 16; e++) w16[e] = pack_bf16x2(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1]));
-                if (kj < p.T) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(row + c0);
-#pragma unroll
-                    for (int e = 0; e < 4; e++) dst[e] = make_uint4(w16[4 * e], w16[4 * e + 1], w16[4 * e + 2], w16[4 * e + 3]);
-                }
+            if constexpr (!C::DV_BY_DRAIN) {
+                // epilogue of the item: dV rows, this warp's half of the columns
+                if (!(ok = mbar_wait_warp(bar(C::B_KDONE), (uint32_t)(pass & 1), abort_flag))) break;
+                tc_fence_after();
+                __nv_bfloat16 *row = p.dv + ((size_t)I.bkv * p.T + (size_t)min(kj, p.T - 1)) * D + I.h * C::DH;
+                bwd_row_out(tmem + lane_base + C::COL_DV, row, hc * (C::DH / 2), (hc + 1) * (C::DH / 2), kj < p.T);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::B_EPI_DONE));
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::B_EPI_DONE));
         }
     } else {
         setmaxnreg_inc<C::REG_DRAIN>();
-        // -------------------------------- dQ drain (warps 8..11), dK epilogue
+        // -------------------------------- dQ drain (warps 8..11), dK (and dV) epilogue
         const int t = threadIdx.x - 32 * C::W_DRAIN;  // TMEM lane of this thread
         const uint32_t lane_base = (uint32_t)((warp - C::W_DRAIN) * 32) << 16;
         bool ok = true;
@@ -797,25 +811,13 @@ __global__ void __launch_bounds__(512, 1)
                 }
             }
             if (!ok) break;
-            // epilogue of the item: dK rows
+            // epilogue of the item: dK rows (and dV rows where the drain warps take them)
             if (!(ok = mbar_wait_warp(bar(C::B_KDONE), (uint32_t)(pass & 1), abort_flag))) break;
             tc_fence_after();
             const int kj = I.k0 + t;
-            __nv_bfloat16 *row = p.dk + ((size_t)I.bkv * p.T + (size_t)min(kj, p.T - 1)) * D + I.h * C::DH;
-#pragma unroll 1
-            for (int c0 = 0; c0 < C::DH; c0 += 32) {
-                uint32_t o[32];
-                tmem_ld32(tmem + lane_base + C::COL_DK + c0, o);
-                tmem_ld_wait(o);
-                uint32_t w16[16];
-#pragma unroll
-                for (int e = 0; e < 16; e++) w16[e] = pack_bf16x2(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1]));
-                if (kj < p.T) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(row + c0);
-#pragma unroll
-                    for (int e = 0; e < 4; e++) dst[e] = make_uint4(w16[4 * e], w16[4 * e + 1], w16[4 * e + 2], w16[4 * e + 3]);
-                }
-            }
+            const size_t roff = ((size_t)I.bkv * p.T + (size_t)min(kj, p.T - 1)) * D + I.h * C::DH;
+            bwd_row_out(tmem + lane_base + C::COL_DK, p.dk + roff, 0, C::DH, kj < p.T);
+            if constexpr (C::DV_BY_DRAIN) bwd_row_out(tmem + lane_base + C::COL_DV, p.dv + roff, 0, C::DH, kj < p.T);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(C::B_EPI_DONE));

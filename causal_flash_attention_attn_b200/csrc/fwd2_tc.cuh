@@ -33,7 +33,10 @@ struct Fwd2Tc {
     static constexpr int NCB = D / 64;
     static constexpr uint32_t CB = 128 * 128;          // column block of a 128-row tile
     static constexpr uint32_t TILE = NCB * CB;         // one 128 x D bf16 tile
-    static constexpr int NSTAGE = D == 128 ? 4 : 8;
+    // K/V ring: four tiles (K and V of two KV tiles). At head dim 64 eight were
+    // slower on short sequences: the larger first burst of loads from every CTA
+    // delays the first scores (T = 512: forward 38.8 against 39.3 us)
+    static constexpr int NSTAGE = 4;
     // Q buffers (tiles A and B each): two at head dim 64, so that the next work
     // item's queries load while the current item runs; one at head dim 128,
     // where shared memory has no room for a second
