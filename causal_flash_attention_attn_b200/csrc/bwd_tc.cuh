@@ -41,10 +41,11 @@
 // during phase B, and dP^T(i + 1) during phase A of step i + 1.
 //
 // Roles (512 threads): warps 0-7 compute (warp w: key rows = TMEM lanes
-// 32 (w % 4).., query-row half w / 4 of the step), warps 8-11 dQ drain + dK
-// epilogue, warp 12 loads (TMA for tiles, plain loads for LSE and Delta), warp
-// 13 issues MMAs and owns TMEM, warps 14-15 idle (see BwdTc for the register
-// split).
+// 32 (w % 4).., query-row half w / 4 of the step; they also write each item's
+// dV rows, except at head dim 64), warps 8-11 dQ drain + dK epilogue (+ dV at
+// head dim 64), warp 12 loads (TMA for tiles, plain loads for LSE and Delta),
+// warp 13 issues MMAs and owns TMEM, warps 14-15 idle (see BwdTc for the
+// register split).
 #pragma once
 
 #include "sm100.cuh"
