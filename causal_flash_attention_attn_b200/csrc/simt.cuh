@@ -70,12 +70,21 @@ constexpr size_t simt_fwd_smem() {
     return sizeof(float) * (size_t)(kSimtRows * DK + kSimtTile * (DK + 1) + kSimtTile * (DV + 1));
 }
 
+// Minimum resident CTAs a kernel asks ptxas to allow for: as many as its shared
+// memory admits on one SM (228 KB, 1 KB of it reserved per CTA), at most eight.
+// The register cap this implies never costs occupancy that shared memory does not
+// already cost, and it leaves ptxas room to keep the accumulators out of local memory.
+constexpr int simt_min_blocks(size_t smem) {
+    return (int)(233472 / (smem + 1024)) < 8 ? (int)(233472 / (smem + 1024)) : 8;
+}
+
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(kSimtThreads) simt_fwd(const T *__restrict__ q, const T *__restrict__ k,
-                                                         const T *__restrict__ v, T *__restrict__ o,
-                                                         float *__restrict__ lse, int Hq, int Hkv, int T_,
-                                                         float scale, int window, float softcap,
-                                                         const float *__restrict__ sink, float *__restrict__ max_logit) {
+__global__ void __launch_bounds__(kSimtThreads, simt_min_blocks(simt_fwd_smem<DK, DV>()))
+    simt_fwd(const T *__restrict__ q, const T *__restrict__ k,
+             const T *__restrict__ v, T *__restrict__ o,
+             float *__restrict__ lse, int Hq, int Hkv, int T_,
+             float scale, int window, float softcap,
+             const float *__restrict__ sink, float *__restrict__ max_logit) {
     extern __shared__ float sm[];
     float *sQ = sm;
     float *sK = sQ + kSimtRows * DK;
@@ -154,11 +163,12 @@ constexpr size_t simt_bwd_dq_smem() {
 }
 
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(kSimtThreads) simt_bwd_dq(const T *__restrict__ q, const T *__restrict__ k,
-                                                            const T *__restrict__ v, const float *__restrict__ lse,
-                                                            const T *__restrict__ dO, const float *__restrict__ delta,
-                                                            T *__restrict__ dq, int Hq, int Hkv, int T_, float scale,
-                                                            int window, float softcap) {
+__global__ void __launch_bounds__(kSimtThreads, simt_min_blocks(simt_bwd_dq_smem<DK, DV>()))
+    simt_bwd_dq(const T *__restrict__ q, const T *__restrict__ k,
+                const T *__restrict__ v, const float *__restrict__ lse,
+                const T *__restrict__ dO, const float *__restrict__ delta,
+                T *__restrict__ dq, int Hq, int Hkv, int T_, float scale,
+                int window, float softcap) {
     extern __shared__ float sm[];
     float *sQ = sm;
     float *sdO = sQ + kSimtRows * DK;
@@ -231,12 +241,13 @@ constexpr size_t simt_bwd_dkdv_smem() {
 }
 
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(kSimtThreads) simt_bwd_dkdv(const T *__restrict__ q, const T *__restrict__ k,
-                                                              const T *__restrict__ v, const float *__restrict__ lse,
-                                                              const T *__restrict__ dO,
-                                                              const float *__restrict__ delta, T *__restrict__ dk,
-                                                              T *__restrict__ dv, int Hq, int Hkv, int T_,
-                                                              float scale, int window, float softcap) {
+__global__ void __launch_bounds__(kSimtThreads, simt_min_blocks(simt_bwd_dkdv_smem<DK, DV>()))
+    simt_bwd_dkdv(const T *__restrict__ q, const T *__restrict__ k,
+                  const T *__restrict__ v, const float *__restrict__ lse,
+                  const T *__restrict__ dO,
+                  const float *__restrict__ delta, T *__restrict__ dk,
+                  T *__restrict__ dv, int Hq, int Hkv, int T_,
+                  float scale, int window, float softcap) {
     extern __shared__ float sm[];
     float *sK = sm;                          // [16][DK] key rows of this block
     float *sV = sK + kSimtRows * DK;         // [16][DV]
