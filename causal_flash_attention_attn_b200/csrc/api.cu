@@ -51,6 +51,14 @@ forge_status check_scalars(float scale, int window, float softcap) {
 
 int effective_window(int window, int T) { return (window >= T) ? 0 : window; }
 
+// Grid for kernels that take one (batch, head) pair per block row: the pairs go
+// on y, and past the 65535 that y allows, on z (the kernels' `pair_index`); x
+// is the kernel's own split of the rows or keys.
+dim3 pair_grid(unsigned x, long long pairs) {
+    const long long y = pairs < 65535 ? pairs : 65535;
+    return dim3(x, (unsigned)y, (unsigned)((pairs + y - 1) / y));
+}
+
 // ------------------------------------------------------------- workspace layout
 // [ delta: B*Hq*T f32, 256-aligned ][ dq accumulator: B*Hq*Tpad*D f32 (bf16 only) ]
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -266,10 +274,10 @@ forge_status fwd_simt(const void *q, const void *k, const void *v, void *o, floa
                       float scale, int window, float softcap, const float *sink, float *max_logit, cudaStream_t st) {
     const size_t sm = simt_fwd_smem<DK, DV>();
     if (set_smem(simt_fwd<T_, DK, DV>, sm) != FORGE_OK) return FORGE_ERR_CUDA;
-    dim3 grid((T + kSimtRows - 1) / kSimtRows, B * Hq);
+    const dim3 grid = pair_grid((unsigned)((T + kSimtRows - 1) / kSimtRows), (long long)B * Hq);
     simt_fwd<T_, DK, DV><<<grid, kSimtThreads, sm, st>>>(static_cast<const T_ *>(q), static_cast<const T_ *>(k),
                                                      static_cast<const T_ *>(v), static_cast<T_ *>(o), lse, Hq, Hkv,
-                                                     T, scale, window, softcap, sink, max_logit);
+                                                     T, scale, window, softcap, sink, max_logit, B * Hq);
     return launch_status();
 }
 
@@ -280,17 +288,17 @@ forge_status bwd_simt(const void *q, const void *k, const void *v, const float *
     const size_t sm1 = simt_bwd_dq_smem<DK, DV>(), sm2 = simt_bwd_dkdv_smem<DK, DV>();
     if (set_smem(simt_bwd_dq<T_, DK, DV>, sm1) != FORGE_OK || set_smem(simt_bwd_dkdv<T_, DK, DV>, sm2) != FORGE_OK)
         return FORGE_ERR_CUDA;
-    dim3 g1((T + kSimtRows - 1) / kSimtRows, B * Hq);
+    const dim3 g1 = pair_grid((unsigned)((T + kSimtRows - 1) / kSimtRows), (long long)B * Hq);
     simt_bwd_dq<T_, DK, DV><<<g1, kSimtThreads, sm1, st>>>(
         static_cast<const T_ *>(q), static_cast<const T_ *>(k), static_cast<const T_ *>(v), lse,
-        static_cast<const T_ *>(dO), delta, static_cast<T_ *>(dq), Hq, Hkv, T, scale, window, softcap);
+        static_cast<const T_ *>(dO), delta, static_cast<T_ *>(dq), Hq, Hkv, T, scale, window, softcap, B * Hq);
     forge_status s = launch_status();
     if (s != FORGE_OK) return s;
-    dim3 g2((T + kSimtRows - 1) / kSimtRows, B * Hkv);
+    const dim3 g2 = pair_grid((unsigned)((T + kSimtRows - 1) / kSimtRows), (long long)B * Hkv);
     simt_bwd_dkdv<T_, DK, DV><<<g2, kSimtThreads, sm2, st>>>(
         static_cast<const T_ *>(q), static_cast<const T_ *>(k), static_cast<const T_ *>(v), lse,
         static_cast<const T_ *>(dO), delta, static_cast<T_ *>(dk), static_cast<T_ *>(dv), Hq, Hkv, T, scale, window,
-        softcap);
+        softcap, B * Hkv);
     return launch_status();
 }
 
@@ -426,7 +434,7 @@ template <typename T_, int D, int MG>
 forge_status decode_split_launch(const void *q, const void *kc, const void *vc, const DecParams &p, cudaStream_t st) {
     using C = DecCfg<T_, D>;
     if (set_smem(decode_split<T_, D, MG>, C::smem(MG)) != FORGE_OK) return FORGE_ERR_CUDA;
-    decode_split<T_, D, MG><<<dim3((unsigned)p.nsplit, (unsigned)(p.B * p.Hkv)), kDecThreads,
+    decode_split<T_, D, MG><<<pair_grid((unsigned)p.nsplit, (long long)p.B * p.Hkv), kDecThreads,
                               C::smem(p.Hq / p.Hkv), st>>>(static_cast<const T_ *>(q), static_cast<const T_ *>(kc),
                                                            static_cast<const T_ *>(vc), p);
     return launch_status();
@@ -445,7 +453,7 @@ forge_status decode_pick(const void *q, const void *kc, const void *vc, const De
     if constexpr (decode_warp_fits<T_, D, MG>()) {
         using C = DecWCfg<T_, D, MG>;
         if (set_smem(decode_split_warp<T_, D, MG>, C::SMEM) != FORGE_OK) return FORGE_ERR_CUDA;
-        decode_split_warp<T_, D, MG><<<dim3((unsigned)p.nsplit, (unsigned)(p.B * p.Hkv)), kDecWarps * 32, C::SMEM,
+        decode_split_warp<T_, D, MG><<<pair_grid((unsigned)p.nsplit, (long long)p.B * p.Hkv), kDecWarps * 32, C::SMEM,
                                        st>>>(static_cast<const T_ *>(q), static_cast<const T_ *>(kc),
                                              static_cast<const T_ *>(vc), p);
         return launch_status();

@@ -103,7 +103,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_split(const T_ *__restrict
     using C = DecCfg<T_, D>;
     extern __shared__ __align__(16) uint8_t dsm[];
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-    const int bkv = blockIdx.y, b = bkv / p.Hkv, hkv = bkv % p.Hkv, split = blockIdx.x;
+    const int bkv = pair_index(), b = bkv / p.Hkv, hkv = bkv % p.Hkv, split = blockIdx.x;
+    if (bkv >= p.B * p.Hkv) return;
     const int G = p.Hq / p.Hkv;
     float *q_s = reinterpret_cast<float *>(dsm);  // [G][SQ][QP], pre-scaled
     float *p_s = q_s + G * C::SQ * C::QP;         // [G][KT] scores, then probabilities
@@ -425,7 +426,8 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_split_warp(const T_ *__
     using C = DecWCfg<T_, D, MG>;
     extern __shared__ __align__(16) uint8_t dsm[];
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-    const int bkv = blockIdx.y, b = bkv / p.Hkv, hkv = bkv % p.Hkv, split = blockIdx.x;
+    const int bkv = pair_index(), b = bkv / p.Hkv, hkv = bkv % p.Hkv, split = blockIdx.x;
+    if (bkv >= p.B * p.Hkv) return;
     const int G = p.Hq / p.Hkv;
     const uint32_t ring = smem_u32(dsm) + (uint32_t)(warp * C::NST * C::STAGEB);
     const uint32_t bars = smem_u32(dsm + C::OFF_BAR) + (uint32_t)(warp * C::NST * 8);

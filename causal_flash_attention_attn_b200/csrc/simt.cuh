@@ -44,6 +44,11 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
+// Index of the (batch, head) pair a block works on. Launches put the pairs on
+// grid y and, past the 65535 that y allows, on z (host side: `pair_grid`); the
+// blocks of the last z slice beyond the pair count return before any work.
+__device__ __forceinline__ int pair_index() { return (int)(blockIdx.y + gridDim.y * blockIdx.z); }
+
 // Visible iff kj <= qi and (window == 0 or kj > qi - window).
 __device__ __forceinline__ bool visible(int qi, int kj, int window) {
     return kj <= qi && (window == 0 || kj > qi - window);
@@ -84,13 +89,14 @@ __global__ void __launch_bounds__(kSimtThreads, simt_min_blocks(simt_fwd_smem<DK
              const T *__restrict__ v, T *__restrict__ o,
              float *__restrict__ lse, int Hq, int Hkv, int T_,
              float scale, int window, float softcap,
-             const float *__restrict__ sink, float *__restrict__ max_logit) {
+             const float *__restrict__ sink, float *__restrict__ max_logit, int npairs) {
     extern __shared__ float sm[];
     float *sQ = sm;
     float *sK = sQ + kSimtRows * DK;
     float *sV = sK + kSimtTile * (DK + 1);
     constexpr int NT = DV / 32;
-    const int bh = blockIdx.y, b = bh / Hq, hq = bh % Hq, hkv = hq / (Hq / Hkv);
+    const int bh = pair_index(), b = bh / Hq, hq = bh % Hq, hkv = hq / (Hq / Hkv);
+    if (bh >= npairs) return;
     const int r0 = blockIdx.x * kSimtRows;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const T *Qb = q + (size_t)bh * T_ * DK;
@@ -168,14 +174,15 @@ __global__ void __launch_bounds__(kSimtThreads, simt_min_blocks(simt_bwd_dq_smem
                 const T *__restrict__ v, const float *__restrict__ lse,
                 const T *__restrict__ dO, const float *__restrict__ delta,
                 T *__restrict__ dq, int Hq, int Hkv, int T_, float scale,
-                int window, float softcap) {
+                int window, float softcap, int npairs) {
     extern __shared__ float sm[];
     float *sQ = sm;
     float *sdO = sQ + kSimtRows * DK;
     float *sK = sdO + kSimtRows * DV;
     float *sV = sK + kSimtTile * (DK + 1);
     constexpr int NT = DK / 32;
-    const int bh = blockIdx.y, b = bh / Hq, hq = bh % Hq, hkv = hq / (Hq / Hkv);
+    const int bh = pair_index(), b = bh / Hq, hq = bh % Hq, hkv = hq / (Hq / Hkv);
+    if (bh >= npairs) return;
     const int r0 = blockIdx.x * kSimtRows;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const T *Kb = k + (size_t)(b * Hkv + hkv) * T_ * DK;
@@ -247,7 +254,7 @@ __global__ void __launch_bounds__(kSimtThreads, simt_min_blocks(simt_bwd_dkdv_sm
                   const T *__restrict__ dO,
                   const float *__restrict__ delta, T *__restrict__ dk,
                   T *__restrict__ dv, int Hq, int Hkv, int T_,
-                  float scale, int window, float softcap) {
+                  float scale, int window, float softcap, int npairs) {
     extern __shared__ float sm[];
     float *sK = sm;                          // [16][DK] key rows of this block
     float *sV = sK + kSimtRows * DK;         // [16][DV]
@@ -256,7 +263,8 @@ __global__ void __launch_bounds__(kSimtThreads, simt_min_blocks(simt_bwd_dkdv_sm
     float *sL = sdO + kSimtTile * (DV + 1);  // [32]
     float *sD = sL + kSimtTile;              // [32]
     constexpr int NK = DK / 32, NV = DV / 32;
-    const int bkv = blockIdx.y, b = bkv / Hkv, hkv = bkv % Hkv;
+    const int bkv = pair_index(), b = bkv / Hkv, hkv = bkv % Hkv;
+    if (bkv >= npairs) return;
     const int G = Hq / Hkv;
     const int r0 = blockIdx.x * kSimtRows;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
